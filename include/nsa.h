@@ -1,0 +1,182 @@
+/*
+ * nsa.h — C ABI of libnsa.so: Native Sparse Attention (NSA) forward on one
+ * NVIDIA B200 (sm_100a), causal prefill and KV-cache decode.
+ *
+ * The method (sources, cited by page title and section):
+ *   "Native Sparse Attention" lesson, aiengineeringfromscratch.com (Phase 10,
+ *   lesson 17), sections "Concept / three parallel branches" and "Compute budget";
+ *   "Разреженное внимание — NSA и DSA", ai.flicky.cc (stage 5.5, lesson 02),
+ *   section "NSA: три ветви" (equation for o_t), "Ветвь отбора", "Практика".
+ *
+ * For each query position t and query head h (KV head g = h / G, G = H_q/H_kv):
+ *   o_t = g_cmp * Attn(q, K_cmp, V_cmp) + g_slc * Attn(q, K_slc, V_slc)
+ *       + g_win * Attn(q, K_win, V_win)
+ * where K_cmp/V_cmp are compressed block summaries (blocks of l tokens, stride s),
+ * K_slc/V_slc are the raw tokens of the top-n selection blocks (size l') chosen
+ * per GQA group from the compressed-attention probabilities, and K_win/V_win are
+ * the last w tokens. Softmax scale 1/sqrt(d_k) unless `scale` is set.
+ *
+ * Conventions shared by every entry point:
+ *  - Memory: every pointer argument is DEVICE memory unless its comment says
+ *    HOST. The caller allocates and owns all buffers, including the workspace;
+ *    the library allocates no memory and keeps no state between calls (except
+ *    the opt-in profiler's CUDA events, see nsa_profile_enable).
+ *  - Layout: row-major, contiguous, 16-byte aligned base pointers. bf16 is
+ *    IEEE bfloat16 (2 bytes); fp32 is IEEE binary32.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). Returns once enqueued.
+ *  - Errors: arguments are validated on the host before anything is launched;
+ *    on any error nothing is written and nothing is launched.
+ *    NSA_ERR_INVALID_ARG: null/misaligned pointer, non-positive size,
+ *    inconsistent lengths. NSA_ERR_UNSUPPORTED: valid but not built (head dims,
+ *    group size, block parameters; see below). NSA_ERR_WORKSPACE: ws_bytes below
+ *    nsa_workspace_size(). NSA_ERR_CUDA: a CUDA launch or driver call failed.
+ *    NSA_ERR_DEVICE_CHECK: returned only by nsa_check_device_status() when a
+ *    kernel recorded a failure (a bounded wait ran out).
+ *  - Supported: d_k in {64, 128, 192}, d_v in {64, 128}, G in {1, 2, 4, 8, 16},
+ *    l_cmp = 32, stride = 16, l_sel = 64, 1 <= top_n <= 32, window >= 1,
+ *    force_first + force_local <= top_n, batch <= NSA_MAX_BATCH.
+ *  - Workspace: the first 256 bytes hold a device status word. Call
+ *    nsa_workspace_init() once on a new workspace before its first use.
+ */
+#ifndef NSA_H_
+#define NSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NSA_MAX_BATCH 128
+
+typedef enum {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARG = 1,
+  NSA_ERR_UNSUPPORTED = 2,
+  NSA_ERR_WORKSPACE = 3,
+  NSA_ERR_CUDA = 4,
+  NSA_ERR_DEVICE_CHECK = 5
+} nsa_status_t;
+
+/* Method parameters (NSA-ru "NSA: три ветви"): compression block l_cmp with
+ * stride `stride`; selection block l_sel; top_n selected blocks per GQA group,
+ * of which force_first initial blocks and force_local local blocks (the block
+ * holding t and the ones just before it) are always taken; sliding window of
+ * `window` keys ending at t; scale = softmax scale, 0 means 1/sqrt(d_k). */
+typedef struct {
+  int32_t l_cmp, stride, l_sel, top_n, window, force_first, force_local;
+  float scale;
+} nsa_params_t;
+
+/* Head geometry: H_q query heads share H_kv key/value heads (GQA, G = H_q/H_kv). */
+typedef struct {
+  int32_t H_q, H_kv, d_k, d_v;
+} nsa_heads_t;
+
+enum { NSA_OP_COMPRESS = 0, NSA_OP_PREFILL = 1, NSA_OP_DECODE = 2 };
+
+/* Bytes of workspace `op` needs. `batch` = number of sequences;
+ * `total_tokens` = sum of sequence lengths (prefill), ignored otherwise;
+ * `max_len` = longest sequence (prefill) or upper bound of the cache lengths
+ * (decode). Returns 0 for invalid arguments. */
+size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* params,
+                          int32_t batch, int64_t total_tokens, int32_t max_len);
+
+/* Zero the workspace header (status word) on `stream`. */
+nsa_status_t nsa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the device status word. Returns NSA_OK,
+ * NSA_ERR_DEVICE_CHECK (a kernel recorded a failed bounded wait; its outputs are
+ * not valid) or NSA_ERR_CUDA. */
+nsa_status_t nsa_check_device_status(void* workspace, void* stream);
+
+/* Block compression (NSA-ru "Сжатая ветвь"; NSA-lesson "Concept"): for every
+ * sequence b and every whole block i (i*stride + l_cmp <= len_b):
+ *   k_cmp[i] = sum_{r<l} sum_e (k[i*stride + r, g, e] + pe_k[r, e]) * w_ck[r*d_k + e, :]
+ * and the same for v with w_cv, pe_v. The flattened block is token-major.
+ * Arithmetic: k, v and W rounded to bf16 once, fp32 accumulation; the position
+ * term sum(pe*W) is added in fp32; outputs rounded to bf16.
+ *   k        bf16, token t of sequence b at row tok_offset[b] + t: [*, H_kv, d_k]
+ *   v        bf16, same rows: [*, H_kv, d_v]
+ *   w_ck     fp32 [l_cmp*d_k, d_k];  pe_k fp32 [l_cmp, d_k]
+ *   w_cv     fp32 [l_cmp*d_v, d_v];  pe_v fp32 [l_cmp, d_v]
+ *   tok_offset HOST int64 [batch]: first row of each sequence in k / v
+ *   seq_len    HOST int32 [batch]: tokens of each sequence (>= 0)
+ *   cmp_offset HOST int64 [batch]: first output row of each sequence
+ *   k_cmp    bf16 out: rows cmp_offset[b] .. + n_cmp(len_b) - 1 of [*, H_kv, d_k]
+ *   v_cmp    bf16 out: same rows of [*, H_kv, d_v]
+ * n_cmp(L) = (L - l_cmp)/stride + 1 for L >= l_cmp, else 0. Packed prefill uses
+ * tok_offset = cu_seqlens[b], cmp_offset = running sum of n_cmp; a batched
+ * cache [B, Lmax, H_kv, d] uses tok_offset = b*Lmax, cmp_offset = b*Lmax_cmp. */
+nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const float* pe_k,
+                          const float* w_cv, const float* pe_v, const int64_t* tok_offset,
+                          const int32_t* seq_len, const int64_t* cmp_offset, int32_t batch,
+                          const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
+                          void* v_cmp, void* workspace, size_t ws_bytes, void* stream);
+
+/* Causal NSA prefill over packed variable-length sequences (NSA-ru "NSA: три
+ * ветви"; NSA-lesson "Concept"). Positions restart at 0 in every sequence.
+ *   q        bf16 [N, H_q, d_k], N = cu_seqlens[batch]
+ *   k, v     bf16 [N, H_kv, d_k], [N, H_kv, d_v]
+ *   k_cmp, v_cmp bf16 [sum_b n_cmp(len_b), H_kv, d_k / d_v], packed in sequence
+ *            order (as written by nsa_compress with cmp_offset = running sum)
+ *   gates    fp32 [N, H_q, 3] in the order (cmp, slc, win)
+ *   cu_seqlens HOST int32 [batch + 1], non-decreasing, cu_seqlens[0] = 0
+ *   out      bf16 out [N, H_q, d_v]
+ *   sel_out  int32 out or NULL: [N, H_kv, top_n] selected block indices per
+ *            (token, KV head), ascending, padded with -1
+ *   imp_out  fp32 out or NULL: [N, H_kv, n_blk(max_len)] selection-block
+ *            importance (entries beyond the token's own block are unspecified)
+ * The workspace (nsa_workspace_size(NSA_OP_PREFILL, ...)) must not overlap any
+ * argument. Selection ties go to the lower block index. */
+nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void* k_cmp,
+                         const void* v_cmp, const float* gates, const int32_t* cu_seqlens,
+                         int32_t batch, const nsa_heads_t* heads, const nsa_params_t* params,
+                         void* out, int32_t* sel_out, float* imp_out, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* NSA decode: one new query per sequence against a KV cache that already holds
+ * the new token, so the query sits at position cache_lens[b] - 1.
+ *   q            bf16 [batch, H_q, d_k]
+ *   k_cache      bf16 [batch, Lmax, H_kv, d_k];  v_cache bf16 [batch, Lmax, H_kv, d_v]
+ *   k_cmp_cache  bf16 [batch, Lmax_cmp, H_kv, d_k]; v_cmp_cache likewise with d_v;
+ *                entries 0 .. n_cmp(cache_lens[b]) - 1 must be valid
+ *   cache_lens   DEVICE int32 [batch], 1 <= cache_lens[b] <= max_len <= Lmax
+ *   gates        fp32 [batch, H_q, 3] (cmp, slc, win)
+ *   out          bf16 out [batch, H_q, d_v]
+ *   sel_out      int32 out or NULL: [batch, H_kv, top_n], ascending, -1 padded
+ *   imp_out      fp32 out or NULL: [batch, H_kv, n_blk(max_len)]
+ * `max_len` (HOST) bounds the lengths and sizes the launch; lengths above it
+ * are an error recorded in the device status word (the sequence is skipped). */
+nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const void* k_cmp_cache, const void* v_cmp_cache,
+                        const int32_t* cache_lens, int32_t batch, int32_t Lmax, int32_t Lmax_cmp,
+                        int32_t max_len, const float* gates, const nsa_heads_t* heads,
+                        const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Opt-in per-kernel timing (no compute change). While enabled, every entry point
+ * records a CUDA event pair on its stream around each of its kernel launches.
+ * nsa_profile_read() waits for the recorded events, writes for each of the
+ * first n_slots kernel slots the accumulated milliseconds and launch count since
+ * the previous read, and resets them. Slot names: nsa_profile_slot_name(). The
+ * events are created on first use and reused; this is the only state the
+ * library keeps between calls. Returns NSA_ERR_CUDA if an event query fails. */
+#define NSA_PROFILE_SLOTS 10
+nsa_status_t nsa_profile_enable(int32_t enable);
+nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots);
+const char* nsa_profile_slot_name(int32_t slot);
+
+/* Human-readable name of a status code (static string). */
+const char* nsa_status_string(nsa_status_t status);
+
+/* Text of the last CUDA error seen by this thread's calls (static per thread). */
+const char* nsa_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_H_ */

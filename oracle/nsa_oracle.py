@@ -269,7 +269,8 @@ def prefill(q, k, v, kc, vc, gates, p, rows=None, sel_override=None):
     Returns dict(out [len(rows), H_q, d_v], sel {(t,g): list}, imp {(t,g): array},
     rows).
     """
-    q, k, v, kc, vc, gates = (_f64(a) for a in (q, k, v, kc, vc, gates))
+    # q and gates are read row by row (only the requested rows are converted)
+    k, v, kc, vc = (_f64(a) for a in (k, v, kc, vc))
     T = q.shape[0]
     rows = list(range(T)) if rows is None else [int(r) for r in rows]
     out = np.zeros((len(rows), q.shape[1], v.shape[2]))
@@ -278,7 +279,7 @@ def prefill(q, k, v, kc, vc, gates, p, rows=None, sel_override=None):
         ov = None
         if sel_override is not None:
             ov = {g: sel_override[(t, g)] for g in range(k.shape[1]) if (t, g) in sel_override}
-        o, sels, imps, _ = nsa_row(t, q[t], k, v, kc, vc, gates[t], p, ov)
+        o, sels, imps, _ = nsa_row(t, _f64(q[t]), k, v, kc, vc, _f64(gates[t]), p, ov)
         out[n] = o
         for g in range(k.shape[1]):
             sel[(t, g)] = sels[g]

@@ -1,0 +1,301 @@
+"""Python binding of libnsa.so — NSA (Native Sparse Attention) forward on B200.
+
+Thin ctypes layer over the C ABI declared in include/nsa.h: every function here
+only checks and marshals arguments (torch tensors -> device pointers, the
+current CUDA stream) and calls the entry point of the same name. All compute
+runs in the library's sm_100a kernels; there is no fallback: if the shared
+library is missing or cannot be loaded, every call raises.
+
+Convenience helpers at the bottom (`compress`, `prefill`, `decode`) allocate
+outputs and the workspace with torch and then call the entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnsa.so")
+
+NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_DEVICE_CHECK = range(6)
+NSA_OP_COMPRESS, NSA_OP_PREFILL, NSA_OP_DECODE = 0, 1, 2
+NSA_MAX_BATCH = 128
+
+# every symbol include/nsa.h declares
+EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
+            "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
+            "nsa_status_string", "nsa_last_error_detail")
+NSA_PROFILE_SLOTS = 10
+
+
+class NSAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {status_name(status)}" + (f" ({detail})" if detail else ""))
+
+
+class Params(ctypes.Structure):
+    """nsa_params_t"""
+    _fields_ = [("l_cmp", ctypes.c_int32), ("stride", ctypes.c_int32), ("l_sel", ctypes.c_int32),
+                ("top_n", ctypes.c_int32), ("window", ctypes.c_int32), ("force_first", ctypes.c_int32),
+                ("force_local", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class Heads(ctypes.Structure):
+    """nsa_heads_t"""
+    _fields_ = [("H_q", ctypes.c_int32), ("H_kv", ctypes.c_int32), ("d_k", ctypes.c_int32),
+                ("d_v", ctypes.c_int32)]
+
+
+def make_params(l_cmp=32, stride=16, l_sel=64, top_n=16, window=512, force_first=1, force_local=2,
+                scale=0.0) -> Params:
+    return Params(l_cmp, stride, l_sel, top_n, window, force_first, force_local, float(scale))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnsa.so once. Raises if it is missing (no CPU fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libnsa.so not built at {LIB_PATH}; run python -m sparse_attention_long_nsa_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    L.nsa_workspace_size.restype = SZ
+    L.nsa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(Heads), ctypes.POINTER(Params), I32, I64, I32]
+    L.nsa_workspace_init.restype = ctypes.c_int
+    L.nsa_workspace_init.argtypes = [P, SZ, P]
+    L.nsa_check_device_status.restype = ctypes.c_int
+    L.nsa_check_device_status.argtypes = [P, P]
+    L.nsa_compress.restype = ctypes.c_int
+    L.nsa_compress.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params),
+                               P, P, P, SZ, P]
+    L.nsa_prefill.restype = ctypes.c_int
+    L.nsa_prefill.argtypes = [P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params), P, P, P,
+                              P, SZ, P]
+    L.nsa_decode.restype = ctypes.c_int
+    L.nsa_decode.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, P, ctypes.POINTER(Heads),
+                             ctypes.POINTER(Params), P, P, P, P, SZ, P]
+    L.nsa_profile_enable.restype = ctypes.c_int
+    L.nsa_profile_enable.argtypes = [I32]
+    L.nsa_profile_read.restype = ctypes.c_int
+    L.nsa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I32]
+    L.nsa_profile_slot_name.restype = ctypes.c_char_p
+    L.nsa_profile_slot_name.argtypes = [I32]
+    L.nsa_status_string.restype = ctypes.c_char_p
+    L.nsa_status_string.argtypes = [ctypes.c_int]
+    L.nsa_last_error_detail.restype = ctypes.c_char_p
+    L.nsa_last_error_detail.argtypes = []
+    _lib = L
+    return L
+
+
+def status_name(s: int) -> str:
+    try:
+        return lib().nsa_status_string(s).decode()
+    except Exception:
+        return f"status {s}"
+
+
+def _check(s: int, where: str):
+    if s != NSA_OK:
+        detail = lib().nsa_last_error_detail().decode() if s == NSA_ERR_CUDA or s == NSA_ERR_DEVICE_CHECK else ""
+        raise NSAError(s, where, detail)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, device_kind="cuda") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    if device_kind == "cuda" and t.device.type != "cuda":
+        raise ValueError("expected a CUDA tensor")
+    if device_kind == "cpu" and t.device.type != "cpu":
+        raise ValueError("expected a host tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def nsa_workspace_size(op: int, heads: Heads, params: Params, batch: int, total_tokens: int, max_len: int) -> int:
+    return int(lib().nsa_workspace_size(op, ctypes.byref(heads), ctypes.byref(params), batch, total_tokens,
+                                        max_len))
+
+
+def nsa_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().nsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "nsa_workspace_init")
+
+
+def nsa_check_device_status(ws: torch.Tensor, stream=None):
+    _check(lib().nsa_check_device_status(_ptr(ws), _stream(stream)), "nsa_check_device_status")
+
+
+def nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, heads: Heads, params: Params,
+                 k_cmp, v_cmp, ws, stream=None):
+    """tok_offset/cmp_offset: host int64 [B]; seq_len: host int32 [B]."""
+    B = int(seq_len.numel())
+    s = lib().nsa_compress(_ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16), _ptr(w_ck, torch.float32),
+                           _ptr(pe_k, torch.float32), _ptr(w_cv, torch.float32), _ptr(pe_v, torch.float32),
+                           _ptr(tok_offset, torch.int64, "cpu"), _ptr(seq_len, torch.int32, "cpu"),
+                           _ptr(cmp_offset, torch.int64, "cpu"), B, ctypes.byref(heads), ctypes.byref(params),
+                           _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream))
+    _check(s, "nsa_compress")
+
+
+def nsa_prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, out, sel_out=None,
+                imp_out=None, ws=None, stream=None):
+    """cu_seqlens: host int32 [B+1]."""
+    B = int(cu_seqlens.numel()) - 1
+    s = lib().nsa_prefill(_ptr(q, torch.bfloat16), _ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16),
+                          _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16), _ptr(gates, torch.float32),
+                          _ptr(cu_seqlens, torch.int32, "cpu"), B, ctypes.byref(heads), ctypes.byref(params),
+                          _ptr(out, torch.bfloat16), _ptr(sel_out, torch.int32), _ptr(imp_out, torch.float32),
+                          _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(s, "nsa_prefill")
+
+
+def nsa_decode(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens, max_len: int, gates, heads: Heads,
+               params: Params, out, sel_out=None, imp_out=None, ws=None, stream=None):
+    """cache_lens: device int32 [B]; caches [B, Lmax, H_kv, d] and [B, Lmax_cmp, H_kv, d]."""
+    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
+    Lc = int(k_cmp_cache.shape[1]) if k_cmp_cache is not None else 0
+    s = lib().nsa_decode(_ptr(q, torch.bfloat16), _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                         _ptr(k_cmp_cache, torch.bfloat16), _ptr(v_cmp_cache, torch.bfloat16),
+                         _ptr(cache_lens, torch.int32), B, Lmax, Lc, int(max_len), _ptr(gates, torch.float32),
+                         ctypes.byref(heads), ctypes.byref(params), _ptr(out, torch.bfloat16),
+                         _ptr(sel_out, torch.int32), _ptr(imp_out, torch.float32), _ptr(ws),
+                         ws.numel() * ws.element_size(), _stream(stream))
+    _check(s, "nsa_decode")
+
+
+def nsa_profile_enable(enable: bool):
+    _check(lib().nsa_profile_enable(1 if enable else 0), "nsa_profile_enable")
+
+
+def nsa_profile_read() -> dict:
+    """{slot name: (total ms, launches)} accumulated since the previous read."""
+    n = NSA_PROFILE_SLOTS
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(lib().nsa_profile_read(ms, cnt, n), "nsa_profile_read")
+    return {lib().nsa_profile_slot_name(i).decode(): (float(ms[i]), int(cnt[i])) for i in range(n)}
+
+
+# ---------------------------------------------------------------------------
+# convenience helpers (allocation with torch, then the entry points)
+# ---------------------------------------------------------------------------
+
+def n_cmp(L: int, l: int = 32, s: int = 16) -> int:
+    return (L - l) // s + 1 if L >= l else 0
+
+
+def n_blk(L: int, l_sel: int = 64) -> int:
+    return -(-L // l_sel)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    nsa_workspace_init(ws)
+    return ws
+
+
+def compress(k, v, w_ck, pe_k, w_cv, pe_v, seqlens, heads: Heads, params: Params, ws=None, out=None):
+    """Packed prefill layout: sequences back to back in k/v. Returns (k_cmp, v_cmp)."""
+    seqlens = [int(x) for x in seqlens]
+    tok = torch.tensor([sum(seqlens[:b]) for b in range(len(seqlens))], dtype=torch.int64)
+    ncs = [n_cmp(L, params.l_cmp, params.stride) for L in seqlens]
+    cmp_off = torch.tensor([sum(ncs[:b]) for b in range(len(ncs))], dtype=torch.int64)
+    total = sum(ncs)
+    dev = k.device
+    if out is None:
+        k_cmp = torch.empty((max(total, 1), heads.H_kv, heads.d_k), dtype=torch.bfloat16, device=dev)
+        v_cmp = torch.empty((max(total, 1), heads.H_kv, heads.d_v), dtype=torch.bfloat16, device=dev)
+    else:
+        k_cmp, v_cmp = out
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, len(seqlens), 0, 0), dev)
+    nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok, torch.tensor(seqlens, dtype=torch.int32), cmp_off, heads,
+                 params, k_cmp, v_cmp, ws)
+    return k_cmp[:total], v_cmp[:total]
+
+
+def compress_cache(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, heads: Heads, params: Params, ws=None):
+    """Compressed caches [B, Lmax_cmp, H_kv, d] for batched caches [B, Lmax, H_kv, d]."""
+    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
+    Lc = max(n_cmp(Lmax, params.l_cmp, params.stride), 1)
+    dev = k_cache.device
+    kc = torch.zeros((B, Lc, heads.H_kv, heads.d_k), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros((B, Lc, heads.H_kv, heads.d_v), dtype=torch.bfloat16, device=dev)
+    lens_l = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, B, 0, 0), dev)
+    nsa_compress(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v,
+                 torch.tensor([b * Lmax for b in range(B)], dtype=torch.int64),
+                 torch.tensor(lens_l, dtype=torch.int32),
+                 torch.tensor([b * Lc for b in range(B)], dtype=torch.int64), heads, params, kc, vc, ws)
+    return kc, vc
+
+
+def prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, ws=None, want_sel=False,
+            want_imp=False):
+    """Returns out (and sel / imp when asked)."""
+    cu = cu_seqlens.to("cpu", torch.int32).contiguous()
+    B = cu.numel() - 1
+    N = int(cu[-1])
+    max_len = int((cu[1:] - cu[:-1]).max()) if B > 0 else 0
+    dev = q.device
+    out = torch.empty((N, heads.H_q, heads.d_v), dtype=torch.bfloat16, device=dev)
+    sel = torch.empty((N, heads.H_kv, params.top_n), dtype=torch.int32, device=dev) if want_sel else None
+    imp = (torch.zeros((N, heads.H_kv, n_blk(max_len, params.l_sel)), dtype=torch.float32, device=dev)
+           if want_imp else None)
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_PREFILL, heads, params, B, N, max_len), dev)
+    nsa_prefill(q, k, v, k_cmp, v_cmp, gates, cu, heads, params, out, sel, imp, ws)
+    res = [out]
+    if want_sel:
+        res.append(sel)
+    if want_imp:
+        res.append(imp)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def decode(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens_dev, max_len, gates, heads: Heads,
+           params: Params, ws=None, want_sel=False, want_imp=False):
+    B = int(q.shape[0])
+    dev = q.device
+    out = torch.empty((B, heads.H_q, heads.d_v), dtype=torch.bfloat16, device=dev)
+    sel = torch.empty((B, heads.H_kv, params.top_n), dtype=torch.int32, device=dev) if want_sel else None
+    imp = (torch.zeros((B, heads.H_kv, n_blk(max_len, params.l_sel)), dtype=torch.float32, device=dev)
+           if want_imp else None)
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_DECODE, heads, params, B, 0, max_len), dev)
+    nsa_decode(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens_dev, max_len, gates, heads, params, out,
+               sel, imp, ws)
+    res = [out]
+    if want_sel:
+        res.append(sel)
+    if want_imp:
+        res.append(imp)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def default_scale(d_k: int) -> float:
+    return 1.0 / math.sqrt(d_k)

@@ -1,0 +1,233 @@
+// Block compression: k_cmp[i] = vec(x[i*s : i*s+l] + pe) . W  (per KV head).
+//
+// "Разреженное внимание — NSA и DSA" (ai.flicky.cc), section "NSA: три ветви",
+// compression branch: overlapping blocks of l tokens with stride s, each mapped
+// to one key and one value by a learned map. The map here is one linear layer W
+// [l*d_in, d_out] of the token-major flattened block plus a position embedding
+// pe [l, d_in] added to every token; by linearity the embedding contributes the
+// constant row vec(pe).W, which the prep kernel computes once in fp32.
+//
+// The GEMM runs on the 5th-generation tensor cores: M = 128 compressed rows of
+// one KV head, N = d_out, K = l*d_in, bf16 operands staged in 128-byte-swizzled
+// shared memory, fp32 accumulator in tensor memory (tcgen05.mma issued by one
+// thread), read back with tcgen05.ld for the bias-add + bf16 epilogue.
+// Operand rows are a strided gather (row i starts at token i*s), so they are
+// fetched with cp.async rather than a tensor map.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nsa {
+
+// ---------------------------------------------------------------------------
+// prep: wt[n][k] = bf16(w[k][n]); partial[kt][n] = sum over the 32 rows of tile
+// kt of pe_flat[k] * w[k][n]; bias[n] = sum_kt partial[kt][n] (fixed order)
+// ---------------------------------------------------------------------------
+__global__ void compress_transpose_kernel(const float* __restrict__ w, const float* __restrict__ pe,
+                                          int K, int N, __nv_bfloat16* __restrict__ wt,
+                                          float* __restrict__ partial) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  for (int r = ty; r < 32; r += 8) {
+    const int k = k0 + r, n = n0 + tx;
+    tile[r][tx] = (k < K && n < N) ? w[(size_t)k * N + n] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int n = n0 + r, k = k0 + tx;
+    if (n < N && k < K) wt[(size_t)n * K + k] = __float2bfloat16_rn(tile[tx][r]);
+  }
+  if (ty == 0) {
+    const int n = n0 + tx;
+    float s = 0.f;
+    for (int r = 0; r < 32; ++r) {
+      const int k = k0 + r;
+      if (k < K) s = fmaf(pe[k], tile[r][tx], s);
+    }
+    if (n < N) partial[(size_t)blockIdx.y * N + n] = s;
+  }
+}
+
+__global__ void compress_bias_kernel(const float* __restrict__ partial, int KT, int N,
+                                     float* __restrict__ bias) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float s = 0.f;
+  for (int kt = 0; kt < KT; ++kt) s += partial[(size_t)kt * N + n];
+  bias[n] = s;
+}
+
+cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
+                                 float* partial, float* bias, cudaStream_t st) {
+  dim3 grid((N + 31) / 32, (K + 31) / 32);
+  compress_transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(
+      w, pe, K, N, static_cast<__nv_bfloat16*>(wt_bf16), partial);
+  compress_bias_kernel<<<(N + 127) / 128, 128, 0, st>>>(partial, (K + 31) / 32, N, bias);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// GEMM
+// ---------------------------------------------------------------------------
+constexpr int kCmpStages = 4;
+constexpr int kTileM = 128;
+
+template <int D_OUT>
+struct CompressSmem {
+  static constexpr int A_BYTES = kTileM * 128;            // 128 rows x 64 bf16
+  static constexpr int B_BYTES = D_OUT * 128;             // D_OUT rows x 64 bf16
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int TOTAL = kCmpStages * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ int find_seq(const SeqTable& t, int tile) {
+  int b = 0;
+  while (b + 1 < t.n && t.tile_prefix[b + 1] <= tile) ++b;
+  return b;
+}
+
+template <int D_IN, int D_OUT>
+__global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArgs a) {
+  using S = CompressSmem<D_OUT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + kCmpStages * S::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + kCmpStages + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x;
+  const int b = find_seq(a.seqs, tile);
+  const int g = blockIdx.y;
+  const int L = a.seqs.len[b];
+  const int ncmp = n_cmp_of(L, a.l, a.s);
+  const int i0 = (tile - a.seqs.tile_prefix[b]) * kTileM;
+  const int64_t tok0 = a.seqs.tok_off[b];
+  const int K = a.l * D_IN;
+  const int nkb = K / 64;
+  constexpr uint32_t TM_COLS = D_OUT <= 64 ? 64 : (D_OUT <= 128 ? 128 : 256);
+
+  if (tid == 0) {
+    for (int i = 0; i <= kCmpStages; ++i) mbar_init(&mma_done[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+  const __nv_bfloat16* wt = static_cast<const __nv_bfloat16*>(a.wt);
+  const size_t row_stride = (size_t)a.H_kv * D_IN;   // elements between tokens
+
+  auto load_stage = [&](int st, int kb) {
+    uint8_t* A = smem + st * S::STAGE;
+    uint8_t* Bm = A + S::A_BYTES;
+    const int f0 = kb * 64;
+    const int r = f0 / D_IN, e0 = f0 % D_IN;
+    {  // A: one 128-byte row per thread
+      const int row = tid;
+      const int ci = i0 + row;
+      const bool ok = ci < ncmp;
+      const __nv_bfloat16* src =
+          x + (size_t)(tok0 + (int64_t)(ok ? ci : 0) * a.s + r) * row_stride + (size_t)g * D_IN + e0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) cp_async16_zfill(A + sw128(row, c), src + c * 8, ok);
+    }
+    // B: D_OUT rows of W^T, 8 chunks each
+    for (int idx = tid; idx < D_OUT * 8; idx += 128) {
+      const int n = idx >> 3, c = idx & 7;
+      cp_async16(Bm + sw128(n, c), wt + (size_t)n * K + f0 + c * 8);
+    }
+  };
+
+  const uint32_t idesc = umma_idesc_bf16(kTileM, D_OUT, false, false);
+  bool ok = true;
+  for (int kb = 0; kb < nkb + kCmpStages - 1; ++kb) {
+    if (kb < nkb) {
+      const int st = kb % kCmpStages;
+      if (kb >= kCmpStages) {
+        if (!mbar_wait(&mma_done[st], ((kb / kCmpStages) - 1) & 1, abort_flag, a.status, 101)) {
+          ok = false;
+        }
+      }
+      if (ok) load_stage(st, kb);
+    }
+    cp_async_commit();
+    const int c = kb - (kCmpStages - 1);
+    if (c >= 0) {
+      cp_async_wait<kCmpStages - 1>();
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (*abort_flag) { ok = false; break; }
+      if (tid == 0) {
+        tc_fence_after();
+        const int st = c % kCmpStages;
+        const uint32_t a_addr = smem_u32(smem + st * S::STAGE);
+        const uint32_t b_addr = a_addr + S::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = umma_desc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t db = umma_desc_sw128(b_addr + kk * 32, 16, 1024);
+          umma_ss(tmem_d, da, db, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&mma_done[st]);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  // all MMAs done: commit a final barrier
+  if (tid == 0 && ok) umma_commit(&mma_done[kCmpStages]);
+  __syncthreads();
+  if (ok && !*abort_flag) ok = mbar_wait(&mma_done[kCmpStages], 0, abort_flag, a.status, 102);
+  tc_fence_after();
+
+  if (ok) {
+    // epilogue: warp w owns accumulator rows 32w .. 32w+31 (TMEM lanes)
+    const int row = warp * 32 + lane;
+    const int ci = i0 + row;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+    const size_t orow = ((size_t)(a.seqs.cmp_off[b] + ci) * a.H_kv + g) * D_OUT;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D_OUT; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem_d + ((uint32_t)(warp * 32) << 16) + c0, v);
+      tmem_ld_wait();
+      if (ci < ncmp) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(v[2 * j] + a.bias[c0 + 2 * j], v[2 * j + 1] + a.bias[c0 + 2 * j + 1]);
+        uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem_d, TM_COLS);
+}
+
+template <int D_IN, int D_OUT>
+static cudaError_t launch_gemm_t(const CompressArgs& a, int n_tiles, cudaStream_t st) {
+  using S = CompressSmem<D_OUT>;
+  auto kern = compress_gemm_kernel<D_IN, D_OUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_tiles, a.H_kv);
+  kern<<<grid, 128, S::TOTAL, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compress_gemm(int d_in, int d_out, const CompressArgs& a, int n_tiles,
+                                 cudaStream_t st) {
+  if (n_tiles <= 0) return cudaSuccess;
+  if (d_in == 64 && d_out == 64) return launch_gemm_t<64, 64>(a, n_tiles, st);
+  if (d_in == 128 && d_out == 128) return launch_gemm_t<128, 128>(a, n_tiles, st);
+  if (d_in == 192 && d_out == 192) return launch_gemm_t<192, 192>(a, n_tiles, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nsa

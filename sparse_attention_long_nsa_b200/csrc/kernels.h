@@ -1,0 +1,103 @@
+// Internal launch interface between the C-ABI host layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nsa {
+
+constexpr int kMaxBatch = 128;
+
+// Opt-in per-kernel timing: CUDA events recorded on the launching stream around
+// each launch (see nsa_profile_enable / nsa_profile_read in include/nsa.h).
+enum ProfSlot {
+  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_CMP_ATTN, P_TOPN, P_SEL_ATTN, P_WIN_ATTN,
+  P_DEC_CMP, P_DEC_SELECT, P_DEC_FINE, P_DEC_COMBINE, P_COUNT
+};
+void prof_begin(int slot, cudaStream_t st);
+void prof_end(int slot, cudaStream_t st, int launches);
+
+// Per-launch sequence table, passed by value as a kernel parameter.
+struct SeqTable {
+  int32_t n;                         // sequences
+  int32_t tile_prefix[kMaxBatch + 1];// first tile id of each sequence
+  int64_t tok_off[kMaxBatch];        // first token row
+  int64_t cmp_off[kMaxBatch];        // first compressed row
+  int32_t len[kMaxBatch];            // tokens
+};
+
+__host__ __device__ inline int n_cmp_of(int L, int l, int s) { return L >= l ? (L - l) / s + 1 : 0; }
+
+// ----- compression (block summaries) -----
+struct CompressArgs {
+  const void* x;          // bf16 [*, H_kv, d_in]
+  const void* wt;         // bf16 [d_out, l*d_in] (W transposed, rounded)
+  const float* bias;      // fp32 [d_out] = vec(pe) . W
+  void* out;              // bf16 [*, H_kv, d_out]
+  int H_kv, l, s;
+  uint32_t* status;
+  SeqTable seqs;
+};
+cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
+                                 float* partial, float* bias, cudaStream_t st);
+cudaError_t launch_compress_gemm(int d_in, int d_out, const CompressArgs& a, int n_tiles,
+                                 cudaStream_t st);
+
+// ----- prefill -----
+struct PrefillArgs {
+  const void* q;          // bf16 [N, H_q, d_k]
+  const void* k;          // bf16 [N, H_kv, d_k]
+  const void* v;          // bf16 [N, H_kv, d_v]
+  const void* kc;         // bf16 [Nc, H_kv, d_k]
+  const void* vc;         // bf16 [Nc, H_kv, d_v]
+  const float* gates;     // fp32 [N, H_q, 3]
+  float* acc;             // fp32 [N, H_q, d_v] (g_cmp*o_cmp + g_slc*o_slc)
+  float* imp;             // fp32 [N, H_kv, nb_stride]
+  int32_t* sel;           // int32 [N, H_kv, top_n]
+  void* out;              // bf16 [N, H_q, d_v]
+  int H_q, H_kv, G, d_k, d_v;
+  int l, s, ls, top_n, window, force_first, force_local;
+  int nb_stride;
+  float scale_log2;       // softmax scale * log2(e)
+  uint32_t* status;
+  SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens
+};
+struct PrefillMaps {
+  CUtensorMap q, k, v, kc, vc;
+};
+cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
+cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st);
+cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int64_t n_tokens, cudaStream_t st);
+cudaError_t launch_win_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
+
+// ----- decode -----
+struct DecodeArgs {
+  const void* q;          // bf16 [B, H_q, d_k]
+  const void* kcache;     // bf16 [B, Lmax, H_kv, d_k]
+  const void* vcache;     // bf16 [B, Lmax, H_kv, d_v]
+  const void* kc;         // bf16 [B, Lmax_cmp, H_kv, d_k]
+  const void* vc;         // bf16 [B, Lmax_cmp, H_kv, d_v]
+  const int32_t* lens;    // int32 [B]
+  const float* gates;     // fp32 [B, H_q, 3]
+  void* out;              // bf16 [B, H_q, d_v]
+  int32_t* sel;           // int32 [B, H_kv, top_n]
+  float* imp;             // fp32 [B, H_kv, nb_stride]
+  float* part;            // split partials (workspace)
+  float* ocmp;            // fp32 [B, H_q, d_v] g_cmp * o_cmp (workspace)
+  int B, Lmax, Lmax_cmp, max_len;
+  int H_q, H_kv, G, d_k, d_v;
+  int l, s, ls, top_n, window, force_first, force_local;
+  int nb_stride;
+  int n_cmp_chunks;              // D1 splits per (b, g), 512 compressed keys each
+  int n_sw_chunks;               // D3 splits per (b, g), 4 blocks of l_sel keys each
+  float scale_log2;
+  uint32_t* status;
+};
+struct DecodeMaps {
+  CUtensorMap k, v, kc, vc;
+};
+size_t decode_partials_floats(const DecodeArgs& a);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
+
+}  // namespace nsa

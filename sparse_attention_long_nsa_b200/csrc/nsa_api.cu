@@ -1,0 +1,502 @@
+// C-ABI host layer of libnsa.so: argument validation, workspace carving,
+// tensor-map encoding and the launch sequence of each entry point.
+// See include/nsa.h for the contract of every function.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/nsa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace nsa;
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+nsa_status_t cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_detail, sizeof(g_detail), "%s: %s", where, cudaGetErrorString(e));
+  return NSA_ERR_CUDA;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool heads_supported(const nsa_heads_t* h) {
+  const int G = h->H_kv > 0 ? h->H_q / h->H_kv : 0;
+  const bool dk = h->d_k == 64 || h->d_k == 128 || h->d_k == 192;
+  const bool dv = h->d_v == 64 || h->d_v == 128;
+  const bool g = G == 1 || G == 2 || G == 4 || G == 8 || G == 16;
+  return dk && dv && g;
+}
+
+nsa_status_t check_heads(const nsa_heads_t* h) {
+  if (!h || h->H_q <= 0 || h->H_kv <= 0 || h->d_k <= 0 || h->d_v <= 0) return NSA_ERR_INVALID_ARG;
+  if (h->H_q % h->H_kv != 0) return NSA_ERR_INVALID_ARG;
+  if (!heads_supported(h)) return NSA_ERR_UNSUPPORTED;
+  return NSA_OK;
+}
+
+nsa_status_t check_params(const nsa_params_t* p, bool need_selection) {
+  if (!p) return NSA_ERR_INVALID_ARG;
+  if (p->l_cmp <= 0 || p->stride <= 0 || p->l_sel <= 0) return NSA_ERR_INVALID_ARG;
+  if (p->l_cmp % p->stride != 0 || p->l_sel % p->stride != 0) return NSA_ERR_INVALID_ARG;
+  if (!(p->scale >= 0.f)) return NSA_ERR_INVALID_ARG;
+  if (need_selection) {
+    if (p->top_n <= 0 || p->window <= 0 || p->force_first < 0 || p->force_local < 0)
+      return NSA_ERR_INVALID_ARG;
+    if (p->force_first + p->force_local > p->top_n) return NSA_ERR_INVALID_ARG;
+    if (p->top_n > 32) return NSA_ERR_UNSUPPORTED;
+  }
+  if (p->l_cmp != 32 || p->stride != 16 || (need_selection && p->l_sel != 64))
+    return NSA_ERR_UNSUPPORTED;
+  return NSA_OK;
+}
+
+// blocks of the decode fine pass: the selected ones plus those the window touches
+int max_union_blocks(const nsa_params_t* p) { return p->top_n + (p->window + p->l_sel - 1) / p->l_sel + 1; }
+
+float softmax_scale(const nsa_params_t* p, int d_k) {
+  return p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)d_k);
+}
+
+int n_blk_of(int L, int ls) { return (L + ls - 1) / ls; }
+
+// ---- workspace layouts ----
+struct CompressWs {
+  size_t wt_k, wt_v, part_k, part_v, bias_k, bias_v, total;
+};
+CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p) {
+  CompressWs w{};
+  size_t off = 256;
+  const size_t Kk = (size_t)p->l_cmp * h->d_k, Kv = (size_t)p->l_cmp * h->d_v;
+  w.wt_k = off; off = align256(off + Kk * h->d_k * 2);
+  w.wt_v = off; off = align256(off + Kv * h->d_v * 2);
+  w.part_k = off; off = align256(off + ((Kk + 31) / 32) * h->d_k * 4);
+  w.part_v = off; off = align256(off + ((Kv + 31) / 32) * h->d_v * 4);
+  w.bias_k = off; off = align256(off + (size_t)h->d_k * 4);
+  w.bias_v = off; off = align256(off + (size_t)h->d_v * 4);
+  w.total = off;
+  return w;
+}
+
+struct PrefillWs {
+  size_t acc, imp, sel, total;
+  int nb;
+};
+PrefillWs prefill_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t N, int max_len) {
+  PrefillWs w{};
+  size_t off = 256;
+  w.nb = n_blk_of(max_len, p->l_sel);
+  w.acc = off; off = align256(off + (size_t)N * h->H_q * h->d_v * 4);
+  w.imp = off; off = align256(off + (size_t)N * h->H_kv * w.nb * 4);
+  w.sel = off; off = align256(off + (size_t)N * h->H_kv * p->top_n * 4);
+  w.total = off;
+  return w;
+}
+
+void fill_decode_args(DecodeArgs& a, const nsa_heads_t* h, const nsa_params_t* p, int B, int Lmax,
+                      int Lmax_cmp, int max_len) {
+  a.B = B; a.Lmax = Lmax; a.Lmax_cmp = Lmax_cmp; a.max_len = max_len;
+  a.H_q = h->H_q; a.H_kv = h->H_kv; a.G = h->H_q / h->H_kv; a.d_k = h->d_k; a.d_v = h->d_v;
+  a.l = p->l_cmp; a.s = p->stride; a.ls = p->l_sel; a.top_n = p->top_n; a.window = p->window;
+  a.force_first = p->force_first; a.force_local = p->force_local;
+  a.nb_stride = n_blk_of(max_len, p->l_sel);
+  a.n_cmp_chunks = (n_cmp_of(max_len, p->l_cmp, p->stride) + 511) / 512;
+  if (a.n_cmp_chunks < 1) a.n_cmp_chunks = 1;
+  a.n_sw_chunks = (max_union_blocks(p) + 3) / 4;
+  a.scale_log2 = softmax_scale(p, h->d_k) * 1.4426950408889634f;
+}
+
+struct DecodeWs {
+  size_t part, ocmp, sel, imp, total;
+};
+DecodeWs decode_ws(const DecodeArgs& a) {
+  DecodeWs w{};
+  size_t off = 256;
+  w.part = off; off = align256(off + decode_partials_floats(a) * 4);
+  w.ocmp = off; off = align256(off + (size_t)a.B * a.H_q * a.d_v * 4);
+  w.sel = off; off = align256(off + (size_t)a.B * a.H_kv * a.top_n * 4);
+  w.imp = off; off = align256(off + (size_t)a.B * a.H_kv * a.nb_stride * 4);
+  w.total = off;
+  return w;
+}
+
+// ---- tensor maps ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over a [rows, heads, dim] tensor; box = (64 elements, bh heads, br rows),
+// 128-byte swizzle. Coordinates: (element, head, row).
+bool make_map_3d(CUtensorMap* m, const void* base, int dim, int heads, int64_t rows, int bh, int br) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * heads * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)bh, (cuuint32_t)br};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---- opt-in profiler ----
+struct ProfRec {
+  int slot, launches;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<ProfRec> recs;
+  cudaEvent_t open[P_COUNT] = {};
+  double total_ms[P_COUNT] = {};
+  int64_t launches[P_COUNT] = {};
+  cudaEvent_t get() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+
+const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "cmp_attn", "topn", "sel_attn", "win_attn",
+                                   "dec_cmp", "dec_select", "dec_fine", "dec_combine"};
+
+}  // namespace
+
+namespace nsa {
+void prof_begin(int slot, cudaStream_t st) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.on) return;
+  cudaEvent_t e = p.get();
+  cudaEventRecord(e, st);
+  p.open[slot] = e;
+}
+void prof_end(int slot, cudaStream_t st, int launches) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.on || !p.open[slot]) return;
+  cudaEvent_t e = p.get();
+  cudaEventRecord(e, st);
+  p.recs.push_back({slot, launches, p.open[slot], e});
+  p.open[slot] = nullptr;
+}
+}  // namespace nsa
+
+extern "C" {
+
+nsa_status_t nsa_profile_enable(int32_t enable) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  p.on = enable != 0;
+  return NSA_OK;
+}
+
+nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots) {
+  if (n_slots < 0 || (n_slots > 0 && (!ms_out || !launches_out))) return NSA_ERR_INVALID_ARG;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (const ProfRec& r : p.recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "nsa_profile_read");
+    p.total_ms[r.slot] += ms;
+    p.launches[r.slot] += r.launches;
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.recs.clear();
+  for (int i = 0; i < n_slots; ++i) {
+    ms_out[i] = i < P_COUNT ? p.total_ms[i] : 0.0;
+    launches_out[i] = i < P_COUNT ? p.launches[i] : 0;
+  }
+  for (int i = 0; i < P_COUNT; ++i) { p.total_ms[i] = 0.0; p.launches[i] = 0; }
+  return NSA_OK;
+}
+
+const char* nsa_profile_slot_name(int32_t slot) {
+  return (slot >= 0 && slot < P_COUNT) ? kSlotNames[slot] : "";
+}
+
+
+const char* nsa_status_string(nsa_status_t s) {
+  switch (s) {
+    case NSA_OK: return "NSA_OK";
+    case NSA_ERR_INVALID_ARG: return "NSA_ERR_INVALID_ARG";
+    case NSA_ERR_UNSUPPORTED: return "NSA_ERR_UNSUPPORTED";
+    case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE";
+    case NSA_ERR_CUDA: return "NSA_ERR_CUDA";
+    case NSA_ERR_DEVICE_CHECK: return "NSA_ERR_DEVICE_CHECK";
+  }
+  return "NSA_UNKNOWN_STATUS";
+}
+
+const char* nsa_last_error_detail(void) { return g_detail; }
+
+size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* params, int32_t batch,
+                          int64_t total_tokens, int32_t max_len) {
+  if (check_heads(heads) != NSA_OK) return 0;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return 0;
+  switch (op) {
+    case NSA_OP_COMPRESS:
+      if (check_params(params, false) != NSA_OK) return 0;
+      return compress_ws(heads, params).total;
+    case NSA_OP_PREFILL:
+      if (check_params(params, true) != NSA_OK || total_tokens < 0 || max_len < 0) return 0;
+      return prefill_ws(heads, params, total_tokens, max_len).total;
+    case NSA_OP_DECODE: {
+      if (check_params(params, true) != NSA_OK || max_len <= 0 || max_union_blocks(params) > 64) return 0;
+      DecodeArgs a{};
+      fill_decode_args(a, heads, params, batch, max_len, n_cmp_of(max_len, params->l_cmp, params->stride),
+                       max_len);
+      return decode_ws(a).total;
+    }
+  }
+  return 0;
+}
+
+nsa_status_t nsa_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || ws_bytes < 256 || !aligned16(workspace)) return NSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "nsa_workspace_init");
+}
+
+nsa_status_t nsa_check_device_status(void* workspace, void* stream) {
+  if (!workspace) return NSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "nsa_check_device_status");
+  if (h[0] != 0) {
+    snprintf(g_detail, sizeof(g_detail), "device status 0x%x at site %u", h[0], h[1]);
+    e = cudaMemsetAsync(workspace, 0, 256, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "nsa_check_device_status(clear)");
+    return NSA_ERR_DEVICE_CHECK;
+  }
+  return NSA_OK;
+}
+
+nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const float* pe_k, const float* w_cv,
+                          const float* pe_v, const int64_t* tok_offset, const int32_t* seq_len,
+                          const int64_t* cmp_offset, int32_t batch, const nsa_heads_t* heads,
+                          const nsa_params_t* params, void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, false)) != NSA_OK) return s;
+  if (heads->d_k != 64 && heads->d_k != 128 && heads->d_k != 192) return NSA_ERR_UNSUPPORTED;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!k || !v || !w_ck || !pe_k || !w_cv || !pe_v || !tok_offset || !seq_len || !cmp_offset || !k_cmp ||
+      !v_cmp || !workspace)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(workspace))
+    return NSA_ERR_INVALID_ARG;
+  const CompressWs w = compress_ws(heads, params);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+
+  SeqTable t{};
+  t.n = batch;
+  int tiles = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (seq_len[b] < 0 || tok_offset[b] < 0 || cmp_offset[b] < 0) return NSA_ERR_INVALID_ARG;
+    t.tile_prefix[b] = tiles;
+    t.tok_off[b] = tok_offset[b];
+    t.cmp_off[b] = cmp_offset[b];
+    t.len[b] = seq_len[b];
+    tiles += (n_cmp_of(seq_len[b], params->l_cmp, params->stride) + 127) / 128;
+  }
+  t.tile_prefix[batch] = tiles;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Kk = params->l_cmp * heads->d_k, Kv = params->l_cmp * heads->d_v;
+  prof_begin(P_COMPRESS_PREP, st);
+  cudaError_t e = launch_compress_prep(w_ck, pe_k, Kk, heads->d_k, ws + w.wt_k, (float*)(ws + w.part_k),
+                                       (float*)(ws + w.bias_k), st);
+  if (e == cudaSuccess)
+    e = launch_compress_prep(w_cv, pe_v, Kv, heads->d_v, ws + w.wt_v, (float*)(ws + w.part_v),
+                             (float*)(ws + w.bias_v), st);
+  prof_end(P_COMPRESS_PREP, st, 4);
+  if (e != cudaSuccess) return cuda_fail(e, "compress prep");
+  if (tiles == 0) return NSA_OK;
+
+  CompressArgs a{};
+  a.H_kv = heads->H_kv; a.l = params->l_cmp; a.s = params->stride;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.seqs = t;
+  prof_begin(P_COMPRESS_GEMM, st);
+  a.x = k; a.wt = ws + w.wt_k; a.bias = (const float*)(ws + w.bias_k); a.out = k_cmp;
+  e = launch_compress_gemm(heads->d_k, heads->d_k, a, tiles, st);
+  if (e == cudaSuccess) {
+    a.x = v; a.wt = ws + w.wt_v; a.bias = (const float*)(ws + w.bias_v); a.out = v_cmp;
+    e = launch_compress_gemm(heads->d_v, heads->d_v, a, tiles, st);
+  }
+  prof_end(P_COMPRESS_GEMM, st, 2);
+  if (e != cudaSuccess) return cuda_fail(e, "compress gemm");
+  return NSA_OK;
+}
+
+nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void* k_cmp, const void* v_cmp,
+                         const float* gates, const int32_t* cu_seqlens, int32_t batch, const nsa_heads_t* heads,
+                         const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, true)) != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !gates || !cu_seqlens || !out || !workspace) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
+      !aligned16(gates))
+    return NSA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return NSA_ERR_INVALID_ARG;
+  int max_len = 0;
+  int64_t ncmp_total = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (L < 0) return NSA_ERR_INVALID_ARG;
+    if (L > max_len) max_len = L;
+    ncmp_total += n_cmp_of(L, params->l_cmp, params->stride);
+  }
+  const int64_t N = cu_seqlens[batch];
+  if (ncmp_total > 0 && (!k_cmp || !v_cmp || !aligned16(k_cmp) || !aligned16(v_cmp))) return NSA_ERR_INVALID_ARG;
+  const PrefillWs w = prefill_ws(heads, params, N, max_len);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+  if (N == 0) return NSA_OK;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.kc = k_cmp; a.vc = v_cmp; a.gates = gates;
+  a.acc = (float*)(ws + w.acc);
+  a.imp = imp_out ? imp_out : (float*)(ws + w.imp);
+  a.sel = sel_out ? sel_out : (int32_t*)(ws + w.sel);
+  a.out = out;
+  a.H_q = heads->H_q; a.H_kv = heads->H_kv; a.G = heads->H_q / heads->H_kv;
+  a.d_k = heads->d_k; a.d_v = heads->d_v;
+  a.l = params->l_cmp; a.s = params->stride; a.ls = params->l_sel; a.top_n = params->top_n;
+  a.window = params->window; a.force_first = params->force_first; a.force_local = params->force_local;
+  a.nb_stride = w.nb;
+  a.scale_log2 = softmax_scale(params, heads->d_k) * 1.4426950408889634f;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+
+  const int tok_per_tile = 128 / a.G;
+  SeqTable t{};
+  t.n = batch;
+  int tiles = 0;
+  int64_t coff = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+    t.tile_prefix[b] = tiles;
+    t.tok_off[b] = cu_seqlens[b];
+    t.cmp_off[b] = coff;
+    t.len[b] = L;
+    tiles += (L + tok_per_tile - 1) / tok_per_tile;
+    coff += n_cmp_of(L, params->l_cmp, params->stride);
+  }
+  t.tile_prefix[batch] = tiles;
+  a.seqs = t;
+
+  PrefillMaps m;
+  memset(&m, 0, sizeof(m));
+  const void* kc_base = ncmp_total > 0 ? k_cmp : k;
+  const void* vc_base = ncmp_total > 0 ? v_cmp : v;
+  if (!make_map_3d(&m.q, q, heads->d_k, heads->H_q, N, a.G, tok_per_tile) ||
+      !make_map_3d(&m.k, k, heads->d_k, heads->H_kv, N, 1, 64) ||
+      !make_map_3d(&m.v, v, heads->d_v, heads->H_kv, N, 1, 64) ||
+      !make_map_3d(&m.kc, kc_base, heads->d_k, heads->H_kv, ncmp_total, 1, 64) ||
+      !make_map_3d(&m.vc, vc_base, heads->d_v, heads->H_kv, ncmp_total, 1, 64)) {
+    snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
+    return NSA_ERR_CUDA;
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_begin(P_CMP_ATTN, st);
+  cudaError_t e = launch_cmp_attn(a, m, tiles, st);
+  prof_end(P_CMP_ATTN, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "compressed attention");
+  prof_begin(P_TOPN, st);
+  e = launch_topn(a, N, st);
+  prof_end(P_TOPN, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "top-n selection");
+  prof_begin(P_SEL_ATTN, st);
+  e = launch_sel_attn(a, m, N, st);
+  prof_end(P_SEL_ATTN, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "selected attention");
+  prof_begin(P_WIN_ATTN, st);
+  e = launch_win_attn(a, m, tiles, st);
+  prof_end(P_WIN_ATTN, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "window attention");
+  return NSA_OK;
+}
+
+nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* k_cmp_cache,
+                        const void* v_cmp_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
+                        int32_t Lmax_cmp, int32_t max_len, const float* gates, const nsa_heads_t* heads,
+                        const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, true)) != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !cache_lens || !gates || !out || !workspace) return NSA_ERR_INVALID_ARG;
+  if (max_len <= 0 || Lmax < max_len) return NSA_ERR_INVALID_ARG;
+  if (Lmax_cmp < n_cmp_of(max_len, params->l_cmp, params->stride)) return NSA_ERR_INVALID_ARG;
+  if (Lmax_cmp > 0 && (!k_cmp_cache || !v_cmp_cache)) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace) ||
+      (k_cmp_cache && !aligned16(k_cmp_cache)) || (v_cmp_cache && !aligned16(v_cmp_cache)))
+    return NSA_ERR_INVALID_ARG;
+  if (max_union_blocks(params) > 64) return NSA_ERR_UNSUPPORTED;
+  DecodeArgs a{};
+  fill_decode_args(a, heads, params, batch, Lmax, Lmax_cmp, max_len);
+  const DecodeWs w = decode_ws(a);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.q = q; a.kcache = k_cache; a.vcache = v_cache; a.kc = k_cmp_cache; a.vc = v_cmp_cache;
+  a.lens = cache_lens; a.gates = gates; a.out = out;
+  a.sel = sel_out ? sel_out : (int32_t*)(ws + w.sel);
+  a.imp = imp_out ? imp_out : (float*)(ws + w.imp);
+  a.part = (float*)(ws + w.part);
+  a.ocmp = (float*)(ws + w.ocmp);
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  DecodeMaps m;
+  memset(&m, 0, sizeof(m));
+  const int64_t rows = (int64_t)batch * Lmax, crows = (int64_t)batch * Lmax_cmp;
+  if (!make_map_3d(&m.k, k_cache, heads->d_k, heads->H_kv, rows, 1, 64) ||
+      !make_map_3d(&m.v, v_cache, heads->d_v, heads->H_kv, rows, 1, 64) ||
+      !make_map_3d(&m.kc, crows > 0 ? k_cmp_cache : k_cache, heads->d_k, heads->H_kv, crows > 0 ? crows : rows, 1, 64) ||
+      !make_map_3d(&m.vc, crows > 0 ? v_cmp_cache : v_cache, heads->d_v, heads->H_kv, crows > 0 ? crows : rows, 1, 64)) {
+    snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
+    return NSA_ERR_CUDA;
+  }
+  cudaError_t e = launch_decode(a, m, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode");
+  return NSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments on the host and sizes workspaces."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_long_nsa_b200 as nsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(nsa.LIB_PATH):
+        from sparse_attention_long_nsa_b200 import build
+        build.build()
+    return nsa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _header_functions()
+    assert declared, "no functions parsed from include/nsa.h"
+    assert set(declared) == set(nsa.EXPORTED)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for s, name in enumerate(["NSA_OK", "NSA_ERR_INVALID_ARG", "NSA_ERR_UNSUPPORTED", "NSA_ERR_WORKSPACE",
+                              "NSA_ERR_CUDA", "NSA_ERR_DEVICE_CHECK"]):
+        assert nsa.status_name(s) == name
+
+
+def test_workspace_size_host_only(L):
+    h = nsa.Heads(64, 4, 192, 128)
+    p = nsa.make_params(top_n=16, window=512)
+    ws = nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, h, p, 1, 8192, 8192)
+    # acc fp32 [N,Hq,dv] + importance [N,Hkv,128] + selection [N,Hkv,16]
+    assert ws >= 8192 * 64 * 128 * 4 + 8192 * 4 * 128 * 4 + 8192 * 4 * 16 * 4
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, h, p, 1, 0, 0) > 32 * 192 * 192 * 2
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_DECODE, h, p, 32, 0, 65536) > 0
+    # invalid / unsupported arguments give 0
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, nsa.Heads(64, 5, 192, 128), p, 1, 10, 10) == 0
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, nsa.Heads(64, 4, 100, 128), p, 1, 10, 10) == 0
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, h, nsa.make_params(top_n=2), 1, 10, 10) == 0
+    assert nsa.nsa_workspace_size(7, h, p, 1, 10, 10) == 0
+
+
+def _call_prefill(L, heads, params, cu, ptr=16, ws_bytes=1 << 30, batch=None):
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    P = ctypes.c_void_p(ptr)
+    return L.nsa_prefill(P, P, P, P, P, P, cu_arr, len(cu) - 1 if batch is None else batch, ctypes.byref(heads),
+                         ctypes.byref(params), P, None, None, P, ws_bytes, None)
+
+
+def test_prefill_argument_validation_launches_nothing(L):
+    h = nsa.Heads(64, 4, 192, 128)
+    p = nsa.make_params()
+    assert _call_prefill(L, h, p, [0, 100], ptr=0) == nsa.NSA_ERR_INVALID_ARG          # null pointers
+    assert _call_prefill(L, h, p, [0, 100], ptr=8) == nsa.NSA_ERR_INVALID_ARG          # misaligned
+    assert _call_prefill(L, h, p, [1, 100]) == nsa.NSA_ERR_INVALID_ARG                 # cu_seqlens[0] != 0
+    assert _call_prefill(L, h, p, [0, 100, 50]) == nsa.NSA_ERR_INVALID_ARG             # decreasing
+    assert _call_prefill(L, h, p, [0, 100], batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert _call_prefill(L, h, p, [0, 100], ws_bytes=16) == nsa.NSA_ERR_WORKSPACE
+    assert _call_prefill(L, nsa.Heads(64, 4, 96, 128), p, [0, 100]) == nsa.NSA_ERR_UNSUPPORTED
+    assert _call_prefill(L, nsa.Heads(60, 4, 192, 128), p, [0, 100]) == nsa.NSA_ERR_UNSUPPORTED   # G = 15
+    assert _call_prefill(L, nsa.Heads(64, 3, 192, 128), p, [0, 100]) == nsa.NSA_ERR_INVALID_ARG
+    assert _call_prefill(L, h, nsa.make_params(l_cmp=30), [0, 100]) == nsa.NSA_ERR_INVALID_ARG   # l % s != 0
+    assert _call_prefill(L, h, nsa.make_params(l_sel=40), [0, 100]) == nsa.NSA_ERR_INVALID_ARG   # l' % s != 0
+    assert _call_prefill(L, h, nsa.make_params(top_n=2), [0, 100]) == nsa.NSA_ERR_INVALID_ARG    # n < forced
+    assert _call_prefill(L, h, nsa.make_params(l_cmp=64, stride=32), [0, 100]) == nsa.NSA_ERR_UNSUPPORTED
+    assert _call_prefill(L, h, nsa.make_params(top_n=40), [0, 100]) == nsa.NSA_ERR_UNSUPPORTED
+
+
+def test_decode_and_compress_validation(L):
+    h = nsa.Heads(64, 4, 192, 128)
+    p = nsa.make_params()
+    P = ctypes.c_void_p(16)
+    # max_len above Lmax
+    assert L.nsa_decode(P, P, P, P, P, P, 2, 100, 5, 200, P, ctypes.byref(h), ctypes.byref(p), P, None, None, P,
+                        1 << 30, None) == nsa.NSA_ERR_INVALID_ARG
+    # compressed cache too short for max_len
+    assert L.nsa_decode(P, P, P, P, P, P, 2, 1000, 5, 1000, P, ctypes.byref(h), ctypes.byref(p), P, None, None, P,
+                        1 << 30, None) == nsa.NSA_ERR_INVALID_ARG
+    # window too large for the decode union buffer
+    assert L.nsa_decode(P, P, P, P, P, P, 2, 1000, 61, 1000, P, ctypes.byref(h),
+                        ctypes.byref(nsa.make_params(window=8192)), P, None, None, P, 1 << 30,
+                        None) == nsa.NSA_ERR_UNSUPPORTED
+    i64 = (ctypes.c_int64 * 1)(0)
+    i32 = (ctypes.c_int32 * 1)(-5)
+    assert L.nsa_compress(P, P, P, P, P, P, i64, i32, i64, 1, ctypes.byref(h), ctypes.byref(p), P, P, P, 1 << 30,
+                          None) == nsa.NSA_ERR_INVALID_ARG
+    i32[0] = 100
+    assert L.nsa_compress(P, P, P, P, P, P, i64, i32, i64, 1, ctypes.byref(h), ctypes.byref(p), P, P, P, 8,
+                          None) == nsa.NSA_ERR_WORKSPACE
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(nsa, "_lib", None)
+    monkeypatch.setattr(nsa, "LIB_PATH", "/nonexistent/libnsa.so")
+    with pytest.raises(ImportError):
+        nsa.lib()

@@ -1,0 +1,145 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle
+on the same seeded inputs. See tests/nsa_parity.py for the acceptance rules."""
+import numpy as np
+import pytest
+import torch
+
+import nsa_workloads as W
+import sparse_attention_long_nsa_b200 as nsa
+from oracle import nsa_oracle as O
+from tests import nsa_parity as NP
+
+pytestmark = pytest.mark.gpu
+
+CFG = W.CONFIGS
+
+
+def test_prefill_tiny_full():
+    """1024-token GQA-4 prefill, every row compared."""
+    st = NP.run_prefill_case(CFG["prefill_tiny_1k"], [1024], n_random_rows=1024)
+    assert max(st["max_abs"]) <= NP.TOL_MAX
+
+
+@pytest.mark.parametrize("seqlens", [[100, 1000, 37], [31, 32, 33, 64, 65], [1], [700]])
+def test_prefill_tiny_varlen(seqlens):
+    NP.run_prefill_case(CFG["prefill_tiny_1k"], seqlens, n_random_rows=400, seed=7)
+
+
+@pytest.mark.parametrize("seqlens", [[1500], [700, 64, 1300]])
+def test_prefill_gqa16_ragged(seqlens):
+    """H_q=64, H_kv=4, d_k=192, d_v=128 at lengths spanning several tiles and a ragged tail."""
+    NP.run_prefill_case(CFG["prefill_8k"], seqlens, n_random_rows=128, seed=11)
+
+
+def test_prefill_8k_sampled():
+    """The benched 8K prefill, in the same launch configuration, on sampled rows."""
+    NP.run_prefill_case(CFG["prefill_8k"], [8192], n_random_rows=160)
+
+
+def test_prefill_64k_sampled():
+    NP.run_prefill_case(CFG["prefill_64k"], [65536], n_random_rows=48)
+
+
+def _dense_ref(inp, G, scale):
+    q = inp["q"].double().permute(1, 0, 2)[None]
+    k = inp["k"].double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    v = inp["v"].double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=scale)[0].permute(1, 0, 2)
+
+
+@pytest.mark.parametrize("branch", ["slc", "win"])
+def test_prefill_dense_reduction(branch):
+    """top-n covering every block (gates 0,1,0) or a window >= T (gates 0,0,1)
+    reduces NSA to dense causal attention."""
+    cfg = W.small_config(T=1000, H_q=16, H_kv=1, d_k=128, d_v=128, top_n=16, window=64, seed=5)
+    T = cfg.T
+    inp = W.make_prefill_inputs(cfg, device="cuda")
+    e = torch.zeros_like(inp["gates"])
+    e[..., 1 if branch == "slc" else 2] = 1.0
+    over = dict(top_n=16) if branch == "slc" else dict(window=T + 3)
+    heads = NP.heads_of(cfg)
+    par = NP.params_of(cfg, **over)
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [T], heads, par)
+    out = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, e, inp["cu_seqlens"], heads, par)
+    torch.cuda.synchronize()
+    ref = _dense_ref(inp, cfg.G, 1.0 / np.sqrt(cfg.d_k)).cpu().numpy()
+    NP.assert_close(NP.f64(out), ref, f"dense reduction ({branch})")
+
+
+def test_prefill_gate_linearity():
+    cfg = CFG["prefill_tiny_1k"]
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=[777])
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [777], heads, par)
+    full = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par).double()
+    acc = torch.zeros_like(full)
+    for b in range(3):
+        e = torch.zeros_like(inp["gates"])
+        e[..., b] = 1.0
+        ob = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, e, inp["cu_seqlens"], heads, par).double()
+        acc += inp["gates"][..., b:b + 1].double() * ob
+    NP.assert_close(full.cpu().numpy(), acc.cpu().numpy(), "gate linearity")
+
+
+def test_prefill_deterministic():
+    cfg = CFG["prefill_tiny_1k"]
+    inp = W.make_prefill_inputs(cfg, device="cuda")
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [1024], heads, par)
+    a = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par,
+                    want_sel=True)
+    b = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par,
+                    want_sel=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_compress_mean_pool_on_gpu():
+    """Averaging weights, no position embedding, stride = block: the compressed
+    keys are the block means (up to bf16 rounding of the weights 1/32)."""
+    cfg = CFG["prefill_tiny_1k"]
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=[640])
+    d = cfg.d_k
+    Wm = torch.cat([torch.eye(d)] * 32, 0).cuda() / 32
+    pe = torch.zeros(32, d, device="cuda")
+    heads = NP.heads_of(cfg)
+    kc, _ = nsa.compress(inp["k"], inp["v"], Wm, pe, Wm, pe, [640], heads, NP.params_of(cfg))
+    # stride 16 rows; blocks starting at multiples of 32 are rows 0, 2, 4, ...
+    means = inp["k"].double().reshape(20, 32, 1, d).mean(1)
+    NP.assert_close(NP.f64(kc[0::2]), means.cpu().numpy(), "mean-pool compression", relative_to_rms=True)
+
+
+@pytest.mark.parametrize("lens", [[8192, 3000, 33, 1], [31, 32, 64, 65, 127, 128, 129, 1000]])
+def test_decode_small(lens):
+    cfg = CFG["decode_64k"]
+    NP.run_decode_case(cfg, lens, seed=3)
+
+
+def test_decode_matches_prefill_last_row():
+    """The decode kernels and the prefill kernels agree on the last position."""
+    cfg = CFG["prefill_8k"]
+    T = 3000
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=[T])
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [T], heads, par)
+    out_p, sel_p = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par,
+                               want_sel=True)
+    lens = torch.tensor([T], dtype=torch.int32, device="cuda")
+    out_d, sel_d = nsa.decode(inp["q"][T - 1:T].contiguous(), inp["k"][None], inp["v"][None], kc[None], vc[None],
+                              lens, T, inp["gates"][T - 1:T].contiguous(), heads, par, want_sel=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sel_p[T - 1], sel_d[0])
+    NP.assert_close(NP.f64(out_d[0]), NP.f64(out_p[T - 1]), "decode vs prefill")
+
+
+def test_decode_64k_sampled():
+    cfg = CFG["decode_64k"]
+    NP.run_decode_case(cfg, [cfg.T] * cfg.B, batch_rows=[0, 13, 31])
+
+
+def test_decode_varlen_sampled():
+    cfg = CFG["decode_varlen"]
+
+    def pick(lens):
+        order = np.argsort(lens)
+        return [int(order[0]), int(order[len(lens) // 2]), int(order[-1])]
+    NP.run_decode_case(cfg, None, batch_rows=pick)
