@@ -14,12 +14,22 @@
 //    iff j <= i and i - j < w). One online-softmax pass; the epilogue writes
 //    out = bf16(acc + g_win * o_win), acc already holding the other branches.
 //
-// Tile: M = 128 rows = (128/G tokens) x (G heads of one KV group), so every
-// K/V tile staged in shared memory serves the whole GQA group. Roles:
-//   warps 0-3  softmax + epilogue, one accumulator row (TMEM lane) per thread
-//   warp 4     TMA producer (Q once, then K/V tiles of 64 keys, 2-stage ring)
-//   warp 5     tcgen05.mma issuer (S = Q.K^T into TMEM; O_tile = P.V with P
-//              read from TMEM and V as an MN-major shared-memory operand)
+// A CTA owns two query tiles of M = 128 rows, each (128/G tokens) x (G heads of
+// one KV group), so every K/V tile staged in shared memory serves the group's
+// heads of 2*128/G tokens. Roles (320 threads):
+//   warps 0-3 / 4-7  softmax warpgroup of query tile 0 / 1, one accumulator row
+//                    (TMEM lane) per thread
+//   warp 8           TMA producer (both Q tiles once, then K/V tiles of 64 keys
+//                    through a 3-stage ring)
+//   warp 9           tcgen05.mma issuer, alternating the two tiles so that one
+//                    tile's softmax overlaps the other tile's products:
+//                    QK0(j) QK1(j) | PV0(j) QK0(j+1) PV1(j) QK1(j+1) | ...
+// S = Q.K^T lands in TMEM; the softmax threads read it with tcgen05.ld, write P
+// (bf16) back to TMEM, and O += P.V runs with A = P from TMEM and V as an
+// MN-major shared-memory operand, accumulating in TMEM. The window pass keeps a
+// reference max per row and rescales O in TMEM only when the running max grows
+// by more than 8 (log2 units); exact, since O and the denominator always share
+// the reference.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -27,12 +37,15 @@ namespace nsa {
 
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kKeyTile = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr float kRescaleThreshold = 8.f;
 
-// TMEM column map (512 allocated)
-constexpr uint32_t kColS0 = 0, kColS1 = 64, kColP0 = 128, kColP1 = 160, kColO = 256;
+// TMEM columns (512 allocated): S, P and O of query tile q
+__device__ __forceinline__ uint32_t col_s(int q) { return q ? 64u : 0u; }
+__device__ __forceinline__ uint32_t col_p(int q) { return q ? 160u : 128u; }
+__device__ __forceinline__ uint32_t col_o(int q) { return q ? 384u : 256u; }
 
 struct Bars {
   uint64_t q_full;
@@ -41,19 +54,18 @@ struct Bars {
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t p_full[2];
-  uint64_t o_full;
-  uint64_t o_free;
+  uint64_t o_done[2];
   uint32_t tmem_base;
   int abort;
 };
 
 template <int DK, int DV>
 struct TcSmem {
-  static constexpr int Q_BYTES = 128 * DK * 2;
+  static constexpr int Q_BYTES = 128 * DK * 2;   // one query tile
   static constexpr int K_BYTES = kKeyTile * DK * 2;
   static constexpr int V_BYTES = kKeyTile * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int TOTAL = 1024 + Q_BYTES + kStages * STAGE + (int)sizeof(Bars) + 64;
+  static constexpr int TOTAL = 1024 + 2 * Q_BYTES + kStages * STAGE + (int)sizeof(Bars) + 64;
 };
 
 __device__ __forceinline__ int seq_of_tile(const SeqTable& t, int tile) {
@@ -69,6 +81,13 @@ __device__ __forceinline__ int cmp_visible_dev(int t, int l, int s) {
   return t >= l - 1 ? (t - l + 1) / s + 1 : 0;
 }
 
+// 2^x on the MUFU unit (PTX ex2.approx.ftz.f32; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 }  // namespace
 
 // MODE 0: compressed attention + importance; MODE 1: window attention + combine
@@ -77,24 +96,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
   using S = TcSmem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* Qs = smem;
-  uint8_t* KVs = smem + S::Q_BYTES;
+  uint8_t* Qs = smem;                                 // [2][Q_BYTES]
+  uint8_t* KVs = smem + 2 * S::Q_BYTES;               // [kStages][STAGE]
   Bars* bars = reinterpret_cast<Bars*>(KVs + kStages * S::STAGE);
   volatile int* abort_flag = &bars->abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G;
-  const int TOK = 128 / G;
+  const int TOK = 128 / G;                            // tokens per query tile
   const int tile = blockIdx.x;
   const int g = blockIdx.y;
   const int b = seq_of_tile(a.seqs, tile);
   const int L = a.seqs.len[b];
   const int64_t tok0 = a.seqs.tok_off[b];
-  const int t0 = (tile - a.seqs.tile_prefix[b]) * TOK;
-  const int t_last = min(t0 + TOK - 1, L - 1);
+  const int t0 = (tile - a.seqs.tile_prefix[b]) * 2 * TOK;
+  const int t_last = min(t0 + 2 * TOK - 1, L - 1);
 
-  // key tiles
-  int nk, key0;   // number of 64-key tiles and the first key (sequence-local)
+  // key tiles shared by both query tiles
+  int nk, key0;
   if (MODE == 0) {
     const int nv = cmp_visible_dev(t_last, a.l, a.s);
     nk = (nv + kKeyTile - 1) / kKeyTile;
@@ -104,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
     key0 = (lo / kKeyTile) * kKeyTile;
     nk = (t_last - key0) / kKeyTile + 1;
   }
-  const int n_s = (MODE == 0) ? 2 * nk : nk;   // S tiles produced
+  const int n_s = (MODE == 0) ? 2 * nk : nk;         // S tiles per query tile
 
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
@@ -113,9 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->s_free[i], 128);
       mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_done[i], 1);
     }
-    mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->o_free, 128);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -125,155 +143,149 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nk > 0) {
       prefetch_tmap(&m.q);
       const CUtensorMap* mk = MODE == 0 ? &m.kc : &m.k;
       const CUtensorMap* mv = MODE == 0 ? &m.vc : &m.v;
       const int64_t krow0 = MODE == 0 ? a.seqs.cmp_off[b] : tok0;
-      mbar_arrive_expect_tx(&bars->q_full, S::Q_BYTES);
-      for (int kb = 0; kb < DK / 64; ++kb)
-        tma_load_3d(Qs + kb * 16384, &m.q, &bars->q_full, kb * 64, g * G, (int)(tok0 + t0));
-      int it = 0;
-      const int passes = MODE == 0 ? 2 : 1;
-      bool ok = true;
-      for (int pass = 0; pass < passes && ok; ++pass) {
-        const bool with_v = (MODE == 1) || pass == 1;
-        for (int j = 0; j < nk; ++j, ++it) {
-          const int st = it % kStages;
-          if (it >= kStages &&
-              !mbar_wait(&bars->kv_empty[st], ((it / kStages) - 1) & 1, abort_flag, a.status, 201)) {
-            ok = false;
-            break;
-          }
-          uint8_t* Ks = KVs + st * S::STAGE;
-          uint8_t* Vs = Ks + S::K_BYTES;
-          mbar_arrive_expect_tx(&bars->kv_full[st], S::K_BYTES + (with_v ? S::V_BYTES : 0));
-          const int row = (int)(krow0 + key0 + j * kKeyTile);
-          for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->kv_full[st], kb * 64, g, row);
-          if (with_v)
-            for (int vb = 0; vb < DV / 64; ++vb) tma_load_3d(Vs + vb * 8192, mv, &bars->kv_full[st], vb * 64, g, row);
-        }
+      mbar_arrive_expect_tx(&bars->q_full, 2 * S::Q_BYTES);
+      for (int qt = 0; qt < 2; ++qt)
+        for (int kb = 0; kb < DK / 64; ++kb)
+          tma_load_3d(Qs + qt * S::Q_BYTES + kb * 16384, &m.q, &bars->q_full, kb * 64, g * G,
+                      (int)(tok0 + t0 + qt * TOK));
+      for (int jj = 0; jj < n_s; ++jj) {
+        const int st = jj % kStages;
+        const int j = (MODE == 0 && jj >= nk) ? jj - nk : jj;
+        const bool with_v = (MODE == 1) || jj >= nk;
+        if (jj >= kStages &&
+            !mbar_wait(&bars->kv_empty[st], ((jj / kStages) - 1) & 1, abort_flag, a.status, 201))
+          break;
+        uint8_t* Ks = KVs + st * S::STAGE;
+        mbar_arrive_expect_tx(&bars->kv_full[st], S::K_BYTES + (with_v ? S::V_BYTES : 0));
+        const int row = (int)(krow0 + key0 + j * kKeyTile);
+        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->kv_full[st], kb * 64, g, row);
+        if (with_v)
+          for (int vb = 0; vb < DV / 64; ++vb)
+            tma_load_3d(Ks + S::K_BYTES + vb * 8192, mv, &bars->kv_full[st], vb * 64, g, row);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nk > 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(128, kKeyTile, false, false);
       const uint32_t idesc_pv = umma_idesc_bf16(128, DV, false, true);
       const uint32_t q_addr = smem_u32(Qs);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.status, 211);
-      int it = 0;          // K/V stage counter
-      int pv = 0;          // PV products issued
-      int prev_st = 0;
-      auto issue_pv = [&](int jp, int st) -> bool {
-        // P_jp ready, previous O tile consumed
-        if (!mbar_wait(&bars->p_full[jp & 1], (jp >> 1) & 1, abort_flag, a.status, 212)) return false;
-        if (pv >= 1 && !mbar_wait(&bars->o_free, (pv - 1) & 1, abort_flag, a.status, 213)) return false;
+      auto qk = [&](int q, int jj) -> bool {
+        if (jj >= 1 && !mbar_wait(&bars->s_free[q], (jj - 1) & 1, abort_flag, a.status, 212)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(KVs + st * S::STAGE + S::K_BYTES);
-        const uint32_t p_col = (jp & 1) ? kColP1 : kColP0;
+        const uint32_t k_addr = smem_u32(KVs + (jj % kStages) * S::STAGE);
+        const uint32_t qa = q_addr + q * S::Q_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t dq = umma_desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t dk = umma_desc_sw128(k_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + col_s(q), dq, dk, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->s_full[q]);
+        return true;
+      };
+      auto pv = [&](int q, int jj, int jp) -> bool {
+        if (!mbar_wait(&bars->p_full[q], jp & 1, abort_flag, a.status, 213)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(KVs + (jj % kStages) * S::STAGE + S::K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < kKeyTile / 16; ++kk) {
           const uint64_t dv = umma_desc_sw128(v_addr + kk * 2048, 8192, 1024);
-          umma_ts(tmem + kColO, tmem + p_col + kk * 8, dv, idesc_pv, kk > 0 ? 1u : 0u);
+          umma_ts(tmem + col_o(q), tmem + col_p(q) + kk * 8, dv, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->o_full);
-        umma_commit(&bars->kv_empty[st]);
-        ++pv;
+        umma_commit(&bars->o_done[q]);
         return true;
       };
-      for (int jj = 0; jj < n_s && ok; ++jj, ++it) {
-        const int st = it % kStages;
-        if (!mbar_wait(&bars->kv_full[st], (it / kStages) & 1, abort_flag, a.status, 214)) { ok = false; break; }
-        const int sb = jj & 1;
-        if (jj >= 2 && !mbar_wait(&bars->s_free[sb], ((jj - 2) >> 1) & 1, abort_flag, a.status, 215)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(KVs + st * S::STAGE);
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint64_t dq = umma_desc_sw128(q_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t dk = umma_desc_sw128(k_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          umma_ss(tmem + (sb ? kColS1 : kColS0), dq, dk, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars->s_full[sb]);
+      if (ok) ok = mbar_wait(&bars->kv_full[0], 0, abort_flag, a.status, 214);
+      if (ok) ok = qk(0, 0) && qk(1, 0);
+      for (int jj = 0; jj < n_s && ok; ++jj) {
+        const int st = jj % kStages;
         const bool pv_pass = (MODE == 1) || jj >= nk;
-        const int jp = MODE == 1 ? jj : jj - nk;   // index within the PV pass
-        if (!pv_pass) {
-          umma_commit(&bars->kv_empty[st]);      // K-only stage is free once S is done
-        } else if (jp >= 1) {
-          if (!issue_pv(jp - 1, prev_st)) { ok = false; break; }
+        const int jp = MODE == 1 ? jj : jj - nk;
+        const bool more = jj + 1 < n_s;
+        if (pv_pass && !pv(0, jj, jp)) break;
+        if (more) {
+          const int s1 = jj + 1;
+          if (!mbar_wait(&bars->kv_full[s1 % kStages], (s1 / kStages) & 1, abort_flag, a.status, 215)) break;
+          if (!qk(0, s1)) break;
         }
-        prev_st = st;
+        if (pv_pass && !pv(1, jj, jp)) break;
+        umma_commit(&bars->kv_empty[st]);   // every product reading stage st has been issued
+        if (more && !qk(1, jj + 1)) break;
       }
-      if (ok) issue_pv(MODE == 1 ? nk - 1 : nk - 1, prev_st);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int r = tid;                 // accumulator row
+    // ------------------------------------------------------------ softmax warpgroups
+    const int q = warp >> 2;                 // query tile
+    const int r = tid & 127;                 // row within the tile = TMEM lane
     const int tt = r / G, hh = r % G;
-    const int t = t0 + tt;
+    const int t = t0 + q * TOK + tt;
     const bool valid = t < L;
     const int h = g * G + hh;
-    const int64_t n = tok0 + t;        // global token row
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float o_acc[DV];
-#pragma unroll
-    for (int i = 0; i < DV; ++i) o_acc[i] = 0.f;
-    float row_m = -1e30f, row_l = 0.f;
+    const int64_t n = tok0 + t;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t colS = tmem + lane_base + col_s(q);
+    const uint32_t colP = tmem + lane_base + col_p(q);
+    const uint32_t colO = tmem + lane_base + col_o(q);
     const float sc = a.scale_log2;
+    float row_m = -1e30f, row_l = 0.f;
     bool ok = true;
-
-    // visibility of key c of tile j for this row
     int nvis = 0, wlo = 0;
     if (MODE == 0) nvis = valid ? cmp_visible_dev(t, a.l, a.s) : 0;
     else wlo = max(0, t - a.window + 1);
-
-    // importance state (MODE 0): tile j covers blocks 16j .. 16j+16
-    float carry = 0.f;
     const int jt = t / a.ls;
-    const int nb_stride = a.nb_stride;
-    float* imp_row = a.imp + ((size_t)n * a.H_kv + g) * nb_stride;
+    float* imp_row = a.imp + ((size_t)n * a.H_kv + g) * a.nb_stride;
+    float carry = 0.f;
+    float linv = 0.f;
 
     auto load_s = [&](int jj, float* sv) -> bool {
-      const int sb = jj & 1;
-      if (!mbar_wait(&bars->s_full[sb], (jj >> 1) & 1, abort_flag, a.status, 221)) return false;
+      if (!mbar_wait(&bars->s_full[q], jj & 1, abort_flag, a.status, 221)) return false;
       tc_fence_after();
-      const uint32_t col = sb ? kColS1 : kColS0;
 #pragma unroll
-      for (int c = 0; c < kKeyTile; c += 16) tmem_ld16(tmem + lane_base + col + c, sv + c);
+      for (int c = 0; c < kKeyTile; c += 16) tmem_ld16(colS + c, sv + c);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars->s_free[sb]);
+      mbar_arrive(&bars->s_free[q]);
       return true;
     };
-    auto store_p = [&](int jp, const float* p) {
-      const uint32_t col = (jp & 1) ? kColP1 : kColP0;
+    // P tile jp into TMEM once PV(jp-1) has finished reading the previous one
+    auto store_p = [&](int jp, const float* p, float alpha) -> bool {
+      if (jp >= 1) {
+        if (!mbar_wait(&bars->o_done[q], (jp - 1) & 1, abort_flag, a.status, 222)) return false;
+        tc_fence_after();
+        if (MODE == 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // rescale this row of O (rare: the running max grew past the threshold)
+#pragma unroll 1
+          for (int c = 0; c < DV; c += 16) {
+            float ov[16];
+            tmem_ld16(colO + c, ov);
+            tmem_ld_wait();
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(ov[i] * alpha);
+            tmem_st8(colO + c, w);
+            tmem_st8(colO + c + 8, w + 8);
+          }
+        }
+      }
 #pragma unroll
       for (int c = 0; c < kKeyTile / 16; ++c) {
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(p[c * 16 + 2 * i], p[c * 16 + 2 * i + 1]);
-        tmem_st8(tmem + lane_base + col + c * 8, pk);
+        tmem_st8(colP + c * 8, pk);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[jp & 1]);
-    };
-    auto add_o = [&](int jp, float alpha) -> bool {
-      if (!mbar_wait(&bars->o_full, jp & 1, abort_flag, a.status, 222)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < DV; c += 16) {
-        float ov[16];
-        tmem_ld16(tmem + lane_base + kColO + c, ov);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) o_acc[c + i] = fmaf(o_acc[c + i], alpha, ov[i]);
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->o_free);
+      mbar_arrive(&bars->p_full[q]);
       return true;
     };
 
@@ -285,71 +297,56 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
         float mx = -1e30f;
 #pragma unroll
         for (int c = 0; c < kKeyTile; ++c) {
-          const int i = j * kKeyTile + c;
-          sv[c] = (i < nvis) ? sv[c] * sc : -INFINITY;
+          sv[c] = (j * kKeyTile + c < nvis) ? sv[c] * sc : -INFINITY;
           mx = fmaxf(mx, sv[c]);
         }
         const float m_new = fmaxf(row_m, mx);
         float sum = 0.f;
 #pragma unroll
-        for (int c = 0; c < kKeyTile; ++c) sum += exp2f(sv[c] - m_new);
-        row_l = row_l * exp2f(row_m - m_new) + sum;
+        for (int c = 0; c < kKeyTile; ++c) sum += ex2(sv[c] - m_new);
+        row_l = row_l * ex2(row_m - m_new) + sum;
         row_m = m_new;
       }
-      const float linv = row_l > 0.f ? 1.f / row_l : 0.f;
-      // ---- pass 2: probabilities, importance, P.V
+      linv = row_l > 0.f ? 1.f / row_l : 0.f;
+      // ---- pass 2: probabilities, importance, O += P.V
       for (int j = 0; j < nk && ok; ++j) {
         float sv[kKeyTile];
         if (!load_s(nk + j, sv)) { ok = false; break; }
 #pragma unroll
-        for (int c = 0; c < kKeyTile; ++c) {
-          const int i = j * kKeyTile + c;
-          sv[c] = (i < nvis) ? exp2f(sv[c] * sc - row_m) * linv : 0.f;
-        }
-        store_p(j, sv);
-        // spread over selection blocks: compressed token i = 4q + u covers tokens
-        // [16i, 16i + 32): u in {0,1,2} -> 2p into block q; u = 3 -> p into q and q+1
+        for (int c = 0; c < kKeyTile; ++c)
+          sv[c] = (j * kKeyTile + c < nvis) ? ex2(sv[c] * sc - row_m) * linv : 0.f;
+        if (!store_p(j, sv, 1.f)) { ok = false; break; }
+        // spread over selection blocks: compressed token i = 4u' + u covers tokens
+        // [16i, 16i + 32): u in {0,1,2} -> 2p into block u'; u = 3 -> p into u' and u'+1
         float blk[17];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float* pp = sv + 4 * q;
-          blk[q] = 2.f * (pp[0] + pp[1] + pp[2]) + pp[3];
+        for (int qb = 0; qb < 16; ++qb) {
+          const float* pp = sv + 4 * qb;
+          blk[qb] = 2.f * (pp[0] + pp[1] + pp[2]) + pp[3];
         }
         blk[16] = 0.f;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) blk[q + 1] += sv[4 * q + 3];
-        // sum over the G heads of this token (G consecutive lanes); the carry
-        // from the previous tile is already a group sum, so it is added after
+        for (int qb = 0; qb < 16; ++qb) blk[qb + 1] += sv[4 * qb + 3];
+        // sum over the G heads of this token (G consecutive lanes); the carry from
+        // the previous tile is already a group sum, so it is added after
 #pragma unroll
-        for (int q = 0; q < 17; ++q) {
-          float x = blk[q];
+        for (int qb = 0; qb < 17; ++qb) {
+          float x = blk[qb];
           for (int off = G >> 1; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-          blk[q] = x;
+          blk[qb] = x;
         }
         blk[0] += carry;
         carry = blk[16];
-        if (valid) {
-          for (int q = hh; q < 16; q += G) {
-            const int jb = j * 16 + q;
-            if (jb <= jt) imp_row[jb] = blk[q];
+        if (valid)
+          for (int qb = hh; qb < 16; qb += G) {
+            const int jb = j * 16 + qb;
+            if (jb <= jt) imp_row[jb] = blk[qb];
           }
-        }
-        if (j >= 1 && !add_o(j - 1, 1.f)) { ok = false; break; }
       }
-      if (ok && nk > 0 && !add_o(nk - 1, 1.f)) ok = false;
-      if (ok && valid) {
-        // the carried block and blocks no visible compressed token reaches
+      if (ok && valid)   // the carried block and blocks no visible compressed token reaches
         for (int jb = nk * 16 + hh; jb <= jt; jb += G) imp_row[jb] = (jb == nk * 16) ? carry : 0.f;
-        float* dst = a.acc + ((size_t)n * a.H_q + h) * DV;
-        const float gc = a.gates[((size_t)n * a.H_q + h) * 3 + 0];
-#pragma unroll
-        for (int c = 0; c < DV; c += 4)
-          *reinterpret_cast<float4*>(dst + c) =
-              make_float4(gc * o_acc[c], gc * o_acc[c + 1], gc * o_acc[c + 2], gc * o_acc[c + 3]);
-      }
     } else {
-      // ---- window: single online-softmax pass
-      float alpha_prev = 1.f;
+      // ---- window: one online-softmax pass with a lazily rescaled reference max
       for (int j = 0; j < nk && ok; ++j) {
         float sv[kKeyTile];
         if (!load_s(j, sv)) { ok = false; break; }
@@ -361,38 +358,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
           sv[c] = vis ? sv[c] * sc : -INFINITY;
           mx = fmaxf(mx, sv[c]);
         }
-        const float m_new = fmaxf(row_m, mx);
-        const float alpha = exp2f(row_m - m_new);
+        float alpha = 1.f;
+        if (mx > row_m + kRescaleThreshold) {
+          alpha = ex2(row_m - mx);
+          row_l *= alpha;
+          row_m = mx;
+        }
         float sum = 0.f;
 #pragma unroll
         for (int c = 0; c < kKeyTile; ++c) {
-          sv[c] = exp2f(sv[c] - m_new);
+          sv[c] = ex2(sv[c] - row_m);
           sum += sv[c];
         }
-        row_l = row_l * alpha + sum;
-        row_m = m_new;
-        store_p(j, sv);
-        if (j >= 1 && !add_o(j - 1, alpha_prev)) { ok = false; break; }
-        alpha_prev = alpha;
+        row_l += sum;
+        if (!store_p(j, sv, alpha)) { ok = false; break; }
       }
-      if (ok && !add_o(nk - 1, alpha_prev)) ok = false;
-      if (ok && valid) {
-        const float linv = row_l > 0.f ? 1.f / row_l : 0.f;
-        const float gw = a.gates[((size_t)n * a.H_q + h) * 3 + 2] * linv;
-        const float* src = a.acc + ((size_t)n * a.H_q + h) * DV;
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + h) * DV;
+      linv = row_l > 0.f ? 1.f / row_l : 0.f;
+    }
+
+    // ---- epilogue: O (TMEM) -> output
+    const int n_pv = nk;
+    if (ok && n_pv > 0) ok = mbar_wait(&bars->o_done[q], (n_pv - 1) & 1, abort_flag, a.status, 223);
+    tc_fence_after();
+    if (ok && n_pv > 0) {
+      const float* gsrc = a.gates + ((size_t)n * a.H_q + h) * 3;
+      float* accp = a.acc + ((size_t)n * a.H_q + h) * DV;
+#pragma unroll 1
+      for (int c = 0; c < DV; c += 32) {
+        float ov[32];
+        tmem_ld16(colO + c, ov);
+        tmem_ld16(colO + c + 16, ov + 16);
+        tmem_ld_wait();
+        if (!valid) continue;
+        if (MODE == 0) {
+          const float gc = gsrc[0];   // P was normalised already
 #pragma unroll
-        for (int c = 0; c < DV; c += 8) {
-          const float4 a0 = *reinterpret_cast<const float4*>(src + c);
-          const float4 a1 = *reinterpret_cast<const float4*>(src + c + 4);
-          uint4 pk;
-          pk.x = pack_bf16x2(fmaf(gw, o_acc[c + 0], a0.x), fmaf(gw, o_acc[c + 1], a0.y));
-          pk.y = pack_bf16x2(fmaf(gw, o_acc[c + 2], a0.z), fmaf(gw, o_acc[c + 3], a0.w));
-          pk.z = pack_bf16x2(fmaf(gw, o_acc[c + 4], a1.x), fmaf(gw, o_acc[c + 5], a1.y));
-          pk.w = pack_bf16x2(fmaf(gw, o_acc[c + 6], a1.z), fmaf(gw, o_acc[c + 7], a1.w));
-          *reinterpret_cast<uint4*>(dst + c) = pk;
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(accp + c + i) =
+                make_float4(gc * ov[i], gc * ov[i + 1], gc * ov[i + 2], gc * ov[i + 3]);
+        } else {
+          const float gw = gsrc[2] * linv;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + h) * DV + c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const float4 a0 = *reinterpret_cast<const float4*>(accp + c + i);
+            const float4 a1 = *reinterpret_cast<const float4*>(accp + c + i + 4);
+            uint4 pk;
+            pk.x = pack_bf16x2(fmaf(gw, ov[i + 0], a0.x), fmaf(gw, ov[i + 1], a0.y));
+            pk.y = pack_bf16x2(fmaf(gw, ov[i + 2], a0.z), fmaf(gw, ov[i + 3], a0.w));
+            pk.z = pack_bf16x2(fmaf(gw, ov[i + 4], a1.x), fmaf(gw, ov[i + 5], a1.y));
+            pk.w = pack_bf16x2(fmaf(gw, ov[i + 6], a1.z), fmaf(gw, ov[i + 7], a1.w));
+            *reinterpret_cast<uint4*>(dst + i) = pk;
+          }
         }
       }
+    }
+    if (MODE == 0 && nk == 0 && valid) {
+      // no compressed token visible to any row: o_cmp = 0, importance 0
+      for (int jb = hh; jb <= jt; jb += G) imp_row[jb] = 0.f;
+      float* accp = a.acc + ((size_t)n * a.H_q + h) * DV;
+      for (int c = 0; c < DV; c += 4) *reinterpret_cast<float4*>(accp + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 

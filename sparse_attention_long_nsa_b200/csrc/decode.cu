@@ -14,8 +14,10 @@
 //       g_cmp * o_cmp, reduce the block sums over the group's heads into the
 //       importance, run the top-n selection.
 //   D3  split over the union of selected blocks and window blocks, 4 blocks per
-//       CTA: one score tile serves both branches, each with its own softmax.
-//   D4  merge the D3 partials and write out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
+//       CTA: one score tile serves both branches, each with its own softmax. The
+//       last CTA of each (sequence, KV head) to finish (atomic counter, no
+//       waiting) merges the partials and writes
+//       out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
 #include "common.cuh"
 #include "kernels.h"
 #include "topn.cuh"
@@ -48,22 +50,29 @@ struct DecSmem {
 __device__ __forceinline__ int n_cmp_dev(int L, int l, int s) { return L >= l ? (L - l) / s + 1 : 0; }
 
 struct PartLayout {
-  size_t cp, tp, fp;   // offsets (floats)
+  // offsets in floats; every row of DV floats starts 16-byte aligned
+  size_t cp_o, cp_ml, tp, fp_o, fp_ml, cnt, total;
   int n_tiles;
 };
 __host__ __device__ inline PartLayout part_layout(const DecodeArgs& a) {
   PartLayout p;
+  const size_t BG = (size_t)a.B * a.H_kv;
   p.n_tiles = a.n_cmp_chunks * kTilesPerChunk;
-  p.cp = 0;
-  p.tp = p.cp + (size_t)a.B * a.H_kv * a.n_cmp_chunks * a.G * (a.d_v + 2);
-  p.fp = p.tp + (size_t)a.B * a.H_kv * p.n_tiles * a.G * kTP;
+  p.cp_o = 0;                                                      // [BG][nch][G][DV]
+  p.cp_ml = p.cp_o + BG * a.n_cmp_chunks * a.G * a.d_v;            // [BG][nch][G][2]
+  p.tp = p.cp_ml + BG * a.n_cmp_chunks * a.G * 2;                  // [BG][tiles][18][G]
+  p.tp = (p.tp + 3) & ~size_t(3);
+  p.fp_o = p.tp + BG * p.n_tiles * kTP * a.G;                      // [BG][nsw][2][G][DV]
+  p.fp_ml = p.fp_o + BG * a.n_sw_chunks * 2 * a.G * a.d_v;         // [BG][nsw][2][G][2]
+  p.cnt = p.fp_ml + BG * a.n_sw_chunks * 2 * a.G * 2;              // [BG] int counters
+  p.total = p.cnt + BG;
   return p;
 }
 
-// merge 4 staged warp states ([w][16][DV+2]) into one row state, for row < G,
-// writing (o relative to M, M, L) to dst[row][DV+2]
+// merge 4 staged warp states ([w][16][DV+2]) into one state per row < G:
+// o relative to the merged max M -> dst_o[row][DV], (M, L) -> dst_ml[row][2]
 template <int DV>
-__device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst, int tid) {
+__device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_o, float* dst_ml, int tid) {
   const int per_row = (kDecConsumers * 32) / 16;
   const int row = tid / per_row, part = tid % per_row;
   if (row >= G) return;
@@ -79,20 +88,17 @@ __device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst,
   for (int c = part * span; c < (part + 1) * span; ++c) {
     float v = 0.f;
     for (int w = 0; w < kDecConsumers; ++w) v += f[w] * stg[(w * 16 + row) * (DV + 2) + c];
-    dst[row * (DV + 2) + c] = v;
+    dst_o[row * DV + c] = v;
   }
   if (part == 0) {
-    dst[row * (DV + 2) + DV] = M;
-    dst[row * (DV + 2) + DV + 1] = Ls;
+    dst_ml[row * 2 + 0] = M;
+    dst_ml[row * 2 + 1] = Ls;
   }
 }
 
 }  // namespace
 
-size_t decode_partials_floats(const DecodeArgs& a) {
-  const PartLayout p = part_layout(a);
-  return p.fp + (size_t)a.B * a.H_kv * a.n_sw_chunks * 2 * a.G * (a.d_v + 2);
-}
+size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total; }
 
 // ---------------------------------------------------------------------------
 // D1: compressed keys, split-K
@@ -182,30 +188,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       // block sums: compressed key 4q+u covers tokens [16(4q+u), +32): u<3 -> 2p
-      // into block q of the tile, u = 3 -> p into q and q+1 (17 relative blocks)
+      // into block q of the tile, u = 3 -> p into q and q+1 (17 relative blocks).
+      // Tile partial layout [18][G]: row 0 = reference max per head, rows 1..17 =
+      // block sums per head.
       {
+        const int tile = (c0 / 64) + i;
+        float* tpb = a.part + pl.tp + (((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * kTP * G;
         const int row = lane >> 1, half = lane & 1;
         if (row < G) {
-          const int tile = (c0 / 64) + i;
-          float* tp = a.part + pl.tp + ((((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * G + row) * kTP;
           const float* pr = ps + row * 64;
           const int q0 = half * 8;
           for (int q = q0; q < q0 + 8; ++q) {
             float v = 2.f * (pr[4 * q] + pr[4 * q + 1] + pr[4 * q + 2]) + pr[4 * q + 3];
             if (q > 0) v += pr[4 * q - 1];
-            tp[1 + q] = v;
+            tpb[(1 + q) * G + row] = v;
           }
-          if (half == 1) tp[1 + 16] = pr[63];
+          if (half == 1) tpb[17 * G + row] = pr[63];
         }
-      }
-      // m_ref of each row: lane (row%8)*4 holds m for rows r0 and r0+8
-      {
-        const int tile = (c0 / 64) + i;
         if ((lane & 3) == 0) {
           const int r0 = lane >> 2;
-          float* base = a.part + pl.tp + ((((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * G) * kTP;
-          if (r0 < G) base[r0 * kTP] = rs.m[0];
-          if (r0 + 8 < G) base[(r0 + 8) * kTP] = rs.m[1];
+          if (r0 < G) tpb[r0] = rs.m[0];
+          if (r0 + 8 < G) tpb[r0 + 8] = rs.m[1];
         }
       }
       __syncwarp();
@@ -215,17 +218,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
     float* stg = reinterpret_cast<float*>(ring);
     rs.stage(stg + warp * 16 * (DV + 2), lane);
     named_bar_sync(1, kDecConsumers * 32);
-    float* cp = a.part + pl.cp + (((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk) * G * (DV + 2);
-    merge_warps<DV>(stg, G, cp, tid);
+    const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
+    merge_warps<DV>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
   }
   __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
-// D2: merge compressed chunks, importance, selection
+// D2: merge compressed chunks, importance, selection (one CTA per (b, g))
 // ---------------------------------------------------------------------------
+constexpr int kSelThreadsD2 = 256;
+
 template <int DV, int PER>
-__global__ void __launch_bounds__(128) dec_select_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeArgs a) {
   extern __shared__ float sm[];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = a.G;
@@ -237,57 +242,68 @@ __global__ void __launch_bounds__(128) dec_select_kernel(const DecodeArgs a) {
   const int t = L - 1;
   const int jt = t / a.ls;
   const PartLayout pl = part_layout(a);
-  float* Mh = sm;             // [16]
-  float* Li = sm + 16;        // [16] 1/L
-  float* imp_s = sm + 32;     // [nb_stride]
-  const float* cp = a.part + pl.cp + ((size_t)b * a.H_kv + g) * a.n_cmp_chunks * G * (DV + 2);
-  const float* tp = a.part + pl.tp + ((size_t)b * a.H_kv + g) * pl.n_tiles * G * kTP;
+  const size_t bg = (size_t)b * a.H_kv + g;
+  float* Mh = sm;                           // [16]
+  float* Li = sm + 16;                      // [16] 1/L
+  float* Fc = sm + 32;                      // [nch][16]   chunk factors
+  float* Ft = Fc + a.n_cmp_chunks * 16;     // [ntl][16]   tile factors (incl. 1/L)
+  float* imp_s = Ft + pl.n_tiles * 16;      // [nb_stride]
+  const float* cpo = a.part + pl.cp_o + bg * a.n_cmp_chunks * G * DV;
+  const float* cpm = a.part + pl.cp_ml + bg * a.n_cmp_chunks * G * 2;
+  const float* tp = a.part + pl.tp + bg * pl.n_tiles * kTP * G;
+  if (tid == 0) reinterpret_cast<int*>(a.part + pl.cnt)[bg] = 0;   // D3 completion counter
   if (tid < G) {
     float M = -1e30f;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, cp[((size_t)c * G + tid) * (DV + 2) + DV]);
+    for (int c = 0; c < nch; ++c)
+      if (cpm[(c * G + tid) * 2 + 1] > 0.f) M = fmaxf(M, cpm[(c * G + tid) * 2]);
     float Ls = 0.f;
     for (int c = 0; c < nch; ++c) {
-      const float* r = cp + ((size_t)c * G + tid) * (DV + 2);
-      if (r[DV + 1] > 0.f) Ls += exp2f(r[DV] - M) * r[DV + 1];
+      const float l = cpm[(c * G + tid) * 2 + 1];
+      const float f = l > 0.f ? exp2f(cpm[(c * G + tid) * 2] - M) : 0.f;
+      Fc[c * 16 + tid] = f;
+      Ls += f * l;
     }
     Mh[tid] = M;
     Li[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
   __syncthreads();
-  // g_cmp * o_cmp
-  for (int idx = tid; idx < G * DV; idx += blockDim.x) {
-    const int h = idx / DV, c = idx % DV;
-    float v = 0.f;
-    for (int ch = 0; ch < nch; ++ch) {
-      const float* r = cp + ((size_t)ch * G + h) * (DV + 2);
-      if (r[DV + 1] > 0.f) v += exp2f(r[DV] - Mh[h]) * r[c];
+  for (int idx = tid; idx < ntl * G; idx += kSelThreadsD2) {
+    const int tj = idx / G, h = idx % G;
+    Ft[tj * 16 + h] = exp2f(tp[(size_t)tj * kTP * G + h] - Mh[h]) * Li[h];
+  }
+  // g_cmp * o_cmp, 4 values per thread
+  for (int idx = tid; idx < G * (DV / 4); idx += kSelThreadsD2) {
+    const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < nch; ++c) {
+      const float f = Fc[c * 16 + h];
+      const float4 v = *reinterpret_cast<const float4*>(cpo + ((size_t)c * G + h) * DV + c4);
+      acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
     }
     const int hq = g * G + h;
-    a.ocmp[((size_t)b * a.H_q + hq) * DV + c] = a.gates[((size_t)b * a.H_q + hq) * 3 + 0] * v * Li[h];
+    const float sc = a.gates[((size_t)b * a.H_q + hq) * 3 + 0] * Li[h];
+    *reinterpret_cast<float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4) =
+        make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
   }
-  // importance of blocks 0..jt
-  for (int j = tid; j <= jt; j += blockDim.x) {
+  __syncthreads();
+  // importance of blocks 0..jt: tile tj holds blocks 16 tj .. 16 tj + 16
+  for (int j = tid; j <= jt; j += kSelThreadsD2) {
     const int tj = j >> 4, q = j & 15;
     float v = 0.f;
-    for (int h = 0; h < G; ++h) {
-      float x = 0.f;
-      if (tj < ntl) {
-        const float* r = tp + ((size_t)tj * G + h) * kTP;
-        x += exp2f(r[0] - Mh[h]) * r[1 + q];
-      }
-      if (q == 0 && tj >= 1 && tj - 1 < ntl) {
-        const float* r = tp + ((size_t)(tj - 1) * G + h) * kTP;
-        x += exp2f(r[0] - Mh[h]) * r[1 + 16];
-      }
-      v += x * Li[h];
+    if (tj < ntl) {
+      const float* r = tp + ((size_t)tj * kTP + 1 + q) * G;
+      for (int h = 0; h < G; ++h) v += Ft[tj * 16 + h] * r[h];
+    }
+    if (q == 0 && tj >= 1 && tj - 1 < ntl) {
+      const float* r = tp + ((size_t)(tj - 1) * kTP + 17) * G;
+      for (int h = 0; h < G; ++h) v += Ft[(tj - 1) * 16 + h] * r[h];
     }
     imp_s[j] = v;
-    a.imp[((size_t)b * a.H_kv + g) * a.nb_stride + j] = v;
+    a.imp[bg * a.nb_stride + j] = v;
   }
   __syncthreads();
   if (tid < 32)
-    warp_topn<PER>(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + ((size_t)b * a.H_kv + g) * a.top_n,
-                   tid);
+    warp_topn<PER>(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, tid);
 }
 
 // ---------------------------------------------------------------------------
@@ -315,7 +331,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   const int wlo = max(0, t - a.window + 1);
   const int G = a.G;
   const PartLayout pl = part_layout(a);
-  float* fp = a.part + pl.fp + (((size_t)b * a.H_kv + g) * a.n_sw_chunks + cc) * 2 * G * (DV + 2);
+  const size_t bg = (size_t)b * a.H_kv + g;
+  float* fpo = a.part + pl.fp_o + (bg * a.n_sw_chunks + cc) * 2 * G * DV;
+  float* fpm = a.part + pl.fp_ml + (bg * a.n_sw_chunks + cc) * 2 * G * 2;
 
   if (tid < 32) sel_s[tid] = tid < a.top_n ? a.sel[((size_t)b * a.H_kv + g) * a.top_n + tid] : -1;
   __syncthreads();
@@ -403,47 +421,60 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     rs_sel.stage(stg + warp * 16 * (DV + 2), lane);
     rs_win.stage(stg + (kDecConsumers + warp) * 16 * (DV + 2), lane);
     named_bar_sync(1, kDecConsumers * 32);
-    merge_warps<DV>(stg, G, fp, tid);
-    merge_warps<DV>(stg + kDecConsumers * 16 * (DV + 2), G, fp + G * (DV + 2), tid);
+    merge_warps<DV>(stg, G, fpo, fpm, tid);
+    merge_warps<DV>(stg + kDecConsumers * 16 * (DV + 2), G, fpo + G * DV, fpm + G * 2, tid);
+  }
+  // the last CTA of this (b, g) to get here combines the three branches
+  __shared__ int last;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const int done = atomicAdd(reinterpret_cast<int*>(a.part + pl.cnt) + bg, 1);
+    last = done == a.n_sw_chunks - 1;
   }
   __syncthreads();
-}
-
-// ---------------------------------------------------------------------------
-// D4: merge the fine partials and combine the three branches
-// ---------------------------------------------------------------------------
-template <int DV>
-__global__ void __launch_bounds__(256) dec_combine_kernel(const DecodeArgs a) {
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int G = a.G;
-  const int L = a.lens[b];
-  if (L < 1 || L > a.max_len) return;
-  const PartLayout pl = part_layout(a);
-  const float* fp = a.part + pl.fp + ((size_t)b * a.H_kv + g) * a.n_sw_chunks * 2 * G * (DV + 2);
-  for (int idx = tid; idx < G * DV; idx += blockDim.x) {
-    const int h = idx / DV, c = idx % DV;
-    const int hq = g * G + h;
-    float res = a.ocmp[((size_t)b * a.H_q + hq) * DV + c];
-#pragma unroll
-    for (int br = 0; br < 2; ++br) {
-      float M = -1e30f;
-      for (int cc = 0; cc < a.n_sw_chunks; ++cc) {
-        const float* r = fp + (((size_t)cc * 2 + br) * G + h) * (DV + 2);
-        if (r[DV + 1] > 0.f) M = fmaxf(M, r[DV]);
-      }
-      float num = 0.f, den = 0.f;
-      for (int cc = 0; cc < a.n_sw_chunks; ++cc) {
-        const float* r = fp + (((size_t)cc * 2 + br) * G + h) * (DV + 2);
-        if (r[DV + 1] > 0.f) {
-          const float f = exp2f(r[DV] - M);
-          num += f * r[c];
-          den += f * r[DV + 1];
-        }
-      }
-      const float gate = a.gates[((size_t)b * a.H_q + hq) * 3 + 1 + br];
-      res += den > 0.f ? gate * num / den : 0.f;
+  if (!last) return;
+  __threadfence();
+  float* fac = reinterpret_cast<float*>(ring);       // [2][nsw][16] factors, then [2][16] 1/den
+  const float* po = a.part + pl.fp_o + bg * a.n_sw_chunks * 2 * G * DV;
+  const volatile float* pm = a.part + pl.fp_ml + bg * a.n_sw_chunks * 2 * G * 2;
+  float* inv = fac + 2 * a.n_sw_chunks * 16;
+  if (tid < 2 * G) {
+    const int br = tid / G, h = tid % G;
+    float M = -1e30f;
+    for (int c = 0; c < a.n_sw_chunks; ++c) {
+      const size_t r = (((size_t)c * 2 + br) * G + h) * 2;
+      if (pm[r + 1] > 0.f) M = fmaxf(M, pm[r]);
     }
-    static_cast<__nv_bfloat16*>(a.out)[((size_t)b * a.H_q + hq) * DV + c] = __float2bfloat16_rn(res);
+    float den = 0.f;
+    for (int c = 0; c < a.n_sw_chunks; ++c) {
+      const size_t r = (((size_t)c * 2 + br) * G + h) * 2;
+      const float f = pm[r + 1] > 0.f ? exp2f(pm[r] - M) : 0.f;
+      fac[(br * a.n_sw_chunks + c) * 16 + h] = f;
+      den += f * pm[r + 1];
+    }
+    const float gate = a.gates[((size_t)b * a.H_q + g * G + h) * 3 + 1 + br];
+    inv[br * 16 + h] = den > 0.f ? gate / den : 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * (DV / 4); idx += kDecThreads) {
+    const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
+    const int hq = g * G + h;
+    float4 res = *reinterpret_cast<const float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4);
+    for (int br = 0; br < 2; ++br) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < a.n_sw_chunks; ++c) {
+        const float f = fac[(br * a.n_sw_chunks + c) * 16 + h];
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(po + (((size_t)c * 2 + br) * G + h) * DV + c4));
+        acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
+      }
+      const float s_ = inv[br * 16 + h];
+      res.x += s_ * acc.x; res.y += s_ * acc.y; res.z += s_ * acc.z; res.w += s_ * acc.w;
+    }
+    uint2 pk;
+    pk.x = pack_bf16x2(res.x, res.y);
+    pk.y = pack_bf16x2(res.z, res.w);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)b * a.H_q + hq) * DV + c4) = pk;
   }
 }
 
@@ -463,15 +494,26 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int per = (a.nb_stride + 31) / 32;
-  const size_t sm2 = (32 + (size_t)a.nb_stride) * 4;
+  const size_t sm2 = (32 + (size_t)a.n_cmp_chunks * 16 + (size_t)a.n_cmp_chunks * kTilesPerChunk * 16 +
+                      (size_t)a.nb_stride) * 4;
+  if (sm2 > 48 * 1024) {
+    cudaError_t e2 = cudaSuccess;
+    if (per <= 4) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    else if (per <= 8) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    else if (per <= 16) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    else if (per <= 32) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    else if (per <= 64) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    else e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    if (e2 != cudaSuccess) return e2;
+  }
   dim3 g2(a.H_kv, a.B);
   prof_begin(P_DEC_SELECT, st);
-  if (per <= 4) dec_select_kernel<DV, 4><<<g2, 128, sm2, st>>>(a);
-  else if (per <= 8) dec_select_kernel<DV, 8><<<g2, 128, sm2, st>>>(a);
-  else if (per <= 16) dec_select_kernel<DV, 16><<<g2, 128, sm2, st>>>(a);
-  else if (per <= 32) dec_select_kernel<DV, 32><<<g2, 128, sm2, st>>>(a);
-  else if (per <= 64) dec_select_kernel<DV, 64><<<g2, 128, sm2, st>>>(a);
-  else if (per <= 128) dec_select_kernel<DV, 128><<<g2, 128, sm2, st>>>(a);
+  if (per <= 4) dec_select_kernel<DV, 4><<<g2, kSelThreadsD2, sm2, st>>>(a);
+  else if (per <= 8) dec_select_kernel<DV, 8><<<g2, kSelThreadsD2, sm2, st>>>(a);
+  else if (per <= 16) dec_select_kernel<DV, 16><<<g2, kSelThreadsD2, sm2, st>>>(a);
+  else if (per <= 32) dec_select_kernel<DV, 32><<<g2, kSelThreadsD2, sm2, st>>>(a);
+  else if (per <= 64) dec_select_kernel<DV, 64><<<g2, kSelThreadsD2, sm2, st>>>(a);
+  else if (per <= 128) dec_select_kernel<DV, 128><<<g2, kSelThreadsD2, sm2, st>>>(a);
   else return cudaErrorInvalidValue;
   prof_end(P_DEC_SELECT, st, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -479,9 +521,6 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
   k3<<<dim3(a.n_sw_chunks, a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
   prof_end(P_DEC_FINE, st, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prof_begin(P_DEC_COMBINE, st);
-  dec_combine_kernel<DV><<<dim3(a.H_kv, a.B), 256, 0, st>>>(a);
-  prof_end(P_DEC_COMBINE, st, 1);
   return cudaGetLastError();
 }
 

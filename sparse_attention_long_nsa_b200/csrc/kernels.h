@@ -61,14 +61,14 @@ struct PrefillArgs {
   int nb_stride;
   float scale_log2;       // softmax scale * log2(e)
   uint32_t* status;
-  SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens
+  SeqTable seqs;          // tile_prefix counts CTA tiles of 2 x 128/G tokens
 };
 struct PrefillMaps {
   CUtensorMap q, k, v, kc, vc;
 };
 cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st);
-cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int64_t n_tokens, cudaStream_t st);
+cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 cudaError_t launch_win_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 
 // ----- decode -----

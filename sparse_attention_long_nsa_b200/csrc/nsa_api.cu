@@ -405,7 +405,7 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   a.scale_log2 = softmax_scale(params, heads->d_k) * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws);
 
-  const int tok_per_tile = 128 / a.G;
+  const int tok_per_tile = 2 * (128 / a.G);   // two 128-row query tiles per attention CTA
   SeqTable t{};
   t.n = batch;
   int tiles = 0;
@@ -426,7 +426,7 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   memset(&m, 0, sizeof(m));
   const void* kc_base = ncmp_total > 0 ? k_cmp : k;
   const void* vc_base = ncmp_total > 0 ? v_cmp : v;
-  if (!make_map_3d(&m.q, q, heads->d_k, heads->H_q, N, a.G, tok_per_tile) ||
+  if (!make_map_3d(&m.q, q, heads->d_k, heads->H_q, N, a.G, 128 / a.G) ||
       !make_map_3d(&m.k, k, heads->d_k, heads->H_kv, N, 1, 64) ||
       !make_map_3d(&m.v, v, heads->d_v, heads->H_kv, N, 1, 64) ||
       !make_map_3d(&m.kc, kc_base, heads->d_k, heads->H_kv, ncmp_total, 1, 64) ||
@@ -445,7 +445,7 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   prof_end(P_TOPN, st, 1);
   if (e != cudaSuccess) return cuda_fail(e, "top-n selection");
   prof_begin(P_SEL_ATTN, st);
-  e = launch_sel_attn(a, m, N, st);
+  e = launch_sel_attn(a, m, tiles, st);
   prof_end(P_SEL_ATTN, st, 1);
   if (e != cudaSuccess) return cuda_fail(e, "selected attention");
   prof_begin(P_WIN_ATTN, st);

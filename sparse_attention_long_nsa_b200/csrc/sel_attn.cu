@@ -27,6 +27,15 @@ namespace nsa {
 
 namespace {
 
+__device__ __forceinline__ int seq_of_tile(const SeqTable& t, int tile) {
+  int lo = 0, hi = t.n - 1;
+  while (lo < hi) {   // last b with tile_prefix[b] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (t.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ int seq_of_token(const SeqTable& t, int64_t row) {
   int lo = 0, hi = t.n - 1;
   while (lo < hi) {   // last b with tok_off[b] <= row and len > 0 reaching it
@@ -72,20 +81,33 @@ cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st)
 
 // ---------------------------------------------------------------------------
 // selected-block attention
+//
+// CTA = 8 consecutive tokens of one sequence x one KV head; consumer warp w owns
+// token t0 + w (its G heads are the 16 MMA rows). The blocks the 8 tokens
+// selected are merged into one ascending union; each union block is loaded once
+// by TMA into a 4-stage ring and used by every warp whose token selected it
+// (the forced blocks 0, jt-1, jt are shared by all 8). Every warp walks the
+// whole union in order (waiting for each stage, computing only on its own
+// blocks) so the stage barriers stay in phase; once all 8 warps released a
+// stage, lane 0 of warp 0 refills it with the block 4 positions ahead (8 warps,
+// two per SM sub-partition, keep the full register budget). Each warp adds
+// g_slc * o_slc of its own token to the fp32 accumulator from its fragments.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int kSelStages = 4;
-constexpr int kSelConsumers = 4;
-constexpr int kSelThreads = (kSelConsumers + 1) * 32;
+constexpr int kSelTok = 8;                        // tokens (consumer warps) per CTA
+constexpr int kSelThreads = kSelTok * 32;       // warp 0 lane 0 also refills the ring
+constexpr int kSelMaxUnion = kSelTok * 32;        // top_n <= 32
 
 template <int DK, int DV>
 struct SelSmem {
   static constexpr int K_BYTES = 64 * DK * 2;
   static constexpr int V_BYTES = 64 * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int MERGE = kSelConsumers * 16 * (DV + 2) * 4;
   static constexpr int RING = kSelStages * STAGE;
-  static constexpr int TOTAL = 1024 + (RING > MERGE ? RING : MERGE) + 1024;
+  // ring | barriers (2 * stages) | union list | union masks | flags | bitmap [nb_stride]
+  static constexpr int FIXED = 1024 + RING + 2 * kSelStages * 8 + kSelMaxUnion * 8 + 64;
+  static int total(int nb_stride) { return FIXED + nb_stride * 4; }
 };
 }  // namespace
 
@@ -96,55 +118,95 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (S::RING > S::MERGE ? S::RING : S::MERGE));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING);
   uint64_t* empty = full + kSelStages;
-  int* sel_s = reinterpret_cast<int*>(empty + kSelStages);     // [32]
-  volatile int* abort_flag = sel_s + 32;
+  int* uni = reinterpret_cast<int*>(empty + kSelStages);        // [kSelMaxUnion]
+  uint32_t* umask = reinterpret_cast<uint32_t*>(uni + kSelMaxUnion);
+  int* nuni = reinterpret_cast<int*>(umask + kSelMaxUnion);
+  volatile int* abort_flag = nuni + 1;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(nuni + 16);         // [nb_stride] warp bits per block
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n = blockIdx.x / a.H_kv;
-  const int g = blockIdx.x % a.H_kv;
-  const int b = seq_of_token(a.seqs, n);
-  const int t = (int)(n - a.seqs.tok_off[b]);
-  const int64_t tok0 = a.seqs.tok_off[b];
   const int G = a.G;
+  const int TOK = 256 / G, SUB = TOK / kSelTok;   // host tiles hold 2 x 128/G tokens
+  const int tile = blockIdx.x / SUB, sub = blockIdx.x % SUB;
+  const int g = blockIdx.y;
+  const int b = seq_of_tile(a.seqs, tile);
+  const int L = a.seqs.len[b];
+  const int64_t tok0 = a.seqs.tok_off[b];
+  const int t0 = (tile - a.seqs.tile_prefix[b]) * TOK + sub * kSelTok;
+  if (t0 >= L) return;   // whole CTA past the end of its sequence (uniform)
+  const int t_last = min(t0 + kSelTok - 1, L - 1);
+  const int jt_max = t_last / a.ls;
 
-  if (tid < 32) sel_s[tid] = tid < a.top_n ? a.sel[((size_t)n * a.H_kv + g) * a.top_n + tid] : -1;
+  for (int j = tid; j <= jt_max; j += kSelThreads) bm[j] = 0u;
   if (tid == 0) {
-    for (int i = 0; i < kSelStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < kSelStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kSelTok); }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  int nsel = 0;
-  while (nsel < a.top_n && sel_s[nsel] >= 0) ++nsel;
-
-  if (warp == kSelConsumers) {
-    if (lane == 0) {
-      for (int i = 0; i < nsel; ++i) {
-        const int st = i % kSelStages;
-        if (i >= kSelStages && !mbar_wait(&empty[st], ((i / kSelStages) - 1) & 1, abort_flag, a.status, 301)) break;
-        uint8_t* Ks = ring + st * S::STAGE;
-        uint8_t* Vs = Ks + S::K_BYTES;
-        const int row = (int)(tok0 + (int64_t)sel_s[i] * a.ls);
-        mbar_arrive_expect_tx(&full[st], S::STAGE);
-        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
-        for (int vb = 0; vb < DV / 64; ++vb) tma_load_3d(Vs + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
+  // mark the blocks each token selected
+  const int t = t0 + warp;
+  const bool has_tok = warp < kSelTok && t < L;
+  const int64_t n = tok0 + t;
+  if (has_tok && lane < a.top_n) {
+    const int j = a.sel[((size_t)n * a.H_kv + g) * a.top_n + lane];
+    if (j >= 0 && j <= jt_max) atomicOr(&bm[j], 1u << warp);
+  }
+  __syncthreads();
+  // compact the union in ascending block order (warp 0)
+  if (warp == 0) {
+    int cnt = 0;
+    for (int j0 = 0; j0 <= jt_max; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t m = j <= jt_max ? bm[j] : 0u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, m != 0u);
+      if (m != 0u) {
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        uni[pos] = j;
+        umask[pos] = m;
       }
+      cnt += __popc(bal);
     }
-  } else {
-    uint32_t qa[DK / 16][4];
-    RowState<DV> rs;
-    rs.init();
+    if (lane == 0) *nuni = cnt;
+  }
+  __syncthreads();
+  const int nu = *nuni;
+
+  auto issue = [&](int u) {
+    const int st = u % kSelStages;
+    uint8_t* Ks = ring + st * S::STAGE;
+    const int row = (int)(tok0 + (int64_t)uni[u] * a.ls);
+    mbar_arrive_expect_tx(&full[st], S::STAGE);
+    for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
+    for (int vb = 0; vb < DV / 64; ++vb) tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
+  };
+  const bool producer = warp == 0 && lane == 0;
+  if (producer)
+    for (int u = 0; u < nu && u < kSelStages; ++u) issue(u);
+
+  uint32_t qa[DK / 16][4];
+  RowState<DV> rs;
+  rs.init();
+  if (has_tok) {
     const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)n * a.H_q + (size_t)g * G) * DK;
     load_q_frags<DK>(qa, qp, G, lane);
-    for (int i = warp; i < nsel; i += kSelConsumers) {
-      const int st = i % kSelStages;
-      if (!mbar_wait(&full[st], (i / kSelStages) & 1, abort_flag, a.status, 302)) break;
+  }
+  const uint32_t bit = 1u << warp;
+  bool ok = true;
+  for (int u = 0; u < nu; ++u) {
+    const int st = u % kSelStages;
+    // warp-uniform outcome of the (bounded) wait
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kSelStages) & 1, abort_flag, a.status, 302))) {
+      ok = false;
+      break;
+    }
+    if (umask[u] & bit) {
       const uint32_t kb = smem_u32(ring + st * S::STAGE);
       float s[8][4];
       warp_qk<DK>(qa, kb, s, lane);
-      const int key0 = sel_s[i] * a.ls + (lane & 3) * 2;
+      const int key0 = uni[u] * a.ls + (lane & 3) * 2;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
@@ -156,36 +218,43 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
       }
       rs.update(s);
       warp_pv<DV>(s, kb + S::K_BYTES, rs.o, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
     }
-    rs.finish();
-    // publish the partial state once every consumer is done with the ring
-    named_bar_sync(1, kSelConsumers * 32);
-    rs.stage(reinterpret_cast<float*>(ring) + warp * 16 * (DV + 2), lane);
-    named_bar_sync(1, kSelConsumers * 32);
-    // merge: thread handles (row, dv range)
-    const float* base = reinterpret_cast<const float*>(ring);
-    const int per_row = (kSelConsumers * 32) / 16;   // threads per row
-    const int row = tid / per_row;
-    const int part = tid % per_row;
-    if (row < G) {
-      float M = -1e30f;
-      for (int w = 0; w < kSelConsumers; ++w) M = fmaxf(M, base[(w * 16 + row) * (DV + 2) + DV]);
-      float wsc[kSelConsumers], Lsum = 0.f;
-      for (int w = 0; w < kSelConsumers; ++w) {
-        const float* rw = base + (w * 16 + row) * (DV + 2);
-        wsc[w] = rw[DV + 1] > 0.f ? exp2f(rw[DV] - M) : 0.f;
-        Lsum += wsc[w] * rw[DV + 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (warp == 0 && u + kSelStages < nu) {
+      // once every warp is done with this stage, refill it
+      bool p_ok = true;
+      if (producer) {
+        p_ok = mbar_wait(&empty[st], (u / kSelStages) & 1, abort_flag, a.status, 301);
+        if (p_ok) issue(u + kSelStages);
       }
-      const int h = g * G + row;
-      const float gs = a.gates[((size_t)n * a.H_q + h) * 3 + 1] / Lsum;
-      float* dst = a.acc + ((size_t)n * a.H_q + h) * DV;
-      const int span = DV / per_row;
-      for (int c = part * span; c < (part + 1) * span; ++c) {
-        float v = 0.f;
-        for (int w = 0; w < kSelConsumers; ++w) v += wsc[w] * base[(w * 16 + row) * (DV + 2) + c];
-        dst[c] += gs * v;
+      if (!__shfl_sync(0xffffffffu, p_ok, 0)) {
+        ok = false;
+        break;
+      }
+    }
+  }
+  {
+    rs.finish();
+    if (has_tok && ok) {
+      // acc[n, h, :] += g_slc * o / l for the group's heads (rows lane/4, lane/4 + 8)
+      const int r0 = lane >> 2, cq = (lane & 3) * 2;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int row = r0 + half * 8;
+        if (row < G) {
+          const int h = g * G + row;
+          const float gs = a.gates[((size_t)n * a.H_q + h) * 3 + 1] / rs.l[half];
+          float* dst = a.acc + ((size_t)n * a.H_q + h) * DV;
+#pragma unroll
+          for (int i = 0; i < DV / 8; ++i) {
+            float2* p = reinterpret_cast<float2*>(dst + i * 8 + cq);
+            float2 v = *p;
+            v.x += gs * rs.o[i][2 * half];
+            v.y += gs * rs.o[i][2 * half + 1];
+            *p = v;
+          }
+        }
       }
     }
   }
@@ -193,25 +262,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
 }
 
 template <int DK, int DV>
-static cudaError_t launch_sel_t(const PrefillArgs& a, const PrefillMaps& m, int64_t n_tokens, cudaStream_t st) {
+static cudaError_t launch_sel_t(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
   using S = SelSmem<DK, DV>;
   auto kern = sel_attn_kernel<DK, DV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
+  const int smem = S::total(a.nb_stride);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = n_tokens * a.H_kv;
-  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, kSelThreads, S::TOTAL, st>>>(a, m);
+  const int sub = (256 / a.G) / kSelTok;
+  kern<<<dim3(n_tiles * sub, a.H_kv), kSelThreads, smem, st>>>(a, m);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int64_t n_tokens, cudaStream_t st) {
-  if (n_tokens == 0) return cudaSuccess;
-  if (a.d_k == 192 && a.d_v == 128) return launch_sel_t<192, 128>(a, m, n_tokens, st);
-  if (a.d_k == 64 && a.d_v == 64) return launch_sel_t<64, 64>(a, m, n_tokens, st);
-  if (a.d_k == 128 && a.d_v == 128) return launch_sel_t<128, 128>(a, m, n_tokens, st);
-  if (a.d_k == 192 && a.d_v == 64) return launch_sel_t<192, 64>(a, m, n_tokens, st);
-  if (a.d_k == 64 && a.d_v == 128) return launch_sel_t<64, 128>(a, m, n_tokens, st);
-  if (a.d_k == 128 && a.d_v == 64) return launch_sel_t<128, 64>(a, m, n_tokens, st);
+cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
+  if (n_tiles == 0) return cudaSuccess;
+  if (a.d_k == 192 && a.d_v == 128) return launch_sel_t<192, 128>(a, m, n_tiles, st);
+  if (a.d_k == 64 && a.d_v == 64) return launch_sel_t<64, 64>(a, m, n_tiles, st);
+  if (a.d_k == 128 && a.d_v == 128) return launch_sel_t<128, 128>(a, m, n_tiles, st);
+  if (a.d_k == 192 && a.d_v == 64) return launch_sel_t<192, 64>(a, m, n_tiles, st);
+  if (a.d_k == 64 && a.d_v == 128) return launch_sel_t<64, 128>(a, m, n_tiles, st);
+  if (a.d_k == 128 && a.d_v == 64) return launch_sel_t<128, 64>(a, m, n_tiles, st);
   return cudaErrorInvalidValue;
 }
 
