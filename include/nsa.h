@@ -116,6 +116,34 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
                           const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
                           void* v_cmp, void* workspace, size_t ws_bytes, void* stream);
 
+/* nsa_compress without a workspace argument, for callers that cannot allocate
+ * device memory where they compress: code that runs while a CUDA graph is being
+ * captured, engines that fix their memory plan ahead of time and forbid
+ * allocation on the serving path, plugins inside a framework that owns every
+ * device allocation. There is no counterpart in the pages describing NSA: this
+ * is an interface convenience. Same arguments, layouts, arithmetic and results
+ * as nsa_compress, minus workspace/ws_bytes.
+ *  - Scratch: a file-scope device array of NSA_NOALLOC_SCRATCH_BYTES (4 MiB)
+ *    inside libnsa.so; every GPU that loads the library keeps it reserved until
+ *    the process exits. Calls that would need more scratch than that return
+ *    NSA_ERR_WORKSPACE (with a message in nsa_last_error_detail()); no supported
+ *    head size needs more (d_k = 192, d_v = 128 needs 3.6 MB).
+ *  - Allocates nothing: no cudaMalloc/cudaFree or allocating library call.
+ *  - Set-up: the first call on a device looks up the array's device address for
+ *    the current device (cudaGetSymbolAddress); make that first call before any
+ *    stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the last
+ *    call's contents (each call clears the status word it needs zeroed). Calls
+ *    whose work overlaps on the GPU (different streams, or different host
+ *    threads) race on the array and must be serialised by the caller.
+ *  - nsa_check_device_status() does not apply (the status word is internal). */
+#define NSA_NOALLOC_SCRATCH_BYTES 4194304
+nsa_status_t nsa_compress_noalloc(const void* k, const void* v, const float* w_ck, const float* pe_k,
+                                  const float* w_cv, const float* pe_v, const int64_t* tok_offset,
+                                  const int32_t* seq_len, const int64_t* cmp_offset, int32_t batch,
+                                  const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
+                                  void* v_cmp, void* stream);
+
 /* Causal NSA prefill over packed variable-length sequences (NSA-ru "NSA: три
  * ветви"; NSA-lesson "Concept"). Positions restart at 0 in every sequence.
  *   q        bf16 [N, H_q, d_k], N = cu_seqlens[batch]

@@ -24,10 +24,11 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_DEVICE_CHECK = range(6)
 NSA_OP_COMPRESS, NSA_OP_PREFILL, NSA_OP_DECODE = 0, 1, 2
 NSA_MAX_BATCH = 128
+NSA_NOALLOC_SCRATCH_BYTES = 4194304
 
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
-            "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
+            "nsa_compress_noalloc", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
 NSA_PROFILE_SLOTS = 10
 
@@ -77,6 +78,9 @@ def lib() -> ctypes.CDLL:
     L.nsa_compress.restype = ctypes.c_int
     L.nsa_compress.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params),
                                P, P, P, SZ, P]
+    L.nsa_compress_noalloc.restype = ctypes.c_int
+    L.nsa_compress_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
+                                       ctypes.POINTER(Params), P, P, P]
     L.nsa_prefill.restype = ctypes.c_int
     L.nsa_prefill.argtypes = [P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params), P, P, P,
                               P, SZ, P]
@@ -158,6 +162,20 @@ def nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, 
                            _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream))
     _check(s, "nsa_compress")
+
+
+def nsa_compress_noalloc(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, heads: Heads,
+                         params: Params, k_cmp, v_cmp, stream=None):
+    """nsa_compress without a workspace: scratch is a fixed device array inside
+    the library (see include/nsa.h). Calls that overlap on the GPU race."""
+    B = int(seq_len.numel())
+    s = lib().nsa_compress_noalloc(_ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16), _ptr(w_ck, torch.float32),
+                                   _ptr(pe_k, torch.float32), _ptr(w_cv, torch.float32), _ptr(pe_v, torch.float32),
+                                   _ptr(tok_offset, torch.int64, "cpu"), _ptr(seq_len, torch.int32, "cpu"),
+                                   _ptr(cmp_offset, torch.int64, "cpu"), B, ctypes.byref(heads),
+                                   ctypes.byref(params), _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16),
+                                   _stream(stream))
+    _check(s, "nsa_compress_noalloc")
 
 
 def nsa_prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, out, sel_out=None,

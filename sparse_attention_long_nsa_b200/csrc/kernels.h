@@ -16,6 +16,7 @@ enum ProfSlot {
   P_DEC_CMP, P_DEC_SELECT, P_DEC_FINE, P_DEC_COMBINE, P_COUNT
 };
 void prof_begin(int slot, cudaStream_t st);
+void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()
 void prof_end(int slot, cudaStream_t st, int launches);
 
 // Per-launch sequence table, passed by value as a kernel parameter.

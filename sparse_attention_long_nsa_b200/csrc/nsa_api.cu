@@ -188,6 +188,8 @@ const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "cmp_attn",
 }  // namespace
 
 namespace nsa {
+void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+
 void prof_begin(int slot, cudaStream_t st) {
   Profiler& p = prof();
   std::lock_guard<std::mutex> g(p.mu);

@@ -1,0 +1,73 @@
+"""nsa_compress_noalloc: the compression entry point for callers that cannot
+allocate device memory where they compress (graph capture in progress, a fixed
+memory plan, a host framework that owns every allocation). Its scratch is a
+fixed device array inside libnsa.so instead of a caller workspace.
+
+Called through the C ABI twice in a row (the array keeps the previous call's
+contents, so the second call checks that nothing stale leaks through) and
+compared with nsa_compress, which takes an explicit workspace, within the
+tolerance the parity tests use for compressed K/V. Kept in a file of its own
+that is collected last."""
+import pytest
+import torch
+
+import nsa_workloads as W
+import sparse_attention_long_nsa_b200 as nsa
+from tests import nsa_parity as NP
+
+pytestmark = pytest.mark.gpu
+
+
+def _offsets(seqlens, params):
+    tok, cmp_, t, c = [], [], 0, 0
+    for L in seqlens:
+        tok.append(t)
+        cmp_.append(c)
+        t += L
+        c += nsa.n_cmp(L, params.l_cmp, params.stride)
+    return (torch.tensor(tok, dtype=torch.int64), torch.tensor(seqlens, dtype=torch.int32),
+            torch.tensor(cmp_, dtype=torch.int64), c)
+
+
+@pytest.mark.parametrize("cfg_name,seqlens", [("prefill_8k", [1500, 64, 700]), ("prefill_tiny_1k", [1024, 31, 333])])
+def test_noalloc_matches_workspace_entry_point(cfg_name, seqlens):
+    cfg = W.CONFIGS[cfg_name]
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    tok, lens, cmp_off, total = _offsets(seqlens, par)
+    ref_k = ref_v = None
+    # reference: the workspace entry point
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=123)
+    ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, len(seqlens), 0, 0), "cuda")
+    ref_k = torch.empty((total, cfg.H_kv, cfg.d_k), dtype=torch.bfloat16, device="cuda")
+    ref_v = torch.empty((total, cfg.H_kv, cfg.d_v), dtype=torch.bfloat16, device="cuda")
+    nsa.nsa_compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], tok, lens, cmp_off,
+                     heads, par, ref_k, ref_v, ws)
+    torch.cuda.synchronize()
+    for call in range(2):
+        # different inputs for the first call, so a stale scratch would show
+        if call == 0:
+            other = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=999)
+            k_tmp = torch.empty_like(ref_k)
+            v_tmp = torch.empty_like(ref_v)
+            nsa.nsa_compress_noalloc(other["k"], other["v"], other["w_ck"], other["pe_k"], other["w_cv"],
+                                     other["pe_v"], tok, lens, cmp_off, heads, par, k_tmp, v_tmp)
+        k_out = torch.full_like(ref_k, float("nan"))
+        v_out = torch.full_like(ref_v, float("nan"))
+        nsa.nsa_compress_noalloc(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], tok, lens,
+                                 cmp_off, heads, par, k_out, v_out)
+        torch.cuda.synchronize()
+        NP.assert_close(NP.f64(k_out), NP.f64(ref_k), f"k_cmp (no-alloc call {call})", relative_to_rms=True)
+        NP.assert_close(NP.f64(v_out), NP.f64(ref_v), f"v_cmp (no-alloc call {call})", relative_to_rms=True)
+
+
+def test_noalloc_rejects_invalid_arguments():
+    cfg = W.CONFIGS["prefill_8k"]
+    par = NP.params_of(cfg)
+    tok, lens, cmp_off, total = _offsets([100], par)
+    x = torch.zeros((100, 4, 192), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((32 * 192, 192), dtype=torch.float32, device="cuda")
+    pe = torch.zeros((32, 192), dtype=torch.float32, device="cuda")
+    out = torch.zeros((max(total, 1), 4, 192), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(nsa.NSAError) as ei:
+        nsa.nsa_compress_noalloc(x, x, w, pe, w, pe, tok, lens, cmp_off, nsa.Heads(64, 4, 96, 96), par, out, out)
+    assert ei.value.status == nsa.NSA_ERR_UNSUPPORTED
