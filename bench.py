@@ -235,7 +235,7 @@ def run_nsa(args, rank, ws):
     k_cmp = torch.empty((nc, cfg.H_kv, cfg.d_k), dtype=torch.bfloat16, device=dev)
     v_cmp = torch.empty((nc, cfg.H_kv, cfg.d_v), dtype=torch.bfloat16, device=dev)
     out = torch.empty((T, cfg.H_q, cfg.d_v), dtype=torch.bfloat16, device=dev)
-    ws_c = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, 1, 0, 0), dev)
+    ws_c = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, 1, T, T), dev)
     ws_p = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, heads, par, 1, T, T), dev)
     tok = torch.zeros(1, dtype=torch.int64)
     seq = torch.tensor([T], dtype=torch.int32)

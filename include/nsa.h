@@ -78,7 +78,9 @@ typedef struct {
 enum { NSA_OP_COMPRESS = 0, NSA_OP_PREFILL = 1, NSA_OP_DECODE = 2 };
 
 /* Bytes of workspace `op` needs. `batch` = number of sequences;
- * `total_tokens` = sum of sequence lengths (prefill), ignored otherwise;
+ * `total_tokens` = sum of sequence lengths (prefill; for NSA_OP_COMPRESS it sizes
+ * optional room that lets nsa_compress split its reduction across more SMs when
+ * the output rows are packed; 0 gives the minimum, which is always valid);
  * `max_len` = longest sequence (prefill) or upper bound of the cache lengths
  * (decode). Returns 0 for invalid arguments. */
 size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* params,

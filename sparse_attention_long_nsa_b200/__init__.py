@@ -249,7 +249,8 @@ def compress(k, v, w_ck, pe_k, w_cv, pe_v, seqlens, heads: Heads, params: Params
     else:
         k_cmp, v_cmp = out
     if ws is None:
-        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, len(seqlens), 0, 0), dev)
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, len(seqlens), sum(seqlens), 0),
+                             dev)
     nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok, torch.tensor(seqlens, dtype=torch.int32), cmp_off, heads,
                  params, k_cmp, v_cmp, ws)
     return k_cmp[:total], v_cmp[:total]

@@ -81,13 +81,6 @@ __device__ __forceinline__ int cmp_visible_dev(int t, int l, int s) {
   return t >= l - 1 ? (t - l + 1) / s + 1 : 0;
 }
 
-// 2^x on the MUFU unit (PTX ex2.approx.ftz.f32; 2^-inf = 0)
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 }  // namespace
 
 // MODE 0: compressed attention + importance; MODE 1: window attention + combine

@@ -63,6 +63,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -85,6 +89,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > NSA_WAIT_LIMIT_NS) {
+      *abort_flag = 1;
+      if (status) {
+        atomicOr(status, DEV_ERR_TIMEOUT);
+        atomicExch(status + 1, site);
+      }
+      return false;
+    }
+  }
+}
+
+// Bounded wait until a shared-memory word equals `want` (written by another warp
+// of the same CTA). Same failure handling as mbar_wait.
+__device__ __forceinline__ bool smem_wait_eq(const volatile int* word, int want, volatile int* abort_flag,
+                                             uint32_t* status, uint32_t site) {
+  if (*word == want) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(20);
+    if (*word == want) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > NSA_WAIT_LIMIT_NS) {
       *abort_flag = 1;
@@ -276,6 +301,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
+
+// 2^x on the MUFU unit (PTX ex2.approx.ftz.f32, relative error ~2^-22; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // ---------------------------------------------------------------------------
 // warp-level mma.sync (m16n8k16, bf16 -> fp32) and ldmatrix, for the 16-row

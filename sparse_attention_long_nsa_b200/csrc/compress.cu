@@ -10,7 +10,9 @@
 // The GEMM runs on the 5th-generation tensor cores: M = 128 compressed rows of
 // one KV head, N = d_out, K = l*d_in, bf16 operands staged in 128-byte-swizzled
 // shared memory, fp32 accumulator in tensor memory (tcgen05.mma issued by one
-// thread), read back with tcgen05.ld for the bias-add + bf16 epilogue.
+// thread), read back with tcgen05.ld for the bias-add + bf16 epilogue. When the
+// rows give too few CTAs to fill the GPU, the K = l*d_in reduction is split over
+// grid.z into fp32 partial sums that a small kernel adds in a fixed order.
 // Operand rows are a strided gather (row i starts at token i*s), so they are
 // fetched with cp.async rather than a tensor map.
 #include "common.cuh"
@@ -104,7 +106,8 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
   const int i0 = (tile - a.seqs.tile_prefix[b]) * kTileM;
   const int64_t tok0 = a.seqs.tok_off[b];
   const int K = a.l * D_IN;
-  const int nkb = K / 64;
+  const int kb0 = blockIdx.z * a.kb_per_split;                 // this CTA's share of K
+  const int nkb = min(K / 64 - kb0, a.kb_per_split);
   constexpr uint32_t TM_COLS = D_OUT <= 64 ? 64 : (D_OUT <= 128 ? 128 : 256);
 
   if (tid == 0) {
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
   auto load_stage = [&](int st, int kb) {
     uint8_t* A = smem + st * S::STAGE;
     uint8_t* Bm = A + S::A_BYTES;
-    const int f0 = kb * 64;
+    const int f0 = (kb0 + kb) * 64;
     const int r = f0 / D_IN, e0 = f0 % D_IN;
     {  // A: one 128-byte row per thread
       const int row = tid;
@@ -196,12 +199,19 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
       tmem_ld16(tmem_d + ((uint32_t)(warp * 32) << 16) + c0, v);
       tmem_ld_wait();
       if (ci < ncmp) {
-        uint32_t pk[8];
+        if (a.ksplit == 1) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(v[2 * j] + a.bias[c0 + 2 * j], v[2 * j + 1] + a.bias[c0 + 2 * j + 1]);
-        uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int j = 0; j < 8; ++j)
+            pk[j] = pack_bf16x2(v[2 * j] + a.bias[c0 + 2 * j], v[2 * j + 1] + a.bias[c0 + 2 * j + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.part + (size_t)blockIdx.z * a.rows_total * a.H_kv * D_OUT + orow + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
       }
     }
   }
@@ -216,8 +226,34 @@ static cudaError_t launch_gemm_t(const CompressArgs& a, int n_tiles, cudaStream_
   auto kern = compress_gemm_kernel<D_IN, D_OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
   if (e != cudaSuccess) return e;
-  dim3 grid(n_tiles, a.H_kv);
+  dim3 grid(n_tiles, a.H_kv, a.ksplit);
   kern<<<grid, 128, S::TOTAL, st>>>(a);
+  return cudaGetLastError();
+}
+
+// out[r, :] = bf16(sum_z part[z, r, :] + bias) over the packed output rows, the
+// partial sums added in a fixed order (deterministic)
+__global__ void compress_finalize_kernel(const float* __restrict__ part, int ksplit, int64_t n4, int d_out,
+                                         const float* __restrict__ bias, __nv_bfloat16* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+  if (i >= n4) return;
+  float4 acc = reinterpret_cast<const float4*>(part)[i];
+  for (int z = 1; z < ksplit; ++z) {
+    const float4 v = reinterpret_cast<const float4*>(part)[(size_t)z * n4 + i];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  const int c = (int)((i * 4) % d_out);
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x + bias[c], acc.y + bias[c + 1]);
+  pk.y = pack_bf16x2(acc.z + bias[c + 2], acc.w + bias[c + 3]);
+  reinterpret_cast<uint2*>(out)[i] = pk;
+}
+
+cudaError_t launch_compress_finalize(int d_out, const CompressArgs& a, cudaStream_t st) {
+  const int64_t n4 = a.rows_total * a.H_kv * d_out / 4;
+  if (n4 <= 0) return cudaSuccess;
+  compress_finalize_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(a.part, a.ksplit, n4, d_out, a.bias,
+                                                                          static_cast<__nv_bfloat16*>(a.out));
   return cudaGetLastError();
 }
 

@@ -13,10 +13,9 @@
 //   D2  per (sequence, KV head): merge the chunks, normalise, finish
 //       g_cmp * o_cmp, reduce the block sums over the group's heads into the
 //       importance, run the top-n selection.
-//   D3  split over the union of selected blocks and window blocks, 4 blocks per
-//       CTA: one score tile serves both branches, each with its own softmax. The
-//       last CTA of each (sequence, KV head) to finish (atomic counter, no
-//       waiting) merges the partials and writes
+//   D3  one CTA per (sequence, KV head) streams the union of the selected
+//       blocks and the window blocks once; one score tile serves both branches,
+//       each with its own softmax; it writes
 //       out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
 #include "common.cuh"
 #include "kernels.h"
@@ -101,125 +100,191 @@ __device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_
 size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total; }
 
 // ---------------------------------------------------------------------------
-// D1: compressed keys, split-K
+// D1: compressed keys, split into 512-key chunks. Persistent: one CTA per SM walks
+// the (sequence, KV head, chunk) items round-robin; the producer warp keeps the
+// ring full across item boundaries (Q of the next item double-buffered), so the
+// HBM stream never drains between items.
 // ---------------------------------------------------------------------------
+template <int DK, int DV>
+struct D1Smem {
+  static constexpr int STAGE = 64 * (DK + DV) * 2;
+  static constexpr int RING = kDecStages * STAGE;
+  static constexpr int QBUF = (DK / 64) * 16 * 128;                 // one item's Q, 16 rows
+  static constexpr int STG = kDecConsumers * 16 * (DV + 2) * 4;      // per-warp states for the merge
+  static constexpr int PSCR = kDecConsumers * 16 * 64 * 4;           // probabilities for block sums
+  static constexpr int TOTAL = 1024 + RING + 2 * QBUF + STG + PSCR + 256;
+};
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArgs a,
                                                                  const __grid_constant__ DecodeMaps mp) {
-  using S = DecSmem<DK, DV>;
+  using S = D1Smem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  float* pscr = reinterpret_cast<float*>(smem + S::BODY);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BODY + S::PSCR);
+  uint8_t* qbuf = smem + S::RING;
+  float* stg = reinterpret_cast<float*>(qbuf + 2 * S::QBUF);
+  float* pscr = stg + S::STG / 4;
+  uint64_t* full = reinterpret_cast<uint64_t*>(pscr + S::PSCR / 4);
   uint64_t* empty = full + kDecStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
+  uint64_t* q_full = empty + kDecStages;     // [2]
+  uint64_t* q_empty = q_full + 2;            // [2]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(q_empty + 2);
+  volatile int* item_abort = abort_flag + 1;   // abort flag as seen at an item end, same for all warps
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int L = a.lens[b];
-  if (L < 1 || L > a.max_len) {
-    if (tid == 0 && chunk == 0 && g == 0) atomicOr(a.status, DEV_ERR_BOUNDS);
-    return;
-  }
-  const int nc = n_cmp_dev(L, a.l, a.s);
-  const int c0 = chunk * kCmpChunk;
-  if (c0 >= nc) return;
-  const int ntl = min(kTilesPerChunk, (nc - c0 + 63) / 64);
   const int G = a.G;
   const PartLayout pl = part_layout(a);
+  const int n_items = a.B * a.H_kv * a.n_cmp_chunks;
 
   if (tid == 0) {
     for (int i = 0; i < kDecStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], kDecConsumers); }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
+  // item -> (b, g, chunk); returns the number of 64-key tiles (0: nothing to do)
+  auto item_tiles = [&](int item, int& b, int& g, int& chunk) -> int {
+    chunk = item % a.n_cmp_chunks;
+    const int bg = item / a.n_cmp_chunks;
+    g = bg % a.H_kv;
+    b = bg / a.H_kv;
+    const int L = a.lens[b];
+    if (L < 1 || L > a.max_len) {
+      if (chunk == 0 && g == 0 && tid == 0) atomicOr(a.status, DEV_ERR_BOUNDS);
+      return 0;
+    }
+    const int nc = n_cmp_dev(L, a.l, a.s);
+    const int c0 = chunk * kCmpChunk;
+    return c0 < nc ? min(kTilesPerChunk, (nc - c0 + 63) / 64) : 0;
+  };
+
   if (warp == kDecConsumers) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int row0 = b * a.Lmax_cmp + c0;
-      for (int i = 0; i < ntl; ++i) {
-        const int st = i % kDecStages;
-        if (i >= kDecStages && !mbar_wait(&empty[st], ((i / kDecStages) - 1) & 1, abort_flag, a.status, 401)) break;
-        uint8_t* Ks = ring + st * S::STAGE;
-        mbar_arrive_expect_tx(&full[st], S::STAGE);
-        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.kc, &full[st], kb * 64, g, row0 + i * 64);
-        for (int vb = 0; vb < DV / 64; ++vb)
-          tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.vc, &full[st], vb * 64, g, row0 + i * 64);
+      int u = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        int b, g, chunk;
+        const int ntl = item_tiles(item, b, g, chunk);
+        if (ntl == 0) continue;
+        const int qi = it & 1;
+        if (it >= 2 && !mbar_wait(&q_empty[qi], ((it >> 1) - 1) & 1, abort_flag, a.status, 403)) break;
+        mbar_arrive_expect_tx(&q_full[qi], (uint32_t)(DK / 64) * G * 128);
+        for (int kb = 0; kb < DK / 64; ++kb)
+          tma_load_3d(qbuf + qi * S::QBUF + kb * 2048, &mp.q, &q_full[qi], kb * 64, g * G, b);
+        const int row0 = b * a.Lmax_cmp + chunk * kCmpChunk;
+        for (int i = 0; i < ntl; ++i, ++u) {
+          const int st = u % kDecStages;
+          if (u >= kDecStages && !mbar_wait(&empty[st], ((u / kDecStages) - 1) & 1, abort_flag, a.status, 401)) {
+            ok = false;
+            break;
+          }
+          uint8_t* Ks = ring + st * S::STAGE;
+          mbar_arrive_expect_tx(&full[st], S::STAGE);
+          for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.kc, &full[st], kb * 64, g, row0 + i * 64);
+          for (int vb = 0; vb < DV / 64; ++vb)
+            tma_load_3d(Ks + DK * 128 + vb * 8192, &mp.vc, &full[st], vb * 64, g, row0 + i * 64);
+        }
+        ++it;
       }
     }
   } else {
-    uint32_t qa[DK / 16][4];
-    RowState<DV> rs;
-    rs.init();
-    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
-    load_q_frags<DK>(qa, qp, G, lane);
+    // ------------------------------------------------------------ consumers
     float* ps = pscr + warp * 16 * 64;
-    for (int i = warp; i < ntl; i += kDecConsumers) {
-      const int st = i % kDecStages;
-      if (!mbar_wait(&full[st], (i / kDecStages) & 1, abort_flag, a.status, 402)) break;
-      const uint32_t kb = smem_u32(ring + st * S::STAGE);
-      float s[8][4];
-      warp_qk<DK>(qa, kb, s, lane);
-      const int kc0 = c0 + i * 64 + (lane & 3) * 2;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool vis = kc0 + nt * 8 + e < nc;
-          s[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
-          s[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
+    int u_base = 0, it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      int b, g, chunk;
+      const int ntl = item_tiles(item, b, g, chunk);
+      if (ntl == 0) continue;
+      const int qi = it & 1;
+      const int nc = n_cmp_dev(a.lens[b], a.l, a.s);
+      const int c0 = chunk * kCmpChunk;
+      // every warp reaches the three item-end barriers even when a wait gave up
+      ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qi], (it >> 1) & 1, abort_flag, a.status, 404));
+      const uint32_t qbase = smem_u32(qbuf + qi * S::QBUF);
+      RowState<DV> rs;
+      rs.init();
+      for (int i = warp; i < ntl && ok; i += kDecConsumers) {
+        const int u = u_base + i;
+        const int st = u % kDecStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kDecStages) & 1, abort_flag, a.status, 402))) {
+          ok = false;
+          break;
         }
-      }
-      rs.update(s);   // s now holds exp2(x - m) for the running max m
-      // stage probabilities for the block sums of this tile
-      {
-        const int r0 = lane >> 2, cq = (lane & 3) * 2;
+        const uint32_t kb = smem_u32(ring + st * S::STAGE);
+        float s[8][4];
+        warp_qk_sq<DK>(qbase, 2048, 0, kb, s, lane);
+        const int kc0 = c0 + i * 64 + (lane & 3) * 2;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
-          ps[r0 * 64 + nt * 8 + cq] = s[nt][0];
-          ps[r0 * 64 + nt * 8 + cq + 1] = s[nt][1];
-          ps[(r0 + 8) * 64 + nt * 8 + cq] = s[nt][2];
-          ps[(r0 + 8) * 64 + nt * 8 + cq + 1] = s[nt][3];
-        }
-      }
-      warp_pv<DV>(s, kb + S::K_BYTES, rs.o, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      // block sums: compressed key 4q+u covers tokens [16(4q+u), +32): u<3 -> 2p
-      // into block q of the tile, u = 3 -> p into q and q+1 (17 relative blocks).
-      // Tile partial layout [18][G]: row 0 = reference max per head, rows 1..17 =
-      // block sums per head.
-      {
-        const int tile = (c0 / 64) + i;
-        float* tpb = a.part + pl.tp + (((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * kTP * G;
-        const int row = lane >> 1, half = lane & 1;
-        if (row < G) {
-          const float* pr = ps + row * 64;
-          const int q0 = half * 8;
-          for (int q = q0; q < q0 + 8; ++q) {
-            float v = 2.f * (pr[4 * q] + pr[4 * q + 1] + pr[4 * q + 2]) + pr[4 * q + 3];
-            if (q > 0) v += pr[4 * q - 1];
-            tpb[(1 + q) * G + row] = v;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool vis = kc0 + nt * 8 + e < nc;
+            s[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
+            s[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
           }
-          if (half == 1) tpb[17 * G + row] = pr[63];
         }
-        if ((lane & 3) == 0) {
-          const int r0 = lane >> 2;
-          if (r0 < G) tpb[r0] = rs.m[0];
-          if (r0 + 8 < G) tpb[r0 + 8] = rs.m[1];
+        rs.update(s);   // s now holds exp2(x - m) for the running max m
+        {
+          const int r0 = lane >> 2, cq = (lane & 3) * 2;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt) {
+            ps[r0 * 64 + nt * 8 + cq] = s[nt][0];
+            ps[r0 * 64 + nt * 8 + cq + 1] = s[nt][1];
+            ps[(r0 + 8) * 64 + nt * 8 + cq] = s[nt][2];
+            ps[(r0 + 8) * 64 + nt * 8 + cq + 1] = s[nt][3];
+          }
         }
+        warp_pv<DV>(s, kb + DK * 128, rs.o, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+        // block sums: compressed key 4q+u covers tokens [16(4q+u), +32): u<3 -> 2p
+        // into block q of the tile, u = 3 -> p into q and q+1 (17 relative blocks).
+        // Tile partial layout [18][G]: row 0 = reference max per head, rows 1..17 =
+        // block sums per head.
+        {
+          const int tile = c0 / 64 + i;
+          float* tpb = a.part + pl.tp + (((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * kTP * G;
+          const int row = lane >> 1, half = lane & 1;
+          if (row < G) {
+            const float* pr = ps + row * 64;
+            const int q0 = half * 8;
+            for (int q = q0; q < q0 + 8; ++q) {
+              float v = 2.f * (pr[4 * q] + pr[4 * q + 1] + pr[4 * q + 2]) + pr[4 * q + 3];
+              if (q > 0) v += pr[4 * q - 1];
+              tpb[(1 + q) * G + row] = v;
+            }
+            if (half == 1) tpb[17 * G + row] = pr[63];
+          }
+          if ((lane & 3) == 0) {
+            const int r0 = lane >> 2;
+            if (r0 < G) tpb[r0] = rs.m[0];
+            if (r0 + 8 < G) tpb[r0 + 8] = rs.m[1];
+          }
+        }
+        __syncwarp();
+      }
+      rs.finish();
+      named_bar_sync(1, kDecConsumers * 32);
+      if (tid == 0) *item_abort = *abort_flag;
+      rs.stage(stg + warp * 16 * (DV + 2), lane);
+      named_bar_sync(1, kDecConsumers * 32);
+      const bool aborted = *item_abort != 0;   // written before the barrier: same in every warp
+      if (!aborted) {
+        const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
+        merge_warps<DV>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
       }
       __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qi]);
+      named_bar_sync(1, kDecConsumers * 32);   // merge done before the staging area is rewritten
+      if (aborted) break;
+      u_base += ntl;
+      ++it;
     }
-    rs.finish();
-    named_bar_sync(1, kDecConsumers * 32);
-    float* stg = reinterpret_cast<float*>(ring);
-    rs.stage(stg + warp * 16 * (DV + 2), lane);
-    named_bar_sync(1, kDecConsumers * 32);
-    const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
-    merge_warps<DV>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
   }
   __syncthreads();
 }
@@ -307,7 +372,12 @@ __global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeA
 }
 
 // ---------------------------------------------------------------------------
-// D3: selected blocks and window, split over the union of their blocks
+// D3: selected blocks and window for one (sequence, KV head) per CTA. The
+// ascending union of the selected blocks and the blocks the window touches is
+// streamed once through the TMA ring; consumer warp w takes union positions
+// w, w+4, ...; one score tile serves both branches, each with its own online
+// softmax. At the end the four warps' states are merged in shared memory and
+// out = g_cmp o_cmp + g_slc o_slc + g_win o_win is written.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeArgs a,
@@ -318,52 +388,87 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BODY + S::PSCR);
   uint64_t* empty = full + kDecStages;
-  int* sel_s = reinterpret_cast<int*>(empty + kDecStages);   // [32]
-  int* uni = sel_s + 32;                                       // [64]
+  int* uni = reinterpret_cast<int*>(empty + kDecStages);      // [64]
   int* nuni = uni + 64;
   volatile int* abort_flag = nuni + 1;
+  uint32_t* flags = reinterpret_cast<uint32_t*>(nuni + 2);     // [64] 1 = selected block
+  uint8_t* qs = smem + S::BODY;                                 // Q: DK/64 chunks of [16 rows][128 B]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cc = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.x, b = blockIdx.y;
   const int L = a.lens[b];
   if (L < 1 || L > a.max_len) return;
   const int t = L - 1, jt = t / a.ls;
   const int wlo = max(0, t - a.window + 1);
   const int G = a.G;
-  const PartLayout pl = part_layout(a);
   const size_t bg = (size_t)b * a.H_kv + g;
-  float* fpo = a.part + pl.fp_o + (bg * a.n_sw_chunks + cc) * 2 * G * DV;
-  float* fpm = a.part + pl.fp_ml + (bg * a.n_sw_chunks + cc) * 2 * G * 2;
 
-  if (tid < 32) sel_s[tid] = tid < a.top_n ? a.sel[((size_t)b * a.H_kv + g) * a.top_n + tid] : -1;
-  __syncthreads();
   if (tid == 0) {
-    // ascending union of the selected blocks and the blocks the window touches
-    int ns = 0;
-    while (ns < a.top_n && sel_s[ns] >= 0) ++ns;
-    int i = 0, w = wlo / a.ls, n = 0;
-    while (i < ns || w <= jt) {
-      int v;
-      if (w > jt || (i < ns && sel_s[i] < w)) v = sel_s[i++];
-      else if (i < ns && sel_s[i] == w) { v = w; ++i; ++w; }
-      else v = w++;
-      if (n < 64) uni[n++] = v;
-    }
-    *nuni = n;
     for (int k = 0; k < kDecStages; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
     *abort_flag = 0;
     fence_mbar_init();
   }
+  {
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
+    for (int idx = tid; idx < 16 * (DK / 8); idx += kDecThreads) {   // 16-byte chunks
+      const int row = idx / (DK / 8), c = idx % (DK / 8);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < G) v = *reinterpret_cast<const uint4*>(qp + (size_t)row * DK + c * 8);
+      *reinterpret_cast<uint4*>(qs + (c >> 3) * 2048 + sw128(row, c & 7)) = v;
+    }
+  }
+  if (warp == 0) {
+    // union of the selected blocks (ascending, -1 padded) and the window blocks
+    // [wlo / l', jt], merged with a ballot over the candidate range
+    const int32_t* sel = a.sel + bg * a.top_n;
+    const int wb = wlo / a.ls;
+    int cnt = 0, si = 0;
+    int ns = 0;
+    for (int i = lane; i < a.top_n; i += 32) ns += sel[i] >= 0;
+    ns = __reduce_add_sync(0xffffffffu, ns);
+    // walk block indices in chunks of 32: a block is in the union if it is
+    // selected or inside the window range
+    int next_sel = ns > 0 ? sel[0] : 0x7fffffff;
+    for (int j0 = 0; j0 <= jt; j0 += 32) {
+      // skip chunks with neither a selected block nor window blocks
+      if (j0 + 31 < wb && next_sel > j0 + 31) {
+        // jump to the chunk of whichever comes first: the next selected block or the window
+        const int target = next_sel < wb ? next_sel : wb;
+        j0 = (target / 32) * 32 - 32;
+        continue;
+      }
+      const int j = j0 + lane;
+      bool is_sel = false;
+      for (int i = si; i < ns; ++i) {
+        const int v = sel[i];
+        if (v > j0 + 31) break;
+        is_sel |= (v == j);
+      }
+      const bool in = j <= jt && (is_sel || j >= wb);
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (pos < 64) {
+          uni[pos] = j;
+          flags[pos] = is_sel ? 1u : 0u;
+        }
+      }
+      cnt += __popc(bal);
+      while (si < ns && sel[si] <= j0 + 31) ++si;
+      next_sel = si < ns ? sel[si] : 0x7fffffff;
+    }
+    if (lane == 0) *nuni = cnt < 64 ? cnt : 64;
+  }
   __syncthreads();
-  const int first = cc * kFineBlocks;
-  const int nblk = max(0, min(kFineBlocks, *nuni - first));
+  const int nu = *nuni;
 
   if (warp == kDecConsumers) {
     if (lane == 0) {
-      for (int i = 0; i < nblk; ++i) {
-        const int st = i % kDecStages;
+      for (int u = 0; u < nu; ++u) {
+        const int st = u % kDecStages;
+        if (u >= kDecStages && !mbar_wait(&empty[st], ((u / kDecStages) - 1) & 1, abort_flag, a.status, 411)) break;
         uint8_t* Ks = ring + st * S::STAGE;
-        const int row = b * a.Lmax + uni[first + i] * a.ls;
+        const int row = b * a.Lmax + uni[u] * a.ls;
         mbar_arrive_expect_tx(&full[st], S::STAGE);
         for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
         for (int vb = 0; vb < DV / 64; ++vb)
@@ -374,32 +479,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     RowState<DV> rs_sel, rs_win;
     rs_sel.init();
     rs_win.init();
-    if (warp < nblk) {
-      uint32_t qa[DK / 16][4];
-      const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
-      load_q_frags<DK>(qa, qp, G, lane);
-      const int st = warp;
-      if (mbar_wait(&full[st], 0, abort_flag, a.status, 411)) {
-        const uint32_t kb = smem_u32(ring + st * S::STAGE);
-        const int blk = uni[first + warp];
-        bool in_sel = false;
-        for (int k = 0; k < a.top_n; ++k) in_sel |= (sel_s[k] == blk);
-        float s[8][4];
-        warp_qk<DK>(qa, kb, s, lane);
-        const int key0 = blk * a.ls + (lane & 3) * 2;
-        float x[8][4];
+    const uint32_t qbase = smem_u32(qs);
+    for (int u = warp; u < nu; u += kDecConsumers) {
+      const int st = u % kDecStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kDecStages) & 1, abort_flag, a.status, 412))) break;
+      const uint32_t kb = smem_u32(ring + st * S::STAGE);
+      const int blk = uni[u];
+      const bool in_sel = flags[u] != 0u;
+      float s[8][4];
+      warp_qk_sq<DK>(qbase, 16 * 128, 0, kb, s, lane);
+      const int key0 = blk * a.ls + (lane & 3) * 2;
+      float x[8][4];
+      if (in_sel) {
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int tau = key0 + nt * 8 + e;
-            const bool vis = in_sel && tau <= t;
+            const bool vis = key0 + nt * 8 + e <= t;
             x[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
             x[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
           }
         }
         rs_sel.update(x);
         warp_pv<DV>(x, kb + S::K_BYTES, rs_sel.o, lane);
+      }
+      if (blk * a.ls + a.ls - 1 >= wlo) {
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
@@ -413,83 +517,70 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
         rs_win.update(x);
         warp_pv<DV>(x, kb + S::K_BYTES, rs_win.o, lane);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
     }
     rs_sel.finish();
     rs_win.finish();
-    named_bar_sync(1, kDecConsumers * 32);
+    named_bar_sync(1, kDecConsumers * 32);   // every block consumed: the ring is free
     float* stg = reinterpret_cast<float*>(ring);
     rs_sel.stage(stg + warp * 16 * (DV + 2), lane);
     rs_win.stage(stg + (kDecConsumers + warp) * 16 * (DV + 2), lane);
     named_bar_sync(1, kDecConsumers * 32);
-    merge_warps<DV>(stg, G, fpo, fpm, tid);
-    merge_warps<DV>(stg + kDecConsumers * 16 * (DV + 2), G, fpo + G * DV, fpm + G * 2, tid);
-  }
-  // the last CTA of this (b, g) to get here combines the three branches
-  __shared__ int last;
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const int done = atomicAdd(reinterpret_cast<int*>(a.part + pl.cnt) + bg, 1);
-    last = done == a.n_sw_chunks - 1;
-  }
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  float* fac = reinterpret_cast<float*>(ring);       // [2][nsw][16] factors, then [2][16] 1/den
-  const float* po = a.part + pl.fp_o + bg * a.n_sw_chunks * 2 * G * DV;
-  const volatile float* pm = a.part + pl.fp_ml + bg * a.n_sw_chunks * 2 * G * 2;
-  float* inv = fac + 2 * a.n_sw_chunks * 16;
-  if (tid < 2 * G) {
-    const int br = tid / G, h = tid % G;
-    float M = -1e30f;
-    for (int c = 0; c < a.n_sw_chunks; ++c) {
-      const size_t r = (((size_t)c * 2 + br) * G + h) * 2;
-      if (pm[r + 1] > 0.f) M = fmaxf(M, pm[r]);
-    }
-    float den = 0.f;
-    for (int c = 0; c < a.n_sw_chunks; ++c) {
-      const size_t r = (((size_t)c * 2 + br) * G + h) * 2;
-      const float f = pm[r + 1] > 0.f ? exp2f(pm[r] - M) : 0.f;
-      fac[(br * a.n_sw_chunks + c) * 16 + h] = f;
-      den += f * pm[r + 1];
-    }
-    const float gate = a.gates[((size_t)b * a.H_q + g * G + h) * 3 + 1 + br];
-    inv[br * 16 + h] = den > 0.f ? gate / den : 0.f;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * (DV / 4); idx += kDecThreads) {
-    const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
-    const int hq = g * G + h;
-    float4 res = *reinterpret_cast<const float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4);
-    for (int br = 0; br < 2; ++br) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c = 0; c < a.n_sw_chunks; ++c) {
-        const float f = fac[(br * a.n_sw_chunks + c) * 16 + h];
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(po + (((size_t)c * 2 + br) * G + h) * DV + c4));
-        acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
+    // merge the four warps of each branch and combine: thread per (row, 4 columns)
+    for (int idx = tid; idx < G * (DV / 4); idx += kDecConsumers * 32) {
+      const int row = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
+      const int hq = g * G + row;
+      float4 res = *reinterpret_cast<const float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4);
+#pragma unroll
+      for (int br = 0; br < 2; ++br) {
+        const float* base = stg + (size_t)br * kDecConsumers * 16 * (DV + 2);
+        float M = -1e30f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) {
+          const float* r = base + (w * 16 + row) * (DV + 2);
+          if (r[DV + 1] > 0.f) M = fmaxf(M, r[DV]);
+        }
+        float den = 0.f;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kDecConsumers; ++w) {
+          const float* r = base + (w * 16 + row) * (DV + 2);
+          if (r[DV + 1] > 0.f) {
+            const float f = ex2(r[DV] - M);
+            den += f * r[DV + 1];
+            num.x += f * r[c4]; num.y += f * r[c4 + 1]; num.z += f * r[c4 + 2]; num.w += f * r[c4 + 3];
+          }
+        }
+        const float gate = a.gates[((size_t)b * a.H_q + hq) * 3 + 1 + br];
+        const float sc = den > 0.f ? gate / den : 0.f;
+        res.x += sc * num.x; res.y += sc * num.y; res.z += sc * num.z; res.w += sc * num.w;
       }
-      const float s_ = inv[br * 16 + h];
-      res.x += s_ * acc.x; res.y += s_ * acc.y; res.z += s_ * acc.z; res.w += s_ * acc.w;
+      uint2 pk;
+      pk.x = pack_bf16x2(res.x, res.y);
+      pk.y = pack_bf16x2(res.z, res.w);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)b * a.H_q + hq) * DV + c4) = pk;
     }
-    uint2 pk;
-    pk.x = pack_bf16x2(res.x, res.y);
-    pk.y = pack_bf16x2(res.z, res.w);
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + ((size_t)b * a.H_q + hq) * DV + c4) = pk;
   }
+  __syncthreads();
 }
 
-// ---------------------------------------------------------------------------
 template <int DK, int DV>
 static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st) {
   using S = DecSmem<DK, DV>;
   cudaError_t e;
   auto k1 = dec_cmp_kernel<DK, DV>;
   auto k3 = dec_fine_kernel<DK, DV>;
-  if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL)) != cudaSuccess) return e;
+  using S1 = D1Smem<DK, DV>;
+  if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, S1::TOTAL)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL)) != cudaSuccess) return e;
   if (a.Lmax_cmp > 0) {
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int n_items = a.B * a.H_kv * a.n_cmp_chunks;
     prof_begin(P_DEC_CMP, st);
-    k1<<<dim3(a.n_cmp_chunks, a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
+    k1<<<n_items < n_sm ? n_items : n_sm, kDecThreads, S1::TOTAL, st>>>(a, m);
     prof_end(P_DEC_CMP, st, 1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -518,7 +609,7 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
   prof_end(P_DEC_SELECT, st, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prof_begin(P_DEC_FINE, st);
-  k3<<<dim3(a.n_sw_chunks, a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
+  k3<<<dim3(a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
   prof_end(P_DEC_FINE, st, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return cudaGetLastError();

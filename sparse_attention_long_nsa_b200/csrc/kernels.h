@@ -37,6 +37,10 @@ struct CompressArgs {
   const float* bias;      // fp32 [d_out] = vec(pe) . W
   void* out;              // bf16 [*, H_kv, d_out]
   int H_kv, l, s;
+  int ksplit;             // split of the K = l*d_in reduction over grid.z (1: no split)
+  int kb_per_split;       // 64-wide K blocks per split
+  float* part;            // fp32 [ksplit][rows_total][H_kv][d_out] partial sums (ksplit > 1)
+  int64_t rows_total;     // output rows (packed: sum of n_cmp)
   uint32_t* status;
   SeqTable seqs;
 };
@@ -44,6 +48,7 @@ cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, 
                                  float* partial, float* bias, cudaStream_t st);
 cudaError_t launch_compress_gemm(int d_in, int d_out, const CompressArgs& a, int n_tiles,
                                  cudaStream_t st);
+cudaError_t launch_compress_finalize(int d_out, const CompressArgs& a, cudaStream_t st);
 
 // ----- prefill -----
 struct PrefillArgs {
@@ -66,6 +71,7 @@ struct PrefillArgs {
 };
 struct PrefillMaps {
   CUtensorMap q, k, v, kc, vc;
+  CUtensorMap q8;   // q with a box of 8 tokens x G heads (selected-block attention)
 };
 cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st);
@@ -97,6 +103,7 @@ struct DecodeArgs {
 };
 struct DecodeMaps {
   CUtensorMap k, v, kc, vc;
+  CUtensorMap q;   // q [B, H_q, d_k] with a box of one sequence's G heads
 };
 size_t decode_partials_floats(const DecodeArgs& a);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);

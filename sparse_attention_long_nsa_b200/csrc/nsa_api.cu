@@ -65,10 +65,13 @@ float softmax_scale(const nsa_params_t* p, int d_k) {
 int n_blk_of(int L, int ls) { return (L + ls - 1) / ls; }
 
 // ---- workspace layouts ----
+constexpr int kMaxKSplit = 16;
 struct CompressWs {
-  size_t wt_k, wt_v, part_k, part_v, bias_k, bias_v, total;
+  size_t wt_k, wt_v, part_k, part_v, bias_k, bias_v, ksum, total;
 };
-CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p) {
+// `rows` bounds the packed compressed rows; it sizes the split-K partial sums
+// (none when 0). Everything before `ksum` is the fixed minimum.
+CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t rows) {
   CompressWs w{};
   size_t off = 256;
   const size_t Kk = (size_t)p->l_cmp * h->d_k, Kv = (size_t)p->l_cmp * h->d_v;
@@ -78,6 +81,9 @@ CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p) {
   w.part_v = off; off = align256(off + ((Kv + 31) / 32) * h->d_v * 4);
   w.bias_k = off; off = align256(off + (size_t)h->d_k * 4);
   w.bias_v = off; off = align256(off + (size_t)h->d_v * 4);
+  w.ksum = off;
+  const size_t dmax = (size_t)(h->d_k > h->d_v ? h->d_k : h->d_v);
+  if (rows > 0) off = align256(off + (size_t)kMaxKSplit * (size_t)rows * h->H_kv * dmax * 4);
   w.total = off;
   return w;
 }
@@ -265,9 +271,12 @@ size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* 
   if (check_heads(heads) != NSA_OK) return 0;
   if (batch <= 0 || batch > NSA_MAX_BATCH) return 0;
   switch (op) {
-    case NSA_OP_COMPRESS:
-      if (check_params(params, false) != NSA_OK) return 0;
-      return compress_ws(heads, params).total;
+    case NSA_OP_COMPRESS: {
+      if (check_params(params, false) != NSA_OK || total_tokens < 0) return 0;
+      // packed rows are at most total_tokens / stride (+1 per sequence)
+      const int64_t rows = total_tokens > 0 ? total_tokens / params->stride + batch : 0;
+      return compress_ws(heads, params, rows).total;
+    }
     case NSA_OP_PREFILL:
       if (check_params(params, true) != NSA_OK || total_tokens < 0 || max_len < 0) return 0;
       return prefill_ws(heads, params, total_tokens, max_len).total;
@@ -320,19 +329,22 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
     return NSA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(workspace))
     return NSA_ERR_INVALID_ARG;
-  const CompressWs w = compress_ws(heads, params);
+  const CompressWs w = compress_ws(heads, params, 0);
   if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
 
   SeqTable t{};
   t.n = batch;
   int tiles = 0;
+  int64_t rows_total = 0;   // packed output rows; -1 when the rows are not packed
   for (int b = 0; b < batch; ++b) {
     if (seq_len[b] < 0 || tok_offset[b] < 0 || cmp_offset[b] < 0) return NSA_ERR_INVALID_ARG;
     t.tile_prefix[b] = tiles;
     t.tok_off[b] = tok_offset[b];
     t.cmp_off[b] = cmp_offset[b];
     t.len[b] = seq_len[b];
-    tiles += (n_cmp_of(seq_len[b], params->l_cmp, params->stride) + 127) / 128;
+    const int nc = n_cmp_of(seq_len[b], params->l_cmp, params->stride);
+    tiles += (nc + 127) / 128;
+    if (rows_total >= 0) rows_total = (cmp_offset[b] == rows_total) ? rows_total + nc : -1;
   }
   t.tile_prefix[batch] = tiles;
 
@@ -353,14 +365,36 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
   a.H_kv = heads->H_kv; a.l = params->l_cmp; a.s = params->stride;
   a.status = reinterpret_cast<uint32_t*>(ws);
   a.seqs = t;
-  prof_begin(P_COMPRESS_GEMM, st);
-  a.x = k; a.wt = ws + w.wt_k; a.bias = (const float*)(ws + w.bias_k); a.out = k_cmp;
-  e = launch_compress_gemm(heads->d_k, heads->d_k, a, tiles, st);
-  if (e == cudaSuccess) {
-    a.x = v; a.wt = ws + w.wt_v; a.bias = (const float*)(ws + w.bias_v); a.out = v_cmp;
-    e = launch_compress_gemm(heads->d_v, heads->d_v, a, tiles, st);
+  a.part = (float*)(ws + w.ksum);
+  a.rows_total = rows_total > 0 ? rows_total : 0;
+  // split K when the row tiles alone leave SMs idle, the rows are packed and the
+  // workspace has room for the partial sums
+  int ks = 1;
+  if (rows_total > 0) {
+    const int ctas = tiles * heads->H_kv;
+    ks = (2 * 148 + ctas - 1) / ctas;
+    if (ks > kMaxKSplit) ks = kMaxKSplit;
+    const size_t dmax = (size_t)(heads->d_k > heads->d_v ? heads->d_k : heads->d_v);
+    while (ks > 1 && w.ksum + (size_t)ks * rows_total * heads->H_kv * dmax * 4 > ws_bytes) ks >>= 1;
   }
-  prof_end(P_COMPRESS_GEMM, st, 2);
+  int launches = 0;
+  auto run = [&](const void* x, const void* wt, const float* bias, void* out, int d) -> cudaError_t {
+    a.x = x; a.wt = wt; a.bias = bias; a.out = out;
+    const int nkb = params->l_cmp * d / 64;
+    a.kb_per_split = (nkb + ks - 1) / ks;
+    a.ksplit = (nkb + a.kb_per_split - 1) / a.kb_per_split;
+    cudaError_t err = launch_compress_gemm(d, d, a, tiles, st);
+    ++launches;
+    if (err == cudaSuccess && a.ksplit > 1) {
+      err = launch_compress_finalize(d, a, st);
+      ++launches;
+    }
+    return err;
+  };
+  prof_begin(P_COMPRESS_GEMM, st);
+  e = run(k, ws + w.wt_k, (const float*)(ws + w.bias_k), k_cmp, heads->d_k);
+  if (e == cudaSuccess) e = run(v, ws + w.wt_v, (const float*)(ws + w.bias_v), v_cmp, heads->d_v);
+  prof_end(P_COMPRESS_GEMM, st, launches);
   if (e != cudaSuccess) return cuda_fail(e, "compress gemm");
   return NSA_OK;
 }
@@ -432,7 +466,8 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
       !make_map_3d(&m.k, k, heads->d_k, heads->H_kv, N, 1, 64) ||
       !make_map_3d(&m.v, v, heads->d_v, heads->H_kv, N, 1, 64) ||
       !make_map_3d(&m.kc, kc_base, heads->d_k, heads->H_kv, ncmp_total, 1, 64) ||
-      !make_map_3d(&m.vc, vc_base, heads->d_v, heads->H_kv, ncmp_total, 1, 64)) {
+      !make_map_3d(&m.vc, vc_base, heads->d_v, heads->H_kv, ncmp_total, 1, 64) ||
+      !make_map_3d(&m.q8, q, heads->d_k, heads->H_q, N, a.G, 8)) {
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
     return NSA_ERR_CUDA;
   }
@@ -492,7 +527,8 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
   if (!make_map_3d(&m.k, k_cache, heads->d_k, heads->H_kv, rows, 1, 64) ||
       !make_map_3d(&m.v, v_cache, heads->d_v, heads->H_kv, rows, 1, 64) ||
       !make_map_3d(&m.kc, crows > 0 ? k_cmp_cache : k_cache, heads->d_k, heads->H_kv, crows > 0 ? crows : rows, 1, 64) ||
-      !make_map_3d(&m.vc, crows > 0 ? v_cmp_cache : v_cache, heads->d_v, heads->H_kv, crows > 0 ? crows : rows, 1, 64)) {
+      !make_map_3d(&m.vc, crows > 0 ? v_cmp_cache : v_cache, heads->d_v, heads->H_kv, crows > 0 ? crows : rows, 1, 64) ||
+      !make_map_3d(&m.q, q, heads->d_k, heads->H_q, batch, heads->H_q / heads->H_kv, 1)) {
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
     return NSA_ERR_CUDA;
   }

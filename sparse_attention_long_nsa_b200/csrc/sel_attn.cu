@@ -83,20 +83,20 @@ cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st)
 // selected-block attention
 //
 // CTA = 8 consecutive tokens of one sequence x one KV head; consumer warp w owns
-// token t0 + w (its G heads are the 16 MMA rows). The blocks the 8 tokens
-// selected are merged into one ascending union; each union block is loaded once
-// by TMA into a 4-stage ring and used by every warp whose token selected it
-// (the forced blocks 0, jt-1, jt are shared by all 8). Every warp walks the
-// whole union in order (waiting for each stage, computing only on its own
-// blocks) so the stage barriers stay in phase; once all 8 warps released a
-// stage, lane 0 of warp 0 refills it with the block 4 positions ahead (8 warps,
-// two per SM sub-partition, keep the full register budget). Each warp adds
+// token t0 + w (its G heads are the 16 MMA rows; Q for the 8 tokens is staged in
+// shared memory by one TMA box). The blocks the 8 tokens selected are merged into
+// one ascending union; a producer warp streams each union block once through a
+// 4-stage TMA ring, and every warp whose token selected it computes on it (the
+// forced blocks 0, jt-1, jt are shared by all 8). Warps wait only for their own
+// blocks: the producer publishes which union position a stage holds, and a
+// stage is refilled once the warps that needed its block released it (the
+// producer itself stands in for the warps that did not need it). Each warp adds
 // g_slc * o_slc of its own token to the fp32 accumulator from its fragments.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int kSelStages = 4;
 constexpr int kSelTok = 8;                        // tokens (consumer warps) per CTA
-constexpr int kSelThreads = kSelTok * 32;       // warp 0 lane 0 also refills the ring
+constexpr int kSelThreads = (kSelTok + 1) * 32;   // + producer warp
 constexpr int kSelMaxUnion = kSelTok * 32;        // top_n <= 32
 
 template <int DK, int DV>
@@ -105,8 +105,10 @@ struct SelSmem {
   static constexpr int V_BYTES = 64 * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int RING = kSelStages * STAGE;
-  // ring | barriers (2 * stages) | union list | union masks | flags | bitmap [nb_stride]
-  static constexpr int FIXED = 1024 + RING + 2 * kSelStages * 8 + kSelMaxUnion * 8 + 64;
+  static constexpr int Q_MAX = kSelTok * 16 * DK * 2;   // 8 tokens x G <= 16 heads
+  // Q | ring | barriers | stage tags | union list | union masks | flags | bitmap [nb_stride]
+  static constexpr int FIXED = 1024 + Q_MAX + RING + (2 * kSelStages + 1) * 8 + kSelStages * 4 +
+                               kSelMaxUnion * 8 + 64;
   static int total(int nb_stride) { return FIXED + nb_stride * 4; }
 };
 }  // namespace
@@ -117,10 +119,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
   using S = SelSmem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING);
+  uint8_t* qs = smem;                                            // [DK/64][8*G rows][128 B]
+  uint8_t* ring = smem + S::Q_MAX;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + S::RING);
   uint64_t* empty = full + kSelStages;
-  int* uni = reinterpret_cast<int*>(empty + kSelStages);        // [kSelMaxUnion]
+  uint64_t* q_full = empty + kSelStages;
+  volatile int* stage_tag = reinterpret_cast<volatile int*>(q_full + 1);   // union position held
+  int* uni = const_cast<int*>(stage_tag) + kSelStages;          // [kSelMaxUnion]
   uint32_t* umask = reinterpret_cast<uint32_t*>(uni + kSelMaxUnion);
   int* nuni = reinterpret_cast<int*>(umask + kSelMaxUnion);
   volatile int* abort_flag = nuni + 1;
@@ -138,10 +143,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
   if (t0 >= L) return;   // whole CTA past the end of its sequence (uniform)
   const int t_last = min(t0 + kSelTok - 1, L - 1);
   const int jt_max = t_last / a.ls;
+  const uint32_t qchunk = (uint32_t)kSelTok * G * 128;
 
   for (int j = tid; j <= jt_max; j += kSelThreads) bm[j] = 0u;
   if (tid == 0) {
-    for (int i = 0; i < kSelStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kSelTok); }
+    for (int i = 0; i < kSelStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kSelTok);
+      stage_tag[i] = -1;
+    }
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -155,8 +166,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
     if (j >= 0 && j <= jt_max) atomicOr(&bm[j], 1u << warp);
   }
   __syncthreads();
-  // compact the union in ascending block order (warp 0)
-  if (warp == 0) {
+  // compact the union in ascending block order (producer warp)
+  if (warp == kSelTok) {
     int cnt = 0;
     for (int j0 = 0; j0 <= jt_max; j0 += 32) {
       const int j = j0 + lane;
@@ -174,67 +185,64 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
   __syncthreads();
   const int nu = *nuni;
 
-  auto issue = [&](int u) {
-    const int st = u % kSelStages;
-    uint8_t* Ks = ring + st * S::STAGE;
-    const int row = (int)(tok0 + (int64_t)uni[u] * a.ls);
-    mbar_arrive_expect_tx(&full[st], S::STAGE);
-    for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
-    for (int vb = 0; vb < DV / 64; ++vb) tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
-  };
-  const bool producer = warp == 0 && lane == 0;
-  if (producer)
-    for (int u = 0; u < nu && u < kSelStages; ++u) issue(u);
-
-  uint32_t qa[DK / 16][4];
-  RowState<DV> rs;
-  rs.init();
-  if (has_tok) {
-    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)n * a.H_q + (size_t)g * G) * DK;
-    load_q_frags<DK>(qa, qp, G, lane);
-  }
-  const uint32_t bit = 1u << warp;
-  bool ok = true;
-  for (int u = 0; u < nu; ++u) {
-    const int st = u % kSelStages;
-    // warp-uniform outcome of the (bounded) wait
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kSelStages) & 1, abort_flag, a.status, 302))) {
-      ok = false;
-      break;
+  if (warp == kSelTok) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, (uint32_t)(DK / 64) * qchunk);
+      for (int kb = 0; kb < DK / 64; ++kb)
+        tma_load_3d(qs + kb * qchunk, &mp.q8, q_full, kb * 64, g * G, (int)(tok0 + t0));
+      for (int u = 0; u < nu; ++u) {
+        const int st = u % kSelStages;
+        if (u >= kSelStages && !mbar_wait(&empty[st], ((u / kSelStages) - 1) & 1, abort_flag, a.status, 301)) break;
+        stage_tag[st] = u;
+        uint8_t* Ks = ring + st * S::STAGE;
+        const int row = (int)(tok0 + (int64_t)uni[u] * a.ls);
+        mbar_arrive_expect_tx(&full[st], S::STAGE);
+        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
+        for (int vb = 0; vb < DV / 64; ++vb)
+          tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
+        const uint32_t others = kSelTok - __popc(umask[u]);   // warps that will not release it
+        if (others) mbar_arrive_cnt(&empty[st], others);
+      }
     }
-    if (umask[u] & bit) {
-      const uint32_t kb = smem_u32(ring + st * S::STAGE);
-      float s[8][4];
-      warp_qk<DK>(qa, kb, s, lane);
-      const int key0 = uni[u] * a.ls + (lane & 3) * 2;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool vis = key0 + nt * 8 + e <= t;
-          s[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
-          s[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
+  } else {
+    // ------------------------------------------------------------ consumers
+    RowState<DV> rs;
+    rs.init();
+    const uint32_t bit = 1u << warp;
+    bool ok = true;
+    if (has_tok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, a.status, 303));
+      const uint32_t qbase = smem_u32(qs);
+      for (int u = 0; u < nu && ok; ++u) {
+        if (!(umask[u] & bit)) continue;
+        const int st = u % kSelStages;
+        // the stage must hold union position u before its barrier phase is meaningful
+        bool w = smem_wait_eq(&stage_tag[st], u, abort_flag, a.status, 304) &&
+                 mbar_wait(&full[st], (u / kSelStages) & 1, abort_flag, a.status, 302);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
         }
+        const uint32_t kb = smem_u32(ring + st * S::STAGE);
+        float s[8][4];
+        warp_qk_sq<DK>(qbase, qchunk, warp * G, kb, s, lane);
+        const int key0 = uni[u] * a.ls + (lane & 3) * 2;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool vis = key0 + nt * 8 + e <= t;
+            s[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
+            s[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
+          }
+        }
+        rs.update(s);
+        warp_pv<DV>(s, kb + S::K_BYTES, rs.o, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
       }
-      rs.update(s);
-      warp_pv<DV>(s, kb + S::K_BYTES, rs.o, lane);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-    if (warp == 0 && u + kSelStages < nu) {
-      // once every warp is done with this stage, refill it
-      bool p_ok = true;
-      if (producer) {
-        p_ok = mbar_wait(&empty[st], (u / kSelStages) & 1, abort_flag, a.status, 301);
-        if (p_ok) issue(u + kSelStages);
-      }
-      if (!__shfl_sync(0xffffffffu, p_ok, 0)) {
-        ok = false;
-        break;
-      }
-    }
-  }
-  {
     rs.finish();
     if (has_tok && ok) {
       // acc[n, h, :] += g_slc * o / l for the group's heads (rows lane/4, lane/4 + 8)

@@ -50,6 +50,32 @@ __device__ __forceinline__ void warp_qk(const uint32_t (&qa)[DK / 16][4], uint32
   }
 }
 
+// Same as warp_qk with Q read from shared memory (TMA box [rows][64] per 64-wide
+// chunk, 128-byte swizzle, chunks `qchunk` bytes apart); rows qrow0 .. qrow0+15.
+template <int DK>
+__device__ __forceinline__ void warp_qk_sq(uint32_t qbase, uint32_t qchunk, int qrow0, uint32_t kbase,
+                                           float (&s)[8][4], int lane) {
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+  const int mi = lane >> 3, rr = lane & 7;
+  const uint32_t qrow = (uint32_t)(qrow0 + (lane & 15));
+#pragma unroll
+  for (int kk = 0; kk < DK / 16; ++kk) {
+    uint32_t qa[4];
+    ldmatrix_x4(qa, qbase + (kk >> 2) * qchunk + sw128(qrow, (kk & 3) * 2 + (lane >> 4)));
+    const uint32_t box = kbase + (kk >> 2) * 8192;
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      const int key = np * 16 + (mi >> 1) * 8 + rr;
+      const int chunk = (kk & 3) * 2 + (mi & 1);
+      uint32_t bfr[4];
+      ldmatrix_x4(bfr, box + sw128(key, chunk));
+      mma_bf16_16816(s[2 * np], qa, bfr);
+      mma_bf16_16816(s[2 * np + 1], qa, bfr + 2);
+    }
+  }
+}
+
 // o += P V for one tile, P given as fp32 probabilities in the score layout.
 template <int DV>
 __device__ __forceinline__ void warp_pv(const float (&p)[8][4], uint32_t vbase, float (&o)[DV / 8][4], int lane) {
@@ -105,16 +131,16 @@ struct RowState {
     mx0 = quad_max(mx0);
     mx1 = quad_max(mx1);
     const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-    const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);
+    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
     m[0] = mn0;
     m[1] = mn1;
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-      x[nt][0] = exp2f(x[nt][0] - mn0);
-      x[nt][1] = exp2f(x[nt][1] - mn0);
-      x[nt][2] = exp2f(x[nt][2] - mn1);
-      x[nt][3] = exp2f(x[nt][3] - mn1);
+      x[nt][0] = ex2(x[nt][0] - mn0);
+      x[nt][1] = ex2(x[nt][1] - mn0);
+      x[nt][2] = ex2(x[nt][2] - mn1);
+      x[nt][3] = ex2(x[nt][3] - mn1);
       s0 += x[nt][0] + x[nt][1];
       s1 += x[nt][2] + x[nt][3];
     }
