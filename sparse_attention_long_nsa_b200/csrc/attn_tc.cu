@@ -55,6 +55,7 @@ struct Bars {
   uint64_t s_free[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
+  uint64_t drain;       // MMA issuer: all its products finished (exit path)
   uint32_t tmem_base;
   int abort;
 };
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
       mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_done[i], 1);
     }
+    mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
         for (int kb = 0; kb < DK / 64; ++kb)
           tma_load_3d(Qs + qt * S::Q_BYTES + kb * 16384, &m.q, &bars->q_full, kb * 64, g * G,
                       (int)(tok0 + t0 + qt * TOK));
+      int issued = 0;
       for (int jj = 0; jj < n_s; ++jj) {
         const int st = jj % kStages;
         const int j = (MODE == 0 && jj >= nk) ? jj - nk : jj;
@@ -155,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
         if (jj >= kStages &&
             !mbar_wait(&bars->kv_empty[st], ((jj / kStages) - 1) & 1, abort_flag, a.status, 201))
           break;
+        issued = jj + 1;
         uint8_t* Ks = KVs + st * S::STAGE;
         mbar_arrive_expect_tx(&bars->kv_full[st], S::K_BYTES + (with_v ? S::V_BYTES : 0));
         const int row = (int)(krow0 + key0 + j * kKeyTile);
@@ -162,6 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
         if (with_v)
           for (int vb = 0; vb < DV / 64; ++vb)
             tma_load_3d(Ks + S::K_BYTES + vb * 8192, mv, &bars->kv_full[st], vb * 64, g, row);
+      }
+      if (*abort_flag) {   // let the copies still in flight land before the CTA exits
+        mbar_wait_drain(&bars->q_full, 0);
+        for (int v = issued - kStages < 0 ? 0 : issued - kStages; v < issued; ++v)
+          mbar_wait_drain(&bars->kv_full[v % kStages], (v / kStages) & 1);
       }
     }
   } else if (warp == 9) {
@@ -214,6 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const PrefillArgs 
         umma_commit(&bars->kv_empty[st]);   // every product reading stage st has been issued
         if (more && !qk(1, jj + 1)) break;
       }
+      // every issued product has finished before the CTA releases tensor memory
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups

@@ -101,6 +101,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Time-bounded wait that ignores the abort flag: used on the exit path to let
+// copies / MMAs this CTA issued land before it leaves (returns false if the
+// phase does not complete within NSA_WAIT_LIMIT_NS).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > NSA_WAIT_LIMIT_NS) return false;
+  return true;
+}
+
 // Bounded wait until a shared-memory word equals `want` (written by another warp
 // of the same CTA). Same failure handling as mbar_wait.
 __device__ __forceinline__ bool smem_wait_eq(const volatile int* word, int want, volatile int* abort_flag,

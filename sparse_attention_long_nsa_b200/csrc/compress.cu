@@ -181,10 +181,12 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
     }
   }
   cp_async_wait<0>();
-  // all MMAs done: commit a final barrier
-  if (tid == 0 && ok) umma_commit(&mma_done[kCmpStages]);
+  // all MMAs done: commit a final barrier (also on the abort path, so that no
+  // product is still running when tensor memory is released)
+  if (tid == 0) umma_commit(&mma_done[kCmpStages]);
   __syncthreads();
   if (ok && !*abort_flag) ok = mbar_wait(&mma_done[kCmpStages], 0, abort_flag, a.status, 102);
+  else if (tid == 0) mbar_wait_drain(&mma_done[kCmpStages], 0);
   tc_fence_after();
 
   if (ok) {

@@ -26,18 +26,26 @@ namespace nsa {
 
 namespace {
 
-constexpr int kDecStages = 4;
+// Key tiles of 32 keys (20 KB of K+V at d 192/128) in an 8-stage ring: each of
+// the 4 consumer warps computes on one stage while the next tiles are in flight.
+constexpr int kTileKeys = 32;
+constexpr int kNT = kTileKeys / 8;     // 8-key MMA n-tiles per tile
+constexpr int kDecStages = 8;
 constexpr int kDecConsumers = 4;
 constexpr int kDecThreads = (kDecConsumers + 1) * 32;
-constexpr int kCmpChunk = 512;         // compressed keys per D1 CTA
-constexpr int kTilesPerChunk = kCmpChunk / 64;
-constexpr int kFineBlocks = 4;         // 64-key blocks per D3 CTA
-constexpr int kTP = 18;                // tile partial: m_ref + 17 block sums
+// compressed-key pass: consumer warps + producer warp
+constexpr int kD1Stages = 8;
+constexpr int kD1Consumers = 4;
+constexpr int kD1Threads = (kD1Consumers + 1) * 32;
+constexpr int kCmpChunk = 512;         // compressed keys per D1 work item
+constexpr int kTilesPerChunk = kCmpChunk / kTileKeys;
+constexpr int kBlkPerTile = kTileKeys / 4;   // selection blocks a tile of compressed keys covers
+constexpr int kTP = kBlkPerTile + 2;   // tile partial: m_ref + block sums (+1 spilling into the next)
 
 template <int DK, int DV>
 struct DecSmem {
-  static constexpr int K_BYTES = 64 * DK * 2;
-  static constexpr int V_BYTES = 64 * DV * 2;
+  static constexpr int K_BYTES = kTileKeys * DK * 2;
+  static constexpr int V_BYTES = kTileKeys * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int RING = kDecStages * STAGE;
   static constexpr int MERGE = 2 * kDecConsumers * 16 * (DV + 2) * 4;
@@ -68,25 +76,25 @@ __host__ __device__ inline PartLayout part_layout(const DecodeArgs& a) {
   return p;
 }
 
-// merge 4 staged warp states ([w][16][DV+2]) into one state per row < G:
+// merge NW staged warp states ([w][16][DV+2]) into one state per row < G:
 // o relative to the merged max M -> dst_o[row][DV], (M, L) -> dst_ml[row][2]
-template <int DV>
+template <int DV, int NW = kDecConsumers>
 __device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_o, float* dst_ml, int tid) {
-  const int per_row = (kDecConsumers * 32) / 16;
+  const int per_row = (NW * 32) / 16;
   const int row = tid / per_row, part = tid % per_row;
   if (row >= G) return;
   float M = -1e30f;
-  for (int w = 0; w < kDecConsumers; ++w) M = fmaxf(M, stg[(w * 16 + row) * (DV + 2) + DV]);
-  float f[kDecConsumers], Ls = 0.f;
-  for (int w = 0; w < kDecConsumers; ++w) {
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, stg[(w * 16 + row) * (DV + 2) + DV]);
+  float f[NW], Ls = 0.f;
+  for (int w = 0; w < NW; ++w) {
     const float* r = stg + (w * 16 + row) * (DV + 2);
-    f[w] = r[DV + 1] > 0.f ? exp2f(r[DV] - M) : 0.f;
+    f[w] = r[DV + 1] > 0.f ? ex2(r[DV] - M) : 0.f;
     Ls += f[w] * r[DV + 1];
   }
   const int span = DV / per_row;
   for (int c = part * span; c < (part + 1) * span; ++c) {
     float v = 0.f;
-    for (int w = 0; w < kDecConsumers; ++w) v += f[w] * stg[(w * 16 + row) * (DV + 2) + c];
+    for (int w = 0; w < NW; ++w) v += f[w] * stg[(w * 16 + row) * (DV + 2) + c];
     dst_o[row * DV + c] = v;
   }
   if (part == 0) {
@@ -107,16 +115,16 @@ size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct D1Smem {
-  static constexpr int STAGE = 64 * (DK + DV) * 2;
-  static constexpr int RING = kDecStages * STAGE;
+  static constexpr int STAGE = kTileKeys * (DK + DV) * 2;
+  static constexpr int RING = kD1Stages * STAGE;
   static constexpr int QBUF = (DK / 64) * 16 * 128;                 // one item's Q, 16 rows
-  static constexpr int STG = kDecConsumers * 16 * (DV + 2) * 4;      // per-warp states for the merge
-  static constexpr int PSCR = kDecConsumers * 16 * 64 * 4;           // probabilities for block sums
+  static constexpr int STG = kD1Consumers * 16 * (DV + 2) * 4;       // per-warp states for the merge
+  static constexpr int PSCR = kD1Consumers * 16 * kTileKeys * 4;     // probabilities for block sums
   static constexpr int TOTAL = 1024 + RING + 2 * QBUF + STG + PSCR + 256;
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArgs a,
+__global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs a,
                                                                  const __grid_constant__ DecodeMaps mp) {
   using S = D1Smem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
@@ -126,11 +134,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
   float* stg = reinterpret_cast<float*>(qbuf + 2 * S::QBUF);
   float* pscr = stg + S::STG / 4;
   uint64_t* full = reinterpret_cast<uint64_t*>(pscr + S::PSCR / 4);
-  uint64_t* empty = full + kDecStages;
-  uint64_t* q_full = empty + kDecStages;     // [2]
+  uint64_t* empty = full + kD1Stages;
+  uint64_t* q_full = empty + kD1Stages;     // [2]
   uint64_t* q_empty = q_full + 2;            // [2]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(q_empty + 2);
   volatile int* item_abort = abort_flag + 1;   // abort flag as seen at an item end, same for all warps
+  // ring position each stage currently holds: a consumer waits on a stage's
+  // barrier only once the stage holds its tile (consecutive tiles of one warp are
+  // not consecutive uses of a stage, so a parity wait alone could alias)
+  volatile int* stage_tag = item_abort + 1;    // [kD1Stages]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G;
@@ -138,8 +150,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
   const int n_items = a.B * a.H_kv * a.n_cmp_chunks;
 
   if (tid == 0) {
-    for (int i = 0; i < kDecStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], kDecConsumers); }
+    for (int i = 0; i < kD1Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); stage_tag[i] = -1; }
+    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], kD1Consumers); }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -158,10 +170,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
     }
     const int nc = n_cmp_dev(L, a.l, a.s);
     const int c0 = chunk * kCmpChunk;
-    return c0 < nc ? min(kTilesPerChunk, (nc - c0 + 63) / 64) : 0;
+    return c0 < nc ? min(kTilesPerChunk, (nc - c0 + kTileKeys - 1) / kTileKeys) : 0;
   };
 
-  if (warp == kDecConsumers) {
+  if (warp == kD1Consumers) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int u = 0, it = 0;
@@ -177,23 +189,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
           tma_load_3d(qbuf + qi * S::QBUF + kb * 2048, &mp.q, &q_full[qi], kb * 64, g * G, b);
         const int row0 = b * a.Lmax_cmp + chunk * kCmpChunk;
         for (int i = 0; i < ntl; ++i, ++u) {
-          const int st = u % kDecStages;
-          if (u >= kDecStages && !mbar_wait(&empty[st], ((u / kDecStages) - 1) & 1, abort_flag, a.status, 401)) {
+          const int st = u % kD1Stages;
+          if (u >= kD1Stages && !mbar_wait(&empty[st], ((u / kD1Stages) - 1) & 1, abort_flag, a.status, 401)) {
             ok = false;
             break;
           }
           uint8_t* Ks = ring + st * S::STAGE;
+          stage_tag[st] = u;
           mbar_arrive_expect_tx(&full[st], S::STAGE);
-          for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.kc, &full[st], kb * 64, g, row0 + i * 64);
+          for (int kb = 0; kb < DK / 64; ++kb)
+            tma_load_3d(Ks + kb * (kTileKeys * 128), &mp.kc, &full[st], kb * 64, g, row0 + i * kTileKeys);
           for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_3d(Ks + DK * 128 + vb * 8192, &mp.vc, &full[st], vb * 64, g, row0 + i * 64);
+            tma_load_3d(Ks + DK * kTileKeys * 2 + vb * (kTileKeys * 128), &mp.vc, &full[st], vb * 64, g,
+                        row0 + i * kTileKeys);
         }
         ++it;
+      }
+      if (*abort_flag) {
+        // let the copies still in flight land before the CTA exits
+        for (int v = u - kD1Stages < 0 ? 0 : u - kD1Stages; v < u; ++v)
+          mbar_wait_drain(&full[v % kD1Stages], (v / kD1Stages) & 1);
+        for (int q2 = it - 2 < 0 ? 0 : it - 2; q2 < it; ++q2) mbar_wait_drain(&q_full[q2 & 1], (q2 >> 1) & 1);
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    float* ps = pscr + warp * 16 * 64;
+    float* ps = pscr + warp * 16 * kTileKeys;
     int u_base = 0, it = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -208,19 +229,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
       const uint32_t qbase = smem_u32(qbuf + qi * S::QBUF);
       RowState<DV> rs;
       rs.init();
-      for (int i = warp; i < ntl && ok; i += kDecConsumers) {
+      for (int i = warp; i < ntl && ok; i += kD1Consumers) {
         const int u = u_base + i;
-        const int st = u % kDecStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kDecStages) & 1, abort_flag, a.status, 402))) {
+        const int st = u % kD1Stages;
+        const bool got = smem_wait_eq(&stage_tag[st], u, abort_flag, a.status, 405) &&
+                         mbar_wait(&full[st], (u / kD1Stages) & 1, abort_flag, a.status, 402);
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         const uint32_t kb = smem_u32(ring + st * S::STAGE);
-        float s[8][4];
-        warp_qk_sq<DK>(qbase, 2048, 0, kb, s, lane);
-        const int kc0 = c0 + i * 64 + (lane & 3) * 2;
+        float s[kNT][4];
+        warp_qk_sq<DK, kNT>(qbase, 2048, 0, kb, s, lane);
+        const int kc0 = c0 + i * kTileKeys + (lane & 3) * 2;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const bool vis = kc0 + nt * 8 + e < nc;
@@ -232,33 +255,33 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
         {
           const int r0 = lane >> 2, cq = (lane & 3) * 2;
 #pragma unroll
-          for (int nt = 0; nt < 8; ++nt) {
-            ps[r0 * 64 + nt * 8 + cq] = s[nt][0];
-            ps[r0 * 64 + nt * 8 + cq + 1] = s[nt][1];
-            ps[(r0 + 8) * 64 + nt * 8 + cq] = s[nt][2];
-            ps[(r0 + 8) * 64 + nt * 8 + cq + 1] = s[nt][3];
+          for (int nt = 0; nt < kNT; ++nt) {
+            ps[r0 * kTileKeys + nt * 8 + cq] = s[nt][0];
+            ps[r0 * kTileKeys + nt * 8 + cq + 1] = s[nt][1];
+            ps[(r0 + 8) * kTileKeys + nt * 8 + cq] = s[nt][2];
+            ps[(r0 + 8) * kTileKeys + nt * 8 + cq + 1] = s[nt][3];
           }
         }
-        warp_pv<DV>(s, kb + DK * 128, rs.o, lane);
+        warp_pv<DV, kNT>(s, kb + DK * kTileKeys * 2, rs.o, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
         // block sums: compressed key 4q+u covers tokens [16(4q+u), +32): u<3 -> 2p
-        // into block q of the tile, u = 3 -> p into q and q+1 (17 relative blocks).
-        // Tile partial layout [18][G]: row 0 = reference max per head, rows 1..17 =
-        // block sums per head.
+        // into block q of the tile, u = 3 -> p into q and q+1. Tile partial layout
+        // [kTP][G]: row 0 = reference max per head, rows 1..kBlkPerTile+1 = block
+        // sums per head (the last one spills into the next tile's first block).
         {
-          const int tile = c0 / 64 + i;
+          const int tile = c0 / kTileKeys + i;
           float* tpb = a.part + pl.tp + (((size_t)b * a.H_kv + g) * pl.n_tiles + tile) * kTP * G;
           const int row = lane >> 1, half = lane & 1;
           if (row < G) {
-            const float* pr = ps + row * 64;
-            const int q0 = half * 8;
-            for (int q = q0; q < q0 + 8; ++q) {
+            const float* pr = ps + row * kTileKeys;
+            const int q0 = half * (kBlkPerTile / 2);
+            for (int q = q0; q < q0 + kBlkPerTile / 2; ++q) {
               float v = 2.f * (pr[4 * q] + pr[4 * q + 1] + pr[4 * q + 2]) + pr[4 * q + 3];
               if (q > 0) v += pr[4 * q - 1];
               tpb[(1 + q) * G + row] = v;
             }
-            if (half == 1) tpb[17 * G + row] = pr[63];
+            if (half == 1) tpb[(1 + kBlkPerTile) * G + row] = pr[kTileKeys - 1];
           }
           if ((lane & 3) == 0) {
             const int r0 = lane >> 2;
@@ -269,18 +292,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_cmp_kernel(const DecodeArg
         __syncwarp();
       }
       rs.finish();
-      named_bar_sync(1, kDecConsumers * 32);
+      named_bar_sync(1, kD1Consumers * 32);
       if (tid == 0) *item_abort = *abort_flag;
       rs.stage(stg + warp * 16 * (DV + 2), lane);
-      named_bar_sync(1, kDecConsumers * 32);
+      named_bar_sync(1, kD1Consumers * 32);
       const bool aborted = *item_abort != 0;   // written before the barrier: same in every warp
       if (!aborted) {
         const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
-        merge_warps<DV>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
+        merge_warps<DV, kD1Consumers>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&q_empty[qi]);
-      named_bar_sync(1, kDecConsumers * 32);   // merge done before the staging area is rewritten
+      named_bar_sync(1, kD1Consumers * 32);   // merge done before the staging area is rewritten
       if (aborted) break;
       u_base += ntl;
       ++it;
@@ -303,7 +326,7 @@ __global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeA
   if (L < 1 || L > a.max_len) return;
   const int nc = n_cmp_dev(L, a.l, a.s);
   const int nch = (nc + kCmpChunk - 1) / kCmpChunk;
-  const int ntl = (nc + 63) / 64;
+  const int ntl = (nc + kTileKeys - 1) / kTileKeys;
   const int t = L - 1;
   const int jt = t / a.ls;
   const PartLayout pl = part_layout(a);
@@ -351,18 +374,28 @@ __global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeA
         make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
   }
   __syncthreads();
-  // importance of blocks 0..jt: tile tj holds blocks 16 tj .. 16 tj + 16
+  // importance of blocks 0..jt: tile tj holds blocks kBlkPerTile*tj .. + kBlkPerTile
   for (int j = tid; j <= jt; j += kSelThreadsD2) {
-    const int tj = j >> 4, q = j & 15;
+    const int tj = j / kBlkPerTile, q = j % kBlkPerTile;
     float v = 0.f;
-    if (tj < ntl) {
-      const float* r = tp + ((size_t)tj * kTP + 1 + q) * G;
-      for (int h = 0; h < G; ++h) v += Ft[tj * 16 + h] * r[h];
-    }
-    if (q == 0 && tj >= 1 && tj - 1 < ntl) {
-      const float* r = tp + ((size_t)(tj - 1) * kTP + 17) * G;
-      for (int h = 0; h < G; ++h) v += Ft[(tj - 1) * 16 + h] * r[h];
-    }
+    auto head_sum = [&](int tile, int rowi) -> float {
+      const float* r = tp + ((size_t)tile * kTP + rowi) * G;
+      const float* f = Ft + tile * 16;
+      float acc = 0.f;
+      if ((G & 3) == 0) {
+#pragma unroll 4
+        for (int h = 0; h < G; h += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(r + h);
+          const float4 y = *reinterpret_cast<const float4*>(f + h);
+          acc += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+        }
+      } else {
+        for (int h = 0; h < G; ++h) acc += f[h] * r[h];
+      }
+      return acc;
+    };
+    if (tj < ntl) v += head_sum(tj, 1 + q);
+    if (q == 0 && tj >= 1 && tj - 1 < ntl) v += head_sum(tj - 1, 1 + kBlkPerTile);
     imp_s[j] = v;
     a.imp[bg * a.nb_stride + j] = v;
   }
@@ -374,8 +407,8 @@ __global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeA
 // ---------------------------------------------------------------------------
 // D3: selected blocks and window for one (sequence, KV head) per CTA. The
 // ascending union of the selected blocks and the blocks the window touches is
-// streamed once through the TMA ring; consumer warp w takes union positions
-// w, w+4, ...; one score tile serves both branches, each with its own online
+// streamed once through the TMA ring in 32-key halves; consumer warp w takes
+// half-tiles w, w+4, ...; one score tile serves both branches, each with its own online
 // softmax. At the end the four warps' states are merged in shared memory and
 // out = g_cmp o_cmp + g_slc o_slc + g_win o_win is written.
 // ---------------------------------------------------------------------------
@@ -462,37 +495,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   __syncthreads();
   const int nu = *nuni;
 
+  // work units: the two 32-key halves of every union block
+  const int nh = 2 * nu;
   if (warp == kDecConsumers) {
     if (lane == 0) {
-      for (int u = 0; u < nu; ++u) {
+      int issued = 0;
+      for (int u = 0; u < nh; ++u) {
         const int st = u % kDecStages;
         if (u >= kDecStages && !mbar_wait(&empty[st], ((u / kDecStages) - 1) & 1, abort_flag, a.status, 411)) break;
         uint8_t* Ks = ring + st * S::STAGE;
-        const int row = b * a.Lmax + uni[u] * a.ls;
+        const int row = b * a.Lmax + uni[u >> 1] * a.ls + (u & 1) * kTileKeys;
         mbar_arrive_expect_tx(&full[st], S::STAGE);
-        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, &mp.k, &full[st], kb * 64, g, row);
+        for (int kb = 0; kb < DK / 64; ++kb)
+          tma_load_3d(Ks + kb * (kTileKeys * 128), &mp.k, &full[st], kb * 64, g, row);
         for (int vb = 0; vb < DV / 64; ++vb)
-          tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
+          tma_load_3d(Ks + S::K_BYTES + vb * (kTileKeys * 128), &mp.v, &full[st], vb * 64, g, row);
+        issued = u + 1;
       }
+      if (*abort_flag)   // let the copies still in flight land before the CTA exits
+        for (int v = issued - kDecStages < 0 ? 0 : issued - kDecStages; v < issued; ++v)
+          mbar_wait_drain(&full[v % kDecStages], (v / kDecStages) & 1);
     }
   } else {
     RowState<DV> rs_sel, rs_win;
     rs_sel.init();
     rs_win.init();
     const uint32_t qbase = smem_u32(qs);
-    for (int u = warp; u < nu; u += kDecConsumers) {
+    for (int u = warp; u < nh; u += kDecConsumers) {
       const int st = u % kDecStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kDecStages) & 1, abort_flag, a.status, 412))) break;
       const uint32_t kb = smem_u32(ring + st * S::STAGE);
-      const int blk = uni[u];
-      const bool in_sel = flags[u] != 0u;
-      float s[8][4];
-      warp_qk_sq<DK>(qbase, 16 * 128, 0, kb, s, lane);
-      const int key0 = blk * a.ls + (lane & 3) * 2;
-      float x[8][4];
-      if (in_sel) {
+      const int blk = uni[u >> 1];
+      const bool in_sel = flags[u >> 1] != 0u;
+      const int first_key = blk * a.ls + (u & 1) * kTileKeys;
+      float s[kNT][4];
+      warp_qk_sq<DK, kNT>(qbase, 16 * 128, 0, kb, s, lane);
+      const int key0 = first_key + (lane & 3) * 2;
+      float x[kNT][4];
+      if (in_sel && first_key <= t) {
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const bool vis = key0 + nt * 8 + e <= t;
@@ -501,11 +543,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
           }
         }
         rs_sel.update(x);
-        warp_pv<DV>(x, kb + S::K_BYTES, rs_sel.o, lane);
+        warp_pv<DV, kNT>(x, kb + S::K_BYTES, rs_sel.o, lane);
       }
-      if (blk * a.ls + a.ls - 1 >= wlo) {
+      if (first_key + kTileKeys - 1 >= wlo && first_key <= t) {
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int tau = key0 + nt * 8 + e;
@@ -515,7 +557,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
           }
         }
         rs_win.update(x);
-        warp_pv<DV>(x, kb + S::K_BYTES, rs_win.o, lane);
+        warp_pv<DV, kNT>(x, kb + S::K_BYTES, rs_win.o, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
@@ -580,7 +622,7 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     const int n_items = a.B * a.H_kv * a.n_cmp_chunks;
     prof_begin(P_DEC_CMP, st);
-    k1<<<n_items < n_sm ? n_items : n_sm, kDecThreads, S1::TOTAL, st>>>(a, m);
+    k1<<<n_items < n_sm ? n_items : n_sm, kD1Threads, S1::TOTAL, st>>>(a, m);
     prof_end(P_DEC_CMP, st, 1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -524,10 +524,11 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
   DecodeMaps m;
   memset(&m, 0, sizeof(m));
   const int64_t rows = (int64_t)batch * Lmax, crows = (int64_t)batch * Lmax_cmp;
-  if (!make_map_3d(&m.k, k_cache, heads->d_k, heads->H_kv, rows, 1, 64) ||
-      !make_map_3d(&m.v, v_cache, heads->d_v, heads->H_kv, rows, 1, 64) ||
-      !make_map_3d(&m.kc, crows > 0 ? k_cmp_cache : k_cache, heads->d_k, heads->H_kv, crows > 0 ? crows : rows, 1, 64) ||
-      !make_map_3d(&m.vc, crows > 0 ? v_cmp_cache : v_cache, heads->d_v, heads->H_kv, crows > 0 ? crows : rows, 1, 64) ||
+  // decode streams 32-key tiles
+  if (!make_map_3d(&m.k, k_cache, heads->d_k, heads->H_kv, rows, 1, 32) ||
+      !make_map_3d(&m.v, v_cache, heads->d_v, heads->H_kv, rows, 1, 32) ||
+      !make_map_3d(&m.kc, crows > 0 ? k_cmp_cache : k_cache, heads->d_k, heads->H_kv, crows > 0 ? crows : rows, 1, 32) ||
+      !make_map_3d(&m.vc, crows > 0 ? v_cmp_cache : v_cache, heads->d_v, heads->H_kv, crows > 0 ? crows : rows, 1, 32) ||
       !make_map_3d(&m.q, q, heads->d_k, heads->H_q, batch, heads->H_q / heads->H_kv, 1)) {
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
     return NSA_ERR_CUDA;

@@ -191,9 +191,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
       mbar_arrive_expect_tx(q_full, (uint32_t)(DK / 64) * qchunk);
       for (int kb = 0; kb < DK / 64; ++kb)
         tma_load_3d(qs + kb * qchunk, &mp.q8, q_full, kb * 64, g * G, (int)(tok0 + t0));
+      int issued = 0;
       for (int u = 0; u < nu; ++u) {
         const int st = u % kSelStages;
         if (u >= kSelStages && !mbar_wait(&empty[st], ((u / kSelStages) - 1) & 1, abort_flag, a.status, 301)) break;
+        issued = u + 1;
         stage_tag[st] = u;
         uint8_t* Ks = ring + st * S::STAGE;
         const int row = (int)(tok0 + (int64_t)uni[u] * a.ls);
@@ -203,6 +205,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) sel_attn_kernel(const PrefillA
           tma_load_3d(Ks + S::K_BYTES + vb * 8192, &mp.v, &full[st], vb * 64, g, row);
         const uint32_t others = kSelTok - __popc(umask[u]);   // warps that will not release it
         if (others) mbar_arrive_cnt(&empty[st], others);
+      }
+      if (*abort_flag) {   // let the copies still in flight land before the CTA exits
+        mbar_wait_drain(q_full, 0);
+        for (int v = issued - kSelStages < 0 ? 0 : issued - kSelStages; v < issued; ++v)
+          mbar_wait_drain(&full[v % kSelStages], (v / kSelStages) & 1);
       }
     }
   } else {

@@ -51,21 +51,22 @@ __device__ __forceinline__ void warp_qk(const uint32_t (&qa)[DK / 16][4], uint32
 }
 
 // Same as warp_qk with Q read from shared memory (TMA box [rows][64] per 64-wide
-// chunk, 128-byte swizzle, chunks `qchunk` bytes apart); rows qrow0 .. qrow0+15.
-template <int DK>
+// chunk, 128-byte swizzle, chunks `qchunk` bytes apart); rows qrow0 .. qrow0+15;
+// the key tile has NT*8 keys (K boxes of [NT*8 keys][64], NT*1 KB apart).
+template <int DK, int NT = 8>
 __device__ __forceinline__ void warp_qk_sq(uint32_t qbase, uint32_t qchunk, int qrow0, uint32_t kbase,
-                                           float (&s)[8][4], int lane) {
+                                           float (&s)[NT][4], int lane) {
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+  for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
   const int mi = lane >> 3, rr = lane & 7;
   const uint32_t qrow = (uint32_t)(qrow0 + (lane & 15));
 #pragma unroll
   for (int kk = 0; kk < DK / 16; ++kk) {
     uint32_t qa[4];
     ldmatrix_x4(qa, qbase + (kk >> 2) * qchunk + sw128(qrow, (kk & 3) * 2 + (lane >> 4)));
-    const uint32_t box = kbase + (kk >> 2) * 8192;
+    const uint32_t box = kbase + (kk >> 2) * (NT * 1024);
 #pragma unroll
-    for (int np = 0; np < 4; ++np) {
+    for (int np = 0; np < NT / 2; ++np) {
       const int key = np * 16 + (mi >> 1) * 8 + rr;
       const int chunk = (kk & 3) * 2 + (mi & 1);
       uint32_t bfr[4];
@@ -76,12 +77,51 @@ __device__ __forceinline__ void warp_qk_sq(uint32_t qbase, uint32_t qchunk, int 
   }
 }
 
-// o += P V for one tile, P given as fp32 probabilities in the score layout.
-template <int DV>
-__device__ __forceinline__ void warp_pv(const float (&p)[8][4], uint32_t vbase, float (&o)[DV / 8][4], int lane) {
+// warp_qk_sq with the K reduction split over two independent accumulator sets
+// (even / odd 16-wide steps), halving the dependent MMA chain.
+template <int DK, int NT = 8>
+__device__ __forceinline__ void warp_qk_sq2(uint32_t qbase, uint32_t qchunk, int qrow0, uint32_t kbase,
+                                            float (&s)[NT][4], int lane) {
+  float s2[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+  const int mi = lane >> 3, rr = lane & 7;
+  const uint32_t qrow = (uint32_t)(qrow0 + (lane & 15));
+#pragma unroll
+  for (int kk = 0; kk < DK / 16; ++kk) {
+    uint32_t qa[4];
+    ldmatrix_x4(qa, qbase + (kk >> 2) * qchunk + sw128(qrow, (kk & 3) * 2 + (lane >> 4)));
+    const uint32_t box = kbase + (kk >> 2) * (NT * 1024);
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      const int key = np * 16 + (mi >> 1) * 8 + rr;
+      const int chunk = (kk & 3) * 2 + (mi & 1);
+      uint32_t bfr[4];
+      ldmatrix_x4(bfr, box + sw128(key, chunk));
+      if (kk & 1) {
+        mma_bf16_16816(s2[2 * np], qa, bfr);
+        mma_bf16_16816(s2[2 * np + 1], qa, bfr + 2);
+      } else {
+        mma_bf16_16816(s[2 * np], qa, bfr);
+        mma_bf16_16816(s[2 * np + 1], qa, bfr + 2);
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
+}
+
+// o += P V for one tile of NT*8 keys, P given as fp32 probabilities in the
+// score layout; V boxes of [NT*8 keys][64 dv], NT*1 KB apart.
+template <int DV, int NT = 8>
+__device__ __forceinline__ void warp_pv(const float (&p)[NT][4], uint32_t vbase, float (&o)[DV / 8][4], int lane) {
   const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
+  for (int kk = 0; kk < NT / 2; ++kk) {
     uint32_t pa[4];
     pa[0] = pack_bf16x2(p[2 * kk][0], p[2 * kk][1]);
     pa[1] = pack_bf16x2(p[2 * kk][2], p[2 * kk][3]);
@@ -92,7 +132,7 @@ __device__ __forceinline__ void warp_pv(const float (&p)[8][4], uint32_t vbase, 
       const int key = kk * 16 + (mi & 1) * 8 + rr;
       const int c16 = np * 2 + (mi >> 1);
       uint32_t bfr[4];
-      ldmatrix_x4_trans(bfr, vbase + (c16 >> 3) * 8192 + sw128(key, c16 & 7));
+      ldmatrix_x4_trans(bfr, vbase + (c16 >> 3) * (NT * 1024) + sw128(key, c16 & 7));
       mma_bf16_16816(o[2 * np], pa, bfr);
       mma_bf16_16816(o[2 * np + 1], pa, bfr + 2);
     }
@@ -121,10 +161,11 @@ struct RowState {
   }
   // x: scaled scores (log2 domain, -inf where masked); turns x into
   // probabilities relative to the new running max and rescales o and l.
-  __device__ __forceinline__ void update(float (&x)[8][4]) {
+  template <int NT>
+  __device__ __forceinline__ void update(float (&x)[NT][4]) {
     float mx0 = -1e30f, mx1 = -1e30f;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       mx0 = fmaxf(mx0, fmaxf(x[nt][0], x[nt][1]));
       mx1 = fmaxf(mx1, fmaxf(x[nt][2], x[nt][3]));
     }
@@ -136,7 +177,7 @@ struct RowState {
     m[1] = mn1;
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       x[nt][0] = ex2(x[nt][0] - mn0);
       x[nt][1] = ex2(x[nt][1] - mn0);
       x[nt][2] = ex2(x[nt][2] - mn1);
