@@ -70,7 +70,7 @@ def prefill_work(cfg):
     per_pair = 2 * (cfg.d_k + cfg.d_v) * cfg.H_q
     nc = (T - cfg.l_cmp) // cfg.stride + 1
     comp = 2 * cfg.l_cmp * (cfg.d_k ** 2 + cfg.d_v ** 2) * nc * cfg.H_kv
-    return dict(cmp_attn=pc * per_pair, sel_attn=ps * per_pair, win_attn=pw * per_pair, compress_gemm=comp,
+    return dict(prefill_attn=(pc + ps + pw) * per_pair, compress_gemm=comp,
                 total=(pc + ps + pw) * per_pair + comp,
                 dense_causal=T * (T + 1) // 2 * per_pair)
 

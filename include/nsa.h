@@ -194,7 +194,7 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
  * the previous read, and resets them. Slot names: nsa_profile_slot_name(). The
  * events are created on first use and reused; this is the only state the
  * library keeps between calls. Returns NSA_ERR_CUDA if an event query fails. */
-#define NSA_PROFILE_SLOTS 10
+#define NSA_PROFILE_SLOTS 6
 nsa_status_t nsa_profile_enable(int32_t enable);
 nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots);
 const char* nsa_profile_slot_name(int32_t slot);

@@ -79,16 +79,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase. Returns false (and records the failure in
-// the status word and in the CTA-wide abort flag) when the phase does not
-// complete within NSA_WAIT_LIMIT_NS, or when another thread of the CTA already
-// gave up. A kernel that sees false stops issuing work and goes to its exit path.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps
+// in hardware until the phase completes or about `hint_ns` pass, instead of
+// spinning on the issue slots its neighbours need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Slow path of mbar_wait (kept out of line so that every wait site in a kernel
+// costs one try_wait instruction and a branch in the hot code).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            uint32_t* status, uint32_t site) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > NSA_WAIT_LIMIT_NS) {
       *abort_flag = 1;
@@ -101,13 +113,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait on an mbarrier phase. Returns false (and records the failure in
+// the status word and in the CTA-wide abort flag) when the phase does not
+// complete within NSA_WAIT_LIMIT_NS, or when another thread of the CTA already
+// gave up. A kernel that sees false stops issuing work and goes to its exit path.
+// Waiting threads sleep (suspend hint of 20 us per try), so the abort flag and
+// the clock are polled only every few microseconds.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, status, site);
+}
+
 // Time-bounded wait that ignores the abort flag: used on the exit path to let
 // copies / MMAs this CTA issued land before it leaves (returns false if the
 // phase does not complete within NSA_WAIT_LIMIT_NS).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+static __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
     if (globaltimer_ns() - t0 > NSA_WAIT_LIMIT_NS) return false;
   return true;
 }

@@ -12,8 +12,7 @@ constexpr int kMaxBatch = 128;
 // Opt-in per-kernel timing: CUDA events recorded on the launching stream around
 // each launch (see nsa_profile_enable / nsa_profile_read in include/nsa.h).
 enum ProfSlot {
-  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_CMP_ATTN, P_TOPN, P_SEL_ATTN, P_WIN_ATTN,
-  P_DEC_CMP, P_DEC_SELECT, P_DEC_FINE, P_DEC_COMBINE, P_COUNT
+  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_SELECT, P_DEC_FINE, P_COUNT
 };
 void prof_begin(int slot, cudaStream_t st);
 void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()
@@ -58,25 +57,23 @@ struct PrefillArgs {
   const void* kc;         // bf16 [Nc, H_kv, d_k]
   const void* vc;         // bf16 [Nc, H_kv, d_v]
   const float* gates;     // fp32 [N, H_q, 3]
-  float* acc;             // fp32 [N, H_q, d_v] (g_cmp*o_cmp + g_slc*o_slc)
   float* imp;             // fp32 [N, H_kv, nb_stride]
   int32_t* sel;           // int32 [N, H_kv, top_n]
   void* out;              // bf16 [N, H_q, d_v]
   int H_q, H_kv, G, d_k, d_v;
   int l, s, ls, top_n, window, force_first, force_local;
   int nb_stride;
+  int n_stages;           // K/V ring depth of the fused kernel
   float scale_log2;       // softmax scale * log2(e)
   uint32_t* status;
-  SeqTable seqs;          // tile_prefix counts CTA tiles of 2 x 128/G tokens
+  SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens
 };
 struct PrefillMaps {
-  CUtensorMap q, k, v, kc, vc;
-  CUtensorMap q8;   // q with a box of 8 tokens x G heads (selected-block attention)
+  CUtensorMap k, v, kc, vc;   // boxes of 64 rows x 1 head x 64 elements
+  CUtensorMap q;              // box of 128/G tokens x G heads x 64 elements (one query tile)
 };
-cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
-cudaError_t launch_topn(const PrefillArgs& a, int64_t n_tokens, cudaStream_t st);
-cudaError_t launch_sel_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
-cudaError_t launch_win_attn(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
+int prefill_fused_stages(const PrefillArgs& a);   // 0: does not fit in shared memory
+cudaError_t launch_prefill_fused(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 
 // ----- decode -----
 struct DecodeArgs {

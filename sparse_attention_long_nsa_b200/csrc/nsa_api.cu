@@ -89,14 +89,13 @@ CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t rows
 }
 
 struct PrefillWs {
-  size_t acc, imp, sel, total;
+  size_t imp, sel, total;
   int nb;
 };
 PrefillWs prefill_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t N, int max_len) {
   PrefillWs w{};
   size_t off = 256;
   w.nb = n_blk_of(max_len, p->l_sel);
-  w.acc = off; off = align256(off + (size_t)N * h->H_q * h->d_v * 4);
   w.imp = off; off = align256(off + (size_t)N * h->H_kv * w.nb * 4);
   w.sel = off; off = align256(off + (size_t)N * h->H_kv * p->top_n * 4);
   w.total = off;
@@ -188,8 +187,8 @@ Profiler& prof() {
   return p;
 }
 
-const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "cmp_attn", "topn", "sel_attn", "win_attn",
-                                   "dec_cmp", "dec_select", "dec_fine", "dec_combine"};
+const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_select",
+                                   "dec_fine"};
 
 }  // namespace
 
@@ -429,7 +428,6 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillArgs a{};
   a.q = q; a.k = k; a.v = v; a.kc = k_cmp; a.vc = v_cmp; a.gates = gates;
-  a.acc = (float*)(ws + w.acc);
   a.imp = imp_out ? imp_out : (float*)(ws + w.imp);
   a.sel = sel_out ? sel_out : (int32_t*)(ws + w.sel);
   a.out = out;
@@ -440,8 +438,13 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   a.nb_stride = w.nb;
   a.scale_log2 = softmax_scale(params, heads->d_k) * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.n_stages = prefill_fused_stages(a);
+  if (a.n_stages == 0) {
+    snprintf(g_detail, sizeof(g_detail), "sequence too long for the fused prefill kernel (%d blocks)", w.nb);
+    return NSA_ERR_UNSUPPORTED;
+  }
 
-  const int tok_per_tile = 2 * (128 / a.G);   // two 128-row query tiles per attention CTA
+  const int tok_per_tile = 128 / a.G;   // one 128-row query tile per CTA
   SeqTable t{};
   t.n = batch;
   int tiles = 0;
@@ -465,30 +468,17 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   if (!make_map_3d(&m.q, q, heads->d_k, heads->H_q, N, a.G, 128 / a.G) ||
       !make_map_3d(&m.k, k, heads->d_k, heads->H_kv, N, 1, 64) ||
       !make_map_3d(&m.v, v, heads->d_v, heads->H_kv, N, 1, 64) ||
-      !make_map_3d(&m.kc, kc_base, heads->d_k, heads->H_kv, ncmp_total, 1, 64) ||
-      !make_map_3d(&m.vc, vc_base, heads->d_v, heads->H_kv, ncmp_total, 1, 64) ||
-      !make_map_3d(&m.q8, q, heads->d_k, heads->H_q, N, a.G, 8)) {
+      !make_map_3d(&m.kc, kc_base, heads->d_k, heads->H_kv, ncmp_total > 0 ? ncmp_total : N, 1, 64) ||
+      !make_map_3d(&m.vc, vc_base, heads->d_v, heads->H_kv, ncmp_total > 0 ? ncmp_total : N, 1, 64)) {
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
     return NSA_ERR_CUDA;
   }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  prof_begin(P_CMP_ATTN, st);
-  cudaError_t e = launch_cmp_attn(a, m, tiles, st);
-  prof_end(P_CMP_ATTN, st, 1);
-  if (e != cudaSuccess) return cuda_fail(e, "compressed attention");
-  prof_begin(P_TOPN, st);
-  e = launch_topn(a, N, st);
-  prof_end(P_TOPN, st, 1);
-  if (e != cudaSuccess) return cuda_fail(e, "top-n selection");
-  prof_begin(P_SEL_ATTN, st);
-  e = launch_sel_attn(a, m, tiles, st);
-  prof_end(P_SEL_ATTN, st, 1);
-  if (e != cudaSuccess) return cuda_fail(e, "selected attention");
-  prof_begin(P_WIN_ATTN, st);
-  e = launch_win_attn(a, m, tiles, st);
-  prof_end(P_WIN_ATTN, st, 1);
-  if (e != cudaSuccess) return cuda_fail(e, "window attention");
+  prof_begin(P_PREFILL_ATTN, st);
+  cudaError_t e = launch_prefill_fused(a, m, tiles, st);
+  prof_end(P_PREFILL_ATTN, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attention");
   return NSA_OK;
 }
 

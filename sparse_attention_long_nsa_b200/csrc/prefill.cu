@@ -1,0 +1,740 @@
+// Fused NSA prefill attention on tcgen05: compressed branch + block importance,
+// top-n block selection, sliding window and selected blocks, gated combine.
+//
+// Method ("Разреженное внимание — NSA и DSA", ai.flicky.cc, section "NSA: три
+// ветви"; "Native Sparse Attention" lesson, aiengineeringfromscratch.com, steps
+// 1-5): each query head attends, in three separate softmaxes, to the compressed
+// block summaries it can see, to the raw tokens of the top-n selection blocks its
+// GQA group chose from the compressed attention weights, and to the last w raw
+// tokens; the three outputs are mixed by per-head sigmoid gates.
+//
+// One CTA owns one query tile of M = 128 rows = (128/G tokens) x (G heads of one
+// KV group) and runs every branch for it, so K/V tiles staged in shared memory
+// serve all heads of the group and the only global output is bf16 `out` (plus
+// the optional importance / selection rows):
+//
+//   C1  compressed keys, pass 1: row max and softmax denominator
+//   C2  compressed keys, pass 2: normalised probabilities p; importance of every
+//       selection block (p spread by token overlap, summed over the group's
+//       heads); O_A = g_cmp * P.V_cmp
+//   --  top-n per token (forced first / local blocks, ties to the lower index),
+//       union of the tile's selections
+//   W   window keys, online softmax into O_B; O_A += g_win / l * O_B
+//   S   union blocks, each row masked to its own token's selection (and to
+//       keys <= t inside the current block); online softmax into O_B;
+//       out = bf16(O_A + g_slc / l * O_B)
+//
+// Every tile is 64 keys. Q sits in shared memory (A operand of S = Q.K^T); S has
+// four buffers in tensor memory and the softmax writes its bf16 P over the S
+// columns it has read (A operand of O += P.V). K and V stream through an n-stage
+// TMA ring. Roles (352 threads): warps 0-7 softmax, warpgroup wg = warp / 4
+// taking the tiles j with j % 2 == wg (warp w owns rows 32(w%4)..+31 and all 64
+// keys of the tile; the online reference max of a row passes from each tile to
+// the next through shared memory guarded by mbarriers); warp 8 TMA producer;
+// warp 9 issues the S = Q.K^T products (up to four tiles ahead of the softmax);
+// warp 10 the O += P.V products. Every wait is
+// time-bounded; on a timeout the CTA stops issuing work, lets its own copies and
+// products land and leaves.
+#include "common.cuh"
+#include "kernels.h"
+#include "topn.cuh"
+
+namespace nsa {
+
+namespace {
+
+constexpr int kKeys = 64;
+constexpr int kThreads = 352;
+constexpr int kSmThreads = 256;
+constexpr float kRescaleLog2 = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
+constexpr int kMaxStages = 8;
+
+// tensor-memory columns (512 allocated)
+constexpr int kSBuf = 4;          // S/P buffers of 64 columns: tile j uses buffer j % 4
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColOA = 256;  // finished branches
+constexpr uint32_t kColOB = 384;  // branch in progress
+__device__ __forceinline__ uint32_t col_s(int b) { return kColS + 64u * (uint32_t)b; }
+
+struct FBars {
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
+  uint64_t q_full, s_full[kSBuf], s_free[kSBuf], p_full[kSBuf], pv_done[kSBuf], ob_free, sel_ready, drain, smx;
+  uint64_t xbar[4];      // pair exchange (rows of a quarter, both warpgroups)
+  uint64_t hbar[4][2];   // reference-max hand-off from the tile of one parity to the next tile
+  uint32_t tmem_base;
+  int abort;
+  int nu;
+};
+
+__device__ __forceinline__ int seq_of_tile(const SeqTable& t, int tile) {
+  int lo = 0, hi = t.n - 1;
+  while (lo < hi) {   // last b with tile_prefix[b] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (t.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int cmp_visible_dev(int t, int l, int s) { return t >= l - 1 ? (t - l + 1) / s + 1 : 0; }
+
+// max / sum of N values: 8 interleaved chains, then a tree over the 8 partials
+// (dependency depth N/8 + 3 with only 8 temporaries live next to the values)
+template <int N>
+__device__ __forceinline__ float tree_max(const float* v) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = v[i];
+#pragma unroll
+  for (int i = 8; i < N; ++i) a[i & 7] = fmaxf(a[i & 7], v[i]);
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) a[i] = fmaxf(a[i], a[i + w]);
+  return a[0];
+}
+template <int N>
+__device__ __forceinline__ float tree_sum(const float* v) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = v[i];
+#pragma unroll
+  for (int i = 8; i < N; ++i) a[i & 7] += v[i];
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) a[i] += a[i + w];
+  return a[0];
+}
+
+// one warp scales `ncols` tensor-memory columns of its 32 rows, starting at `col`
+__device__ __noinline__ void tmem_scale_cols(uint32_t col, int ncols, float alpha) {
+  for (int c = 0; c < ncols; c += 16) {
+    float ov[16];
+    tmem_ld16(col + c, ov);
+    tmem_ld_wait();
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(ov[i] * alpha);
+    tmem_st8(col + c, w);
+    tmem_st8(col + c + 8, w + 8);
+  }
+  tmem_st_wait();
+}
+
+// head sum over the G consecutive lanes of one token
+__device__ __forceinline__ float group_sum(float x, int G) {
+  for (int off = G >> 1; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ void topn_any(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
+                                         int lane) {
+  const int per = (jt + 32) / 32;   // candidates 0..jt
+  if (per <= 1) warp_topn<1>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 2) warp_topn<2>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 4) warp_topn<4>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 8) warp_topn<8>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 16) warp_topn<16>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 32) warp_topn<32>(imp, jt, top_n, ff, fl, out, lane);
+  else warp_topn_mem(imp, jt, top_n, ff, fl, out, lane);
+}
+
+}  // namespace
+
+// dynamic shared memory: Q [d_k/64][128 rows][128 B] | ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
+// block masks [nb][MW] | union [nb] | importance carries [nb/16 + 2][128/G] f32
+__host__ __device__ inline size_t fused_fixed_bytes(int nb, int G) {
+  const int tok = 128 / G, mw = (tok + 31) / 32;
+  return sizeof(FBars) + 2 * 2 * 128 * 4 + 2 * 128 * 4 + (size_t)nb * mw * 4 + (size_t)nb * 4 +
+         (size_t)(nb / 16 + 2) * tok * 4 + 64;
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillArgs a,
+                                                                   const __grid_constant__ PrefillMaps mp) {
+  constexpr int K_BYTES = kKeys * DK * 2;
+  constexpr int V_BYTES = kKeys * DV * 2;
+  constexpr int STAGE = K_BYTES + V_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nst = a.n_stages;
+  uint8_t* Qs = smem;                        // Q tile, 128-byte swizzled chunks of 64 columns
+  uint8_t* ring = smem + 128 * DK * 2;
+  FBars* bars = reinterpret_cast<FBars*>(ring + (size_t)nst * STAGE);
+  float* xch = reinterpret_cast<float*>(bars + 1);                 // [slot][warpgroup][row]
+  float* hslot = xch + 512;                                        // [tile parity][row] reference max
+  const int G = a.G;
+  const int TOK = 128 / G, MW = (TOK + 31) / 32;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(hslot + 256);         // [nb][MW] token bits per block
+  int* uni = reinterpret_cast<int*>(bm + (size_t)a.nb_stride * MW);  // union of selected blocks
+  float* cbuf = reinterpret_cast<float*>(uni + a.nb_stride);      // [compressed tile][token] carried mass
+  volatile int* abort_flag = &bars->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, g = blockIdx.y;
+  const int b = seq_of_tile(a.seqs, tile);
+  const int L = a.seqs.len[b];
+  const int64_t tok0 = a.seqs.tok_off[b];
+  const int64_t cmp0 = a.seqs.cmp_off[b];
+  const int t0 = (tile - a.seqs.tile_prefix[b]) * TOK;
+  const int t_last = min(t0 + TOK - 1, L - 1);
+  const int jt_max = t_last / a.ls;
+  const int nkc = (cmp_visible_dev(t_last, a.l, a.s) + kKeys - 1) / kKeys;   // compressed tiles per pass
+  const int key0w = max(0, t0 - a.window + 1);
+  const int nkw = (t_last - key0w) / kKeys + 1;                              // window tiles
+  const int first_w = 2 * nkc, first_s = first_w + nkw;
+
+  for (int i = tid; i < (jt_max + 1) * MW; i += kThreads) bm[i] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < nst; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < kSBuf; ++i) {   // tile j is read and written by warpgroup j & 1 only
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_free[i], kSmThreads / 2);
+      mbar_init(&bars->p_full[i], kSmThreads / 2);
+      mbar_init(&bars->pv_done[i], 1);
+    }
+    mbar_init(&bars->ob_free, kSmThreads);
+    mbar_init(&bars->sel_ready, 1);
+    mbar_init(&bars->drain, 2);   // one commit per MMA issuer
+    mbar_init(&bars->smx, kSmThreads);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars->xbar[i], 64);
+      mbar_init(&bars->hbar[i][0], 32);
+      mbar_init(&bars->hbar[i][1], 32);
+    }
+    bars->abort = 0;
+    bars->nu = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&bars->tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&mp.k);
+      prefetch_tmap(&mp.v);
+      mbar_arrive_expect_tx(&bars->q_full, (uint32_t)(128 * DK * 2));
+#pragma unroll
+      for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Qs + kb * 16384, &mp.q, &bars->q_full, kb * 64, g * G, (int)(tok0 + t0));
+      int issued = 0;
+      bool ok = true;
+      auto load = [&](int j, const CUtensorMap* mk, const CUtensorMap* mv, int row, bool with_v) -> bool {
+        const int st = j % nst;
+        if (j >= nst && !mbar_wait(&bars->kv_empty[st], ((j / nst) - 1) & 1, abort_flag, a.status, 401))
+          return false;
+        uint8_t* Ks = ring + (size_t)st * STAGE;
+        mbar_arrive_expect_tx(&bars->kv_full[st], K_BYTES + (with_v ? V_BYTES : 0));
+#pragma unroll
+        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->kv_full[st], kb * 64, g, row);
+        if (with_v) {
+#pragma unroll
+          for (int vb = 0; vb < DV / 64; ++vb)
+            tma_load_3d(Ks + K_BYTES + vb * 8192, mv, &bars->kv_full[st], vb * 64, g, row);
+        }
+        issued = j + 1;
+        return true;
+      };
+      int j = 0;
+      for (int i = 0; i < nkc && ok; ++i) ok = load(j++, &mp.kc, &mp.vc, (int)(cmp0 + i * kKeys), false);
+      for (int i = 0; i < nkc && ok; ++i) ok = load(j++, &mp.kc, &mp.vc, (int)(cmp0 + i * kKeys), true);
+      for (int i = 0; i < nkw && ok; ++i) ok = load(j++, &mp.k, &mp.v, (int)(tok0 + key0w + i * kKeys), true);
+      if (ok) ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 402);
+      const int nu = ok ? bars->nu : 0;
+      for (int u = 0; u < nu && ok; ++u) ok = load(j++, &mp.k, &mp.v, (int)(tok0 + (int64_t)uni[u] * a.ls), true);
+      if (!ok) {   // let the copies still in flight land before the CTA exits
+        mbar_wait_drain(&bars->q_full, 0);
+        for (int v = issued - nst < 0 ? 0 : issued - nst; v < issued; ++v)
+          mbar_wait_drain(&bars->kv_full[v % nst], (v / nst) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ S = Q.K^T issuer
+    // S(j) goes to buffer j % 4; the buffer is free again once the softmax read
+    // S(j - 4) (pass 1) or P.V(j - 4) consumed the P written over it.
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(128, kKeys, false, false);
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
+      const uint64_t qdesc0 = umma_desc_sw128(smem_u32(Qs), 16, 1024);
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.status, 411);
+      int total = first_s;
+      for (int j = 0; ok; ++j) {
+        if (j == first_s) {
+          ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 414);
+          if (!ok) break;
+          total = first_s + bars->nu;
+        }
+        if (j >= total) break;
+        const int st = j % nst, sb = j & (kSBuf - 1);
+        ok = mbar_wait(&bars->kv_full[st], (j / nst) & 1, abort_flag, a.status, 415);
+        if (ok && j >= kSBuf) {
+          // s_* barriers complete once per tile, p_full / pv_done once per P.V tile (index >= nkc)
+          const int jp = j - kSBuf;
+          ok = (jp >= nkc) ? mbar_wait(&bars->pv_done[sb], ((jp - nkc) >> 2) & 1, abort_flag, a.status, 416)
+                           : mbar_wait(&bars->s_free[sb], (jp >> 2) & 1, abort_flag, a.status, 418);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)st * STAGE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          umma_ss(tmem + col_s(sb), qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                  kd + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_full[sb]);
+        if (j < nkc) umma_commit(&bars->kv_empty[st]);   // pass 1 reads K only
+      }
+      // every product this thread issued has finished before tensor memory is released
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ O += P.V issuer
+    // (P(i) exists only after the softmax read S(i), so Q.K(i) has finished and
+    // releasing the stage after P.V(i) also covers the K half)
+    if (lane == 0) {
+      const uint32_t idesc_pv = umma_idesc_bf16(128, DV, false, true);
+      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring) + K_BYTES, 8192, 1024);
+      bool ok = true;
+      int total = first_s;
+      for (int i = nkc; ok; ++i) {
+        if (i == first_s) {
+          ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 417);
+          if (!ok) break;
+          total = first_s + bars->nu;
+        }
+        if (i >= total) break;
+        const int sb = i & (kSBuf - 1);
+        ok = mbar_wait(&bars->p_full[sb], ((i - nkc) >> 2) & 1, abort_flag, a.status, 412) &&
+             (i != first_s || mbar_wait(&bars->ob_free, 0, abort_flag, a.status, 413));
+        if (!ok) break;
+        tc_fence_after();
+        const bool first = (i == nkc) || (i == first_w) || (i == first_s);
+        const uint32_t ocol = i < first_w ? kColOA : kColOB;
+        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)(i % nst) * STAGE) >> 4);
+        // P (bf16 pairs, 32 columns) sits over the first half of the S columns of its buffer
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          umma_ts(tmem + ocol, tmem + col_s(sb) + (uint32_t)(kk * 8), vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                  (first && kk == 0) ? 0u : 1u);
+        umma_commit(&bars->pv_done[sb]);
+        umma_commit(&bars->kv_empty[i % nst]);
+      }
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    // Warpgroup wg = warp / 4 owns the tiles j with j % 2 == wg (all 64 keys of its
+    // 32 rows); the two warps of a row quarter work on alternate tiles, so one
+    // computes while the other waits. The online reference max of a row is handed
+    // from each tile to the next through shared memory.
+    const int wg = warp >> 2;
+    const int q4 = warp & 3;          // row quarter = TMEM lane quarter
+    const int r = q4 * 32 + lane;     // row = TMEM lane
+    const int tt = r / G, hh = r % G;
+    const int t = t0 + tt;
+    const bool valid = t < L;
+    const int64_t n = tok0 + t;
+    const int hq = g * G + hh;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const float sc = a.scale_log2;    // raw score -> log2 units
+    float gc = 0.f, gsl = 0.f, gw = 0.f;
+    if (valid) {
+      const float* gp = a.gates + ((size_t)n * a.H_q + hq) * 3;
+      gc = gp[0];
+      gsl = gp[1];
+      gw = gp[2];
+    }
+    const int jt = t / a.ls;
+    float* imp_row = a.imp + ((size_t)n * a.H_kv + g) * a.nb_stride;
+
+    bool ok = true;
+    // waits give one answer per warp (the tensor-memory accesses after them are warp-wide)
+    auto uwait = [&](uint64_t* bar, int parity, uint32_t site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)parity, abort_flag, a.status, site));
+    };
+    int xcnt = 0;
+    // value of the other warpgroup for this row (both warps of the quarter call it in step)
+    auto exchange = [&](float mine) -> float {
+      const int slot = xcnt & 1;
+      xch[(slot * 2 + wg) * 128 + r] = mine;
+      mbar_arrive(&bars->xbar[q4]);
+      const bool w = uwait(&bars->xbar[q4], xcnt & 1, 421);
+      ++xcnt;
+      if (!w) ok = false;
+      return xch[(slot * 2 + (1 - wg)) * 128 + r];
+    };
+    // Every tile is handled in two halves of 32 keys (S re-read from tensor memory
+    // where a second pass needs it), so a thread holds 32 scores at a time.
+    float sv[32];
+    int cur_b = 0;   // S/P buffer of the tile being processed (tile j uses buffer j % 4)
+    auto wait_s = [&](int j) -> bool {
+      cur_b = j & (kSBuf - 1);
+      if (!uwait(&bars->s_full[cur_b], (j >> 2) & 1, 422)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // raw scores of keys 32*hf .. 32*hf + 31 of the current tile
+    auto ld_half = [&](int hf) {
+      const uint32_t src = tmem + lane_base + col_s(cur_b) + 32u * hf;
+      tmem_ld16(src, sv);
+      tmem_ld16(src + 16, sv + 16);
+      tmem_ld_wait();
+    };
+    // bf16 P of keys 32*hf .. into columns 16*hf .. of the buffer (S there already read)
+    auto st_half = [&](int hf, float scale) {
+#pragma unroll
+      for (int c = 0; c < 16; c += 8) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(sv[2 * (c + i)] * scale, sv[2 * (c + i) + 1] * scale);
+        tmem_st8(tmem + lane_base + col_s(cur_b) + 16u * hf + c, pk);
+      }
+    };
+    // all S reads of the tile are done (and its P written)
+    auto tile_done = [&](bool with_p) {
+      if (with_p) tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->s_free[cur_b]);
+      if (with_p) mbar_arrive(&bars->p_full[cur_b]);
+    };
+    // P.V of tile i (>= nkc) has finished; p_full / pv_done phases count P.V tiles per buffer
+    auto wait_pv = [&](int i) -> bool {
+      if (!uwait(&bars->pv_done[i & (kSBuf - 1)], ((i - nkc) >> 2) & 1, 424)) return false;
+      tc_fence_after();
+      return true;
+    };
+
+    // ---------------- C1: compressed keys, row max and denominator (per warpgroup, merged)
+    const int nvis = valid ? cmp_visible_dev(t, a.l, a.s) : 0;
+    float m = -1e30f, lp = 0.f;   // raw units
+    for (int j = wg; j < nkc; j += 2) {
+      if (ok) ok = wait_s(j);
+      const bool part = !__all_sync(0xffffffffu, j * kKeys + kKeys <= nvis);
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        if (ok) ld_half(hf);
+        const int c0 = j * kKeys + 32 * hf;
+        if (part) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
+        }
+        const float mn = fmaxf(m, tree_max<32>(sv));
+        const float mo = -mn * sc;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
+        lp = lp * ex2((m - mn) * sc) + tree_sum<32>(sv);
+        m = mn;
+      }
+      if (ok) tile_done(false);
+    }
+    float linv = 0.f, mo_c = 0.f;
+    if (nkc > 0) {   // merge the two warpgroups' (max, sum) in a fixed order
+      const float m_o = exchange(m);
+      const float l_o = exchange(lp);
+      const float m0 = wg == 0 ? m : m_o, m1 = wg == 0 ? m_o : m;
+      const float l0 = wg == 0 ? lp : l_o, l1 = wg == 0 ? l_o : lp;
+      const float mm = fmaxf(m0, m1);
+      const float lc = l0 * ex2((m0 - mm) * sc) + l1 * ex2((m1 - mm) * sc);
+      linv = lc > 0.f ? 1.f / lc : 0.f;
+      mo_c = -mm * sc;
+    }
+
+    // ---------------- C2: probabilities, importance, O_A = g_cmp * P.V_cmp
+    // compressed key i' = 4u' + u spans tokens [16i', 16i' + 32): u in {0,1,2} puts
+    // 2p on selection block u', u = 3 puts p on u' and u' + 1 (overlap / stride).
+    // Each half of a tile covers 8 blocks; the mass carried past the first half
+    // is added here, the one carried past the tile before the selection.
+    for (int i = 0; i < nkc; ++i) {
+      const int j = nkc + i;
+      if ((j & 1) != wg) continue;
+      if (ok) ok = wait_s(j);
+      const bool part = !__all_sync(0xffffffffu, i * kKeys + kKeys <= nvis);
+      float cin = 0.f;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        if (ok) ld_half(hf);
+        const int c0 = i * kKeys + 32 * hf;
+        if (part) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo_c)) * linv;
+        if (ok) st_half(hf, gc);
+        float blk[8];
+#pragma unroll
+        for (int qb = 0; qb < 8; ++qb) blk[qb] = 2.f * (sv[4 * qb] + sv[4 * qb + 1] + sv[4 * qb + 2]) + sv[4 * qb + 3];
+#pragma unroll
+        for (int qb = 0; qb < 7; ++qb) blk[qb + 1] += sv[4 * qb + 3];
+#pragma unroll
+        for (int qb = 0; qb < 8; ++qb) blk[qb] = group_sum(blk[qb], G);
+        const float carry = group_sum(sv[31], G);
+        blk[0] += cin;
+        const int B0 = 16 * i + 8 * hf;
+        if (valid && ok) {
+          for (int qb = hh; qb < 8; qb += G)
+            if (B0 + qb <= jt) imp_row[B0 + qb] = blk[qb];
+          if (hf == 1 && hh == 0) cbuf[i * TOK + tt] = carry;
+        }
+        cin = carry;
+      }
+      if (ok) tile_done(true);
+    }
+
+    // ---------------- top-n per token and the tile's union of selected blocks
+    int smx_phase = 0;
+    auto sm_sync = [&]() {
+      mbar_arrive(&bars->smx);
+      if (!uwait(&bars->smx, smx_phase & 1, 425)) ok = false;
+      ++smx_phase;
+    };
+    sm_sync();
+    for (int tk = warp; tk < TOK && ok; tk += 8) {
+      const int tq = t0 + tk;
+      if (tq >= L) break;
+      const int64_t nq = tok0 + tq;
+      const int jq = tq / a.ls;
+      float* irow = a.imp + ((size_t)nq * a.H_kv + g) * a.nb_stride;
+      // carried mass across compressed-tile boundaries (written by the other tile's warps)
+      for (int i = 1 + lane; i < nkc; i += 32)
+        if (16 * i <= jq) irow[16 * i] += cbuf[(i - 1) * TOK + tk];
+      if (nkc > 0) {
+        for (int jb = 16 * nkc + lane; jb <= jq; jb += 32)
+          irow[jb] = (jb == 16 * nkc) ? cbuf[(nkc - 1) * TOK + tk] : 0.f;
+      } else {
+        for (int jb = lane; jb <= jq; jb += 32) irow[jb] = 0.f;
+      }
+      __syncwarp();
+      int32_t* srow = a.sel + ((size_t)nq * a.H_kv + g) * a.top_n;
+      topn_any(irow, jq, a.top_n, a.force_first, a.force_local, srow, lane);
+      __syncwarp();
+      if (lane < a.top_n) {
+        const int jb = srow[lane];
+        if (jb >= 0) atomicOr(&bm[jb * MW + (tk >> 5)], 1u << (tk & 31));
+      }
+    }
+    sm_sync();
+    if (warp == 0 && ok) {
+      int cnt = 0;
+      for (int j0 = 0; j0 <= jt_max; j0 += 32) {
+        const int jb = j0 + lane;
+        bool any = false;
+        if (jb <= jt_max)
+          for (int w = 0; w < MW; ++w) any |= bm[jb * MW + w] != 0u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, any);
+        if (any) uni[cnt + __popc(bal & ((1u << lane) - 1u))] = jb;
+        cnt += __popc(bal);
+      }
+      if (lane == 0) bars->nu = cnt;
+    }
+    sm_sync();
+    if (tid == 0) mbar_arrive(&bars->sel_ready);
+    const int nu = ok ? bars->nu : 0;
+
+    // ---------------- online phases (window, selected blocks)
+    // Each tile takes the reference max left by the previous tile of the phase,
+    // raises it when its own max exceeds it by more than kRescaleLog2 (rescaling
+    // O_B once the previous product has landed) and hands it to the next tile.
+    const float thr = kRescaleLog2 / sc;
+    float r_last = -1e30f;   // reference this warp's partial sum lp is relative to
+    // mask_half(hf) masks the raw scores in sv of keys 32*hf .. of the tile
+    auto online_tile = [&](int j, int pfirst, bool skip, auto&& mask_half) -> bool {
+      float tmx = -1e30f;
+      if (!skip && ok) {
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          ld_half(hf);
+          mask_half(hf);
+          tmx = fmaxf(tmx, tree_max<32>(sv));
+        }
+      }
+      float m_in = -1e30f;
+      if (j > pfirst) {
+        const int ip = j - 1;
+        if (!uwait(&bars->hbar[q4][ip & 1], ((ip - first_w) >> 1) & 1, 426)) ok = false;
+        m_in = hslot[(ip & 1) * 128 + r];
+      }
+      float ref = m_in, alpha = 1.f;
+      if (tmx > ref + thr) {
+        alpha = ex2((ref - tmx) * sc);
+        ref = tmx;
+      }
+      hslot[(j & 1) * 128 + r] = ref;
+      mbar_arrive(&bars->hbar[q4][j & 1]);
+      if (!ok) return false;
+      lp *= ex2((r_last - m_in) * sc);   // tiles of the other warpgroup may have raised it
+      r_last = ref;
+      const bool had = m_in > -1e29f;
+      if (__any_sync(0xffffffffu, had && alpha != 1.f)) {
+        if (!wait_pv(j - 1)) return false;
+        tmem_scale_cols(tmem + lane_base + kColOB, DV, had ? alpha : 1.f);
+      }
+      lp *= alpha;
+      const float mo = -ref * sc;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        if (skip) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[c] = 0.f;
+        } else {
+          ld_half(hf);
+          mask_half(hf);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
+          lp += tree_sum<32>(sv);
+        }
+        st_half(hf, 1.f);
+      }
+      tile_done(true);
+      return true;
+    };
+    // denominator of the phase ending with tile j_last, both warpgroups summed in a fixed order
+    auto phase_sum = [&](int j_last) -> float {
+      if ((j_last & 1) != wg) {
+        if (!uwait(&bars->hbar[q4][j_last & 1], ((j_last - first_w) >> 1) & 1, 427)) ok = false;
+        const float m_fin = hslot[(j_last & 1) * 128 + r];
+        lp *= ex2((r_last - m_fin) * sc);
+      }
+      const float other = exchange(lp);
+      return wg == 0 ? lp + other : other + lp;
+    };
+
+    // ---------------- W: window keys into O_B, then O_A += g_win / l * O_B
+    const int wlo = t - a.window + 1;
+    lp = 0.f;
+    for (int i = 0; i < nkw; ++i) {
+      const int j = first_w + i;
+      if ((j & 1) != wg) continue;
+      if (ok) ok = wait_s(j);
+      const int k0 = key0w + i * kKeys;
+      const bool part = !__all_sync(0xffffffffu, valid && k0 >= wlo && k0 + kKeys - 1 <= t);
+      auto mask_w = [&](int hf) {
+        if (!part) return;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int tau = k0 + 32 * hf + c;
+          sv[c] = (valid && tau <= t && tau >= wlo) ? sv[c] : -INFINITY;
+        }
+      };
+      if (!online_tile(j, first_w, false, mask_w)) ok = false;
+    }
+    {
+      const float lw = phase_sum(first_s - 1);
+      if (ok) ok = wait_pv(first_s - 1);
+      const float sw = lw > 0.f ? gw / lw : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < DV / 2; c += 16) {
+        const uint32_t cb = lane_base + wg * (DV / 2) + c;
+        float ob[16], oa[16];
+        tmem_ld16(tmem + kColOB + cb, ob);
+        if (nkc > 0) tmem_ld16(tmem + kColOA + cb, oa);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = __float_as_uint((nkc > 0 ? oa[e] : 0.f) + sw * ob[e]);
+        tmem_st8(tmem + kColOA + cb, w);
+        tmem_st8(tmem + kColOA + cb + 8, w + 8);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->ob_free);
+    }
+
+    // ---------------- S: union blocks, each row masked to its token's selection
+    r_last = -1e30f;
+    lp = 0.f;
+    for (int u = 0; u < nu; ++u) {
+      const int j = first_s + u;
+      if ((j & 1) != wg) continue;
+      if (ok) ok = wait_s(j);
+      const int jb = uni[u];
+      const bool mine = valid && ((bm[jb * MW + (tt >> 5)] >> (tt & 31)) & 1u);
+      const int k0 = jb * a.ls;
+      // no row of this warp selected the block: its P rows are zero
+      const bool skip = !__any_sync(0xffffffffu, mine);
+      const bool part = !__all_sync(0xffffffffu, mine && k0 + kKeys - 1 <= t);
+      auto mask_s = [&](int hf) {
+        if (!part) return;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[c] = (mine && k0 + 32 * hf + c <= t) ? sv[c] : -INFINITY;
+      };
+      if (!online_tile(j, first_s, skip, mask_s)) ok = false;
+    }
+    {
+      const float ls_ = nu > 0 ? phase_sum(first_s + nu - 1) : 0.f;
+      if (ok && nu > 0) ok = wait_pv(first_s + nu - 1);
+      const float ss = ls_ > 0.f ? gsl / ls_ : 0.f;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + hq) * DV + wg * (DV / 2);
+#pragma unroll 1
+      for (int c = 0; c < DV / 2; c += 16) {
+        const uint32_t cb = lane_base + wg * (DV / 2) + c;
+        float ob[16], oa[16];
+        tmem_ld16(tmem + kColOB + cb, ob);
+        tmem_ld16(tmem + kColOA + cb, oa);
+        tmem_ld_wait();
+        if (valid && ok) {
+          uint4 pk0, pk1;
+          pk0.x = pack_bf16x2(fmaf(ss, ob[0], oa[0]), fmaf(ss, ob[1], oa[1]));
+          pk0.y = pack_bf16x2(fmaf(ss, ob[2], oa[2]), fmaf(ss, ob[3], oa[3]));
+          pk0.z = pack_bf16x2(fmaf(ss, ob[4], oa[4]), fmaf(ss, ob[5], oa[5]));
+          pk0.w = pack_bf16x2(fmaf(ss, ob[6], oa[6]), fmaf(ss, ob[7], oa[7]));
+          pk1.x = pack_bf16x2(fmaf(ss, ob[8], oa[8]), fmaf(ss, ob[9], oa[9]));
+          pk1.y = pack_bf16x2(fmaf(ss, ob[10], oa[10]), fmaf(ss, ob[11], oa[11]));
+          pk1.z = pack_bf16x2(fmaf(ss, ob[12], oa[12]), fmaf(ss, ob[13], oa[13]));
+          pk1.w = pack_bf16x2(fmaf(ss, ob[14], oa[14]), fmaf(ss, ob[15], oa[15]));
+          *reinterpret_cast<uint4*>(dst + c) = pk0;
+          *reinterpret_cast<uint4*>(dst + c + 8) = pk1;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// largest stage count that fits the opt-in shared memory of one CTA (0: none)
+static int fused_stages(int dk, int dv, int nb, int G) {
+  const size_t stage = (size_t)kKeys * (dk + dv) * 2;
+  const size_t budget = 232448 - 1024 - (size_t)128 * dk * 2 - fused_fixed_bytes(nb, G);
+  int n = (int)(budget / stage);
+  if (n > kMaxStages) n = kMaxStages;
+  return n >= 2 ? n : 0;
+}
+
+int prefill_fused_stages(const PrefillArgs& a) { return fused_stages(a.d_k, a.d_v, a.nb_stride, a.G); }
+
+template <int DK, int DV>
+static cudaError_t launch_fused_t(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
+  auto kern = nsa_prefill_kernel<DK, DV>;
+  const size_t smem =
+      1024 + (size_t)128 * DK * 2 + (size_t)a.n_stages * kKeys * (DK + DV) * 2 + fused_fixed_bytes(a.nb_stride, a.G);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(n_tiles, a.H_kv), kThreads, smem, st>>>(a, m);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_fused(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
+  if (n_tiles == 0) return cudaSuccess;
+  if (a.n_stages < 2 || a.n_stages > kMaxStages) return cudaErrorInvalidValue;
+  if (a.d_k == 192 && a.d_v == 128) return launch_fused_t<192, 128>(a, m, n_tiles, st);
+  if (a.d_k == 64 && a.d_v == 64) return launch_fused_t<64, 64>(a, m, n_tiles, st);
+  if (a.d_k == 128 && a.d_v == 128) return launch_fused_t<128, 128>(a, m, n_tiles, st);
+  if (a.d_k == 192 && a.d_v == 64) return launch_fused_t<192, 64>(a, m, n_tiles, st);
+  if (a.d_k == 64 && a.d_v == 128) return launch_fused_t<64, 128>(a, m, n_tiles, st);
+  if (a.d_k == 128 && a.d_v == 64) return launch_fused_t<128, 64>(a, m, n_tiles, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nsa
