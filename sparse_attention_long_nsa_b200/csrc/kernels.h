@@ -63,7 +63,8 @@ struct PrefillArgs {
   int H_q, H_kv, G, d_k, d_v;
   int l, s, ls, top_n, window, force_first, force_local;
   int nb_stride;
-  int n_stages;           // K/V ring depth of the fused kernel
+  int n_stages;           // K ring depth of the fused kernel
+  int n_vstages;          // V ring depth
   float scale_log2;       // softmax scale * log2(e)
   uint32_t* status;
   SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens
@@ -72,7 +73,7 @@ struct PrefillMaps {
   CUtensorMap k, v, kc, vc;   // boxes of 64 rows x 1 head x 64 elements
   CUtensorMap q;              // box of 128/G tokens x G heads x 64 elements (one query tile)
 };
-int prefill_fused_stages(const PrefillArgs& a);   // 0: does not fit in shared memory
+bool prefill_fused_stages(PrefillArgs& a);   // sets the ring depths; false: does not fit
 cudaError_t launch_prefill_fused(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st);
 
 // ----- decode -----

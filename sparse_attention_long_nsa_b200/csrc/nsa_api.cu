@@ -438,8 +438,7 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   a.nb_stride = w.nb;
   a.scale_log2 = softmax_scale(params, heads->d_k) * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws);
-  a.n_stages = prefill_fused_stages(a);
-  if (a.n_stages == 0) {
+  if (!prefill_fused_stages(a)) {
     snprintf(g_detail, sizeof(g_detail), "sequence too long for the fused prefill kernel (%d blocks)", w.nb);
     return NSA_ERR_UNSUPPORTED;
   }

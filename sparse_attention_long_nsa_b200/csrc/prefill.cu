@@ -26,13 +26,13 @@
 //
 // Every tile is 64 keys. Q sits in shared memory (A operand of S = Q.K^T); S has
 // four buffers in tensor memory and the softmax writes its bf16 P over the S
-// columns it has read (A operand of O += P.V). K and V stream through an n-stage
-// TMA ring. Roles (352 threads): warps 0-7 softmax, warpgroup wg = warp / 4
+// columns it has read (A operand of O += P.V). K and V stream through TMA rings. Roles (384 threads): warps 0-7 softmax, warpgroup wg = warp / 4
 // taking the tiles j with j % 2 == wg (warp w owns rows 32(w%4)..+31 and all 64
 // keys of the tile; the online reference max of a row passes from each tile to
-// the next through shared memory guarded by mbarriers); warp 8 TMA producer;
-// warp 9 issues the S = Q.K^T products (up to four tiles ahead of the softmax);
-// warp 10 the O += P.V products. Every wait is
+// the next through shared memory guarded by mbarriers); warp 8 loads Q and the
+// K tiles, warp 11 the V tiles (separate rings: a K tile is released as soon as
+// its S is computed); warp 9 issues the S = Q.K^T products (up to four tiles
+// ahead of the softmax); warp 10 the O += P.V products. Every wait is
 // time-bounded; on a timeout the CTA stops issuing work, lets its own copies and
 // products land and leaves.
 #include "common.cuh"
@@ -44,7 +44,7 @@ namespace nsa {
 namespace {
 
 constexpr int kKeys = 64;
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kSmThreads = 256;
 constexpr float kRescaleLog2 = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
 constexpr int kMaxStages = 8;
@@ -57,8 +57,8 @@ constexpr uint32_t kColOB = 384;  // branch in progress
 __device__ __forceinline__ uint32_t col_s(int b) { return kColS + 64u * (uint32_t)b; }
 
 struct FBars {
-  uint64_t kv_full[kMaxStages];
-  uint64_t kv_empty[kMaxStages];
+  uint64_t k_full[kMaxStages], k_empty[kMaxStages];   // K ring: released once S = Q.K^T is computed
+  uint64_t v_full[kMaxStages], v_empty[kMaxStages];   // V ring: released once O += P.V is computed
   uint64_t q_full, s_full[kSBuf], s_free[kSBuf], p_full[kSBuf], pv_done[kSBuf], ob_free, sel_ready, drain, smx;
   uint64_t xbar[4];      // pair exchange (rows of a quarter, both warpgroups)
   uint64_t hbar[4][2];   // reference-max hand-off from the tile of one parity to the next tile
@@ -142,7 +142,7 @@ __device__ __forceinline__ void topn_any(const float* imp, int jt, int top_n, in
 
 }  // namespace
 
-// dynamic shared memory: Q [d_k/64][128 rows][128 B] | ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
+// dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
 // block masks [nb][MW] | union [nb] | importance carries [nb/16 + 2][128/G] f32
 __host__ __device__ inline size_t fused_fixed_bytes(int nb, int G) {
   const int tok = 128 / G, mw = (tok + 31) / 32;
@@ -155,13 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
                                                                    const __grid_constant__ PrefillMaps mp) {
   constexpr int K_BYTES = kKeys * DK * 2;
   constexpr int V_BYTES = kKeys * DV * 2;
-  constexpr int STAGE = K_BYTES + V_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int nst = a.n_stages;
+  const int nks = a.n_stages, nvs = a.n_vstages;
   uint8_t* Qs = smem;                        // Q tile, 128-byte swizzled chunks of 64 columns
-  uint8_t* ring = smem + 128 * DK * 2;
-  FBars* bars = reinterpret_cast<FBars*>(ring + (size_t)nst * STAGE);
+  uint8_t* kring = smem + 128 * DK * 2;
+  uint8_t* vring = kring + (size_t)nks * K_BYTES;
+  FBars* bars = reinterpret_cast<FBars*>(vring + (size_t)nvs * V_BYTES);
   float* xch = reinterpret_cast<float*>(bars + 1);                 // [slot][warpgroup][row]
   float* hslot = xch + 512;                                        // [tile parity][row] reference max
   const int G = a.G;
@@ -187,9 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
 
   for (int i = tid; i < (jt_max + 1) * MW; i += kThreads) bm[i] = 0u;
   if (tid == 0) {
-    for (int i = 0; i < nst; ++i) {
-      mbar_init(&bars->kv_full[i], 1);
-      mbar_init(&bars->kv_empty[i], 1);
+    for (int i = 0; i < nks; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < nvs; ++i) {
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
     }
     mbar_init(&bars->q_full, 1);
     for (int i = 0; i < kSBuf; ++i) {   // tile j is read and written by warpgroup j & 1 only
@@ -218,43 +222,65 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ Q and K producer
     if (lane == 0) {
       prefetch_tmap(&mp.k);
-      prefetch_tmap(&mp.v);
       mbar_arrive_expect_tx(&bars->q_full, (uint32_t)(128 * DK * 2));
 #pragma unroll
-      for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Qs + kb * 16384, &mp.q, &bars->q_full, kb * 64, g * G, (int)(tok0 + t0));
+      for (int kb = 0; kb < DK / 64; ++kb)
+        tma_load_3d(Qs + kb * 16384, &mp.q, &bars->q_full, kb * 64, g * G, (int)(tok0 + t0));
       int issued = 0;
       bool ok = true;
-      auto load = [&](int j, const CUtensorMap* mk, const CUtensorMap* mv, int row, bool with_v) -> bool {
-        const int st = j % nst;
-        if (j >= nst && !mbar_wait(&bars->kv_empty[st], ((j / nst) - 1) & 1, abort_flag, a.status, 401))
+      auto load = [&](int j, const CUtensorMap* mk, int row) -> bool {
+        const int st = j % nks;
+        if (j >= nks && !mbar_wait(&bars->k_empty[st], ((j / nks) - 1) & 1, abort_flag, a.status, 401))
           return false;
-        uint8_t* Ks = ring + (size_t)st * STAGE;
-        mbar_arrive_expect_tx(&bars->kv_full[st], K_BYTES + (with_v ? V_BYTES : 0));
+        uint8_t* Ks = kring + (size_t)st * K_BYTES;
+        mbar_arrive_expect_tx(&bars->k_full[st], K_BYTES);
 #pragma unroll
-        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->kv_full[st], kb * 64, g, row);
-        if (with_v) {
-#pragma unroll
-          for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_3d(Ks + K_BYTES + vb * 8192, mv, &bars->kv_full[st], vb * 64, g, row);
-        }
+        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->k_full[st], kb * 64, g, row);
         issued = j + 1;
         return true;
       };
       int j = 0;
-      for (int i = 0; i < nkc && ok; ++i) ok = load(j++, &mp.kc, &mp.vc, (int)(cmp0 + i * kKeys), false);
-      for (int i = 0; i < nkc && ok; ++i) ok = load(j++, &mp.kc, &mp.vc, (int)(cmp0 + i * kKeys), true);
-      for (int i = 0; i < nkw && ok; ++i) ok = load(j++, &mp.k, &mp.v, (int)(tok0 + key0w + i * kKeys), true);
+      for (int pass = 0; pass < 2; ++pass)
+        for (int i = 0; i < nkc && ok; ++i) ok = load(j++, &mp.kc, (int)(cmp0 + i * kKeys));
+      for (int i = 0; i < nkw && ok; ++i) ok = load(j++, &mp.k, (int)(tok0 + key0w + i * kKeys));
       if (ok) ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 402);
       const int nu = ok ? bars->nu : 0;
-      for (int u = 0; u < nu && ok; ++u) ok = load(j++, &mp.k, &mp.v, (int)(tok0 + (int64_t)uni[u] * a.ls), true);
+      for (int u = 0; u < nu && ok; ++u) ok = load(j++, &mp.k, (int)(tok0 + (int64_t)uni[u] * a.ls));
       if (!ok) {   // let the copies still in flight land before the CTA exits
         mbar_wait_drain(&bars->q_full, 0);
-        for (int v = issued - nst < 0 ? 0 : issued - nst; v < issued; ++v)
-          mbar_wait_drain(&bars->kv_full[v % nst], (v / nst) & 1);
+        for (int v = issued - nks < 0 ? 0 : issued - nks; v < issued; ++v)
+          mbar_wait_drain(&bars->k_full[v % nks], (v / nks) & 1);
       }
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ V producer (tiles with P.V only)
+    if (lane == 0) {
+      prefetch_tmap(&mp.v);
+      int issued = 0;
+      bool ok = true;
+      auto load = [&](int vi, const CUtensorMap* mv, int row) -> bool {
+        const int st = vi % nvs;
+        if (vi >= nvs && !mbar_wait(&bars->v_empty[st], ((vi / nvs) - 1) & 1, abort_flag, a.status, 403))
+          return false;
+        uint8_t* Vs = vring + (size_t)st * V_BYTES;
+        mbar_arrive_expect_tx(&bars->v_full[st], V_BYTES);
+#pragma unroll
+        for (int vb = 0; vb < DV / 64; ++vb) tma_load_3d(Vs + vb * 8192, mv, &bars->v_full[st], vb * 64, g, row);
+        issued = vi + 1;
+        return true;
+      };
+      int vi = 0;
+      for (int i = 0; i < nkc && ok; ++i) ok = load(vi++, &mp.vc, (int)(cmp0 + i * kKeys));
+      for (int i = 0; i < nkw && ok; ++i) ok = load(vi++, &mp.v, (int)(tok0 + key0w + i * kKeys));
+      if (ok) ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 404);
+      const int nu = ok ? bars->nu : 0;
+      for (int u = 0; u < nu && ok; ++u) ok = load(vi++, &mp.v, (int)(tok0 + (int64_t)uni[u] * a.ls));
+      if (!ok)
+        for (int v = issued - nvs < 0 ? 0 : issued - nvs; v < issued; ++v)
+          mbar_wait_drain(&bars->v_full[v % nvs], (v / nvs) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ S = Q.K^T issuer
@@ -262,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     // S(j - 4) (pass 1) or P.V(j - 4) consumed the P written over it.
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(128, kKeys, false, false);
-      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(kring), 16, 1024);
       const uint64_t qdesc0 = umma_desc_sw128(smem_u32(Qs), 16, 1024);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.status, 411);
       int total = first_s;
@@ -273,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           total = first_s + bars->nu;
         }
         if (j >= total) break;
-        const int st = j % nst, sb = j & (kSBuf - 1);
-        ok = mbar_wait(&bars->kv_full[st], (j / nst) & 1, abort_flag, a.status, 415);
+        const int st = j % nks, sb = j & (kSBuf - 1);
+        ok = mbar_wait(&bars->k_full[st], (j / nks) & 1, abort_flag, a.status, 415);
         if (ok && j >= kSBuf) {
           // s_* barriers complete once per tile, p_full / pv_done once per P.V tile (index >= nkc)
           const int jp = j - kSBuf;
@@ -283,13 +309,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         }
         if (!ok) break;
         tc_fence_after();
-        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)st * STAGE) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)st * K_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
           umma_ss(tmem + col_s(sb), qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
                   kd + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_full[sb]);
-        if (j < nkc) umma_commit(&bars->kv_empty[st]);   // pass 1 reads K only
+        umma_commit(&bars->k_empty[st]);
       }
       // every product this thread issued has finished before tensor memory is released
       umma_commit(&bars->drain);
@@ -301,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     // releasing the stage after P.V(i) also covers the K half)
     if (lane == 0) {
       const uint32_t idesc_pv = umma_idesc_bf16(128, DV, false, true);
-      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring) + K_BYTES, 8192, 1024);
+      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(vring), 8192, 1024);
       bool ok = true;
       int total = first_s;
       for (int i = nkc; ok; ++i) {
@@ -311,21 +337,22 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           total = first_s + bars->nu;
         }
         if (i >= total) break;
-        const int sb = i & (kSBuf - 1);
-        ok = mbar_wait(&bars->p_full[sb], ((i - nkc) >> 2) & 1, abort_flag, a.status, 412) &&
+        const int sb = i & (kSBuf - 1), vi = i - nkc, vs = vi % nvs;
+        ok = mbar_wait(&bars->v_full[vs], (vi / nvs) & 1, abort_flag, a.status, 419) &&
+             mbar_wait(&bars->p_full[sb], ((i - nkc) >> 2) & 1, abort_flag, a.status, 412) &&
              (i != first_s || mbar_wait(&bars->ob_free, 0, abort_flag, a.status, 413));
         if (!ok) break;
         tc_fence_after();
         const bool first = (i == nkc) || (i == first_w) || (i == first_s);
         const uint32_t ocol = i < first_w ? kColOA : kColOB;
-        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)(i % nst) * STAGE) >> 4);
+        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)vs * V_BYTES) >> 4);
         // P (bf16 pairs, 32 columns) sits over the first half of the S columns of its buffer
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
           umma_ts(tmem + ocol, tmem + col_s(sb) + (uint32_t)(kk * 8), vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
                   (first && kk == 0) ? 0u : 1u);
         umma_commit(&bars->pv_done[sb]);
-        umma_commit(&bars->kv_empty[i % nst]);
+        umma_commit(&bars->v_empty[vs]);
       }
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
@@ -703,22 +730,24 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// largest stage count that fits the opt-in shared memory of one CTA (0: none)
-static int fused_stages(int dk, int dv, int nb, int G) {
-  const size_t stage = (size_t)kKeys * (dk + dv) * 2;
-  const size_t budget = 232448 - 1024 - (size_t)128 * dk * 2 - fused_fixed_bytes(nb, G);
-  int n = (int)(budget / stage);
+// K and V ring depths that fit the opt-in shared memory of one CTA (false: none)
+bool prefill_fused_stages(PrefillArgs& a) {
+  const size_t kb = (size_t)kKeys * a.d_k * 2, vb = (size_t)kKeys * a.d_v * 2;
+  const size_t budget = 232448 - 1024 - (size_t)128 * a.d_k * 2 - fused_fixed_bytes(a.nb_stride, a.G);
+  int n = (int)(budget / (kb + vb));
   if (n > kMaxStages) n = kMaxStages;
-  return n >= 2 ? n : 0;
+  if (n < 2) return false;
+  int nk = n + (int)((budget - (size_t)n * (kb + vb)) / kb);   // spare room holds extra K tiles
+  a.n_stages = nk > kMaxStages ? kMaxStages : nk;
+  a.n_vstages = n;
+  return true;
 }
-
-int prefill_fused_stages(const PrefillArgs& a) { return fused_stages(a.d_k, a.d_v, a.nb_stride, a.G); }
 
 template <int DK, int DV>
 static cudaError_t launch_fused_t(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
   auto kern = nsa_prefill_kernel<DK, DV>;
-  const size_t smem =
-      1024 + (size_t)128 * DK * 2 + (size_t)a.n_stages * kKeys * (DK + DV) * 2 + fused_fixed_bytes(a.nb_stride, a.G);
+  const size_t smem = 1024 + (size_t)128 * DK * 2 + (size_t)a.n_stages * kKeys * DK * 2 +
+                     (size_t)a.n_vstages * kKeys * DV * 2 + fused_fixed_bytes(a.nb_stride, a.G);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(n_tiles, a.H_kv), kThreads, smem, st>>>(a, m);
@@ -727,7 +756,8 @@ static cudaError_t launch_fused_t(const PrefillArgs& a, const PrefillMaps& m, in
 
 cudaError_t launch_prefill_fused(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
   if (n_tiles == 0) return cudaSuccess;
-  if (a.n_stages < 2 || a.n_stages > kMaxStages) return cudaErrorInvalidValue;
+  if (a.n_stages < 2 || a.n_stages > kMaxStages || a.n_vstages < 2 || a.n_vstages > kMaxStages)
+    return cudaErrorInvalidValue;
   if (a.d_k == 192 && a.d_v == 128) return launch_fused_t<192, 128>(a, m, n_tiles, st);
   if (a.d_k == 64 && a.d_v == 64) return launch_fused_t<64, 64>(a, m, n_tiles, st);
   if (a.d_k == 128 && a.d_v == 128) return launch_fused_t<128, 128>(a, m, n_tiles, st);
