@@ -459,6 +459,36 @@ def run_reference(args, rank, ws):
     }
 
 
+def run_case(case):
+    """Two untimed invocations of one workload, for kernel profilers (no JSON line):
+    prefill = compression + prefill of the 8K workload; decode = 8 sequences of the
+    64K decode workload."""
+    import sparse_attention_long_nsa_b200 as nsa
+    dev = torch.device("cuda", 0)
+    if case == "prefill":
+        cfg = PREFILL
+        inp = W.make_prefill_inputs(cfg, device=dev)
+        heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+        par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                              cfg.force_local)
+        for _ in range(2):
+            kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [cfg.T],
+                                  heads, par)
+            nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par)
+    else:
+        cfg = DECODE
+        inp = W.make_decode_inputs(cfg, device=dev, lens=[cfg.T] * 8)
+        heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+        par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                              cfg.force_local)
+        kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                    inp["pe_v"], inp["cache_lens"], heads, par)
+        lens = inp["cache_lens"].to(dev)
+        for _ in range(2):
+            nsa.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens, cfg.T, inp["gates"], heads, par)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,7 +497,12 @@ def main():
     ap.add_argument("--impl", choices=["nsa", "reference"], default="nsa")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["prefill", "decode"], default=None,
+                    help="run two untimed invocations of one workload for a profiler, print nothing")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank, ws = dist_setup(args.gpus)
