@@ -65,6 +65,8 @@ struct PrefillArgs {
   int nb_stride;
   int n_stages;           // K ring depth of the fused kernel
   int n_vstages;          // V ring depth
+  int imp_smem;           // importance and selections of the query tile kept in shared memory
+  int want_imp, want_sel; // caller asked for the importance / selection rows
   float scale_log2;       // softmax scale * log2(e)
   uint32_t* status;
   SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens

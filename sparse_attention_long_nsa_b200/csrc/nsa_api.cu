@@ -430,6 +430,8 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   a.q = q; a.k = k; a.v = v; a.kc = k_cmp; a.vc = v_cmp; a.gates = gates;
   a.imp = imp_out ? imp_out : (float*)(ws + w.imp);
   a.sel = sel_out ? sel_out : (int32_t*)(ws + w.sel);
+  a.want_imp = imp_out != nullptr;
+  a.want_sel = sel_out != nullptr;
   a.out = out;
   a.H_q = heads->H_q; a.H_kv = heads->H_kv; a.G = heads->H_q / heads->H_kv;
   a.d_k = heads->d_k; a.d_v = heads->d_v;

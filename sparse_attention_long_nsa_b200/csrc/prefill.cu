@@ -143,7 +143,8 @@ __device__ __forceinline__ void topn_any(const float* imp, int jt, int top_n, in
 }  // namespace
 
 // dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
-// block masks [nb][MW] | union [nb] | importance carries [nb/16 + 2][128/G] f32
+// block masks [nb][MW] | union [nb] | importance carries [nb/16 + 2][128/G] f32 |
+// (when it fits) importance [128/G][nb] f32 | selections [128/G][32] i32
 __host__ __device__ inline size_t fused_fixed_bytes(int nb, int G) {
   const int tok = 128 / G, mw = (tok + 31) / 32;
   return sizeof(FBars) + 2 * 2 * 128 * 4 + 2 * 128 * 4 + (size_t)nb * mw * 4 + (size_t)nb * 4 +
@@ -169,6 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   uint32_t* bm = reinterpret_cast<uint32_t*>(hslot + 256);         // [nb][MW] token bits per block
   int* uni = reinterpret_cast<int*>(bm + (size_t)a.nb_stride * MW);  // union of selected blocks
   float* cbuf = reinterpret_cast<float*>(uni + a.nb_stride);      // [compressed tile][token] carried mass
+  float* imp_s = cbuf + (size_t)(a.nb_stride / 16 + 2) * TOK;     // [token][nb] when a.imp_smem
+  int32_t* sel_s = reinterpret_cast<int32_t*>(imp_s + (size_t)TOK * a.nb_stride);   // [token][32]
   volatile int* abort_flag = &bars->abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       gw = gp[2];
     }
     const int jt = t / a.ls;
-    float* imp_row = a.imp + ((size_t)n * a.H_kv + g) * a.nb_stride;
+    float* imp_row = a.imp_smem ? imp_s + (size_t)tt * a.nb_stride : a.imp + ((size_t)n * a.H_kv + g) * a.nb_stride;
 
     bool ok = true;
     // waits give one answer per warp (the tensor-memory accesses after them are warp-wide)
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       if (tq >= L) break;
       const int64_t nq = tok0 + tq;
       const int jq = tq / a.ls;
-      float* irow = a.imp + ((size_t)nq * a.H_kv + g) * a.nb_stride;
+      float* irow = a.imp_smem ? imp_s + (size_t)tk * a.nb_stride : a.imp + ((size_t)nq * a.H_kv + g) * a.nb_stride;
       // carried mass across compressed-tile boundaries (written by the other tile's warps)
       for (int i = 1 + lane; i < nkc; i += 32)
         if (16 * i <= jq) irow[16 * i] += cbuf[(i - 1) * TOK + tk];
@@ -541,12 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         for (int jb = lane; jb <= jq; jb += 32) irow[jb] = 0.f;
       }
       __syncwarp();
-      int32_t* srow = a.sel + ((size_t)nq * a.H_kv + g) * a.top_n;
+      int32_t* gsel = a.sel + ((size_t)nq * a.H_kv + g) * a.top_n;
+      int32_t* srow = a.imp_smem ? sel_s + tk * 32 : gsel;
       topn_any(irow, jq, a.top_n, a.force_first, a.force_local, srow, lane);
       __syncwarp();
       if (lane < a.top_n) {
         const int jb = srow[lane];
         if (jb >= 0) atomicOr(&bm[jb * MW + (tk >> 5)], 1u << (tk & 31));
+        if (a.imp_smem && a.want_sel) gsel[lane] = jb;
+      }
+      if (a.imp_smem && a.want_imp) {
+        float* gimp = a.imp + ((size_t)nq * a.H_kv + g) * a.nb_stride;
+        for (int jb = lane; jb <= jq; jb += 32) gimp[jb] = irow[jb];
       }
     }
     sm_sync();
@@ -573,8 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     // O_B once the previous product has landed) and hands it to the next tile.
     const float thr = kRescaleLog2 / sc;
     float r_last = -1e30f;   // reference this warp's partial sum lp is relative to
-    // mask_half(hf) masks the raw scores in sv of keys 32*hf .. of the tile
-    auto online_tile = [&](int j, int pfirst, bool skip, auto&& mask_half) -> bool {
+    // mask_half(hf) masks the raw scores in sv of keys 32*hf .. of the tile; a row
+    // with rowv == false takes no part in the tile (max -inf, p = 0) at no per-key cost
+    auto online_tile = [&](int j, int pfirst, bool skip, bool rowv, auto&& mask_half) -> bool {
       float tmx = -1e30f;
       if (!skip && ok) {
 #pragma unroll 1
@@ -583,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           mask_half(hf);
           tmx = fmaxf(tmx, tree_max<32>(sv));
         }
+        if (!rowv) tmx = -1e30f;
       }
       float m_in = -1e30f;
       if (j > pfirst) {
@@ -606,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         tmem_scale_cols(tmem + lane_base + kColOB, DV, had ? alpha : 1.f);
       }
       lp *= alpha;
-      const float mo = -ref * sc;
+      const float mo = rowv ? -ref * sc : -INFINITY;
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
         if (skip) {
@@ -652,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           sv[c] = (valid && tau <= t && tau >= wlo) ? sv[c] : -INFINITY;
         }
       };
-      if (!online_tile(j, first_w, false, mask_w)) ok = false;
+      if (!online_tile(j, first_w, false, valid, mask_w)) ok = false;
     }
     {
       const float lw = phase_sum(first_s - 1);
@@ -688,13 +699,14 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const int k0 = jb * a.ls;
       // no row of this warp selected the block: its P rows are zero
       const bool skip = !__any_sync(0xffffffffu, mine);
-      const bool part = !__all_sync(0xffffffffu, mine && k0 + kKeys - 1 <= t);
+      // keys after t exist only in a row's own current block
+      const bool part = __any_sync(0xffffffffu, mine && k0 + kKeys - 1 > t);
       auto mask_s = [&](int hf) {
         if (!part) return;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c] = (mine && k0 + 32 * hf + c <= t) ? sv[c] : -INFINITY;
+        for (int c = 0; c < 32; ++c) sv[c] = (k0 + 32 * hf + c <= t) ? sv[c] : -INFINITY;
       };
-      if (!online_tile(j, first_s, skip, mask_s)) ok = false;
+      if (!online_tile(j, first_s, skip, mine, mask_s)) ok = false;
     }
     {
       const float ls_ = nu > 0 ? phase_sum(first_s + nu - 1) : 0.f;
@@ -731,13 +743,19 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
 }
 
 // K and V ring depths that fit the opt-in shared memory of one CTA (false: none)
+static size_t imp_smem_bytes(int nb, int G) { return (size_t)(128 / G) * (nb + 32) * 4; }
+
 bool prefill_fused_stages(PrefillArgs& a) {
   const size_t kb = (size_t)kKeys * a.d_k * 2, vb = (size_t)kKeys * a.d_v * 2;
-  const size_t budget = 232448 - 1024 - (size_t)128 * a.d_k * 2 - fused_fixed_bytes(a.nb_stride, a.G);
+  size_t budget = 232448 - 1024 - (size_t)128 * a.d_k * 2 - fused_fixed_bytes(a.nb_stride, a.G);
   int n = (int)(budget / (kb + vb));
   if (n > kMaxStages) n = kMaxStages;
   if (n < 2) return false;
-  int nk = n + (int)((budget - (size_t)n * (kb + vb)) / kb);   // spare room holds extra K tiles
+  budget -= (size_t)n * (kb + vb);
+  // the tile's importance and selections stay on chip when the room is left over
+  a.imp_smem = budget >= imp_smem_bytes(a.nb_stride, a.G) ? 1 : 0;
+  if (a.imp_smem) budget -= imp_smem_bytes(a.nb_stride, a.G);
+  int nk = n + (int)(budget / kb);   // spare room holds extra K tiles
   a.n_stages = nk > kMaxStages ? kMaxStages : nk;
   a.n_vstages = n;
   return true;
@@ -747,7 +765,8 @@ template <int DK, int DV>
 static cudaError_t launch_fused_t(const PrefillArgs& a, const PrefillMaps& m, int n_tiles, cudaStream_t st) {
   auto kern = nsa_prefill_kernel<DK, DV>;
   const size_t smem = 1024 + (size_t)128 * DK * 2 + (size_t)a.n_stages * kKeys * DK * 2 +
-                     (size_t)a.n_vstages * kKeys * DV * 2 + fused_fixed_bytes(a.nb_stride, a.G);
+                     (size_t)a.n_vstages * kKeys * DV * 2 + fused_fixed_bytes(a.nb_stride, a.G) +
+                     (a.imp_smem ? imp_smem_bytes(a.nb_stride, a.G) : 0);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(n_tiles, a.H_kv), kThreads, smem, st>>>(a, m);
