@@ -293,8 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const uint32_t idesc_qk = umma_idesc_bf16(128, kKeys, false, false);
       const uint64_t kdesc0 = umma_desc_sw128(smem_u32(kring), 16, 1024);
       const uint64_t qdesc0 = umma_desc_sw128(smem_u32(Qs), 16, 1024);
+      uint64_t qd[DK / 16];   // Q operand descriptors, fixed for the CTA
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk) qd[kk] = qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.status, 411);
       int total = first_s;
+      int st = 0;
+      uint32_t kph = 0;   // K ring slot of tile j and its phase parity
       for (int j = 0; ok; ++j) {
         if (j == first_s) {
           ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 414);
@@ -302,8 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           total = first_s + bars->nu;
         }
         if (j >= total) break;
-        const int st = j % nks, sb = j & (kSBuf - 1);
-        ok = mbar_wait(&bars->k_full[st], (j / nks) & 1, abort_flag, a.status, 415);
+        const int sb = j & (kSBuf - 1);
+        ok = mbar_wait(&bars->k_full[st], kph, abort_flag, a.status, 415);
         if (ok && j >= kSBuf) {
           // s_* barriers complete once per tile, p_full / pv_done once per P.V tile (index >= nkc)
           const int jp = j - kSBuf;
@@ -312,13 +317,18 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         }
         if (!ok) break;
         tc_fence_after();
-        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)st * K_BYTES) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)((uint32_t)st * (uint32_t)(K_BYTES >> 4));
+        const uint32_t dcol = tmem + col_s(sb);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          umma_ss(tmem + col_s(sb), qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                  kd + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss(dcol, qd[kk], kd + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), idesc_qk,
+                  kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_full[sb]);
         umma_commit(&bars->k_empty[st]);
+        if (++st == nks) {
+          st = 0;
+          kph ^= 1u;
+        }
       }
       // every product this thread issued has finished before tensor memory is released
       umma_commit(&bars->drain);
@@ -333,6 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const uint64_t vdesc0 = umma_desc_sw128(smem_u32(vring), 8192, 1024);
       bool ok = true;
       int total = first_s;
+      int vs = 0;
+      uint32_t vph = 0;   // V ring slot of P.V tile i and its phase parity
       for (int i = nkc; ok; ++i) {
         if (i == first_s) {
           ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 417);
@@ -340,15 +352,15 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           total = first_s + bars->nu;
         }
         if (i >= total) break;
-        const int sb = i & (kSBuf - 1), vi = i - nkc, vs = vi % nvs;
-        ok = mbar_wait(&bars->v_full[vs], (vi / nvs) & 1, abort_flag, a.status, 419) &&
+        const int sb = i & (kSBuf - 1);
+        ok = mbar_wait(&bars->v_full[vs], vph, abort_flag, a.status, 419) &&
              mbar_wait(&bars->p_full[sb], ((i - nkc) >> 2) & 1, abort_flag, a.status, 412) &&
              (i != first_s || mbar_wait(&bars->ob_free, 0, abort_flag, a.status, 413));
         if (!ok) break;
         tc_fence_after();
         const bool first = (i == nkc) || (i == first_w) || (i == first_s);
         const uint32_t ocol = i < first_w ? kColOA : kColOB;
-        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)vs * V_BYTES) >> 4);
+        const uint64_t vd = vdesc0 + (uint64_t)((uint32_t)vs * (uint32_t)(V_BYTES >> 4));
         // P (bf16 pairs, 32 columns) sits over the first half of the S columns of its buffer
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
@@ -356,6 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
                   (first && kk == 0) ? 0u : 1u);
         umma_commit(&bars->pv_done[sb]);
         umma_commit(&bars->v_empty[vs]);
+        if (++vs == nvs) {
+          vs = 0;
+          vph ^= 1u;
+        }
       }
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
