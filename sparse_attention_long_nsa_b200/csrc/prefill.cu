@@ -238,10 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         const int st = j % nks;
         if (j >= nks && !mbar_wait(&bars->k_empty[st], ((j / nks) - 1) & 1, abort_flag, a.status, 401))
           return false;
-        uint8_t* Ks = kring + (size_t)st * K_BYTES;
+        uint8_t* Ks = kring + (size_t)st * 8192;   // chunk kb of slot st at kb * nks * 8 KB + st * 8 KB
         mbar_arrive_expect_tx(&bars->k_full[st], K_BYTES);
 #pragma unroll
-        for (int kb = 0; kb < DK / 64; ++kb) tma_load_3d(Ks + kb * 8192, mk, &bars->k_full[st], kb * 64, g, row);
+        for (int kb = 0; kb < DK / 64; ++kb)
+          tma_load_3d(Ks + (size_t)kb * nks * 8192, mk, &bars->k_full[st], kb * 64, g, row);
         issued = j + 1;
         return true;
       };
@@ -288,45 +289,69 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   } else if (warp == 9) {
     // ------------------------------------------------------------ S = Q.K^T issuer
     // S(j) goes to buffer j % 4; the buffer is free again once the softmax read
-    // S(j - 4) (pass 1) or P.V(j - 4) consumed the P written over it.
+    // S(j - 4) (pass 1) or P.V(j - 4) consumed the P written over it. Tiles are
+    // taken in pairs (j even): their S buffers are adjacent columns and their K
+    // tiles adjacent rows of the ring (chunk-interleaved slots), so one N = 128
+    // product computes both.
     if (lane == 0) {
-      const uint32_t idesc_qk = umma_idesc_bf16(128, kKeys, false, false);
+      const uint32_t idesc_64 = umma_idesc_bf16(128, kKeys, false, false);
+      const uint32_t idesc_128 = umma_idesc_bf16(128, 2 * kKeys, false, false);
       const uint64_t kdesc0 = umma_desc_sw128(smem_u32(kring), 16, 1024);
       const uint64_t qdesc0 = umma_desc_sw128(smem_u32(Qs), 16, 1024);
       uint64_t qd[DK / 16];   // Q operand descriptors, fixed for the CTA
+      uint32_t koff[DK / 16]; // K operand offsets (16-byte units) inside a slot
 #pragma unroll
-      for (int kk = 0; kk < DK / 16; ++kk) qd[kk] = qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4);
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        qd[kk] = qdesc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4);
+        koff[kk] = (uint32_t)(kk >> 2) * (uint32_t)nks * (8192u >> 4) + (uint32_t)((kk & 3) * 32 >> 4);
+      }
+      auto buf_free = [&](int jj) -> bool {
+        if (jj < kSBuf) return true;
+        // s_* barriers complete once per tile, p_full / pv_done once per P.V tile (index >= nkc)
+        const int jp = jj - kSBuf, sb = jj & (kSBuf - 1);
+        return (jp >= nkc) ? mbar_wait(&bars->pv_done[sb], ((jp - nkc) >> 2) & 1, abort_flag, a.status, 416)
+                           : mbar_wait(&bars->s_free[sb], (jp >> 2) & 1, abort_flag, a.status, 418);
+      };
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.status, 411);
       int total = first_s;
+      bool known = false;
       int st = 0;
       uint32_t kph = 0;   // K ring slot of tile j and its phase parity
-      for (int j = 0; ok; ++j) {
-        if (j == first_s) {
+      for (int j = 0; ok;) {
+        if (!known && j + 1 >= first_s) {
           ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 414);
           if (!ok) break;
           total = first_s + bars->nu;
+          known = true;
         }
         if (j >= total) break;
+        const bool pair = j + 1 < total;   // j and st are even whenever a pair starts
         const int sb = j & (kSBuf - 1);
-        ok = mbar_wait(&bars->k_full[st], kph, abort_flag, a.status, 415);
-        if (ok && j >= kSBuf) {
-          // s_* barriers complete once per tile, p_full / pv_done once per P.V tile (index >= nkc)
-          const int jp = j - kSBuf;
-          ok = (jp >= nkc) ? mbar_wait(&bars->pv_done[sb], ((jp - nkc) >> 2) & 1, abort_flag, a.status, 416)
-                           : mbar_wait(&bars->s_free[sb], (jp >> 2) & 1, abort_flag, a.status, 418);
-        }
+        ok = mbar_wait(&bars->k_full[st], kph, abort_flag, a.status, 415) &&
+             (!pair || mbar_wait(&bars->k_full[st + 1], kph, abort_flag, a.status, 415)) && buf_free(j) &&
+             (!pair || buf_free(j + 1));
         if (!ok) break;
         tc_fence_after();
-        const uint64_t kd = kdesc0 + (uint64_t)((uint32_t)st * (uint32_t)(K_BYTES >> 4));
+        const uint64_t kd = kdesc0 + (uint64_t)((uint32_t)st * (8192u >> 4));
         const uint32_t dcol = tmem + col_s(sb);
+        if (pair) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-          umma_ss(dcol, qd[kk], kd + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), idesc_qk,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < DK / 16; ++kk) umma_ss(dcol, qd[kk], kd + koff[kk], idesc_128, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) umma_ss(dcol, qd[kk], kd + koff[kk], idesc_64, kk > 0 ? 1u : 0u);
+        }
         umma_commit(&bars->s_full[sb]);
         umma_commit(&bars->k_empty[st]);
-        if (++st == nks) {
-          st = 0;
+        if (pair) {
+          umma_commit(&bars->s_full[sb + 1]);
+          umma_commit(&bars->k_empty[st + 1]);
+        }
+        const int adv = pair ? 2 : 1;
+        j += adv;
+        st += adv;
+        if (st >= nks) {
+          st -= nks;
           kph ^= 1u;
         }
       }
@@ -772,7 +797,8 @@ bool prefill_fused_stages(PrefillArgs& a) {
   a.imp_smem = budget >= imp_smem_bytes(a.nb_stride, a.G) ? 1 : 0;
   if (a.imp_smem) budget -= imp_smem_bytes(a.nb_stride, a.G);
   int nk = n + (int)(budget / kb);   // spare room holds extra K tiles
-  a.n_stages = nk > kMaxStages ? kMaxStages : nk;
+  if (nk > kMaxStages) nk = kMaxStages;
+  a.n_stages = nk & ~1;   // even: tiles are computed in pairs of adjacent K slots
   a.n_vstages = n;
   return true;
 }
