@@ -179,7 +179,8 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
  *   sel_out      int32 out or NULL: [batch, H_kv, top_n], ascending, -1 padded
  *   imp_out      fp32 out or NULL: [batch, H_kv, n_blk(max_len)]
  * `max_len` (HOST) bounds the lengths and sizes the launch; lengths above it
- * are an error recorded in the device status word (the sequence is skipped). */
+ * are an error recorded in the device status word (the sequence is skipped).
+ * max_len above 262144 tokens returns NSA_ERR_UNSUPPORTED. */
 nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
                         const void* k_cmp_cache, const void* v_cmp_cache,
                         const int32_t* cache_lens, int32_t batch, int32_t Lmax, int32_t Lmax_cmp,
@@ -194,7 +195,7 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
  * the previous read, and resets them. Slot names: nsa_profile_slot_name(). The
  * events are created on first use and reused; this is the only state the
  * library keeps between calls. Returns NSA_ERR_CUDA if an event query fails. */
-#define NSA_PROFILE_SLOTS 6
+#define NSA_PROFILE_SLOTS 5
 nsa_status_t nsa_profile_enable(int32_t enable);
 nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots);
 const char* nsa_profile_slot_name(int32_t slot);

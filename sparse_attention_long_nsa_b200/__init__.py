@@ -30,7 +30,7 @@ NSA_NOALLOC_SCRATCH_BYTES = 4194304
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
             "nsa_compress_noalloc", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
-NSA_PROFILE_SLOTS = 6
+NSA_PROFILE_SLOTS = 5
 
 
 class NSAError(RuntimeError):

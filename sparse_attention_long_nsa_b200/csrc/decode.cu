@@ -10,9 +10,9 @@
 //   D1  split-K over the compressed cache, 512 keys per CTA: per-chunk online
 //       softmax state (o, m, l) per head, and per 64-key tile the block sums
 //       sum_i exp(s_i - m_ref) * omega(i, j) of the selection blocks it touches.
-//   D2  per (sequence, KV head): merge the chunks, normalise, finish
-//       g_cmp * o_cmp, reduce the block sums over the group's heads into the
-//       importance, run the top-n selection.
+//   D2  (at the start of the D3 CTA of each (sequence, KV head)): merge the
+//       chunks, normalise, finish g_cmp * o_cmp, reduce the block sums over the
+//       group's heads into the importance, run the top-n selection.
 //   D3  one CTA per (sequence, KV head) streams the union of the selected
 //       blocks and the window blocks once; one score tile serves both branches,
 //       each with its own softmax; it writes
@@ -72,7 +72,7 @@ __host__ __device__ inline PartLayout part_layout(const DecodeArgs& a) {
   p.fp_o = p.tp + BG * p.n_tiles * kTP * a.G;                      // [BG][nsw][2][G][DV]
   p.fp_ml = p.fp_o + BG * a.n_sw_chunks * 2 * a.G * a.d_v;         // [BG][nsw][2][G][2]
   p.cnt = p.fp_ml + BG * a.n_sw_chunks * 2 * a.G * 2;              // [BG] int counters
-  p.total = p.cnt + BG;
+  p.total = p.cnt + BG + 16;   // slack: bulk copies round their size up to 16 bytes
   return p;
 }
 
@@ -313,98 +313,6 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
 }
 
 // ---------------------------------------------------------------------------
-// D2: merge compressed chunks, importance, selection (one CTA per (b, g))
-// ---------------------------------------------------------------------------
-constexpr int kSelThreadsD2 = 256;
-
-template <int DV, int PER>
-__global__ void __launch_bounds__(kSelThreadsD2) dec_select_kernel(const DecodeArgs a) {
-  extern __shared__ float sm[];
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int G = a.G;
-  const int L = a.lens[b];
-  if (L < 1 || L > a.max_len) return;
-  const int nc = n_cmp_dev(L, a.l, a.s);
-  const int nch = (nc + kCmpChunk - 1) / kCmpChunk;
-  const int ntl = (nc + kTileKeys - 1) / kTileKeys;
-  const int t = L - 1;
-  const int jt = t / a.ls;
-  const PartLayout pl = part_layout(a);
-  const size_t bg = (size_t)b * a.H_kv + g;
-  float* Mh = sm;                           // [16]
-  float* Li = sm + 16;                      // [16] 1/L
-  float* Fc = sm + 32;                      // [nch][16]   chunk factors
-  float* Ft = Fc + a.n_cmp_chunks * 16;     // [ntl][16]   tile factors (incl. 1/L)
-  float* imp_s = Ft + pl.n_tiles * 16;      // [nb_stride]
-  const float* cpo = a.part + pl.cp_o + bg * a.n_cmp_chunks * G * DV;
-  const float* cpm = a.part + pl.cp_ml + bg * a.n_cmp_chunks * G * 2;
-  const float* tp = a.part + pl.tp + bg * pl.n_tiles * kTP * G;
-  if (tid == 0) reinterpret_cast<int*>(a.part + pl.cnt)[bg] = 0;   // D3 completion counter
-  if (tid < G) {
-    float M = -1e30f;
-    for (int c = 0; c < nch; ++c)
-      if (cpm[(c * G + tid) * 2 + 1] > 0.f) M = fmaxf(M, cpm[(c * G + tid) * 2]);
-    float Ls = 0.f;
-    for (int c = 0; c < nch; ++c) {
-      const float l = cpm[(c * G + tid) * 2 + 1];
-      const float f = l > 0.f ? exp2f(cpm[(c * G + tid) * 2] - M) : 0.f;
-      Fc[c * 16 + tid] = f;
-      Ls += f * l;
-    }
-    Mh[tid] = M;
-    Li[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < ntl * G; idx += kSelThreadsD2) {
-    const int tj = idx / G, h = idx % G;
-    Ft[tj * 16 + h] = exp2f(tp[(size_t)tj * kTP * G + h] - Mh[h]) * Li[h];
-  }
-  // g_cmp * o_cmp, 4 values per thread
-  for (int idx = tid; idx < G * (DV / 4); idx += kSelThreadsD2) {
-    const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < nch; ++c) {
-      const float f = Fc[c * 16 + h];
-      const float4 v = *reinterpret_cast<const float4*>(cpo + ((size_t)c * G + h) * DV + c4);
-      acc.x += f * v.x; acc.y += f * v.y; acc.z += f * v.z; acc.w += f * v.w;
-    }
-    const int hq = g * G + h;
-    const float sc = a.gates[((size_t)b * a.H_q + hq) * 3 + 0] * Li[h];
-    *reinterpret_cast<float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4) =
-        make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
-  }
-  __syncthreads();
-  // importance of blocks 0..jt: tile tj holds blocks kBlkPerTile*tj .. + kBlkPerTile
-  for (int j = tid; j <= jt; j += kSelThreadsD2) {
-    const int tj = j / kBlkPerTile, q = j % kBlkPerTile;
-    float v = 0.f;
-    auto head_sum = [&](int tile, int rowi) -> float {
-      const float* r = tp + ((size_t)tile * kTP + rowi) * G;
-      const float* f = Ft + tile * 16;
-      float acc = 0.f;
-      if ((G & 3) == 0) {
-#pragma unroll 4
-        for (int h = 0; h < G; h += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(r + h);
-          const float4 y = *reinterpret_cast<const float4*>(f + h);
-          acc += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
-        }
-      } else {
-        for (int h = 0; h < G; ++h) acc += f[h] * r[h];
-      }
-      return acc;
-    };
-    if (tj < ntl) v += head_sum(tj, 1 + q);
-    if (q == 0 && tj >= 1 && tj - 1 < ntl) v += head_sum(tj - 1, 1 + kBlkPerTile);
-    imp_s[j] = v;
-    a.imp[bg * a.nb_stride + j] = v;
-  }
-  __syncthreads();
-  if (tid < 32)
-    warp_topn<PER>(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, tid);
-}
-
-// ---------------------------------------------------------------------------
 // D3: selected blocks and window for one (sequence, KV head) per CTA. The
 // ascending union of the selected blocks and the blocks the window touches is
 // streamed once through the TMA ring in 32-key halves; consumer warp w takes
@@ -425,6 +333,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   int* nuni = uni + 64;
   volatile int* abort_flag = nuni + 1;
   uint32_t* flags = reinterpret_cast<uint32_t*>(nuni + 2);     // [64] 1 = selected block
+  uint64_t* d2bar = reinterpret_cast<uint64_t*>(flags + 64);    // bulk copy of the chunk partials
   uint8_t* qs = smem + S::BODY;                                 // Q: DK/64 chunks of [16 rows][128 B]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -438,8 +347,117 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
 
   if (tid == 0) {
     for (int k = 0; k < kDecStages; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
+    mbar_init(d2bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  __syncthreads();
+  // ---- D2 (in this CTA, before the ring is used): merge the compressed chunks of
+  // (b, g), finish g_cmp * o_cmp, form the importance, select the top-n blocks
+  {
+    const PartLayout pl = part_layout(a);
+    const int nc = n_cmp_dev(L, a.l, a.s);
+    const int nch = (nc + kCmpChunk - 1) / kCmpChunk;   // <= 32 (checked on the host)
+    const int ntl = (nc + kTileKeys - 1) / kTileKeys;
+    float* Mh = reinterpret_cast<float*>(ring);   // [16] max per head
+    float* Li = Mh + 16;                          // [16] 1 / denominator
+    float* Fc = Mh + 32;                          // [nch][16] chunk factors
+    float* Ft = Fc + a.n_cmp_chunks * 16;         // [ntl][16] tile factors (incl. 1/L)
+    float* imp_s = Ft + pl.n_tiles * 16;          // [nb_stride]
+    const float* cpo = a.part + pl.cp_o + bg * a.n_cmp_chunks * G * DV;
+    const float* cpm = a.part + pl.cp_ml + bg * a.n_cmp_chunks * G * 2;
+    const float* tp = a.part + pl.tp + bg * pl.n_tiles * kTP * G;
+    // the tile partials and chunk outputs come into shared memory with two bulk
+    // copies when they fit next to the scratch (otherwise they are read in place)
+    float* tp_s = imp_s + ((a.nb_stride + 3) & ~3);
+    const uint32_t tp_bytes = (uint32_t)(((size_t)ntl * kTP * G * 4 + 15) & ~size_t(15));
+    float* cpo_s = tp_s + tp_bytes / 4;
+    const uint32_t cpo_bytes = (uint32_t)((size_t)nch * G * DV * 4);
+    const bool bulk = (size_t)((uint8_t*)cpo_s - ring) + cpo_bytes <= (size_t)S::BODY && nc > 0;
+    if (bulk) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(d2bar, tp_bytes + cpo_bytes);
+        bulk_load(tp_s, tp, tp_bytes, d2bar);
+        bulk_load(cpo_s, cpo, cpo_bytes, d2bar);
+      }
+      const bool got = mbar_wait(d2bar, 0, abort_flag, a.status, 410);
+      if (__syncthreads_or(!got)) {   // one decision for the whole CTA
+        if (tid == 0) mbar_wait_drain(d2bar, 0);   // let the copies land before the CTA leaves
+        return;
+      }
+      tp = tp_s;
+      cpo = cpo_s;
+    }
+    // one warp per head, the chunks in its lanes
+    for (int h = warp; h < G; h += kDecThreads / 32) {
+      float m = -1e30f, l = 0.f;
+      if (lane < nch) {
+        m = cpm[(lane * G + h) * 2];
+        l = cpm[(lane * G + h) * 2 + 1];
+      }
+      float M = l > 0.f ? m : -1e30f;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      const float f = (lane < nch && l > 0.f) ? exp2f(m - M) : 0.f;
+      float Ls = f * l;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+      if (lane < nch) Fc[lane * 16 + h] = f;
+      if (lane == 0) {
+        Mh[h] = M;
+        Li[h] = Ls > 0.f ? 1.f / Ls : 0.f;
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < ntl * G; idx += kDecThreads) {
+      const int tj = idx / G, h = idx % G;
+      Ft[tj * 16 + h] = exp2f(tp[(size_t)tj * kTP * G + h] - Mh[h]) * Li[h];
+    }
+    // g_cmp * o_cmp, 4 values per thread
+    for (int idx = tid; idx < G * (DV / 4); idx += kDecThreads) {
+      const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int c = 0; c < nch; ++c) {
+        const float fc = Fc[c * 16 + h];
+        const float4 v = *reinterpret_cast<const float4*>(cpo + ((size_t)c * G + h) * DV + c4);
+        acc.x += fc * v.x; acc.y += fc * v.y; acc.z += fc * v.z; acc.w += fc * v.w;
+      }
+      const int hq = g * G + h;
+      const float sc = a.gates[((size_t)b * a.H_q + hq) * 3 + 0] * Li[h];
+      *reinterpret_cast<float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4) =
+          make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
+    }
+    __syncthreads();
+    // importance of blocks 0..jt: tile tj holds blocks kBlkPerTile*tj .. + kBlkPerTile
+    for (int j = tid; j <= jt; j += kDecThreads) {
+      const int tj = j / kBlkPerTile, q = j % kBlkPerTile;
+      float v = 0.f;
+      auto head_sum = [&](int tile, int rowi) -> float {
+        const float* rr = tp + ((size_t)tile * kTP + rowi) * G;
+        const float* ff = Ft + tile * 16;
+        float acc = 0.f;
+        if ((G & 3) == 0) {
+#pragma unroll 4
+          for (int h = 0; h < G; h += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(rr + h);
+            const float4 y = *reinterpret_cast<const float4*>(ff + h);
+            acc += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+          }
+        } else {
+          for (int h = 0; h < G; ++h) acc += ff[h] * rr[h];
+        }
+        return acc;
+      };
+      if (tj < ntl) v += head_sum(tj, 1 + q);
+      if (q == 0 && tj >= 1 && tj - 1 < ntl) v += head_sum(tj - 1, 1 + kBlkPerTile);
+      imp_s[j] = v;
+      a.imp[bg * a.nb_stride + j] = v;
+    }
+    __syncthreads();
+    if (warp == 0)
+      warp_topn_any(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, lane);
+    __syncthreads();
   }
   {
     const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
@@ -452,45 +470,63 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   }
   if (warp == 0) {
     // union of the selected blocks (ascending, -1 padded) and the window blocks
-    // [wlo / l', jt], merged with a ballot over the candidate range
+    // [wlo / l', jt]: the selected blocks below the window first, then the window
+    // blocks, each flagged when it was also selected
     const int32_t* sel = a.sel + bg * a.top_n;
     const int wb = wlo / a.ls;
-    int cnt = 0, si = 0;
+    const int nwin = jt - wb + 1;
     int ns = 0;
     for (int i = lane; i < a.top_n; i += 32) ns += sel[i] >= 0;
     ns = __reduce_add_sync(0xffffffffu, ns);
-    // walk block indices in chunks of 32: a block is in the union if it is
-    // selected or inside the window range
-    int next_sel = ns > 0 ? sel[0] : 0x7fffffff;
-    for (int j0 = 0; j0 <= jt; j0 += 32) {
-      // skip chunks with neither a selected block nor window blocks
-      if (j0 + 31 < wb && next_sel > j0 + 31) {
-        // jump to the chunk of whichever comes first: the next selected block or the window
-        const int target = next_sel < wb ? next_sel : wb;
-        j0 = (target / 32) * 32 - 32;
-        continue;
+    if (nwin <= 32 && ns <= 32) {
+      const int si = lane < ns ? sel[lane] : 0x7fffffff;
+      const bool below = lane < ns && si < wb;
+      const uint32_t bb = __ballot_sync(0xffffffffu, below);
+      const int nbelow = __popc(bb);
+      if (below) {
+        const int pos = __popc(bb & ((1u << lane) - 1u));
+        uni[pos] = si;
+        flags[pos] = 1u;
       }
-      const int j = j0 + lane;
-      bool is_sel = false;
-      for (int i = si; i < ns; ++i) {
-        const int v = sel[i];
-        if (v > j0 + 31) break;
-        is_sel |= (v == j);
+      const uint32_t wsel =
+          __reduce_or_sync(0xffffffffu, (lane < ns && si >= wb && si <= jt) ? 1u << (si - wb) : 0u);
+      if (lane < nwin && nbelow + lane < 64) {
+        uni[nbelow + lane] = wb + lane;
+        flags[nbelow + lane] = (wsel >> lane) & 1u;
       }
-      const bool in = j <= jt && (is_sel || j >= wb);
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-        if (pos < 64) {
-          uni[pos] = j;
-          flags[pos] = is_sel ? 1u : 0u;
+      if (lane == 0) *nuni = nbelow + nwin < 64 ? nbelow + nwin : 64;
+    } else {
+      // general walk over the candidate range in chunks of 32 blocks
+      int cnt = 0, sj = 0;
+      int next_sel = ns > 0 ? sel[0] : 0x7fffffff;
+      for (int j0 = 0; j0 <= jt; j0 += 32) {
+        if (j0 + 31 < wb && next_sel > j0 + 31) {   // neither a selected block nor the window here
+          const int target = next_sel < wb ? next_sel : wb;
+          j0 = (target / 32) * 32 - 32;
+          continue;
         }
+        const int j = j0 + lane;
+        bool is_sel = false;
+        for (int i = sj; i < ns; ++i) {
+          const int v = sel[i];
+          if (v > j0 + 31) break;
+          is_sel |= (v == j);
+        }
+        const bool in = j <= jt && (is_sel || j >= wb);
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+          if (pos < 64) {
+            uni[pos] = j;
+            flags[pos] = is_sel ? 1u : 0u;
+          }
+        }
+        cnt += __popc(bal);
+        while (sj < ns && sel[sj] <= j0 + 31) ++sj;
+        next_sel = sj < ns ? sel[sj] : 0x7fffffff;
       }
-      cnt += __popc(bal);
-      while (si < ns && sel[si] <= j0 + 31) ++si;
-      next_sel = si < ns ? sel[si] : 0x7fffffff;
+      if (lane == 0) *nuni = cnt < 64 ? cnt : 64;
     }
-    if (lane == 0) *nuni = cnt < 64 ? cnt : 64;
   }
   __syncthreads();
   const int nu = *nuni;
@@ -626,30 +662,6 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
     prof_end(P_DEC_CMP, st, 1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const int per = (a.nb_stride + 31) / 32;
-  const size_t sm2 = (32 + (size_t)a.n_cmp_chunks * 16 + (size_t)a.n_cmp_chunks * kTilesPerChunk * 16 +
-                      (size_t)a.nb_stride) * 4;
-  if (sm2 > 48 * 1024) {
-    cudaError_t e2 = cudaSuccess;
-    if (per <= 4) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    else if (per <= 8) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    else if (per <= 16) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    else if (per <= 32) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    else if (per <= 64) e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    else e2 = cudaFuncSetAttribute(dec_select_kernel<DV, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    if (e2 != cudaSuccess) return e2;
-  }
-  dim3 g2(a.H_kv, a.B);
-  prof_begin(P_DEC_SELECT, st);
-  if (per <= 4) dec_select_kernel<DV, 4><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else if (per <= 8) dec_select_kernel<DV, 8><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else if (per <= 16) dec_select_kernel<DV, 16><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else if (per <= 32) dec_select_kernel<DV, 32><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else if (per <= 64) dec_select_kernel<DV, 64><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else if (per <= 128) dec_select_kernel<DV, 128><<<g2, kSelThreadsD2, sm2, st>>>(a);
-  else return cudaErrorInvalidValue;
-  prof_end(P_DEC_SELECT, st, 1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prof_begin(P_DEC_FINE, st);
   k3<<<dim3(a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
   prof_end(P_DEC_FINE, st, 1);

@@ -12,7 +12,7 @@ constexpr int kMaxBatch = 128;
 // Opt-in per-kernel timing: CUDA events recorded on the launching stream around
 // each launch (see nsa_profile_enable / nsa_profile_read in include/nsa.h).
 enum ProfSlot {
-  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_SELECT, P_DEC_FINE, P_COUNT
+  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_FINE, P_COUNT
 };
 void prof_begin(int slot, cudaStream_t st);
 void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()

@@ -187,8 +187,7 @@ Profiler& prof() {
   return p;
 }
 
-const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_select",
-                                   "dec_fine"};
+const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_fine"};
 
 }  // namespace
 
@@ -284,6 +283,7 @@ size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* 
       DecodeArgs a{};
       fill_decode_args(a, heads, params, batch, max_len, n_cmp_of(max_len, params->l_cmp, params->stride),
                        max_len);
+      if (a.n_cmp_chunks > 32) return 0;
       return decode_ws(a).total;
     }
   }
@@ -502,6 +502,10 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
   if (max_union_blocks(params) > 64) return NSA_ERR_UNSUPPORTED;
   DecodeArgs a{};
   fill_decode_args(a, heads, params, batch, Lmax, Lmax_cmp, max_len);
+  if (a.n_cmp_chunks > 32) {   // the chunk merge holds one chunk per lane
+    snprintf(g_detail, sizeof(g_detail), "decode cache longer than 262144 tokens");
+    return NSA_ERR_UNSUPPORTED;
+  }
   const DecodeWs w = decode_ws(a);
   if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -128,18 +128,6 @@ __device__ __forceinline__ float group_sum(float x, int G) {
   return x;
 }
 
-__device__ __forceinline__ void topn_any(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
-                                         int lane) {
-  const int per = (jt + 32) / 32;   // candidates 0..jt
-  if (per <= 1) warp_topn<1>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 2) warp_topn<2>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 4) warp_topn<4>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 8) warp_topn<8>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 16) warp_topn<16>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 32) warp_topn<32>(imp, jt, top_n, ff, fl, out, lane);
-  else warp_topn_mem(imp, jt, top_n, ff, fl, out, lane);
-}
-
 }  // namespace
 
 // dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
@@ -587,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       __syncwarp();
       int32_t* gsel = a.sel + ((size_t)nq * a.H_kv + g) * a.top_n;
       int32_t* srow = a.imp_smem ? sel_s + tk * 32 : gsel;
-      topn_any(irow, jq, a.top_n, a.force_first, a.force_local, srow, lane);
+      warp_topn_any(irow, jq, a.top_n, a.force_first, a.force_local, srow, lane);
       __syncwarp();
       if (lane < a.top_n) {
         const int jb = srow[lane];

@@ -19,7 +19,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// All 32 lanes call it. imp: scores of blocks 0..jt (generic pointer).
+// All 32 lanes call it. imp: scores of blocks 0..jt (generic pointer). The free
+// slots are filled in top_n - ff - fl rounds of a warp arg-max: each round takes
+// the largest remaining score (the lowest block index among equal ones), marks
+// it in a per-lane bitmask and removes it; the marked and forced blocks are then
+// written in ascending order.
 template <int PER>
 __device__ __forceinline__ void warp_topn(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
                                           int lane) {
@@ -30,41 +34,53 @@ __device__ __forceinline__ void warp_topn(const float* imp, int jt, int top_n, i
   }
   const int need = top_n - ff - fl;   // K > top_n >= ff + fl: forced sets are disjoint
   uint32_t key[PER];
+  uint32_t chosen = 0u;   // bit i: block i*32 + lane taken
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int j = i * 32 + lane;
     const bool cand = j < K && j >= ff && j <= jt - fl;
-    key[i] = cand ? order_key(imp[j]) : 0u;   // 0 sorts below every real score
+    const bool forced = j < K && (j < ff || j > jt - fl);
+    key[i] = cand ? order_key(imp[j]) : 0u;   // every real score maps above 0
+    if (forced) chosen |= 1u << i;
   }
-  uint32_t x = 0;   // need-th largest candidate key
-  if (need > 0) {
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t y = x | (1u << bit);
-      int c = 0;
+  // (up to 8 scores per lane the scans are short chains; above that they are
+  // split into 8 independent chains joined by a tree)
+  constexpr int NP = PER <= 8 ? 1 : 8;
+  for (int round = 0; round < need; ++round) {
+    uint32_t part[NP];
 #pragma unroll
-      for (int i = 0; i < PER; ++i) c += key[i] >= y;
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= need) x = y;
-    }
+    for (int p = 0; p < NP; ++p) part[p] = key[p];
+#pragma unroll
+    for (int i = NP; i < PER; ++i) part[i % NP] = max(part[i % NP], key[i]);
+#pragma unroll
+    for (int w = NP / 2; w >= 1; w >>= 1)
+#pragma unroll
+      for (int p = 0; p < w; ++p) part[p] = max(part[p], part[p + w]);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, part[0]);
+    uint32_t eq[NP];   // bit i: key[i] == M
+#pragma unroll
+    for (int p = 0; p < NP; ++p) eq[p] = 0u;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) eq[i % NP] |= (key[i] == M ? 1u : 0u) << i;
+#pragma unroll
+    for (int w = NP / 2; w >= 1; w >>= 1)
+#pragma unroll
+      for (int p = 0; p < w; ++p) eq[p] |= eq[p + w];
+    // this lane's lowest block holding M, then the lowest over the warp
+    const uint32_t li = eq[0] ? (uint32_t)((__ffs(eq[0]) - 1) * 32 + lane) : 0xffffffffu;
+    const uint32_t jmin = __reduce_min_sync(0xffffffffu, li);
+    const uint32_t take = (lane == (int)(jmin & 31u)) ? (1u << (jmin >> 5)) : 0u;
+    chosen |= take;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if ((take >> i) & 1u) key[i] = 0u;
   }
-  int gt = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) gt += (need > 0) && key[i] > x;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  int ties_left = need - gt;
   int pos = 0;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
-    const int j = i * 32 + lane;
-    const bool forced = j < K && (j < ff || j > jt - fl);
-    const bool eq = need > 0 && key[i] == x && key[i] != 0u;
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    const int before = __popc(eqm & ((1u << lane) - 1u));
-    const bool take_eq = eq && before < ties_left;
-    ties_left -= min(__popc(eqm), max(ties_left, 0));
-    const bool chosen = forced || (need > 0 && key[i] > x) || take_eq;
-    const uint32_t cm = __ballot_sync(0xffffffffu, chosen);
-    if (chosen) out[pos + __popc(cm & ((1u << lane) - 1u))] = j;
+    const bool c = (chosen >> i) & 1u;
+    const uint32_t cm = __ballot_sync(0xffffffffu, c);
+    if (c) out[pos + __popc(cm & ((1u << lane) - 1u))] = i * 32 + lane;
     pos += __popc(cm);
   }
   for (int i = pos + lane; i < top_n; i += 32) out[i] = -1;
@@ -114,6 +130,19 @@ __device__ __forceinline__ void warp_topn_mem(const float* imp, int jt, int top_
     pos += __popc(cm);
   }
   for (int i = pos + lane; i < top_n; i += 32) out[i] = -1;
+}
+
+// Dispatch on the number of candidates 0..jt (register version up to 1024).
+__device__ __forceinline__ void warp_topn_any(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
+                                              int lane) {
+  const int per = (jt + 32) / 32;
+  if (per <= 1) warp_topn<1>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 2) warp_topn<2>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 4) warp_topn<4>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 8) warp_topn<8>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 16) warp_topn<16>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 32) warp_topn<32>(imp, jt, top_n, ff, fl, out, lane);
+  else warp_topn_mem(imp, jt, top_n, ff, fl, out, lane);
 }
 
 }  // namespace nsa
