@@ -26,15 +26,16 @@
 //
 // Every tile is 64 keys. Q sits in shared memory (A operand of S = Q.K^T); S has
 // four buffers in tensor memory and the softmax writes its bf16 P over the S
-// columns it has read (A operand of O += P.V). K and V stream through TMA rings. Roles (384 threads): warps 0-7 softmax, warpgroup wg = warp / 4
-// taking the tiles j with j % 2 == wg (warp w owns rows 32(w%4)..+31 and all 64
-// keys of the tile; the online reference max of a row passes from each tile to
-// the next through shared memory guarded by mbarriers); warp 8 loads Q and the
-// K tiles, warp 11 the V tiles (separate rings: a K tile is released as soon as
-// its S is computed); warp 9 issues the S = Q.K^T products (up to four tiles
-// ahead of the softmax); warp 10 the O += P.V products. Every wait is
-// time-bounded; on a timeout the CTA stops issuing work, lets its own copies and
-// products land and leaves.
+// columns it has read (A operand of O += P.V). K and V stream through TMA rings.
+// Roles (384 threads): warps 0-7 softmax: warp w owns the 32 rows of tensor-
+// memory lane quarter w % 4 and key columns 32 (w / 4) .. + 31 of every tile; the
+// two warps of a quarter trade their partial row maxima once per tile, so both
+// hold the same reference max. Warp 8 loads Q and the K tiles, warp 11 the V
+// tiles (separate rings: a K tile is released as soon as its S is computed);
+// warp 9 issues the S = Q.K^T products (tiles in pairs, up to four tiles ahead
+// of the softmax); warp 10 the O += P.V products. Every wait is time-bounded; on
+// a timeout the CTA stops issuing work, lets its own copies and products land
+// and leaves.
 #include "common.cuh"
 #include "kernels.h"
 #include "topn.cuh"
@@ -44,7 +45,7 @@ namespace nsa {
 namespace {
 
 constexpr int kKeys = 64;
-constexpr int kThreads = 384;
+constexpr int kThreads = 384;   // 8 softmax warps, K producer, S issuer, P.V issuer, V producer
 constexpr int kSmThreads = 256;
 constexpr float kRescaleLog2 = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
 constexpr int kMaxStages = 8;
@@ -60,8 +61,8 @@ struct FBars {
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];   // K ring: released once S = Q.K^T is computed
   uint64_t v_full[kMaxStages], v_empty[kMaxStages];   // V ring: released once O += P.V is computed
   uint64_t q_full, s_full[kSBuf], s_free[kSBuf], p_full[kSBuf], pv_done[kSBuf], ob_free, sel_ready, drain, smx;
-  uint64_t xbar[4];      // pair exchange (rows of a quarter, both warpgroups)
-  uint64_t hbar[4][2];   // reference-max hand-off from the tile of one parity to the next tile
+  uint64_t xbar[4];      // end-of-phase exchange between the two warps of a row quarter
+  uint64_t pbar[4];      // per-tile max exchange between the two warps of a row quarter
   uint32_t tmem_base;
   int abort;
   int nu;
@@ -123,20 +124,100 @@ __device__ __noinline__ void tmem_scale_cols(uint32_t col, int ncols, float alph
 }
 
 // head sum over the G consecutive lanes of one token
-__device__ __forceinline__ float group_sum(float x, int G) {
+template <int G>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
   for (int off = G >> 1; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
   return x;
 }
 
+// Sums each of the 8 values v[0..7] over the G lanes of a token by recursive
+// halving: at every step a lane keeps half of its values and trades the other
+// half with its partner, so 8 sums over 16 lanes take 8 shuffles instead of 32.
+// On return the lane holds the sums of blocks base .. base + max(1, 8/G) - 1 in
+// v[0..]; the return value is base.
+template <int G>
+__device__ __forceinline__ int group_reduce8(float* v, int lane) {
+  int base = 0;
+  int n = 8;
+#pragma unroll
+  for (int off = G >> 1; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool up = (lane & off) != 0;
+      const int h = n >> 1;
+#pragma unroll
+      for (int k = 0; k < h; ++k) {
+        const float send = up ? v[k] : v[k + h];
+        const float keep = up ? v[k + h] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+      if (up) base += h;
+      n = h;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+  return base;
+}
+
+// Importance of the 8 selection blocks B0 .. B0+7 covered by 32 compressed keys
+// (probabilities h[0..31] of one row), summed over the G heads of the token and
+// written to imp_row by one lane per block; `cin` is the mass carried into block
+// B0 from the previous 32 keys. Returns the mass carried past block B0 + 7.
+template <int G>
+__device__ __forceinline__ float importance32(const float* h, float cin, int lane, bool write, float* imp_row,
+                                              int B0, int jt) {
+  float v[8];
+#pragma unroll
+  for (int qb = 0; qb < 8; ++qb) v[qb] = 2.f * (h[4 * qb] + h[4 * qb + 1] + h[4 * qb + 2]) + h[4 * qb + 3];
+#pragma unroll
+  for (int qb = 0; qb < 7; ++qb) v[qb + 1] += h[4 * qb + 3];
+  const float carry = group_sum<G>(h[31]);
+  const int base = group_reduce8<G>(v, lane);
+  constexpr int kHeld = G >= 8 ? 1 : 8 / G;
+  constexpr int kDup = G > 8 ? G / 8 - 1 : 0;   // lanes holding copies of the same sums
+  if (write && (lane & kDup) == 0) {
+#pragma unroll
+    for (int k = 0; k < kHeld; ++k) {
+      const int qb = base + k;
+      if (B0 + qb <= jt) imp_row[B0 + qb] = v[k] + (qb == 0 ? cin : 0.f);
+    }
+  }
+  return carry;
+}
+
 }  // namespace
 
-// dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 | hand-off [2][128] f32 |
-// block masks [nb][MW] | union [nb] | importance carries [nb/16 + 2][128/G] f32 |
+// Optional in-kernel timeline (compiled only with -DNSA_PREFILL_TRACE): lane 0
+// of every warp of a few CTAs (KV head 0, query tiles 255, 511, 767, 1023)
+// records clock64() at fixed points of each tile's life; nsa_prefill_trace_read
+// copies the records out. Off in the library build.
+#ifdef NSA_PREFILL_TRACE
+constexpr int kTrTiles = 192;
+__device__ unsigned long long g_trace[4][12][kTrTiles][4];
+__device__ unsigned long long g_trace_phase[4][12][8];
+#define TR(j, k)                                                                            \
+  do {                                                                                      \
+    if (tr_cta >= 0 && (threadIdx.x & 31) == 0 && (j) >= 0 && (j) < kTrTiles)                \
+      g_trace[tr_cta][threadIdx.x >> 5][(j)][(k)] = clock64();                              \
+  } while (0)
+#define TRP(k)                                                                              \
+  do {                                                                                      \
+    if (tr_cta >= 0 && (threadIdx.x & 31) == 0) g_trace_phase[tr_cta][threadIdx.x >> 5][(k)] = clock64(); \
+  } while (0)
+#else
+#define TR(j, k) do {} while (0)
+#define TRP(k) do {} while (0)
+#endif
+
+
+// dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 |
+// per-tile maxima [2][2][128] f32 | block masks [nb][MW] | union [nb] | importance carries [nb/8 + 2][128/G] f32 |
 // (when it fits) importance [128/G][nb] f32 | selections [128/G][32] i32
 __host__ __device__ inline size_t fused_fixed_bytes(int nb, int G) {
   const int tok = 128 / G, mw = (tok + 31) / 32;
-  return sizeof(FBars) + 2 * 2 * 128 * 4 + 2 * 128 * 4 + (size_t)nb * mw * 4 + (size_t)nb * 4 +
-         (size_t)(nb / 16 + 2) * tok * 4 + 64;
+  return sizeof(FBars) + 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4 + (size_t)nb * mw * 4 + (size_t)nb * 4 +
+         (size_t)(nb / 8 + 2) * tok * 4 + 64;
 }
 
 template <int DK, int DV>
@@ -152,13 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   uint8_t* vring = kring + (size_t)nks * K_BYTES;
   FBars* bars = reinterpret_cast<FBars*>(vring + (size_t)nvs * V_BYTES);
   float* xch = reinterpret_cast<float*>(bars + 1);                 // [slot][warpgroup][row]
-  float* hslot = xch + 512;                                        // [tile parity][row] reference max
+  float* pxch = xch + 512;                                         // [slot][warpgroup][row] per-tile maxima
   const int G = a.G;
   const int TOK = 128 / G, MW = (TOK + 31) / 32;
-  uint32_t* bm = reinterpret_cast<uint32_t*>(hslot + 256);         // [nb][MW] token bits per block
+  uint32_t* bm = reinterpret_cast<uint32_t*>(pxch + 512);          // [nb][MW] token bits per block
   int* uni = reinterpret_cast<int*>(bm + (size_t)a.nb_stride * MW);  // union of selected blocks
-  float* cbuf = reinterpret_cast<float*>(uni + a.nb_stride);      // [compressed tile][token] carried mass
-  float* imp_s = cbuf + (size_t)(a.nb_stride / 16 + 2) * TOK;     // [token][nb] when a.imp_smem
+  float* cbuf = reinterpret_cast<float*>(uni + a.nb_stride);      // [32-key half][token] carried mass
+  float* imp_s = cbuf + (size_t)(a.nb_stride / 8 + 2) * TOK;      // [token][nb] when a.imp_smem
   int32_t* sel_s = reinterpret_cast<int32_t*>(imp_s + (size_t)TOK * a.nb_stride);   // [token][32]
   volatile int* abort_flag = &bars->abort;
 
@@ -175,6 +256,10 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   const int key0w = max(0, t0 - a.window + 1);
   const int nkw = (t_last - key0w) / kKeys + 1;                              // window tiles
   const int first_w = 2 * nkc, first_s = first_w + nkw;
+#ifdef NSA_PREFILL_TRACE
+  const int tr_cta = (g == 0 && (tile & 255) == 255) ? (tile >> 8) & 3 : -1;
+#endif
+  TRP(0);
 
   for (int i = tid; i < (jt_max + 1) * MW; i += kThreads) bm[i] = 0u;
   if (tid == 0) {
@@ -187,10 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       mbar_init(&bars->v_empty[i], 1);
     }
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < kSBuf; ++i) {   // tile j is read and written by warpgroup j & 1 only
+    for (int i = 0; i < kSBuf; ++i) {   // every softmax thread reads (and writes P into) every tile
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], kSmThreads / 2);
-      mbar_init(&bars->p_full[i], kSmThreads / 2);
+      mbar_init(&bars->s_free[i], kSmThreads);
+      mbar_init(&bars->p_full[i], kSmThreads);
       mbar_init(&bars->pv_done[i], 1);
     }
     mbar_init(&bars->ob_free, kSmThreads);
@@ -199,8 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     mbar_init(&bars->smx, kSmThreads);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&bars->xbar[i], 64);
-      mbar_init(&bars->hbar[i][0], 32);
-      mbar_init(&bars->hbar[i][1], 32);
+      mbar_init(&bars->pbar[i], 64);
     }
     bars->abort = 0;
     bars->nu = 0;
@@ -226,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         const int st = j % nks;
         if (j >= nks && !mbar_wait(&bars->k_empty[st], ((j / nks) - 1) & 1, abort_flag, a.status, 401))
           return false;
+        TR(j, 0);
         uint8_t* Ks = kring + (size_t)st * 8192;   // chunk kb of slot st at kb * nks * 8 KB + st * 8 KB
         mbar_arrive_expect_tx(&bars->k_full[st], K_BYTES);
 #pragma unroll
@@ -257,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         const int st = vi % nvs;
         if (vi >= nvs && !mbar_wait(&bars->v_empty[st], ((vi / nvs) - 1) & 1, abort_flag, a.status, 403))
           return false;
+        TR(vi, 0);
         uint8_t* Vs = vring + (size_t)st * V_BYTES;
         mbar_arrive_expect_tx(&bars->v_full[st], V_BYTES);
 #pragma unroll
@@ -277,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   } else if (warp == 9) {
     // ------------------------------------------------------------ S = Q.K^T issuer
     // S(j) goes to buffer j % 4; the buffer is free again once the softmax read
-    // S(j - 4) (pass 1) or P.V(j - 4) consumed the P written over it. Tiles are
+    // S(j - 4) (C1 tiles) or P.V(j - 4) consumed the P written over it. Tiles are
     // taken in pairs (j even): their S buffers are adjacent columns and their K
     // tiles adjacent rows of the ring (chunk-interleaved slots), so one N = 128
     // product computes both.
@@ -319,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
              (!pair || mbar_wait(&bars->k_full[st + 1], kph, abort_flag, a.status, 415)) && buf_free(j) &&
              (!pair || buf_free(j + 1));
         if (!ok) break;
+        TR(j, 0);
         tc_fence_after();
         const uint64_t kd = kdesc0 + (uint64_t)((uint32_t)st * (8192u >> 4));
         const uint32_t dcol = tmem + col_s(sb);
@@ -335,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
           umma_commit(&bars->s_full[sb + 1]);
           umma_commit(&bars->k_empty[st + 1]);
         }
+        TR(j, 1);
         const int adv = pair ? 2 : 1;
         j += adv;
         st += adv;
@@ -370,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
              mbar_wait(&bars->p_full[sb], ((i - nkc) >> 2) & 1, abort_flag, a.status, 412) &&
              (i != first_s || mbar_wait(&bars->ob_free, 0, abort_flag, a.status, 413));
         if (!ok) break;
+        TR(i, 2);
         tc_fence_after();
         const bool first = (i == nkc) || (i == first_w) || (i == first_s);
         const uint32_t ocol = i < first_w ? kColOA : kColOB;
@@ -381,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
                   (first && kk == 0) ? 0u : 1u);
         umma_commit(&bars->pv_done[sb]);
         umma_commit(&bars->v_empty[vs]);
+        TR(i, 3);
         if (++vs == nvs) {
           vs = 0;
           vph ^= 1u;
@@ -391,10 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // Warpgroup wg = warp / 4 owns the tiles j with j % 2 == wg (all 64 keys of its
-    // 32 rows); the two warps of a row quarter work on alternate tiles, so one
-    // computes while the other waits. The online reference max of a row is handed
-    // from each tile to the next through shared memory.
+    // Warp w owns the 32 rows of tensor-memory lane quarter q4 = w % 4 and key
+    // columns 32*wg .. 32*wg + 31 (wg = w / 4) of every tile. The two warps of a
+    // quarter split each tile: they trade their partial row maxima once per tile
+    // (which also orders both warps' S reads before either writes P over the
+    // buffer), so both hold the same reference max, and each keeps the softmax
+    // denominator of its own columns until the end of the phase.
     const int wg = warp >> 2;
     const int q4 = warp & 3;          // row quarter = TMEM lane quarter
     const int r = q4 * 32 + lane;     // row = TMEM lane
@@ -404,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     const int64_t n = tok0 + t;
     const int hq = g * G + hh;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t colh = 32u * (uint32_t)wg;   // this warp's key columns inside a tile
     const float sc = a.scale_log2;    // raw score -> log2 units
     float gc = 0.f, gsl = 0.f, gw = 0.f;
     if (valid) {
@@ -421,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       return __all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)parity, abort_flag, a.status, site));
     };
     int xcnt = 0;
-    // value of the other warpgroup for this row (both warps of the quarter call it in step)
+    // value of the partner warp for this row (both warps of the quarter call it in step)
     auto exchange = [&](float mine) -> float {
       const int slot = xcnt & 1;
       xch[(slot * 2 + wg) * 128 + r] = mine;
@@ -431,39 +524,63 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       if (!w) ok = false;
       return xch[(slot * 2 + (1 - wg)) * 128 + r];
     };
-    // Every tile is handled in two halves of 32 keys (S re-read from tensor memory
-    // where a second pass needs it), so a thread holds 32 scores at a time.
+    // per-tile max with the partner warp (called by both warps for every online
+    // and C2 tile, whether or not they read S, so the phases stay in step)
+    int pxs = 0;
+    auto pair_max = [&](float mine) -> float {
+      const int slot = pxs & 1;
+      pxch[(slot * 2 + wg) * 128 + r] = mine;
+      mbar_arrive(&bars->pbar[q4]);
+      if (!uwait(&bars->pbar[q4], pxs & 1, 428)) ok = false;
+      ++pxs;
+      return fmaxf(mine, pxch[(slot * 2 + (1 - wg)) * 128 + r]);
+    };
+    // A thread holds the 32 scores of its row and columns for the current tile.
     float sv[32];
+    int cur_j = 0;
+    (void)cur_j;
     int cur_b = 0;   // S/P buffer of the tile being processed (tile j uses buffer j % 4)
     auto wait_s = [&](int j) -> bool {
       cur_b = j & (kSBuf - 1);
+      cur_j = j;
       if (!uwait(&bars->s_full[cur_b], (j >> 2) & 1, 422)) return false;
+      TR(j, 0);
       tc_fence_after();
       return true;
     };
-    // raw scores of keys 32*hf .. 32*hf + 31 of the current tile
-    auto ld_half = [&](int hf) {
-      const uint32_t src = tmem + lane_base + col_s(cur_b) + 32u * hf;
+    // raw scores of this warp's 32 keys of the current tile (two loads, one wait)
+    auto ld32 = [&]() {
+      const uint32_t src = tmem + lane_base + col_s(cur_b) + colh;
       tmem_ld16(src, sv);
       tmem_ld16(src + 16, sv + 16);
       tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) asm volatile("" : "+f"(sv[c]));   // no use before the wait
     };
-    // bf16 P of keys 32*hf .. into columns 16*hf .. of the buffer (S there already read)
-    auto st_half = [&](int hf, float scale) {
+    // bf16 P (sv * scale) of keys colh .. colh + 31 into columns colh/2 .. colh/2 + 15
+    // (P of key pair (2c, 2c+1) sits in column c; both warps' S reads are done)
+    auto st32 = [&](float scale) {
 #pragma unroll
       for (int c = 0; c < 16; c += 8) {
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(sv[2 * (c + i)] * scale, sv[2 * (c + i) + 1] * scale);
-        tmem_st8(tmem + lane_base + col_s(cur_b) + 16u * hf + c, pk);
+        tmem_st8(tmem + lane_base + col_s(cur_b) + colh / 2 + c, pk);
       }
+    };
+    auto st32_zero = [&]() {
+      const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < 16; c += 8) tmem_st8(tmem + lane_base + col_s(cur_b) + colh / 2 + c, z);
     };
     // all S reads of the tile are done (and its P written)
     auto tile_done = [&](bool with_p) {
+      TR(cur_j, 2);
       if (with_p) tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->s_free[cur_b]);
       if (with_p) mbar_arrive(&bars->p_full[cur_b]);
+      TR(cur_j, 3);
     };
     // P.V of tile i (>= nkc) has finished; p_full / pv_done phases count P.V tiles per buffer
     auto wait_pv = [&](int i) -> bool {
@@ -472,31 +589,30 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       return true;
     };
 
-    // ---------------- C1: compressed keys, row max and denominator (per warpgroup, merged)
+    // ---------------- C1: compressed keys, row max and denominator (per warp, merged)
     const int nvis = valid ? cmp_visible_dev(t, a.l, a.s) : 0;
     float m = -1e30f, lp = 0.f;   // raw units
-    for (int j = wg; j < nkc; j += 2) {
+    for (int j = 0; j < nkc; ++j) {
       if (ok) ok = wait_s(j);
-      const bool part = !__all_sync(0xffffffffu, j * kKeys + kKeys <= nvis);
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        if (ok) ld_half(hf);
-        const int c0 = j * kKeys + 32 * hf;
-        if (part) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
-        }
-        const float mn = fmaxf(m, tree_max<32>(sv));
-        const float mo = -mn * sc;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
-        lp = lp * ex2((m - mn) * sc) + tree_sum<32>(sv);
-        m = mn;
+      const int c0 = j * kKeys + (int)colh;
+      const bool part = !__all_sync(0xffffffffu, c0 + 32 <= nvis);
+      if (ok) {
+        ld32();
+        tile_done(false);   // S is in registers: the buffer is free again
       }
-      if (ok) tile_done(false);
+      if (part) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
+      }
+      const float mn = fmaxf(m, tree_max<32>(sv));
+      const float mo = -mn * sc;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
+      lp = lp * ex2((m - mn) * sc) + tree_sum<32>(sv);
+      m = mn;
     }
     float linv = 0.f, mo_c = 0.f;
-    if (nkc > 0) {   // merge the two warpgroups' (max, sum) in a fixed order
+    if (nkc > 0) {   // merge the two warps' (max, sum) in a fixed order
       const float m_o = exchange(m);
       const float l_o = exchange(lp);
       const float m0 = wg == 0 ? m : m_o, m1 = wg == 0 ? m_o : m;
@@ -507,48 +623,42 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       mo_c = -mm * sc;
     }
 
+    TRP(1);
     // ---------------- C2: probabilities, importance, O_A = g_cmp * P.V_cmp
     // compressed key i' = 4u' + u spans tokens [16i', 16i' + 32): u in {0,1,2} puts
     // 2p on selection block u', u = 3 puts p on u' and u' + 1 (overlap / stride).
-    // Each half of a tile covers 8 blocks; the mass carried past the first half
-    // is added here, the one carried past the tile before the selection.
+    // The 32 keys of a warp cover 8 selection blocks; the mass its last key
+    // carries into the next block is added before the selection.
     for (int i = 0; i < nkc; ++i) {
       const int j = nkc + i;
-      if ((j & 1) != wg) continue;
       if (ok) ok = wait_s(j);
-      const bool part = !__all_sync(0xffffffffu, i * kKeys + kKeys <= nvis);
-      float cin = 0.f;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        if (ok) ld_half(hf);
-        const int c0 = i * kKeys + 32 * hf;
-        if (part) {
+      const int c0 = i * kKeys + (int)colh;
+      const bool part = !__all_sync(0xffffffffu, c0 + 32 <= nvis);
+      if (ok) ld32();
+      pair_max(0.f);   // both warps' S reads precede the P stores
+      if (part) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo_c)) * linv;
-        if (ok) st_half(hf, gc);
-        float blk[8];
-#pragma unroll
-        for (int qb = 0; qb < 8; ++qb) blk[qb] = 2.f * (sv[4 * qb] + sv[4 * qb + 1] + sv[4 * qb + 2]) + sv[4 * qb + 3];
-#pragma unroll
-        for (int qb = 0; qb < 7; ++qb) blk[qb + 1] += sv[4 * qb + 3];
-#pragma unroll
-        for (int qb = 0; qb < 8; ++qb) blk[qb] = group_sum(blk[qb], G);
-        const float carry = group_sum(sv[31], G);
-        blk[0] += cin;
-        const int B0 = 16 * i + 8 * hf;
-        if (valid && ok) {
-          for (int qb = hh; qb < 8; qb += G)
-            if (B0 + qb <= jt) imp_row[B0 + qb] = blk[qb];
-          if (hf == 1 && hh == 0) cbuf[i * TOK + tt] = carry;
-        }
-        cin = carry;
+        for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
       }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo_c)) * linv;
+      if (ok) st32(gc);
+      TR(j, 1);
+      const bool wr = valid && ok;
+      const int B0 = 16 * i + 8 * wg;
+      float carry;
+      switch (G) {
+        case 16: carry = importance32<16>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
+        case 8: carry = importance32<8>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
+        case 4: carry = importance32<4>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
+        case 2: carry = importance32<2>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
+        default: carry = importance32<1>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
+      }
+      if (wr && hh == 0) cbuf[(2 * i + wg) * TOK + tt] = carry;
       if (ok) tile_done(true);
     }
 
+    TRP(2);
     // ---------------- top-n per token and the tile's union of selected blocks
     int smx_phase = 0;
     auto sm_sync = [&]() {
@@ -557,18 +667,19 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       ++smx_phase;
     };
     sm_sync();
+    const int nh = 2 * nkc;   // 32-key halves of the compressed tiles
     for (int tk = warp; tk < TOK && ok; tk += 8) {
       const int tq = t0 + tk;
       if (tq >= L) break;
       const int64_t nq = tok0 + tq;
       const int jq = tq / a.ls;
       float* irow = a.imp_smem ? imp_s + (size_t)tk * a.nb_stride : a.imp + ((size_t)nq * a.H_kv + g) * a.nb_stride;
-      // carried mass across compressed-tile boundaries (written by the other tile's warps)
-      for (int i = 1 + lane; i < nkc; i += 32)
-        if (16 * i <= jq) irow[16 * i] += cbuf[(i - 1) * TOK + tk];
-      if (nkc > 0) {
-        for (int jb = 16 * nkc + lane; jb <= jq; jb += 32)
-          irow[jb] = (jb == 16 * nkc) ? cbuf[(nkc - 1) * TOK + tk] : 0.f;
+      // mass carried across the 32-key boundaries (written by the warps of the other half)
+      for (int h = 1 + lane; h < nh; h += 32)
+        if (8 * h <= jq) irow[8 * h] += cbuf[(h - 1) * TOK + tk];
+      if (nh > 0) {
+        for (int jb = 8 * nh + lane; jb <= jq; jb += 32)
+          irow[jb] = (jb == 8 * nh) ? cbuf[(nh - 1) * TOK + tk] : 0.f;
       } else {
         for (int jb = lane; jb <= jq; jb += 32) irow[jb] = 0.f;
       }
@@ -602,75 +713,55 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       if (lane == 0) bars->nu = cnt;
     }
     sm_sync();
+    TRP(3);
     if (tid == 0) mbar_arrive(&bars->sel_ready);
     const int nu = ok ? bars->nu : 0;
 
     // ---------------- online phases (window, selected blocks)
-    // Each tile takes the reference max left by the previous tile of the phase,
-    // raises it when its own max exceeds it by more than kRescaleLog2 (rescaling
-    // O_B once the previous product has landed) and hands it to the next tile.
+    // A tile raises the row's reference max only when its own max exceeds it by
+    // more than kRescaleLog2 (rescaling this warp's half of O_B once the previous
+    // product has landed); p = 2^(s - ref) stays below 2^kRescaleLog2.
     const float thr = kRescaleLog2 / sc;
-    float r_last = -1e30f;   // reference this warp's partial sum lp is relative to
-    // mask_half(hf) masks the raw scores in sv of keys 32*hf .. of the tile; a row
-    // with rowv == false takes no part in the tile (max -inf, p = 0) at no per-key cost
-    auto online_tile = [&](int j, int pfirst, bool skip, bool rowv, auto&& mask_half) -> bool {
+    float m_ref = -1e30f;
+    // mask32() masks the raw scores of this warp's keys; a row with rowv == false
+    // takes no part in the tile (max -inf, p = 0) at no per-key cost
+    auto online_tile = [&](int j, bool skip, bool rowv, auto&& mask32) -> bool {
       float tmx = -1e30f;
       if (!skip && ok) {
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          ld_half(hf);
-          mask_half(hf);
-          tmx = fmaxf(tmx, tree_max<32>(sv));
-        }
+        ld32();
+        mask32();
+        tmx = tree_max<32>(sv);
         if (!rowv) tmx = -1e30f;
       }
-      float m_in = -1e30f;
-      if (j > pfirst) {
-        const int ip = j - 1;
-        if (!uwait(&bars->hbar[q4][ip & 1], ((ip - first_w) >> 1) & 1, 426)) ok = false;
-        m_in = hslot[(ip & 1) * 128 + r];
-      }
-      float ref = m_in, alpha = 1.f;
+      tmx = pair_max(tmx);
+      TR(j, 1);
+      if (!ok) return false;
+      float ref = m_ref, alpha = 1.f;
       if (tmx > ref + thr) {
         alpha = ex2((ref - tmx) * sc);
         ref = tmx;
       }
-      hslot[(j & 1) * 128 + r] = ref;
-      mbar_arrive(&bars->hbar[q4][j & 1]);
-      if (!ok) return false;
-      lp *= ex2((r_last - m_in) * sc);   // tiles of the other warpgroup may have raised it
-      r_last = ref;
-      const bool had = m_in > -1e29f;
+      const bool had = m_ref > -1e29f;
+      m_ref = ref;
       if (__any_sync(0xffffffffu, had && alpha != 1.f)) {
         if (!wait_pv(j - 1)) return false;
-        tmem_scale_cols(tmem + lane_base + kColOB, DV, had ? alpha : 1.f);
+        tmem_scale_cols(tmem + lane_base + kColOB + wg * (DV / 2), DV / 2, had ? alpha : 1.f);
       }
       lp *= alpha;
-      const float mo = rowv ? -ref * sc : -INFINITY;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        if (skip) {
+      if (skip) {
+        st32_zero();
+      } else {
+        const float mo = rowv ? -ref * sc : -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) sv[c] = 0.f;
-        } else {
-          ld_half(hf);
-          mask_half(hf);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
-          lp += tree_sum<32>(sv);
-        }
-        st_half(hf, 1.f);
+        for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo));
+        lp += tree_sum<32>(sv);
+        st32(1.f);
       }
       tile_done(true);
       return true;
     };
-    // denominator of the phase ending with tile j_last, both warpgroups summed in a fixed order
-    auto phase_sum = [&](int j_last) -> float {
-      if ((j_last & 1) != wg) {
-        if (!uwait(&bars->hbar[q4][j_last & 1], ((j_last - first_w) >> 1) & 1, 427)) ok = false;
-        const float m_fin = hslot[(j_last & 1) * 128 + r];
-        lp *= ex2((r_last - m_fin) * sc);
-      }
+    // denominator of the phase, both warps' columns summed in a fixed order
+    auto phase_sum = [&]() -> float {
       const float other = exchange(lp);
       return wg == 0 ? lp + other : other + lp;
     };
@@ -680,22 +771,21 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     lp = 0.f;
     for (int i = 0; i < nkw; ++i) {
       const int j = first_w + i;
-      if ((j & 1) != wg) continue;
       if (ok) ok = wait_s(j);
-      const int k0 = key0w + i * kKeys;
-      const bool part = !__all_sync(0xffffffffu, valid && k0 >= wlo && k0 + kKeys - 1 <= t);
-      auto mask_w = [&](int hf) {
+      const int k0 = key0w + i * kKeys + (int)colh;
+      const bool part = !__all_sync(0xffffffffu, valid && k0 >= wlo && k0 + 31 <= t);
+      auto mask_w = [&]() {
         if (!part) return;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const int tau = k0 + 32 * hf + c;
+          const int tau = k0 + c;
           sv[c] = (valid && tau <= t && tau >= wlo) ? sv[c] : -INFINITY;
         }
       };
-      if (!online_tile(j, first_w, false, valid, mask_w)) ok = false;
+      if (!online_tile(j, false, valid, mask_w)) ok = false;
     }
     {
-      const float lw = phase_sum(first_s - 1);
+      const float lw = phase_sum();
       if (ok) ok = wait_pv(first_s - 1);
       const float sw = lw > 0.f ? gw / lw : 0.f;
 #pragma unroll 1
@@ -716,29 +806,29 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       mbar_arrive(&bars->ob_free);
     }
 
+    TRP(4);
     // ---------------- S: union blocks, each row masked to its token's selection
-    r_last = -1e30f;
+    m_ref = -1e30f;
     lp = 0.f;
     for (int u = 0; u < nu; ++u) {
       const int j = first_s + u;
-      if ((j & 1) != wg) continue;
       if (ok) ok = wait_s(j);
       const int jb = uni[u];
       const bool mine = valid && ((bm[jb * MW + (tt >> 5)] >> (tt & 31)) & 1u);
-      const int k0 = jb * a.ls;
+      const int k0 = jb * a.ls + (int)colh;
       // no row of this warp selected the block: its P rows are zero
       const bool skip = !__any_sync(0xffffffffu, mine);
       // keys after t exist only in a row's own current block
-      const bool part = __any_sync(0xffffffffu, mine && k0 + kKeys - 1 > t);
-      auto mask_s = [&](int hf) {
+      const bool part = __any_sync(0xffffffffu, mine && k0 + 31 > t);
+      auto mask_s = [&]() {
         if (!part) return;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c] = (k0 + 32 * hf + c <= t) ? sv[c] : -INFINITY;
+        for (int c = 0; c < 32; ++c) sv[c] = (k0 + c <= t) ? sv[c] : -INFINITY;
       };
-      if (!online_tile(j, first_s, skip, mine, mask_s)) ok = false;
+      if (!online_tile(j, skip, mine, mask_s)) ok = false;
     }
     {
-      const float ls_ = nu > 0 ? phase_sum(first_s + nu - 1) : 0.f;
+      const float ls_ = nu > 0 ? phase_sum() : 0.f;
       if (ok && nu > 0) ok = wait_pv(first_s + nu - 1);
       const float ss = ls_ > 0.f ? gsl / ls_ : 0.f;
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + hq) * DV + wg * (DV / 2);
@@ -766,6 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     }
   }
 
+  TRP(5);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -817,3 +908,17 @@ cudaError_t launch_prefill_fused(const PrefillArgs& a, const PrefillMaps& m, int
 }
 
 }  // namespace nsa
+
+#ifdef NSA_PREFILL_TRACE
+extern "C" int nsa_prefill_trace_read(void* tiles, void* phases) {
+  if (cudaMemcpyFromSymbol(tiles, nsa::g_trace, sizeof(nsa::g_trace)) != cudaSuccess) return 1;
+  if (cudaMemcpyFromSymbol(phases, nsa::g_trace_phase, sizeof(nsa::g_trace_phase)) != cudaSuccess) return 1;
+  return 0;
+}
+extern "C" int nsa_prefill_trace_clear() {
+  static unsigned long long z[4 * 12 * 192 * 4];
+  if (cudaMemcpyToSymbol(nsa::g_trace, z, sizeof(nsa::g_trace)) != cudaSuccess) return 1;
+  if (cudaMemcpyToSymbol(nsa::g_trace_phase, z, sizeof(nsa::g_trace_phase)) != cudaSuccess) return 1;
+  return 0;
+}
+#endif
