@@ -105,6 +105,19 @@ __device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_
 
 }  // namespace
 
+// Optional timeline of the fine pass (compiled only with -DNSA_DECODE_TRACE): thread
+// 0 of the CTAs of KV head 0 and sequences 0..7 records clock64() at fixed points;
+// nsa_decode_trace_read copies the records out. Off in the library build.
+#ifdef NSA_DECODE_TRACE
+__device__ unsigned long long g_dtrace[8][16];
+#define TRD(k)                                                                   \
+  do {                                                                           \
+    if (blockIdx.x == 0 && blockIdx.y < 8 && threadIdx.x == 0) g_dtrace[blockIdx.y][(k)] = clock64(); \
+  } while (0)
+#else
+#define TRD(k) do {} while (0)
+#endif
+
 size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total; }
 
 // ---------------------------------------------------------------------------
@@ -345,6 +358,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   const int G = a.G;
   const size_t bg = (size_t)b * a.H_kv + g;
 
+  TRD(0);
   if (tid == 0) {
     for (int k = 0; k < kDecStages; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
     mbar_init(d2bar, 1);
@@ -369,7 +383,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     const float* tp = a.part + pl.tp + bg * pl.n_tiles * kTP * G;
     // the tile partials and chunk outputs come into shared memory with two bulk
     // copies when they fit next to the scratch (otherwise they are read in place)
-    float* tp_s = imp_s + ((a.nb_stride + 3) & ~3);
+    uint32_t* ck = reinterpret_cast<uint32_t*>(imp_s + ((a.nb_stride + 3) & ~3));   // top-n scratch [5][32]
+    int* ci = reinterpret_cast<int*>(ck + 5 * 32);
+    float* tp_s = reinterpret_cast<float*>(ci + 5 * 32);
     const uint32_t tp_bytes = (uint32_t)(((size_t)ntl * kTP * G * 4 + 15) & ~size_t(15));
     float* cpo_s = tp_s + tp_bytes / 4;
     const uint32_t cpo_bytes = (uint32_t)((size_t)nch * G * DV * 4);
@@ -388,6 +404,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       tp = tp_s;
       cpo = cpo_s;
     }
+    TRD(1);
     // one warp per head, the chunks in its lanes
     for (int h = warp; h < G; h += kDecThreads / 32) {
       float m = -1e30f, l = 0.f;
@@ -409,6 +426,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       }
     }
     __syncthreads();
+    TRD(2);
     for (int idx = tid; idx < ntl * G; idx += kDecThreads) {
       const int tj = idx / G, h = idx % G;
       Ft[tj * 16 + h] = exp2f(tp[(size_t)tj * kTP * G + h] - Mh[h]) * Li[h];
@@ -429,6 +447,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
           make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
     }
     __syncthreads();
+    TRD(3);
     // importance of blocks 0..jt: tile tj holds blocks kBlkPerTile*tj .. + kBlkPerTile
     for (int j = tid; j <= jt; j += kDecThreads) {
       const int tj = j / kBlkPerTile, q = j % kBlkPerTile;
@@ -455,10 +474,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       a.imp[bg * a.nb_stride + j] = v;
     }
     __syncthreads();
-    if (warp == 0)
+    TRD(4);
+    static_assert(kDecThreads / 32 <= 5, "top-n scratch holds five warps");
+    if (!cta_topn(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, ck, ci, kDecThreads / 32,
+                  warp, lane) &&
+        warp == 0)
       warp_topn_any(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, lane);
     __syncthreads();
   }
+  TRD(5);
   {
     const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
     for (int idx = tid; idx < 16 * (DK / 8); idx += kDecThreads) {   // 16-byte chunks
@@ -529,6 +553,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     }
   }
   __syncthreads();
+  TRD(6);
   const int nu = *nuni;
 
   // work units: the two 32-key halves of every union block
@@ -601,6 +626,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     rs_sel.finish();
     rs_win.finish();
     named_bar_sync(1, kDecConsumers * 32);   // every block consumed: the ring is free
+    TRD(7);
     float* stg = reinterpret_cast<float*>(ring);
     rs_sel.stage(stg + warp * 16 * (DV + 2), lane);
     rs_win.stage(stg + (kDecConsumers + warp) * 16 * (DV + 2), lane);
@@ -641,6 +667,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     }
   }
   __syncthreads();
+  TRD(8);
 }
 
 template <int DK, int DV>
@@ -668,6 +695,12 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return cudaGetLastError();
 }
+
+#ifdef NSA_DECODE_TRACE
+extern "C" int nsa_decode_trace_read(void* dst) {
+  return cudaMemcpyFromSymbol(dst, g_dtrace, sizeof(g_dtrace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st) {
   if (a.d_k == 192 && a.d_v == 128) return launch_dec_t<192, 128>(a, m, st);

@@ -145,4 +145,124 @@ __device__ __forceinline__ void warp_topn_any(const float* imp, int jt, int top_
   else warp_topn_mem(imp, jt, top_n, ff, fl, out, lane);
 }
 
+// Ascending bitonic sort of one int per lane across the warp.
+__device__ __forceinline__ int warp_sort_asc(int v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j >= 1; j >>= 1) {
+      const int o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool up = (lane & k) == 0;          // direction of this k-block
+      const bool lower = (lane & j) == 0;       // this lane keeps the smaller of the pair when up
+      v = (lower == up) ? min(v, o) : max(v, o);
+    }
+  }
+  return v;
+}
+
+// Best `need` free candidates of one slice of blocks, by warp arg-max rounds
+// (ties to the lower block index). Writes round r's (key, block) to ck[r], ci[r];
+// key 0 once the slice has no candidate left.
+template <int PER>
+__device__ __forceinline__ void slice_best(const float* imp, int lo, int hi, int ff, int last_free, int need,
+                                           uint32_t* ck, int* ci, int lane) {
+  uint32_t key[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = lo + i * 32 + lane;
+    key[i] = (j < hi && j >= ff && j <= last_free) ? order_key(imp[j]) : 0u;
+  }
+  for (int round = 0; round < need; ++round) {
+    uint32_t m = key[0];
+#pragma unroll
+    for (int i = 1; i < PER; ++i) m = max(m, key[i]);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, m);
+    uint32_t eq = 0u;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) eq |= (key[i] == M ? 1u : 0u) << i;
+    const uint32_t li = eq ? (uint32_t)((__ffs(eq) - 1) * 32 + lane) : 0xffffffffu;
+    const uint32_t pmin = __reduce_min_sync(0xffffffffu, li);   // lowest position = lowest block
+    if (lane == (int)(pmin & 31u)) {
+      const int i0 = (int)(pmin >> 5);
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (i == i0) key[i] = 0u;
+    }
+    if (lane == 0) {
+      ck[round] = M;
+      ci[round] = M ? lo + (int)pmin : 0x7fffffff;
+    }
+  }
+}
+
+// CTA-wide selection with the same result as warp_topn (block 0 .. ff-1 and the
+// fl blocks ending at jt forced; the other top_n - ff - fl slots to the highest
+// scores, ties to the lower index; ascending, -1 padded). Each of the nw warps
+// picks the best candidates of its slice of the blocks, then warp 0 picks among
+// those (a block in the overall best set is among the best of its own slice).
+// ck/ci: shared scratch of nw * 32 entries each. Every thread of the CTA calls it
+// (it synchronises the CTA); returns false when the candidates do not fit
+// (more than nw * 512 blocks), and then writes nothing.
+__device__ inline bool cta_topn(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out, uint32_t* ck,
+                                int* ci, int nw, int warp, int lane) {
+  const int K = jt + 1;
+  if (K <= top_n) {
+    if (warp == 0)
+      for (int i = lane; i < top_n; i += 32) out[i] = i < K ? i : -1;
+    return true;
+  }
+  const int per = (K + 32 * nw - 1) / (32 * nw);
+  if (per > 16) return false;
+  const int need = top_n - ff - fl;
+  const int pw = per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : per <= 8 ? 8 : 16;
+  const int lo = warp * 32 * pw, hi = min(K, lo + 32 * pw);
+  if (warp < nw && lo < K && need > 0) {
+    uint32_t* wk = ck + warp * 32;
+    int* wi = ci + warp * 32;
+    switch (pw) {
+      case 1: slice_best<1>(imp, lo, hi, ff, jt - fl, need, wk, wi, lane); break;
+      case 2: slice_best<2>(imp, lo, hi, ff, jt - fl, need, wk, wi, lane); break;
+      case 4: slice_best<4>(imp, lo, hi, ff, jt - fl, need, wk, wi, lane); break;
+      case 8: slice_best<8>(imp, lo, hi, ff, jt - fl, need, wk, wi, lane); break;
+      default: slice_best<16>(imp, lo, hi, ff, jt - fl, need, wk, wi, lane); break;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nsl = (K + 32 * pw - 1) / (32 * pw);   // slices that ran
+    // lane l holds entry r = l of every slice: key k[w], block b[w]
+    uint32_t k[8];
+    int bidx[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const bool v = w < nsl && lane < need;
+      k[w] = v ? ck[w * 32 + lane] : 0u;
+      bidx[w] = v ? ci[w * 32 + lane] : 0x7fffffff;
+    }
+    int mine = 0x7fffffff;   // block chosen in round `lane`
+    for (int round = 0; round < need; ++round) {
+      uint32_t m = 0u;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = max(m, k[w]);
+      const uint32_t M = __reduce_max_sync(0xffffffffu, m);
+      int bm = 0x7fffffff;
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        if (k[w] == M) bm = min(bm, bidx[w]);
+      const int B = (int)__reduce_min_sync(0xffffffffu, (uint32_t)bm);
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        if (bidx[w] == B) k[w] = 0u;
+      if (lane == round) mine = B;
+    }
+    // forced blocks in the lanes after the chosen ones
+    const int f = lane - need;
+    if (f >= 0 && f < ff) mine = f;
+    if (f >= ff && f < ff + fl) mine = jt - fl + 1 + (f - ff);
+    const int v = warp_sort_asc(mine, lane);
+    if (lane < top_n) out[lane] = v == 0x7fffffff ? -1 : v;
+  }
+  return true;
+}
+
 }  // namespace nsa
