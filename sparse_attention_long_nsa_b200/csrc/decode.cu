@@ -36,7 +36,7 @@ constexpr int kDecThreads = (kDecConsumers + 1) * 32;
 // compressed-key pass: consumer warps + producer warp
 constexpr int kD1Stages = 8;
 constexpr int kD1Consumers = 4;
-constexpr int kD1Threads = (kD1Consumers + 1) * 32;
+constexpr int kD1Threads = (kD1Consumers + 2) * 32;   // consumers, producer, merger
 constexpr int kCmpChunk = 512;         // compressed keys per D1 work item
 constexpr int kTilesPerChunk = kCmpChunk / kTileKeys;
 constexpr int kBlkPerTile = kTileKeys / 4;   // selection blocks a tile of compressed keys covers
@@ -103,6 +103,40 @@ __device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_
   }
 }
 
+// merge_warps for one warp: lanes 2r, 2r+1 take row r (< G <= 16), half of its columns each
+template <int DV, int NW>
+__device__ __forceinline__ void merge_warps_w32(const float* stg, int G, float* dst_o, float* dst_ml, int lane) {
+  const int row = lane >> 1, part = lane & 1;
+  if (row >= G) return;
+  float M = -1e30f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, stg[(w * 16 + row) * (DV + 2) + DV]);
+  float f[NW], Ls = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const float* r = stg + (w * 16 + row) * (DV + 2);
+    f[w] = r[DV + 1] > 0.f ? ex2(r[DV] - M) : 0.f;
+    Ls += f[w] * r[DV + 1];
+  }
+  const int c0 = part * (DV / 2);
+#pragma unroll 4
+  for (int c = c0; c < c0 + DV / 2; c += 4) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float* r = stg + (w * 16 + row) * (DV + 2) + c;   // 8-byte aligned rows
+      const float2 x = *reinterpret_cast<const float2*>(r);
+      const float2 y = *reinterpret_cast<const float2*>(r + 2);
+      v.x += f[w] * x.x; v.y += f[w] * x.y; v.z += f[w] * y.x; v.w += f[w] * y.y;
+    }
+    *reinterpret_cast<float4*>(dst_o + row * DV + c) = v;
+  }
+  if (part == 0) {
+    dst_ml[row * 2 + 0] = M;
+    dst_ml[row * 2 + 1] = Ls;
+  }
+}
+
 }  // namespace
 
 // Optional timeline of the fine pass (compiled only with -DNSA_DECODE_TRACE): thread
@@ -114,8 +148,15 @@ __device__ unsigned long long g_dtrace[8][16];
   do {                                                                           \
     if (blockIdx.x == 0 && blockIdx.y < 8 && threadIdx.x == 0) g_dtrace[blockIdx.y][(k)] = clock64(); \
   } while (0)
+// compressed pass: CTA 0, per consumer tile of warp 0 / per item
+__device__ unsigned long long g_ctrace[2][64][4];
+#define TRC(kind, i, k)                                                          \
+  do {                                                                           \
+    if (blockIdx.x == 0 && lane == 0 && (i) < 64) g_ctrace[kind][i][k] = clock64(); \
+  } while (0)
 #else
 #define TRD(k) do {} while (0)
+#define TRC(kind, i, k) do {} while (0)
 #endif
 
 size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total; }
@@ -150,12 +191,13 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
   uint64_t* empty = full + kD1Stages;
   uint64_t* q_full = empty + kD1Stages;     // [2]
   uint64_t* q_empty = q_full + 2;            // [2]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(q_empty + 2);
-  volatile int* item_abort = abort_flag + 1;   // abort flag as seen at an item end, same for all warps
+  uint64_t* stg_full = q_empty + 2;          // the consumers' item states are staged
+  uint64_t* stg_free = stg_full + 1;         // the merger has read them
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(stg_free + 1);
   // ring position each stage currently holds: a consumer waits on a stage's
   // barrier only once the stage holds its tile (consecutive tiles of one warp are
   // not consecutive uses of a stage, so a parity wait alone could alias)
-  volatile int* stage_tag = item_abort + 1;    // [kD1Stages]
+  volatile int* stage_tag = abort_flag + 1;    // [kD1Stages]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G;
@@ -165,6 +207,8 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
   if (tid == 0) {
     for (int i = 0; i < kD1Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); stage_tag[i] = -1; }
     for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], kD1Consumers); }
+    mbar_init(stg_full, kD1Consumers * 32);
+    mbar_init(stg_free, 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -207,6 +251,7 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
             ok = false;
             break;
           }
+          TRC(0, u, 2);
           uint8_t* Ks = ring + st * S::STAGE;
           stage_tag[st] = u;
           mbar_arrive_expect_tx(&full[st], S::STAGE);
@@ -225,6 +270,20 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
         for (int q2 = it - 2 < 0 ? 0 : it - 2; q2 < it; ++q2) mbar_wait_drain(&q_full[q2 & 1], (q2 >> 1) & 1);
       }
     }
+  } else if (warp == kD1Consumers + 1) {
+    // ------------------------------------------------------------ merger
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      int b, g, chunk;
+      const int ntl = item_tiles(item, b, g, chunk);
+      if (ntl == 0) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(stg_full, it & 1, abort_flag, a.status, 407))) break;
+      const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
+      merge_warps_w32<DV, kD1Consumers>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, lane);
+      __syncwarp();
+      mbar_arrive(stg_free);
+      ++it;
+    }
   } else {
     // ------------------------------------------------------------ consumers
     float* ps = pscr + warp * 16 * kTileKeys;
@@ -238,7 +297,9 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
       const int nc = n_cmp_dev(a.lens[b], a.l, a.s);
       const int c0 = chunk * kCmpChunk;
       // every warp reaches the three item-end barriers even when a wait gave up
+      if (warp == 0) TRC(1, it, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qi], (it >> 1) & 1, abort_flag, a.status, 404));
+      if (warp == 0) TRC(1, it, 1);
       const uint32_t qbase = smem_u32(qbuf + qi * S::QBUF);
       RowState<DV> rs;
       rs.init();
@@ -251,6 +312,7 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
           ok = false;
           break;
         }
+        if (warp == 0) TRC(0, u, 0);
         const uint32_t kb = smem_u32(ring + st * S::STAGE);
         float s[kNT][4];
         warp_qk_sq<DK, kNT>(qbase, 2048, 0, kb, s, lane);
@@ -277,6 +339,7 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
         }
         warp_pv<DV, kNT>(s, kb + DK * kTileKeys * 2, rs.o, lane);
         __syncwarp();
+        if (warp == 0) TRC(0, u, 1);
         if (lane == 0) mbar_arrive(&empty[st]);
         // block sums: compressed key 4q+u covers tokens [16(4q+u), +32): u<3 -> 2p
         // into block q of the tile, u = 3 -> p into q and q+1. Tile partial layout
@@ -304,20 +367,18 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
         }
         __syncwarp();
       }
+      if (warp == 0) TRC(1, it, 2);
       rs.finish();
-      named_bar_sync(1, kD1Consumers * 32);
-      if (tid == 0) *item_abort = *abort_flag;
-      rs.stage(stg + warp * 16 * (DV + 2), lane);
-      named_bar_sync(1, kD1Consumers * 32);
-      const bool aborted = *item_abort != 0;   // written before the barrier: same in every warp
-      if (!aborted) {
-        const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
-        merge_warps<DV, kD1Consumers>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, tid);
-      }
+      // the merger warp combines the four warps' states while the consumers go on
+      // with the next item; the staging area is single-buffered
+      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(stg_free, (it - 1) & 1, abort_flag, a.status, 406)))
+        ok = false;
+      if (ok) rs.stage(stg + warp * 16 * (DV + 2), lane);
+      mbar_arrive(stg_full);
       __syncwarp();
       if (lane == 0) mbar_arrive(&q_empty[qi]);
-      named_bar_sync(1, kD1Consumers * 32);   // merge done before the staging area is rewritten
-      if (aborted) break;
+      if (warp == 0) TRC(1, it, 3);
+      if (!ok) break;
       u_base += ntl;
       ++it;
     }
@@ -699,6 +760,9 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
 #ifdef NSA_DECODE_TRACE
 extern "C" int nsa_decode_trace_read(void* dst) {
   return cudaMemcpyFromSymbol(dst, g_dtrace, sizeof(g_dtrace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int nsa_decode_ctrace_read(void* dst) {
+  return cudaMemcpyFromSymbol(dst, g_ctrace, sizeof(g_ctrace)) == cudaSuccess ? 0 : 1;
 }
 #endif
 
