@@ -31,7 +31,8 @@ namespace {
 constexpr int kTileKeys = 32;
 constexpr int kNT = kTileKeys / 8;     // 8-key MMA n-tiles per tile
 constexpr int kDecStages = 8;
-constexpr int kDecConsumers = 4;
+constexpr int kDecBranchWarps = 4;                      // consumer warps per branch (selected, window)
+constexpr int kDecConsumers = 2 * kDecBranchWarps;
 constexpr int kDecThreads = (kDecConsumers + 1) * 32;
 // compressed-key pass: consumer warps + producer warp
 constexpr int kD1Stages = 8;
@@ -48,8 +49,8 @@ struct DecSmem {
   static constexpr int V_BYTES = kTileKeys * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int RING = kDecStages * STAGE;
-  static constexpr int MERGE = 2 * kDecConsumers * 16 * (DV + 2) * 4;
-  static constexpr int PSCR = kDecConsumers * 16 * 64 * 4;   // probabilities for block sums
+  static constexpr int MERGE = kDecConsumers * 16 * (DV + 2) * 4;   // one staged state per consumer warp
+  static constexpr int PSCR = 16 * 1024;                              // the group's Q (16 rows x d_k <= 256)
   static constexpr int BODY = (RING > MERGE ? RING : MERGE);
   static constexpr int TOTAL = 1024 + BODY + PSCR + 1024;
 };
@@ -148,8 +149,10 @@ __device__ unsigned long long g_dtrace[8][16];
   do {                                                                           \
     if (blockIdx.x == 0 && blockIdx.y < 8 && threadIdx.x == 0) g_dtrace[blockIdx.y][(k)] = clock64(); \
   } while (0)
-// compressed pass: CTA 0, per consumer tile of warp 0 / per item
+// compressed pass: CTA 0, per consumer tile of warp 0 / per item; every CTA's start / end (global timer)
 __device__ unsigned long long g_ctrace[2][64][4];
+__device__ unsigned long long g_cspan[256][3];
+__device__ unsigned long long g_fspan[512][3];
 #define TRC(kind, i, k)                                                          \
   do {                                                                           \
     if (blockIdx.x == 0 && lane == 0 && (i) < 64) g_ctrace[kind][i][k] = clock64(); \
@@ -203,6 +206,9 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
   const int G = a.G;
   const PartLayout pl = part_layout(a);
   const int n_items = a.B * a.H_kv * a.n_cmp_chunks;
+  // the fine pass may be scheduled on SMs this kernel's CTAs leave; it waits for
+  // this whole grid before it reads the partials
+  pdl_launch_dependents();
 
   if (tid == 0) {
     for (int i = 0; i < kD1Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); stage_tag[i] = -1; }
@@ -212,6 +218,14 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     *abort_flag = 0;
     fence_mbar_init();
   }
+#ifdef NSA_DECODE_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 256) {
+    g_cspan[blockIdx.x][0] = globaltimer_ns();
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_cspan[blockIdx.x][2] = smid;
+  }
+#endif
   __syncthreads();
 
   // item -> (b, g, chunk); returns the number of 64-key tiles (0: nothing to do)
@@ -384,6 +398,9 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     }
   }
   __syncthreads();
+#ifdef NSA_DECODE_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 256) g_cspan[blockIdx.x][1] = globaltimer_ns();
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -420,13 +437,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   const size_t bg = (size_t)b * a.H_kv + g;
 
   TRD(0);
+#ifdef NSA_DECODE_TRACE
+  const int fsp = blockIdx.y * gridDim.x + blockIdx.x;
+  if (threadIdx.x == 0 && fsp < 512) g_fspan[fsp][0] = globaltimer_ns();
+#endif
+  // K/V of one 32-key half of block blk into L2 (the stream reads them from there)
+  auto prefetch_half = [&](int blk, int half) {
+    const int row = b * a.Lmax + blk * a.ls + half * kTileKeys;
+    for (int kb = 0; kb < DK / 64; ++kb) tma_prefetch_3d(&mp.k, kb * 64, g, row);
+    for (int vb = 0; vb < DV / 64; ++vb) tma_prefetch_3d(&mp.v, vb * 64, g, row);
+  };
+  if (warp == kDecConsumers && lane == 0) {
+    // the window does not depend on the selection: its blocks travel to L2 while
+    // the chunk partials are merged and the blocks are selected
+    for (int blk = wlo / a.ls; blk <= jt; ++blk)
+      for (int h = 0; h < 2; ++h)
+        if (blk * a.ls + h * kTileKeys <= t) prefetch_half(blk, h);
+  }
   if (tid == 0) {
-    for (int k = 0; k < kDecStages; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 1); }
+    for (int k = 0; k < kDecStages; ++k) { mbar_init(&full[k], 1); mbar_init(&empty[k], 2); }   // one warp per branch
     mbar_init(d2bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();   // the compressed pass (the previous kernel) has finished: its partials are visible
   // ---- D2 (in this CTA, before the ring is used): merge the compressed chunks of
   // (b, g), finish g_cmp * o_cmp, form the importance, select the top-n blocks
   {
@@ -536,14 +571,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     }
     __syncthreads();
     TRD(4);
-    static_assert(kDecThreads / 32 <= 5, "top-n scratch holds five warps");
-    if (!cta_topn(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, ck, ci, kDecThreads / 32,
+    constexpr int kTopnWarps = 5;   // the top-n scratch holds five warps' candidates
+    if (!cta_topn(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, ck, ci, kTopnWarps,
                   warp, lane) &&
         warp == 0)
       warp_topn_any(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, lane);
     __syncthreads();
   }
   TRD(5);
+  if (warp == kDecConsumers && lane == 0) {   // selected blocks below the window, ahead of the stream
+    const int32_t* sel = a.sel + bg * a.top_n;
+    for (int i = 0; i < a.top_n; ++i) {
+      const int blk = sel[i];
+      if (blk >= 0 && blk < wlo / a.ls) {
+        prefetch_half(blk, 0);
+        prefetch_half(blk, 1);
+      }
+    }
+  }
   {
     const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
     for (int idx = tid; idx < 16 * (DK / 8); idx += kDecThreads) {   // 16-byte chunks
@@ -639,58 +684,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
           mbar_wait_drain(&full[v % kDecStages], (v / kDecStages) & 1);
     }
   } else {
-    RowState<DV> rs_sel, rs_win;
-    rs_sel.init();
-    rs_win.init();
+    // warps 0..3 run the selected branch, warps 4..7 the window branch: warp
+    // (br, wq) takes the 32-key halves u with u % 4 == wq and computes on those its
+    // branch reads; both warps of a half release its stage
+    const int br = warp / kDecBranchWarps, wq = warp % kDecBranchWarps;
+    RowState<DV> rs;
+    rs.init();
     const uint32_t qbase = smem_u32(qs);
-    for (int u = warp; u < nh; u += kDecConsumers) {
+    for (int u = wq; u < nh; u += kDecBranchWarps) {
       const int st = u % kDecStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (u / kDecStages) & 1, abort_flag, a.status, 412))) break;
       const uint32_t kb = smem_u32(ring + st * S::STAGE);
       const int blk = uni[u >> 1];
       const bool in_sel = flags[u >> 1] != 0u;
       const int first_key = blk * a.ls + (u & 1) * kTileKeys;
-      float s[kNT][4];
-      warp_qk_sq<DK, kNT>(qbase, 16 * 128, 0, kb, s, lane);
-      const int key0 = first_key + (lane & 3) * 2;
-      float x[kNT][4];
-      if (in_sel && first_key <= t) {
+      const bool use = first_key <= t && (br == 0 ? in_sel : first_key + kTileKeys - 1 >= wlo);
+      if (use) {
+        float s[kNT][4];
+        warp_qk_sq<DK, kNT>(qbase, 16 * 128, 0, kb, s, lane);
+        const int key0 = first_key + (lane & 3) * 2;
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const bool vis = key0 + nt * 8 + e <= t;
-            x[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
-            x[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
+            const int tau0 = key0 + nt * 8 + e;
+            const bool vis0 = tau0 <= t && (br == 0 || tau0 >= wlo);
+            s[nt][e] = vis0 ? s[nt][e] * a.scale_log2 : -INFINITY;
+            s[nt][2 + e] = vis0 ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
           }
         }
-        rs_sel.update(x);
-        warp_pv<DV, kNT>(x, kb + S::K_BYTES, rs_sel.o, lane);
-      }
-      if (first_key + kTileKeys - 1 >= wlo && first_key <= t) {
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int tau = key0 + nt * 8 + e;
-            const bool vis = tau <= t && tau >= wlo;
-            x[nt][e] = vis ? s[nt][e] * a.scale_log2 : -INFINITY;
-            x[nt][2 + e] = vis ? s[nt][2 + e] * a.scale_log2 : -INFINITY;
-          }
-        }
-        rs_win.update(x);
-        warp_pv<DV, kNT>(x, kb + S::K_BYTES, rs_win.o, lane);
+        rs.update(s);
+        warp_pv<DV, kNT>(s, kb + S::K_BYTES, rs.o, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
-    rs_sel.finish();
-    rs_win.finish();
+    rs.finish();
     named_bar_sync(1, kDecConsumers * 32);   // every block consumed: the ring is free
     TRD(7);
     float* stg = reinterpret_cast<float*>(ring);
-    rs_sel.stage(stg + warp * 16 * (DV + 2), lane);
-    rs_win.stage(stg + (kDecConsumers + warp) * 16 * (DV + 2), lane);
+    rs.stage(stg + warp * 16 * (DV + 2), lane);   // [branch][warp of branch][16][DV + 2]
     named_bar_sync(1, kDecConsumers * 32);
     // merge the four warps of each branch and combine: thread per (row, 4 columns)
     for (int idx = tid; idx < G * (DV / 4); idx += kDecConsumers * 32) {
@@ -699,17 +732,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       float4 res = *reinterpret_cast<const float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4);
 #pragma unroll
       for (int br = 0; br < 2; ++br) {
-        const float* base = stg + (size_t)br * kDecConsumers * 16 * (DV + 2);
+        const float* base = stg + (size_t)br * kDecBranchWarps * 16 * (DV + 2);
         float M = -1e30f;
 #pragma unroll
-        for (int w = 0; w < kDecConsumers; ++w) {
+        for (int w = 0; w < kDecBranchWarps; ++w) {
           const float* r = base + (w * 16 + row) * (DV + 2);
           if (r[DV + 1] > 0.f) M = fmaxf(M, r[DV]);
         }
         float den = 0.f;
         float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kDecConsumers; ++w) {
+        for (int w = 0; w < kDecBranchWarps; ++w) {
           const float* r = base + (w * 16 + row) * (DV + 2);
           if (r[DV + 1] > 0.f) {
             const float f = ex2(r[DV] - M);
@@ -729,6 +762,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   }
   __syncthreads();
   TRD(8);
+#ifdef NSA_DECODE_TRACE
+  if (threadIdx.x == 0 && fsp < 512) g_fspan[fsp][1] = globaltimer_ns();
+#endif
 }
 
 template <int DK, int DV>
@@ -751,7 +787,21 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   prof_begin(P_DEC_FINE, st);
-  k3<<<dim3(a.H_kv, a.B), kDecThreads, S::TOTAL, st>>>(a, m);
+  {
+    // programmatic dependent launch: the fine pass's CTAs start (barriers, L2
+    // prefetch of the window) while the compressed pass finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.H_kv, a.B);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = S::TOTAL;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, k3, a, m)) != cudaSuccess) return e;
+  }
   prof_end(P_DEC_FINE, st, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return cudaGetLastError();
@@ -760,6 +810,12 @@ static cudaError_t launch_dec_t(const DecodeArgs& a, const DecodeMaps& m, cudaSt
 #ifdef NSA_DECODE_TRACE
 extern "C" int nsa_decode_trace_read(void* dst) {
   return cudaMemcpyFromSymbol(dst, g_dtrace, sizeof(g_dtrace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int nsa_decode_fspan_read(void* dst) {
+  return cudaMemcpyFromSymbol(dst, g_fspan, sizeof(g_fspan)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int nsa_decode_cspan_read(void* dst) {
+  return cudaMemcpyFromSymbol(dst, g_cspan, sizeof(g_cspan)) == cudaSuccess ? 0 : 1;
 }
 extern "C" int nsa_decode_ctrace_read(void* dst) {
   return cudaMemcpyFromSymbol(dst, g_ctrace, sizeof(g_ctrace)) == cudaSuccess ? 0 : 1;
