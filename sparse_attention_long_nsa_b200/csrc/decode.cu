@@ -460,6 +460,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     *abort_flag = 0;
     fence_mbar_init();
   }
+  {   // the group's Q (an input: staged before the wait on the previous kernel)
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
+    for (int idx = tid; idx < 16 * (DK / 8); idx += kDecThreads) {   // 16-byte chunks
+      const int row = idx / (DK / 8), c = idx % (DK / 8);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < G) v = *reinterpret_cast<const uint4*>(qp + (size_t)row * DK + c * 8);
+      *reinterpret_cast<uint4*>(qs + (c >> 3) * 2048 + sw128(row, c & 7)) = v;
+    }
+  }
   __syncthreads();
   pdl_wait();   // the compressed pass (the previous kernel) has finished: its partials are visible
   // ---- D2 (in this CTA, before the ring is used): merge the compressed chunks of
@@ -487,10 +496,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     const uint32_t cpo_bytes = (uint32_t)((size_t)nch * G * DV * 4);
     const bool bulk = (size_t)((uint8_t*)cpo_s - ring) + cpo_bytes <= (size_t)S::BODY && nc > 0;
     if (bulk) {
-      if (tid == 0) {
-        mbar_arrive_expect_tx(d2bar, tp_bytes + cpo_bytes);
-        bulk_load(tp_s, tp, tp_bytes, d2bar);
-        bulk_load(cpo_s, cpo, cpo_bytes, d2bar);
+      if (warp == 0) {   // 16 KB pieces from several lanes keep more copies in flight
+        if (lane == 0) mbar_arrive_expect_tx(d2bar, tp_bytes + cpo_bytes);
+        __syncwarp();
+        constexpr uint32_t kPiece = 16384;
+        const uint32_t ntp = (tp_bytes + kPiece - 1) / kPiece, ncp = (cpo_bytes + kPiece - 1) / kPiece;
+        for (uint32_t i = lane; i < ntp + ncp; i += 32) {
+          const bool is_tp = i < ntp;
+          const uint32_t off = (is_tp ? i : i - ntp) * kPiece;
+          const uint32_t tot = is_tp ? tp_bytes : cpo_bytes;
+          const uint32_t n = min(kPiece, tot - off);
+          if (is_tp) bulk_load(reinterpret_cast<uint8_t*>(tp_s) + off, reinterpret_cast<const uint8_t*>(tp) + off, n, d2bar);
+          else bulk_load(reinterpret_cast<uint8_t*>(cpo_s) + off, reinterpret_cast<const uint8_t*>(cpo) + off, n, d2bar);
+        }
       }
       const bool got = mbar_wait(d2bar, 0, abort_flag, a.status, 410);
       if (__syncthreads_or(!got)) {   // one decision for the whole CTA
@@ -587,15 +605,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
         prefetch_half(blk, 0);
         prefetch_half(blk, 1);
       }
-    }
-  }
-  {
-    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.H_q + (size_t)g * G) * DK;
-    for (int idx = tid; idx < 16 * (DK / 8); idx += kDecThreads) {   // 16-byte chunks
-      const int row = idx / (DK / 8), c = idx % (DK / 8);
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < G) v = *reinterpret_cast<const uint4*>(qp + (size_t)row * DK + c * 8);
-      *reinterpret_cast<uint4*>(qs + (c >> 3) * 2048 + sw128(row, c & 7)) = v;
     }
   }
   if (warp == 0) {
