@@ -4,19 +4,22 @@
 // ai.flicky.cc, section "NSA: три ветви"; the cache holds the new token), laid
 // out as coalesced HBM streaming: decode reads every compressed key once and the
 // raw keys of the selected blocks and the window once, so the bound is HBM
-// bandwidth. Every KV tile is loaded once per GQA group (TMA, 64 keys) and
+// bandwidth. Every KV tile (TMA, 32 keys) is loaded once per GQA group and
 // consumed by mma.sync with the group's heads as the 16 rows.
 //
-//   D1  split-K over the compressed cache, 512 keys per CTA: per-chunk online
-//       softmax state (o, m, l) per head, and per 64-key tile the block sums
-//       sum_i exp(s_i - m_ref) * omega(i, j) of the selection blocks it touches.
-//   D2  (at the start of the D3 CTA of each (sequence, KV head)): merge the
-//       chunks, normalise, finish g_cmp * o_cmp, reduce the block sums over the
-//       group's heads into the importance, run the top-n selection.
-//   D3  one CTA per (sequence, KV head) streams the union of the selected
-//       blocks and the window blocks once; one score tile serves both branches,
-//       each with its own softmax; it writes
-//       out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
+//   D1  dec_cmp, persistent over (sequence, KV head, 512-key chunk) items:
+//       per-chunk online softmax state (o, m, l) per head, and per 32-key tile
+//       the block sums sum_i exp(s_i - m_ref) * omega(i, j) of the selection
+//       blocks it touches. A dedicated warp merges the consumer warps' states
+//       while they go on with the next item.
+//   D2  (prologue of the D3 CTA of each (sequence, KV head), after waiting for
+//       D1 through programmatic dependent launch): merge the chunks, normalise,
+//       finish g_cmp * o_cmp, reduce the block sums over the group's heads into
+//       the importance, run the top-n selection over the CTA's warps.
+//   D3  dec_fine streams the union of the selected blocks and the window blocks
+//       once (the window is prefetched into L2 while D2 runs); four warps run
+//       the selected branch and four the window branch, each with its own
+//       softmax; it writes out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
 #include "common.cuh"
 #include "kernels.h"
 #include "topn.cuh"
