@@ -246,7 +246,7 @@ def run_nsa(args, rank, ws):
         # holds clean lines: otherwise the write-back of ~126 MB of dirty lines
         # competes with the first microseconds of the timed kernels
         flush_buf.fill_(1)
-        flush_buf.view(torch.int32).sum()
+        flush_buf.view(torch.int32).max()
 
     def step():
         nsa.nsa_compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], tok, seq, tok,

@@ -80,34 +80,9 @@ __host__ __device__ inline PartLayout part_layout(const DecodeArgs& a) {
   return p;
 }
 
-// merge NW staged warp states ([w][16][DV+2]) into one state per row < G:
-// o relative to the merged max M -> dst_o[row][DV], (M, L) -> dst_ml[row][2]
-template <int DV, int NW = kDecConsumers>
-__device__ __forceinline__ void merge_warps(const float* stg, int G, float* dst_o, float* dst_ml, int tid) {
-  const int per_row = (NW * 32) / 16;
-  const int row = tid / per_row, part = tid % per_row;
-  if (row >= G) return;
-  float M = -1e30f;
-  for (int w = 0; w < NW; ++w) M = fmaxf(M, stg[(w * 16 + row) * (DV + 2) + DV]);
-  float f[NW], Ls = 0.f;
-  for (int w = 0; w < NW; ++w) {
-    const float* r = stg + (w * 16 + row) * (DV + 2);
-    f[w] = r[DV + 1] > 0.f ? ex2(r[DV] - M) : 0.f;
-    Ls += f[w] * r[DV + 1];
-  }
-  const int span = DV / per_row;
-  for (int c = part * span; c < (part + 1) * span; ++c) {
-    float v = 0.f;
-    for (int w = 0; w < NW; ++w) v += f[w] * stg[(w * 16 + row) * (DV + 2) + c];
-    dst_o[row * DV + c] = v;
-  }
-  if (part == 0) {
-    dst_ml[row * 2 + 0] = M;
-    dst_ml[row * 2 + 1] = Ls;
-  }
-}
-
-// merge_warps for one warp: lanes 2r, 2r+1 take row r (< G <= 16), half of its columns each
+// Merge NW staged warp states ([w][16][DV+2]) into one state per row < G, by one
+// warp: lanes 2r, 2r+1 take row r (< G <= 16), half of its columns each; o is
+// written relative to the merged max M -> dst_o[row][DV], (M, L) -> dst_ml[row][2]
 template <int DV, int NW>
 __device__ __forceinline__ void merge_warps_w32(const float* stg, int G, float* dst_o, float* dst_ml, int lane) {
   const int row = lane >> 1, part = lane & 1;
