@@ -273,6 +273,48 @@ def compress_cache(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, heads: Heads,
     return kc, vc
 
 
+def append_plan(lens, Lmax: int, Lmax_cmp: int, l: int = 32, s: int = 16):
+    """Offsets for incremental decode: the newest token of a sequence of length L
+    completes compressed block i = (L - l) / s exactly when L >= l and (L - l) % s == 0;
+    that block's l tokens then start at row b*Lmax + i*s of the batched cache and its
+    summary goes to row b*Lmax_cmp + i. Returns (tok_offset, seq_len, cmp_offset) for
+    nsa_compress, with seq_len 0 for sequences whose newest token completes no block."""
+    tok, sl, co = [], [], []
+    for b, L in enumerate(int(x) for x in lens):
+        if L >= l and (L - l) % s == 0:
+            i = (L - l) // s
+            tok.append(b * Lmax + i * s)
+            sl.append(l)
+            co.append(b * Lmax_cmp + i)
+        else:
+            tok.append(b * Lmax)
+            sl.append(0)
+            co.append(b * Lmax_cmp)
+    return tok, sl, co
+
+
+def compress_append(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, k_cmp, v_cmp, heads: Heads, params: Params,
+                    ws=None) -> int:
+    """Incremental decode: after the batched caches [B, Lmax, H_kv, d] grew to `lens`
+    tokens (one new token per sequence since the last call), write the summary of
+    every block a newest token completed into the compressed caches
+    [B, Lmax_cmp, H_kv, d], in place, with one nsa_compress call. Returns the number
+    of blocks written (0: nothing to do, no launch)."""
+    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
+    Lc = int(k_cmp.shape[1])
+    lens_l = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
+    tok, sl, co = append_plan(lens_l, Lmax, Lc, params.l_cmp, params.stride)
+    n = sum(1 for x in sl if x > 0)
+    if n == 0:
+        return 0
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, B, 0, 0), k_cache.device)
+    nsa_compress(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, torch.tensor(tok, dtype=torch.int64),
+                 torch.tensor(sl, dtype=torch.int32), torch.tensor(co, dtype=torch.int64), heads, params, k_cmp,
+                 v_cmp, ws)
+    return n
+
+
 def prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, ws=None, want_sel=False,
             want_imp=False):
     """Returns out (and sel / imp when asked)."""

@@ -109,3 +109,24 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(nsa, "LIB_PATH", "/nonexistent/libnsa.so")
     with pytest.raises(ImportError):
         nsa.lib()
+
+
+def test_append_plan_matches_block_counts():
+    """Incremental decode: the newest token of a sequence of length L completes a
+    compressed block exactly when n_cmp(L) = n_cmp(L - 1) + 1, and that block is
+    number n_cmp(L) - 1 with tokens [i*s, i*s + l)."""
+    import random
+    rng = random.Random(5)
+    for l, s in ((32, 16), (32, 32), (64, 16), (16, 8)):
+        lens = [rng.randint(1, 3000) for _ in range(64)] + [l - 1, l, l + s - 1, l + s, 1]
+        Lmax, Lc = 4096, nsa.n_cmp(4096, l, s)
+        tok, sl, co = nsa.append_plan(lens, Lmax, Lc, l, s)
+        for b, L in enumerate(lens):
+            new_block = nsa.n_cmp(L, l, s) - nsa.n_cmp(L - 1, l, s)
+            assert new_block in (0, 1)
+            if new_block:
+                i = nsa.n_cmp(L, l, s) - 1
+                assert (sl[b], tok[b], co[b]) == (l, b * Lmax + i * s, b * Lc + i)
+                assert i * s + l == L   # the block ends at the newest token
+            else:
+                assert sl[b] == 0

@@ -143,3 +143,39 @@ def test_decode_varlen_sampled():
         order = np.argsort(lens)
         return [int(order[0]), int(order[len(lens) // 2]), int(order[-1])]
     NP.run_decode_case(cfg, None, batch_rows=pick)
+
+
+def test_decode_incremental_compressed_cache():
+    """A decode loop that appends one token per sequence and step and compresses each
+    newly completed block (compress_append) builds the same compressed caches as the
+    fp64 oracle compressing the grown sequences, and as one call over the whole cache."""
+    cfg = CFG["decode_64k"]
+    lens0, steps = [20, 100, 1001, 4090], 48
+    lens_end = [L + steps for L in lens0]
+    inp = W.make_decode_inputs(cfg, device="cuda", lens=lens_end, seed=31)
+    heads, par, op = NP.heads_of(cfg), NP.params_of(cfg), NP.oracle_params(cfg)
+    kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"],
+                                lens0, heads, par)
+    ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, len(lens0), 0, 0), "cuda")
+    written = 0
+    for step in range(1, steps + 1):
+        written += nsa.compress_append(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                       inp["pe_v"], [L + step for L in lens0], kc, vc, heads, par, ws=ws)
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws)
+    assert written == sum(nsa.n_cmp(L + steps) - nsa.n_cmp(L) for L in lens0)
+    kc1, vc1 = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                  inp["pe_v"], lens_end, heads, par)
+    w_ck, pe_k, w_cv, pe_v = (NP.f64(inp[x]) for x in ("w_ck", "pe_k", "w_cv", "pe_v"))
+    for b, L in enumerate(lens_end):
+        nc = nsa.n_cmp(L)
+        if nc == 0:
+            continue
+        kb, vb = NP.f64(inp["k_cache"][b, :L]), NP.f64(inp["v_cache"][b, :L])
+        NP.assert_close(NP.f64(kc[b, :nc]), O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"]), "appended k_cmp",
+                        relative_to_rms=True)
+        NP.assert_close(NP.f64(vc[b, :nc]), O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]), "appended v_cmp",
+                        relative_to_rms=True)
+        # same kernel arithmetic per block: at most a bf16 rounding step apart from one call
+        d = (kc[b, :nc].float() - kc1[b, :nc].float()).abs()
+        assert float(d.max()) <= 2.0 ** -7 * float(kc1[b, :nc].float().abs().max())
