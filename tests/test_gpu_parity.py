@@ -179,3 +179,21 @@ def test_decode_incremental_compressed_cache():
         # same kernel arithmetic per block: at most a bf16 rounding step apart from one call
         d = (kc[b, :nc].float() - kc1[b, :nc].float()).abs()
         assert float(d.max()) <= 2.0 ** -7 * float(kc1[b, :nc].float().abs().max())
+
+
+# GQA groups of 8, 2 and 1 heads take the other compile-time head reductions of the
+# importance; with them the remaining supported (d_k, d_v) pairs
+GROUP_SHAPES = [(8, 1, 128, 64), (4, 2, 64, 128), (4, 4, 192, 64)]
+
+
+@pytest.mark.parametrize("H_q,H_kv,d_k,d_v", GROUP_SHAPES)
+def test_prefill_group_sizes(H_q, H_kv, d_k, d_v):
+    """Ragged batch with an empty sequence and a one-token sequence."""
+    cfg = W.small_config(T=1100, H_q=H_q, H_kv=H_kv, d_k=d_k, d_v=d_v, top_n=16, window=256, seed=21)
+    NP.run_prefill_case(cfg, [0, 1100, 1, 257], n_random_rows=96, seed=21)
+
+
+@pytest.mark.parametrize("H_q,H_kv,d_k,d_v", GROUP_SHAPES)
+def test_decode_group_sizes(H_q, H_kv, d_k, d_v):
+    cfg = W.small_config(T=3000, H_q=H_q, H_kv=H_kv, d_k=d_k, d_v=d_v, top_n=16, window=256, seed=22)
+    NP.run_decode_case(cfg, lens=[3000, 1, 31, 32, 700], seed=22)
