@@ -40,6 +40,34 @@ DECODE = W.CONFIGS["decode_64k"]
 L2_FLUSH_BYTES = 256 << 20
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernels from one ncu capture each, valid only for the kernel source it was taken
+# on (the bench reports null once that file changes). The decode capture ran 8
+# sequences; its traffic is scaled to the bench's 32 (the stream is per sequence).
+NCU_TRAFFIC = {
+    "prefill_attn": dict(bytes=232.535808e6 + 102.639360e6, src="prefill.cu",
+                         sha1="fe74b5e0732b48a3b4ff97b468fa0b9e4100689f"),
+    "dec_cmp": dict(bytes=(84.101376e6 + 2.978816e6) * 32 / 8, src="decode.cu",
+                    sha1="8f90d6dfe658bdde1789419248f1040cb7999844"),
+}
+
+
+def ncu_traffic(kernel):
+    """Measured bytes per launch for `kernel`, or None when unknown or stale."""
+    import hashlib
+    e = NCU_TRAFFIC.get(kernel)
+    if e is None:
+        return None
+    path = os.path.join(ROOT, "sparse_attention_long_nsa_b200", "csrc", e["src"])
+    try:
+        with open(path, "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != e["sha1"]:
+                return None
+    except OSError:
+        return None
+    return e["bytes"]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -374,7 +402,7 @@ def run_nsa(args, rank, ws):
             "achieved": achieved, "peak": pk["tc"], "unit": "TFLOP/s",
             "frac": (achieved / pk["tc"]) if achieved else None,
             "peak_source": f"{pk['src']} bf16 dense (burst)",
-            "traffic": None,
+            "traffic": ncu_traffic(dominant),
             "ms_per_launch": dom_ms,
             "algorithmic_flop_per_launch": dom_flops,
         },
@@ -393,7 +421,7 @@ def run_nsa(args, rank, ws):
                          "achieved": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9) if d_dom_bytes else None,
                          "peak": pk["hbm"], "unit": "GB/s",
                          "frac": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9 / pk["hbm"]) if d_dom_bytes else None,
-                         "traffic": None},
+                         "traffic": ncu_traffic(d_dom)},
         },
         "cpu_baseline": cpu,
     }
