@@ -273,19 +273,23 @@ def compress_cache(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, heads: Heads,
     return kc, vc
 
 
-def append_plan(lens, Lmax: int, Lmax_cmp: int, l: int = 32, s: int = 16):
-    """Offsets for incremental decode: the newest token of a sequence of length L
-    completes compressed block i = (L - l) / s exactly when L >= l and (L - l) % s == 0;
-    that block's l tokens then start at row b*Lmax + i*s of the batched cache and its
-    summary goes to row b*Lmax_cmp + i. Returns (tok_offset, seq_len, cmp_offset) for
-    nsa_compress, with seq_len 0 for sequences whose newest token completes no block."""
+def append_plan(lens, Lmax: int, Lmax_cmp: int, l: int = 32, s: int = 16, lens_prev=None):
+    """Offsets for incremental decode: when a sequence grows from P to L tokens
+    (P = L - 1 unless lens_prev is given), the compressed blocks i with
+    n_cmp(P) <= i < n_cmp(L) are new; their tokens form one segment that starts at
+    row b*Lmax + n_cmp(P)*s of the batched cache and holds (count - 1)*s + l tokens,
+    and their summaries go to rows b*Lmax_cmp + n_cmp(P) onwards. Returns
+    (tok_offset, seq_len, cmp_offset) for nsa_compress, with seq_len 0 for sequences
+    that completed no block."""
+    lens = [int(x) for x in lens]
+    prev = [L - 1 for L in lens] if lens_prev is None else [int(x) for x in lens_prev]
     tok, sl, co = [], [], []
-    for b, L in enumerate(int(x) for x in lens):
-        if L >= l and (L - l) % s == 0:
-            i = (L - l) // s
-            tok.append(b * Lmax + i * s)
-            sl.append(l)
-            co.append(b * Lmax_cmp + i)
+    for b, (P, L) in enumerate(zip(prev, lens)):
+        i0, i1 = n_cmp(max(P, 0), l, s), n_cmp(L, l, s)
+        if i1 > i0:
+            tok.append(b * Lmax + i0 * s)
+            sl.append((i1 - 1 - i0) * s + l)
+            co.append(b * Lmax_cmp + i0)
         else:
             tok.append(b * Lmax)
             sl.append(0)
@@ -294,17 +298,19 @@ def append_plan(lens, Lmax: int, Lmax_cmp: int, l: int = 32, s: int = 16):
 
 
 def compress_append(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, k_cmp, v_cmp, heads: Heads, params: Params,
-                    ws=None) -> int:
-    """Incremental decode: after the batched caches [B, Lmax, H_kv, d] grew to `lens`
-    tokens (one new token per sequence since the last call), write the summary of
-    every block a newest token completed into the compressed caches
-    [B, Lmax_cmp, H_kv, d], in place, with one nsa_compress call. Returns the number
-    of blocks written (0: nothing to do, no launch)."""
+                    ws=None, lens_prev=None) -> int:
+    """Incremental decode: after the batched caches [B, Lmax, H_kv, d] grew from
+    `lens_prev` (default: one token less) to `lens` tokens, write the summaries of
+    every block completed in between into the compressed caches [B, Lmax_cmp, H_kv,
+    d], in place, with one nsa_compress call. Returns the number of blocks written
+    (0: nothing to do, no launch)."""
     B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
     Lc = int(k_cmp.shape[1])
     lens_l = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
-    tok, sl, co = append_plan(lens_l, Lmax, Lc, params.l_cmp, params.stride)
-    n = sum(1 for x in sl if x > 0)
+    prev_l = None if lens_prev is None else [int(x) for x in (lens_prev.tolist() if hasattr(lens_prev, "tolist")
+                                                                else lens_prev)]
+    tok, sl, co = append_plan(lens_l, Lmax, Lc, params.l_cmp, params.stride, lens_prev=prev_l)
+    n = sum(n_cmp(x, params.l_cmp, params.stride) for x in sl)
     if n == 0:
         return 0
     if ws is None:

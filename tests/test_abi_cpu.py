@@ -130,3 +130,22 @@ def test_append_plan_matches_block_counts():
                 assert i * s + l == L   # the block ends at the newest token
             else:
                 assert sl[b] == 0
+
+
+def test_append_plan_multi_token_growth():
+    """Growth by several tokens: the segment holds exactly the blocks completed
+    between the two lengths (the blocks nsa_compress finds in it)."""
+    import random
+    rng = random.Random(9)
+    for l, s in ((32, 16), (32, 32), (64, 16)):
+        prev = [rng.randint(0, 5000) for _ in range(64)] + [0, l - 1, l, 100]
+        lens = [P + rng.choice([0, 1, 7, 16, 33, 500]) for P in prev]
+        Lmax, Lc = 8192, nsa.n_cmp(8192, l, s)
+        tok, sl, co = nsa.append_plan(lens, Lmax, Lc, l, s, lens_prev=prev)
+        for b, (P, L) in enumerate(zip(prev, lens)):
+            new = list(range(nsa.n_cmp(P, l, s), nsa.n_cmp(L, l, s)))
+            got = [] if sl[b] == 0 else [(tok[b] - b * Lmax) // s + i for i in range(nsa.n_cmp(sl[b], l, s))]
+            assert got == new
+            if new:
+                assert co[b] == b * Lc + new[0] and (tok[b] - b * Lmax) % s == 0
+                assert (tok[b] - b * Lmax) + sl[b] <= L   # the segment ends inside the grown cache
