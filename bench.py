@@ -48,7 +48,7 @@ NCU_TRAFFIC = {
     "prefill_attn": dict(bytes=232.535808e6 + 102.639360e6, src="prefill.cu",
                          sha1="fe74b5e0732b48a3b4ff97b468fa0b9e4100689f"),
     "dec_cmp": dict(bytes=(84.101376e6 + 2.978816e6) * 32 / 8, src="decode.cu",
-                    sha1="8f90d6dfe658bdde1789419248f1040cb7999844"),
+                    sha1="dbff8042aebed087fa021e617ebdf2f0475b1f68"),
 }
 
 

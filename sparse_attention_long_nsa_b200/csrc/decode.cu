@@ -384,10 +384,10 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
 // ---------------------------------------------------------------------------
 // D3: selected blocks and window for one (sequence, KV head) per CTA. The
 // ascending union of the selected blocks and the blocks the window touches is
-// streamed once through the TMA ring in 32-key halves; consumer warp w takes
-// half-tiles w, w+4, ...; one score tile serves both branches, each with its own online
-// softmax. At the end the four warps' states are merged in shared memory and
-// out = g_cmp o_cmp + g_slc o_slc + g_win o_win is written.
+// streamed once through the TMA ring in 32-key halves; warps 0-3 (selected
+// branch) and 4-7 (window) take halves w, w+4, ... and compute on those their
+// branch reads, each warp with one online softmax. The warps' states are merged
+// in shared memory and out = g_cmp o_cmp + g_slc o_slc + g_win o_win is written.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeArgs a,
