@@ -73,7 +73,8 @@ def compress(x, W, pe, l: int, s: int) -> np.ndarray:
 
     Each block of l consecutive tokens starting at i*s gets the position
     embedding pe[r] added to its r-th token, is flattened token-major and mapped
-    by W [l*d, d_out].
+    by W [l*d, d_out]. The blocks are independent; they are evaluated a chunk of
+    blocks at a time (the same formula per block, gathered by token index).
     """
     x = np.asarray(x, dtype=np.float64)
     W = np.asarray(W, dtype=np.float64)
@@ -81,10 +82,13 @@ def compress(x, W, pe, l: int, s: int) -> np.ndarray:
     T, H, d = x.shape
     n = n_cmp(T, l, s)
     out = np.zeros((n, H, W.shape[1]))
-    for i in range(n):
-        blk = x[i * s:i * s + l] + pe[:, None, :]          # [l, H, d]
-        flat = blk.transpose(1, 0, 2).reshape(H, l * d)    # row r*d + e
-        out[i] = flat @ W
+    chunk = 256
+    for i0 in range(0, n, chunk):
+        i = np.arange(i0, min(n, i0 + chunk))
+        tok = i[:, None] * s + np.arange(l)[None, :]          # [c, l] token of row r of block i
+        blk = x[tok] + pe[None, :, None, :]                    # [c, l, H, d]
+        flat = blk.transpose(0, 2, 1, 3).reshape(len(i), H, l * d)   # row r*d + e
+        out[i0:i0 + len(i)] = flat @ W
     return out
 
 
@@ -244,9 +248,9 @@ def nsa_row(t, q_t, k, v, kc, vc, gates_t, p, sel_override=None):
         else:
             sel = select(imp, t, ls, p["top_n"], p["force_first"], p["force_local"])
         idx = selected_keys(sel, t, ls)
-        o_slc[g * G:(g + 1) * G], _ = attend(qg, k[idx, g], v[idx, g], scale)
+        o_slc[g * G:(g + 1) * G], _ = attend(qg, _take(k, idx, g), _take(v, idx, g), scale)
         widx = window_keys(t, p["window"])
-        o_win[g * G:(g + 1) * G], _ = attend(qg, k[widx, g], v[widx, g], scale)
+        o_win[g * G:(g + 1) * G], _ = attend(qg, _take(k, widx, g), _take(v, widx, g), scale)
         sels.append(sel)
         imps.append(imp)
     gt = np.asarray(gates_t, dtype=np.float64)
@@ -258,6 +262,15 @@ def _f64(x):
     if hasattr(x, "detach"):
         x = x.detach().to("cpu").double().numpy()
     return np.asarray(x, dtype=np.float64)
+
+
+def _take(x, idx, g):
+    """Rows idx of head g of x [T, H, d] as float64 (x a numpy array, or a torch
+    tensor of which only these rows are converted)."""
+    if hasattr(x, "detach"):
+        import torch
+        return _f64(x[torch.as_tensor(idx, dtype=torch.long, device=x.device), g])
+    return np.asarray(x[idx, g], dtype=np.float64)
 
 
 def prefill(q, k, v, kc, vc, gates, p, rows=None, sel_override=None):
@@ -312,7 +325,8 @@ def decode(q, k_cache, v_cache, kc_cache, vc_cache, lens, gates, p, batch_rows=N
         L = lens[b]
         t = L - 1
         nc = n_cmp(L, p["l_cmp"], p["stride"])
-        kb, vb = _f64(k_cache[b, :L]), _f64(v_cache[b, :L])
+        # raw keys/values stay in their own dtype; nsa_row converts the rows it reads
+        kb, vb = k_cache[b, :L], v_cache[b, :L]
         kcb, vcb = _f64(kc_cache[b, :nc]), _f64(vc_cache[b, :nc])
         ov = None
         if sel_override is not None:
