@@ -4,17 +4,19 @@
 
 One step = the whole hot path on one batch of synthetic input: block
 compression of K and V, compressed attention + block importance, top-n
-selection, selected-block attention, sliding-window attention + gated combine
-(the 8K prefill: B=1, T=8192, H_q=64, H_kv=4, d_k=192, d_v=128, l=32, stride 16,
-l'=64, top-n 16, w=512). The decode path (B=32 sequences, 64K cache each) is
-timed the same way and reported in the "decode" object of the same line.
+selection, selected-block attention, sliding-window attention + gated combine.
+The headline (`value`) is the largest prefill configuration: B=1, T=65536,
+H_q=64, H_kv=4, d_k=192, d_v=128, l=32, stride 16, l'=64, top-n 16, w=512. The
+same line carries the 8K prefill ("prefill_8k"), the 64K decode ("decode": B=32
+sequences, one query each) and the varlen decode ("decode_varlen": B=64, cache
+lengths drawn in [8192, 131072]), each timed the same way.
 
 N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
 workload (the path needs no exchange between GPUs: independent sequences);
 timings are the max over ranks, value = all ranks' tokens / that time.
 
 --impl reference times the CPU oracle (numpy fp64) on the host cores on a
-bounded sample of the same workload.
+bounded sample of the headline workload.
 """
 from __future__ import annotations
 
@@ -35,27 +37,31 @@ sys.path.insert(0, ROOT)
 import nsa_workloads as W  # noqa: E402
 
 METRIC = "NSA prefill tokens/s & % bf16 TC peak; 64k decode tokens/s & HBM GB/s"
-PREFILL = W.CONFIGS["prefill_8k"]
+PREFILL = W.CONFIGS["prefill_64k"]      # the headline: the largest prefill configuration
+PREFILL_8K = W.CONFIGS["prefill_8k"]
 DECODE = W.CONFIGS["decode_64k"]
+DECODE_VARLEN = W.CONFIGS["decode_varlen"]
 L2_FLUSH_BYTES = 256 << 20
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernels from one ncu capture each, valid only for the kernel source it was taken
-# on (the bench reports null once that file changes). The decode capture ran 8
-# sequences; its traffic is scaled to the bench's 32 (the stream is per sequence).
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel of a workload, from one ncu capture each, valid only for the
+# kernel source it was taken on (the bench reports null once that file changes).
+# Captures of a smaller case are scaled to the bench's launch by the units
+# processed when the traffic grows in proportion: the 64K decode capture ran 8 of
+# the 32 sequences (the compressed stream is per sequence).
 NCU_TRAFFIC = {
-    "prefill_attn": dict(bytes=232.535808e6 + 102.639360e6, src="prefill.cu",
-                         sha1="fe74b5e0732b48a3b4ff97b468fa0b9e4100689f"),
-    "dec_cmp": dict(bytes=(84.101376e6 + 2.978816e6) * 32 / 8, src="decode.cu",
-                    sha1="dbff8042aebed087fa021e617ebdf2f0475b1f68"),
+    ("prefill_attn", "prefill_8k"): dict(bytes=232.535808e6 + 102.639360e6, src="prefill.cu",
+                                         sha1="fe74b5e0732b48a3b4ff97b468fa0b9e4100689f"),
+    ("dec_cmp", "decode_64k"): dict(bytes=(84.101376e6 + 2.978816e6) * 32 / 8, src="decode.cu",
+                                    sha1="dbff8042aebed087fa021e617ebdf2f0475b1f68"),
 }
 
 
-def ncu_traffic(kernel):
-    """Measured bytes per launch for `kernel`, or None when unknown or stale."""
+def ncu_traffic(kernel, workload):
+    """Measured bytes per launch of `kernel` on `workload`, or None when unknown or stale."""
     import hashlib
-    e = NCU_TRAFFIC.get(kernel)
+    e = NCU_TRAFFIC.get((kernel, workload))
     if e is None:
         return None
     path = os.path.join(ROOT, "sparse_attention_long_nsa_b200", "csrc", e["src"])
@@ -103,16 +109,18 @@ def prefill_work(cfg):
                 dense_causal=T * (T + 1) // 2 * per_pair)
 
 
-def decode_bytes(cfg, lens, sel):
+def decode_bytes(cfg, lens, sel, per_seq=False):
     """Unique K/V bytes the decode must read: every compressed key, and the raw
     keys of the selected blocks united with the window (per KV head)."""
     row = (cfg.d_k + cfg.d_v) * 2
     cmp_b = 0
     fine_b = 0
+    seq = []
     sel = sel.cpu().numpy()
     for b, L in enumerate(lens):
         nc = (L - cfg.l_cmp) // cfg.stride + 1 if L >= cfg.l_cmp else 0
         t = L - 1
+        sb = 0
         for g in range(cfg.H_kv):
             keys = set(range(max(0, t - cfg.window + 1), t + 1))
             for j in sel[b, g]:
@@ -120,7 +128,9 @@ def decode_bytes(cfg, lens, sel):
                     keys.update(range(j * cfg.l_sel, min((j + 1) * cfg.l_sel, t + 1)))
             fine_b += len(keys) * row
             cmp_b += nc * row
-    return cmp_b, fine_b
+            sb += (len(keys) + nc) * row
+        seq.append(sb)
+    return (cmp_b, fine_b, seq) if per_seq else (cmp_b, fine_b)
 
 
 # ---------------------------------------------------------------------------
@@ -248,11 +258,36 @@ def timed_steps(step, steps, warmup, flush, ws):
     return max_over_ranks(ms, ws)
 
 
-def run_nsa(args, rank, ws):
+def _make_flush(dev):
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        # evict L2 by writing a buffer twice its size, then read it back so that L2
+        # holds clean lines: otherwise the write-back of ~126 MB of dirty lines
+        # competes with the first microseconds of the timed kernels
+        flush_buf.fill_(1)
+        flush_buf.view(torch.int32).max()
+    return flush
+
+
+def _profiled(step, steps, warmup, flush, ws):
+    """Per-kernel device time of `steps` calls of step() (the library's opt-in
+    event profiler; its events add gaps, so the step time is taken without it).
+    Returns ({kernel: (ms per call, launches per call)}, launches per call)."""
     import sparse_attention_long_nsa_b200 as nsa
-    dev = torch.device("cuda", torch.cuda.current_device())
-    pk = peaks()
-    cfg = PREFILL
+    nsa.nsa_profile_read()
+    nsa.nsa_profile_enable(True)
+    timed_steps(step, steps, warmup, flush, ws)
+    prof = nsa.nsa_profile_read()
+    nsa.nsa_profile_enable(False)
+    n_calls = steps + warmup   # the profile covers warm-up + timed calls
+    kern = {k: (v[0] / n_calls, v[1] / n_calls) for k, v in prof.items() if v[1] > 0}
+    return kern, sum(v[1] for v in kern.values())
+
+
+def bench_prefill(cfg, args, rank, ws, dev, pk, e2e=False, clocks=False):
+    """One step = nsa_compress + nsa_prefill of one sequence of cfg.T tokens."""
+    import sparse_attention_long_nsa_b200 as nsa
     heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
     par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
                           cfg.force_local)
@@ -267,14 +302,7 @@ def run_nsa(args, rank, ws):
     ws_p = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, heads, par, 1, T, T), dev)
     tok = torch.zeros(1, dtype=torch.int64)
     seq = torch.tensor([T], dtype=torch.int32)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def flush():
-        # evict L2 by writing a buffer twice its size, then read it back so that L2
-        # holds clean lines: otherwise the write-back of ~126 MB of dirty lines
-        # competes with the first microseconds of the timed kernels
-        flush_buf.fill_(1)
-        flush_buf.view(torch.int32).max()
+    flush = _make_flush(dev)
 
     def step():
         nsa.nsa_compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], tok, seq, tok,
@@ -282,119 +310,26 @@ def run_nsa(args, rank, ws):
         nsa.nsa_prefill(inp["q"], inp["k"], inp["v"], k_cmp, v_cmp, inp["gates"], cu, heads, par, out, None, None,
                         ws_p)
 
-    # ---- device-timed prefill (the step alone), then a second timed region with
-    # the library's per-kernel event profiler on: its events sit between the
-    # kernels and add gaps, so the step time is taken without them
     step()
     torch.cuda.synchronize()
     nsa.nsa_check_device_status(ws_p)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        ms = timed_steps(step, args.steps, args.warmup, flush, ws)
-    nsa.nsa_profile_read()
-    nsa.nsa_profile_enable(True)
-    psteps = min(args.steps, 50)
-    timed_steps(step, psteps, args.warmup, flush, ws)
-    prof = nsa.nsa_profile_read()
-    nsa.nsa_profile_enable(False)
+    steps = args.steps
+    clk = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if clk:
+        clk.__enter__()
+    ms = timed_steps(step, steps, args.warmup, flush, ws)
+    if clk:
+        clk.__exit__(None, None, None)
+    kern, launches = _profiled(step, min(steps, 20), args.warmup, flush, ws)
     nsa.nsa_check_device_status(ws_p)
-    # the profile covers warm-up + timed steps of the profiled region
-    n_calls = psteps + args.warmup
-    launches = sum(c for _, c in prof.values())
     work = prefill_work(cfg)
-    kern = {k: v for k, v in prof.items() if v[1] > 0}
     dominant = max(kern, key=lambda k: kern[k][0])
     dom_ms = kern[dominant][0] / kern[dominant][1]
     dom_flops = work.get(dominant, 0)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_flops else None
-    tokens = T * ws
-    value = tokens / (ms * 1e-3)
-
-    # ---- end to end through the C ABI with host buffers
-    host = {k: inp[k].to("cpu").pin_memory() for k in ("q", "k", "v", "gates", "w_ck", "pe_k", "w_cv", "pe_v")}
-    dev_bufs = {k: torch.empty_like(inp[k]) for k in host}
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-
-    def e2e_step():
-        for k_, t_ in host.items():
-            dev_bufs[k_].copy_(t_, non_blocking=True)
-        nsa.nsa_compress(dev_bufs["k"], dev_bufs["v"], dev_bufs["w_ck"], dev_bufs["pe_k"], dev_bufs["w_cv"],
-                         dev_bufs["pe_v"], tok, seq, tok, heads, par, k_cmp, v_cmp, ws_c)
-        nsa.nsa_prefill(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], k_cmp, v_cmp, dev_bufs["gates"], cu, heads,
-                        par, out, None, None, ws_p)
-        out_host.copy_(out, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 30))
-    ms_e2e = timed_steps(e2e_step, e2e_steps, args.warmup, flush, ws)
-    torch.cuda.synchronize()
-
-    # ---- decode (64K cache, B=32): caches built once, then timed
-    dcfg = DECODE
-    dinp = W.make_decode_inputs(dcfg, device=dev, seed=dcfg.seed + 97 * rank)
-    dheads = nsa.Heads(dcfg.H_q, dcfg.H_kv, dcfg.d_k, dcfg.d_v)
-    dpar = nsa.make_params(dcfg.l_cmp, dcfg.stride, dcfg.l_sel, dcfg.top_n, dcfg.window, dcfg.force_first,
-                           dcfg.force_local)
-    lens = dinp["cache_lens"]
-    kc, vc = nsa.compress_cache(dinp["k_cache"], dinp["v_cache"], dinp["w_ck"], dinp["pe_k"], dinp["w_cv"],
-                                dinp["pe_v"], lens, dheads, dpar)
-    lens_d = lens.to(dev)
-    Lmax = int(dinp["k_cache"].shape[1])
-    ws_d = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_DECODE, dheads, dpar, dcfg.B, 0, Lmax), dev)
-    dout = torch.empty((dcfg.B, dcfg.H_q, dcfg.d_v), dtype=torch.bfloat16, device=dev)
-    dsel = torch.empty((dcfg.B, dcfg.H_kv, dcfg.top_n), dtype=torch.int32, device=dev)
-
-    def dstep():
-        nsa.nsa_decode(dinp["q"], dinp["k_cache"], dinp["v_cache"], kc, vc, lens_d, Lmax, dinp["gates"], dheads,
-                       dpar, dout, dsel, None, ws_d)
-
-    dstep()
-    torch.cuda.synchronize()
-    nsa.nsa_check_device_status(ws_d)
-    dsteps = max(args.steps, 20)
-    dms = timed_steps(dstep, dsteps, args.warmup, flush, ws)
-    nsa.nsa_check_device_status(ws_d)
-    nsa.nsa_profile_read()
-    nsa.nsa_profile_enable(True)
-    dpsteps = min(dsteps, 50)
-    timed_steps(dstep, dpsteps, args.warmup, flush, ws)
-    dprof = nsa.nsa_profile_read()
-    nsa.nsa_profile_enable(False)
-    cmp_b, fine_b = decode_bytes(dcfg, [int(x) for x in lens], dsel)
-    dbytes = cmp_b + fine_b
-    dgbs = dbytes / (dms * 1e-3) / 1e9
-    dk = {k: v for k, v in dprof.items() if v[1] > 0}
-    d_dom = max(dk, key=lambda k: dk[k][0])
-    d_dom_ms = dk[d_dom][0] / dk[d_dom][1]
-    d_dom_bytes = cmp_b if d_dom == "dec_cmp" else (fine_b if d_dom == "dec_fine" else None)
-
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = oracle_prefill_rate(inp, cfg, budget_s=args.cpu_seconds)
-
-    if rank != 0:
-        return None
     res = {
-        "metric": METRIC,
-        "value": value,
-        "unit": "tokens/s",
-        "n_gpus": ws,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) q/k/v, N(0,1/(l*d)) compression weights, sigmoid(N(0,1)) gates)",
-        "config": {
-            "workload": "prefill_8k: B=1 T=8192 causal, H_q=64 H_kv=4, d_k=192 d_v=128, l=32 stride=16 "
-                        "l'=64 top-n=16 (1 initial + 2 local forced) w=512; step = nsa_compress + nsa_prefill",
-            "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
-            "l2": "flushed before every timed step (256 MB write, then a read of it, outside the events)",
-            "useful_flop_per_step": work["total"], "dense_causal_flop_per_step": work["dense_causal"],
-        },
+        "tokens_per_s": T * ws / (ms * 1e-3), "ms_per_step": ms,
+        "useful_flop_per_step": work["total"], "dense_causal_flop_per_step": work["dense_causal"],
         "tflops_useful": work["total"] / (ms * 1e-3) / 1e12 * ws,
         "tc_frac_useful": work["total"] / (ms * 1e-3) / 1e12 / pk["tc"],
         "roofline": {
@@ -402,29 +337,169 @@ def run_nsa(args, rank, ws):
             "achieved": achieved, "peak": pk["tc"], "unit": "TFLOP/s",
             "frac": (achieved / pk["tc"]) if achieved else None,
             "peak_source": f"{pk['src']} bf16 dense (burst)",
-            "traffic": ncu_traffic(dominant),
+            "traffic": ncu_traffic(dominant, cfg.name),
             "ms_per_launch": dom_ms,
             "algorithmic_flop_per_launch": dom_flops,
         },
-        "kernels_ms_per_step": {k: v[0] / n_calls for k, v in kern.items()},
-        "gpu_launches": int(round(launches / n_calls)) * args.steps,
-        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "clocks": clk.summary(),
-        "decode": {
-            "workload": "decode_64k: B=32 x 1 query, cache 65536 each, H_q=64 H_kv=4, d_k=192 d_v=128",
-            "tokens_per_s": dcfg.B * ws / (dms * 1e-3), "ms_per_step": dms,
-            "bytes_per_step": dbytes, "bytes_compressed": cmp_b, "bytes_fine": fine_b,
-            "hbm_gbs": dgbs, "hbm_frac": dgbs / pk["hbm"], "hbm_peak_gbs": pk["hbm"],
-            "kernels_ms_per_step": {k: v[0] / (dpsteps + args.warmup) for k, v in dk.items()},
-            "roofline": {"kernel": d_dom, "bound": "hbm",
-                         "achieved": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9) if d_dom_bytes else None,
-                         "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9 / pk["hbm"]) if d_dom_bytes else None,
-                         "traffic": ncu_traffic(d_dom)},
+        "kernels_ms_per_step": {k: v[0] for k, v in kern.items()},
+        "launches_per_step": launches,
+    }
+    if clk:
+        res["clocks"] = clk.summary()
+    if e2e:
+        # end to end through the C ABI with host buffers: H2D of the step's inputs
+        # from pinned memory and D2H of the output inside the timed region
+        host = {k: inp[k].to("cpu").pin_memory() for k in ("q", "k", "v", "gates", "w_ck", "pe_k", "w_cv", "pe_v")}
+        dev_bufs = {k: torch.empty_like(inp[k]) for k in host}
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            for k_, t_ in host.items():
+                dev_bufs[k_].copy_(t_, non_blocking=True)
+            nsa.nsa_compress(dev_bufs["k"], dev_bufs["v"], dev_bufs["w_ck"], dev_bufs["pe_k"], dev_bufs["w_cv"],
+                             dev_bufs["pe_v"], tok, seq, tok, heads, par, k_cmp, v_cmp, ws_c)
+            nsa.nsa_prefill(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], k_cmp, v_cmp, dev_bufs["gates"], cu, heads,
+                            par, out, None, None, ws_p)
+            out_host.copy_(out, non_blocking=True)
+
+        ms_e2e = timed_steps(e2e_step, max(3, min(steps, 10)), args.warmup, flush, ws)
+        torch.cuda.synchronize()
+        res["e2e"] = {"value": T * ws / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+                      "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+        del host, dev_bufs, out_host
+    res["_inp"] = inp
+    return res
+
+
+def bench_decode(cfg, args, rank, ws, dev, pk):
+    """One step = nsa_decode of the batch (compressed caches built once before)."""
+    import sparse_attention_long_nsa_b200 as nsa
+    dinp = W.make_decode_inputs(cfg, device=dev, seed=cfg.seed + 97 * rank)
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                          cfg.force_local)
+    lens = dinp["cache_lens"]
+    kc, vc = nsa.compress_cache(dinp["k_cache"], dinp["v_cache"], dinp["w_ck"], dinp["pe_k"], dinp["w_cv"],
+                                dinp["pe_v"], lens, heads, par)
+    lens_d = lens.to(dev)
+    Lmax = int(dinp["k_cache"].shape[1])
+    B = len(lens)
+    ws_d = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_DECODE, heads, par, B, 0, Lmax), dev)
+    dout = torch.empty((B, cfg.H_q, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    dsel = torch.empty((B, cfg.H_kv, cfg.top_n), dtype=torch.int32, device=dev)
+    flush = _make_flush(dev)
+
+    def dstep():
+        nsa.nsa_decode(dinp["q"], dinp["k_cache"], dinp["v_cache"], kc, vc, lens_d, Lmax, dinp["gates"], heads,
+                       par, dout, dsel, None, ws_d)
+
+    dstep()
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws_d)
+    dsteps = max(args.steps, 20)
+    dms = timed_steps(dstep, dsteps, args.warmup, flush, ws)
+    nsa.nsa_check_device_status(ws_d)
+    kern, launches = _profiled(dstep, min(dsteps, 50), args.warmup, flush, ws)
+    lens_l = [int(x) for x in lens]
+    cmp_b, fine_b, per_seq = decode_bytes(cfg, lens_l, dsel, per_seq=True)
+    dbytes = cmp_b + fine_b
+    dgbs = dbytes / (dms * 1e-3) / 1e9
+    d_dom = max(kern, key=lambda k: kern[k][0])
+    d_dom_ms = kern[d_dom][0] / kern[d_dom][1]
+    d_dom_bytes = cmp_b if d_dom == "dec_cmp" else (fine_b if d_dom == "dec_fine" else None)
+    nominal = 8000.0
+    res = {
+        "tokens_per_s": B * ws / (dms * 1e-3), "ms_per_step": dms,
+        "bytes_per_step": dbytes, "bytes_compressed": cmp_b, "bytes_fine": fine_b,
+        "bytes_per_token": dbytes / B,
+        "hbm_gbs": dgbs, "hbm_frac": dgbs / pk["hbm"], "hbm_peak_gbs": pk["hbm"],
+        "hbm_peak_source": f"{pk['src']} copy bandwidth (read+write)",
+        "hbm_frac_vs_8tbs_nominal": dgbs / nominal,
+        "kernels_ms_per_step": {k: v[0] for k, v in kern.items()},
+        "launches_per_step": launches,
+        "roofline": {"kernel": d_dom, "bound": "hbm",
+                     "achieved": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9) if d_dom_bytes else None,
+                     "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": (d_dom_bytes / (d_dom_ms * 1e-3) / 1e9 / pk["hbm"]) if d_dom_bytes else None,
+                     "traffic": ncu_traffic(d_dom, cfg.name)},
+    }
+    if len(set(lens_l)) > 1:
+        # load balance of the ragged batch: bytes per sequence, and the compressed
+        # pass's 512-key work items per CTA of its persistent grid
+        items = sum(cfg.H_kv * -(-nsa.n_cmp(L) // 512) for L in lens_l)
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        grid = min(items, n_sm)
+        res["load_balance"] = {
+            "cache_len_min": min(lens_l), "cache_len_max": max(lens_l),
+            "bytes_per_seq_min": min(per_seq), "bytes_per_seq_max": max(per_seq),
+            "bytes_per_seq_mean": sum(per_seq) / len(per_seq),
+            "dec_cmp_items": items, "dec_cmp_ctas": grid,
+            "dec_cmp_items_per_cta_max": -(-items // grid), "dec_cmp_items_per_cta_mean": items / grid,
+            "dec_fine_ctas": B * cfg.H_kv,
+        }
+    return res
+
+
+def run_nsa(args, rank, ws):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk = peaks()
+    head = bench_prefill(PREFILL, args, rank, ws, dev, pk, e2e=True, clocks=True)
+    inp64 = head.pop("_inp")
+    # CPU baseline: the oracle on a bounded sample of the headline workload
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = oracle_prefill_rate(inp64, PREFILL, budget_s=args.cpu_seconds, last_rows=512)
+    del inp64
+    torch.cuda.empty_cache()
+    p8 = bench_prefill(PREFILL_8K, args, rank, ws, dev, pk)
+    p8.pop("_inp")
+    torch.cuda.empty_cache()
+    dec = bench_decode(DECODE, args, rank, ws, dev, pk)
+    torch.cuda.empty_cache()
+    dvar = bench_decode(DECODE_VARLEN, args, rank, ws, dev, pk)
+    if rank != 0:
+        return None
+    cfg = PREFILL
+    launches = head.pop("launches_per_step")
+    res = {
+        "metric": METRIC,
+        "value": head["tokens_per_s"],
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, N(0,1/(l*d)) compression weights, sigmoid(N(0,1)) gates)",
+        "config": {
+            "workload": "prefill_64k: B=1 T=65536 causal, H_q=64 H_kv=4, d_k=192 d_v=128, l=32 stride=16 "
+                        "l'=64 top-n=16 (1 initial + 2 local forced) w=512; step = nsa_compress + nsa_prefill",
+            "global_batch": ws, "seq_len": cfg.T, "parallelism": f"replicas x{ws}",
+            "l2": "flushed before every timed step (256 MB write, then a read of it, outside the events); "
+                  "the inputs (2.8 GB) are also larger than L2",
+            "useful_flop_per_step": head["useful_flop_per_step"],
+            "dense_causal_flop_per_step": head["dense_causal_flop_per_step"],
         },
+        "tflops_useful": head["tflops_useful"],
+        "tc_frac_useful": head["tc_frac_useful"],
+        "roofline": head["roofline"],
+        "kernels_ms_per_step": head["kernels_ms_per_step"],
+        "gpu_launches": int(round(launches)) * args.steps,
+        "e2e": head["e2e"],
+        "clocks": head["clocks"],
+        "prefill_8k": dict(p8, workload="prefill_8k: as prefill_64k with T=8192"),
+        "decode": dict(dec, workload="decode_64k: B=32 x 1 query, cache 65536 each, H_q=64 H_kv=4, "
+                                     "d_k=192 d_v=128"),
+        "decode_varlen": dict(dvar, workload="decode_varlen: B=64 x 1 query, cache lengths drawn uniformly in "
+                                             "[8192, 131072] (seeded), H_q=64 H_kv=4, d_k=192 d_v=128"),
         "cpu_baseline": cpu,
     }
+    for d in (res["prefill_8k"], res["decode"], res["decode_varlen"]):
+        d.pop("launches_per_step", None)
     return res
 
 
@@ -441,13 +516,10 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def oracle_prefill_rate(inp, cfg, budget_s=15.0, max_rows=None):
-    """Oracle tokens/s on the 8K prefill: the full compression of K and V, plus
-    evenly spaced query rows until the time budget is spent; the rate is T over
-    (compression time + T x mean time per row)."""
+def _oracle_inputs(inp, cfg):
+    """fp64 K/V and the oracle's own compression of them (timed)."""
     from oracle import nsa_oracle as O
     p = cfg.params()
-    T = cfg.T
     k = inp["k"].double().cpu().numpy()
     v = inp["v"].double().cpu().numpy()
     t0 = time.perf_counter()
@@ -455,88 +527,142 @@ def oracle_prefill_rate(inp, cfg, budget_s=15.0, max_rows=None):
                     p["stride"])
     vc = O.compress(v, inp["w_cv"].double().cpu().numpy(), inp["pe_v"].double().cpu().numpy(), p["l_cmp"],
                     p["stride"])
-    t_cmp = time.perf_counter() - t0
-    q = inp["q"]
-    g = inp["gates"]
-    order = np.random.default_rng(0).permutation(T)
-    done = 0
+    return k, v, kc, vc, time.perf_counter() - t0
+
+
+def _oracle_rows(inp, cfg, k, v, kc, vc, rows):
+    """Wall time of the oracle over the given query rows."""
+    from oracle import nsa_oracle as O
     t1 = time.perf_counter()
-    while done < T and (time.perf_counter() - t1) < budget_s and (max_rows is None or done < max_rows):
-        batch = order[done:done + 16]
-        O.prefill(q, k, v, kc, vc, g, p, rows=batch.tolist())
-        done += len(batch)
-    t_rows = time.perf_counter() - t1
+    for i in range(0, len(rows), 16):
+        O.prefill(inp["q"], k, v, kc, vc, inp["gates"], cfg.params(), rows=[int(r) for r in rows[i:i + 16]])
+    return time.perf_counter() - t1
+
+
+def oracle_prefill_rate(inp, cfg, budget_s=15.0, max_rows=None, last_rows=0):
+    """Oracle tokens/s on a prefill workload: the full compression of K and V, plus
+    query rows drawn uniformly until the time budget is spent; the rate is T over
+    (compression time + T x mean time per row). With last_rows, the last rows of
+    the sequence (the most expensive ones) are also timed, within the same budget,
+    and reported as a labelled rows/s slice."""
+    T = cfg.T
+    k, v, kc, vc, t_cmp = _oracle_inputs(inp, cfg)
+    order = np.random.default_rng(0).permutation(T)
+    done, t_rows = 0, 0.0
+    while done < T and t_rows < budget_s and (max_rows is None or done < max_rows):
+        t_rows += _oracle_rows(inp, cfg, k, v, kc, vc, order[done:done + 16])
+        done += len(order[done:done + 16])
     est = t_cmp + T * t_rows / max(done, 1)
-    return {"value": T / est, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"full K/V compression ({t_cmp:.1f} s) + {done} of {T} query rows drawn uniformly "
-                      f"({t_rows:.1f} s); rate = T / (compression + T x mean row time)",
-            "host_cpus": os.cpu_count()}
+    res = {"value": T / est, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+           "sample": f"{cfg.name}: full K/V compression ({t_cmp:.1f} s) + {done} of {T} query rows drawn "
+                     f"uniformly ({t_rows:.1f} s); rate = T / (compression + T x mean row time)",
+           "host_cpus": os.cpu_count()}
+    if last_rows:
+        tail, t_tail = np.arange(T - 1, T - 1 - last_rows, -1), 0.0
+        n = 0
+        while n < len(tail) and t_tail < budget_s:
+            t_tail += _oracle_rows(inp, cfg, k, v, kc, vc, tail[n:n + 16])
+            n += len(tail[n:n + 16])
+        res["last_rows_slice"] = {"rows": n, "of_last": last_rows, "seconds": t_tail, "rows_per_s": n / t_tail,
+                                  "note": "query rows T-1 downwards (the most expensive), compression excluded"}
+    return res
 
 
 def run_reference(args, rank, ws):
+    """The oracle on the host cores, on the nsa arm's workload: the compression of
+    K and V is timed once; every step then times the oracle on 16 query rows drawn
+    uniformly (a bounded sample). value = T / (compression + T x mean row time);
+    ms_per_step is the measured wall time of one step's sample."""
     if rank != 0:
         return None
     cfg = PREFILL
     inp = W.make_prefill_inputs(cfg, device="cpu")
-    vals = []
-    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    k, v, kc, vc, t_cmp = _oracle_inputs(inp, cfg)
+    rng = np.random.default_rng(0)
+    times, rows_done = [], 0
     for i in range(args.warmup + args.steps):
-        r = oracle_prefill_rate(inp, cfg, budget_s=budget, max_rows=64)
+        rows = rng.choice(cfg.T, size=16, replace=False)
+        dt = _oracle_rows(inp, cfg, k, v, kc, vc, rows)
         if i >= args.warmup:
-            vals.append(r)
-    value = float(np.mean([r["value"] for r in vals]))
-    ms = cfg.T / value * 1e3
+            times.append(dt)
+            rows_done += len(rows)
+    row_s = sum(times) / rows_done
+    value = cfg.T / (t_cmp + cfg.T * row_s)
+    sample = (f"{cfg.name}: K/V compression timed once ({t_cmp:.1f} s), then 16 uniformly drawn query rows per "
+              f"step ({rows_done} rows over {args.steps} steps); rate = T / (compression + T x mean row time)")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill_8k (as the nsa arm), CPU oracle on a bounded sample per step",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / len(times) * 1e3,
+        "ms_per_step_basis": "measured wall time of one step's bounded sample (16 rows); value extrapolates "
+                             "the sampled rate to the whole sequence",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} (as the nsa arm), CPU oracle on a bounded sample per step",
                    "global_batch": 1, "seq_len": cfg.T, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": vals[-1]["cores"], "kind": "oracle",
-                         "sample": vals[-1]["sample"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def run_case(case):
-    """Two untimed invocations of one workload, for kernel profilers (no JSON line):
-    prefill = compression + prefill of the 8K workload; decode = 8 sequences of the
-    64K decode workload."""
+def _prefill_case(cfg, dev):
     import sparse_attention_long_nsa_b200 as nsa
+    inp = W.make_prefill_inputs(cfg, device=dev)
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                          cfg.force_local)
+    for _ in range(2):
+        kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [cfg.T],
+                              heads, par)
+        nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par)
+
+
+def _decode_case(cfg, dev, lens=None):
+    import sparse_attention_long_nsa_b200 as nsa
+    inp = W.make_decode_inputs(cfg, device=dev, lens=lens)
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                          cfg.force_local)
+    kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                inp["pe_v"], inp["cache_lens"], heads, par)
+    lens_d = inp["cache_lens"].to(dev)
+    for _ in range(2):
+        nsa.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens_d, int(inp["k_cache"].shape[1]),
+                   inp["gates"], heads, par)
+
+
+# Workloads for kernel profilers (two untimed invocations, no JSON line):
+#   prefill        compression + prefill of the 8K workload
+#   prefill64k_g1  the 64K prefill with one KV group (H_q=16, H_kv=1): the same
+#                  kernel on a quarter of the work units (grid.y = KV groups), for a
+#                  DRAM-traffic capture that stays a few GB on the device
+#   decode         8 sequences of the 64K decode workload
+#   decode_varlen  the varlen decode batch
+CASES = ("prefill", "prefill64k_g1", "decode", "decode_varlen")
+
+
+def run_case(case):
+    import dataclasses
     dev = torch.device("cuda", 0)
     if case == "prefill":
-        cfg = PREFILL
-        inp = W.make_prefill_inputs(cfg, device=dev)
-        heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
-        par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
-                              cfg.force_local)
-        for _ in range(2):
-            kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [cfg.T],
-                                  heads, par)
-            nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par)
+        _prefill_case(PREFILL_8K, dev)
+    elif case == "prefill64k_g1":
+        _prefill_case(dataclasses.replace(PREFILL, name="prefill_64k_g1", H_q=16, H_kv=1), dev)
+    elif case == "decode":
+        _decode_case(DECODE, dev, lens=[DECODE.T] * 8)
     else:
-        cfg = DECODE
-        inp = W.make_decode_inputs(cfg, device=dev, lens=[cfg.T] * 8)
-        heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
-        par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
-                              cfg.force_local)
-        kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
-                                    inp["pe_v"], inp["cache_lens"], heads, par)
-        lens = inp["cache_lens"].to(dev)
-        for _ in range(2):
-            nsa.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens, cfg.T, inp["gates"], heads, par)
+        _decode_case(DECODE_VARLEN, dev)
     torch.cuda.synchronize()
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["nsa", "reference"], default="nsa")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--case", choices=list(CASES), default=None,
                     help="run two untimed invocations of one workload for a profiler, print nothing")
     args = ap.parse_args()
     if args.case:

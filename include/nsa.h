@@ -118,6 +118,38 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
                           const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
                           void* v_cmp, void* workspace, size_t ws_bytes, void* stream);
 
+/* Incremental decode (NSA-ru "NSA: три ветви", compression branch: a summary
+ * exists for every whole block of l_cmp tokens at stride `stride`; the cache
+ * grows one token, or several, at a time). When sequence b of a batched cache
+ * [batch, Lmax, H_kv, d] grows from lens_prev[b] to lens[b] tokens, the blocks
+ * i with n_cmp(lens_prev[b]) <= i < n_cmp(lens[b]) are completed; their tokens
+ * form one segment starting at row b*Lmax + i0*stride. HOST-only planning:
+ *   lens_prev  HOST int32 [batch] or NULL (NULL: lens[b] - 1, one new token)
+ *   lens       HOST int32 [batch], lens_prev[b] <= lens[b] <= Lmax
+ *   tok_offset, seq_len, cmp_offset  HOST out [batch]: the arguments of the
+ *              nsa_compress call that writes the new summaries into rows
+ *              b*Lmax_cmp + i of a compressed cache [batch, Lmax_cmp, H_kv, d]
+ *              (seq_len 0 for sequences that completed no block)
+ *   n_blocks   HOST out or NULL: number of summaries to write
+ * NSA_ERR_INVALID_ARG for inconsistent lengths or Lmax_cmp < n_cmp(Lmax). Any
+ * l_cmp that is a multiple of `stride` is planned (only `l_cmp`, `stride` of
+ * params are read); nsa_compress_append checks what the kernels support. */
+nsa_status_t nsa_compress_append_plan(const int32_t* lens_prev, const int32_t* lens, int32_t batch, int32_t Lmax,
+                                      int32_t Lmax_cmp, const nsa_params_t* params, int64_t* tok_offset,
+                                      int32_t* seq_len, int64_t* cmp_offset, int32_t* n_blocks);
+
+/* Plans as nsa_compress_append_plan and writes the new summaries in place with
+ * one nsa_compress call on `stream` (no launch when no block was completed).
+ * k_cache/v_cache: bf16 [batch, Lmax, H_kv, d_k / d_v]; k_cmp_cache/v_cmp_cache:
+ * bf16 [batch, Lmax_cmp, H_kv, d_k / d_v]; n_blocks: HOST out or NULL. The
+ * workspace is that of nsa_compress (nsa_workspace_size(NSA_OP_COMPRESS, ...,
+ * batch, 0, 0) suffices). */
+nsa_status_t nsa_compress_append(const void* k_cache, const void* v_cache, const float* w_ck, const float* pe_k,
+                                 const float* w_cv, const float* pe_v, const int32_t* lens_prev, const int32_t* lens,
+                                 int32_t batch, int32_t Lmax, int32_t Lmax_cmp, const nsa_heads_t* heads,
+                                 const nsa_params_t* params, void* k_cmp_cache, void* v_cmp_cache,
+                                 int32_t* n_blocks, void* workspace, size_t ws_bytes, void* stream);
+
 /* nsa_compress without a workspace argument, for callers that cannot allocate
  * device memory where they compress: code that runs while a CUDA graph is being
  * captured, engines that fix their memory plan ahead of time and forbid
@@ -187,6 +219,47 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
                         int32_t max_len, const float* gates, const nsa_heads_t* heads,
                         const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Paged KV cache (the same decode as nsa_decode; NSA-lesson introduction: at
+ * long context decode is dominated by reading the KV cache, which serving
+ * systems keep in fixed-size pages). Raw keys/values live in pools of pages:
+ *   k_pool       bf16 [n_pages, page_size, H_kv, d_k]; v_pool likewise with d_v
+ *   block_table  DEVICE int32 [batch, max_pages]: token t of sequence b is row
+ *                t % page_size of page block_table[b][t / page_size]
+ * and the compressed summaries in pools of their own pages:
+ *   k_cmp_pool   bf16 [n_cmp_pages, cmp_page_size, H_kv, d_k]; v_cmp_pool with d_v
+ *   cmp_block_table DEVICE int32 [batch, max_cmp_pages]: summary i of sequence b
+ *                is row i % cmp_page_size of page cmp_block_table[b][i / cmp_page_size]
+ * page_size must be a multiple of 64 (a selection block and a 32-key tile never
+ * straddle pages) and cmp_page_size a multiple of 32 (nor does a tile of 32
+ * summaries). Only the pages a sequence's length reaches are read. Page ids
+ * outside [0, n_pages) are recorded in the status word (nsa_check_device_status
+ * then reports NSA_ERR_DEVICE_CHECK) and read as page 0. Other arguments as in
+ * nsa_decode; max_len <= max_pages * page_size. Results are identical to
+ * nsa_decode on the same contents laid out contiguously. */
+nsa_status_t nsa_decode_paged(const void* q, const void* k_pool, const void* v_pool, int32_t n_pages,
+                              int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                              const void* k_cmp_pool, const void* v_cmp_pool, int32_t n_cmp_pages,
+                              int32_t cmp_page_size, const int32_t* cmp_block_table, int32_t max_cmp_pages,
+                              const int32_t* cache_lens, int32_t batch, int32_t max_len, const float* gates,
+                              const nsa_heads_t* heads, const nsa_params_t* params, void* out, int32_t* sel_out,
+                              float* imp_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Compression into paged caches (layouts as in nsa_decode_paged): writes the
+ * summaries of the blocks completed while the sequences grew from lens_prev to
+ * lens tokens (HOST int32 [batch]; lens_prev NULL means lens - 1; all zeros
+ * builds the whole compressed cache), reading the raw tokens through
+ * block_table and writing through cmp_block_table. n_blocks: HOST out or NULL.
+ * Results are identical to nsa_compress on the same contents laid out
+ * contiguously. Invalid page ids are recorded in the status word (the rows they
+ * would read are taken as zeros, the rows they would write are skipped). */
+nsa_status_t nsa_compress_paged(const void* k_pool, const void* v_pool, int32_t n_pages, int32_t page_size,
+                                const int32_t* block_table, int32_t max_pages, const float* w_ck, const float* pe_k,
+                                const float* w_cv, const float* pe_v, const int32_t* lens_prev, const int32_t* lens,
+                                int32_t batch, void* k_cmp_pool, void* v_cmp_pool, int32_t n_cmp_pages,
+                                int32_t cmp_page_size, const int32_t* cmp_block_table, int32_t max_cmp_pages,
+                                const nsa_heads_t* heads, const nsa_params_t* params, int32_t* n_blocks,
+                                void* workspace, size_t ws_bytes, void* stream);
 
 /* Opt-in per-kernel timing (no compute change). While enabled, every entry point
  * records a CUDA event pair on its stream around each of its kernel launches.

@@ -11,6 +11,7 @@ outputs and the workspace with torch and then call the entry points.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -20,6 +21,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnsa.so")
+# checking build (index checks, test fault injection; include/nsa_check.h): tests only
+CHECK_LIB_PATH = os.path.join(_PKG, "libnsa_check.so")
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_DEVICE_CHECK = range(6)
 NSA_OP_COMPRESS, NSA_OP_PREFILL, NSA_OP_DECODE = 0, 1, 2
@@ -28,9 +31,13 @@ NSA_NOALLOC_SCRATCH_BYTES = 4194304
 
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
-            "nsa_compress_noalloc", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
+            "nsa_compress_append_plan", "nsa_compress_append", "nsa_compress_paged", "nsa_compress_noalloc",
+            "nsa_decode_paged", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
 NSA_PROFILE_SLOTS = 5
+# the checking build exports one more symbol (include/nsa_check.h)
+CHECK_EXPORTED = EXPORTED + ("nsa_test_set_fault",)
+FAULT_NONE, FAULT_DECODE_FINE_TILE, FAULT_PREFILL_K_TILE = 0, 1, 2
 
 
 class NSAError(RuntimeError):
@@ -58,6 +65,7 @@ def make_params(l_cmp=32, stride=16, l_sel=64, top_n=16, window=512, force_first
 
 
 _lib = None
+_loaded = {}
 
 
 def lib() -> ctypes.CDLL:
@@ -65,9 +73,37 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libnsa.so not built at {LIB_PATH}; run python -m sparse_attention_long_nsa_b200.build")
-    L = ctypes.CDLL(LIB_PATH)
+    _lib = _load(LIB_PATH)
+    return _lib
+
+
+@contextlib.contextmanager
+def checking_library():
+    """Route every entry point of this module through libnsa_check.so (the
+    checking build) inside the `with` block; the library build is restored after."""
+    global _lib
+    prev = lib()
+    _lib = _load(CHECK_LIB_PATH)
+    try:
+        yield _lib
+    finally:
+        _lib = prev
+
+
+def nsa_test_set_fault(site: int):
+    """Checking build only (include/nsa_check.h): make a producer withhold a tile."""
+    L = lib()
+    if not hasattr(L, "nsa_test_set_fault"):
+        raise RuntimeError("nsa_test_set_fault exists only in the checking build (use checking_library())")
+    _check(L.nsa_test_set_fault(int(site)), "nsa_test_set_fault")
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path in _loaded:
+        return _loaded[path]
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built at {path}; run python -m sparse_attention_long_nsa_b200.build")
+    L = ctypes.CDLL(path)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     L.nsa_workspace_size.restype = SZ
     L.nsa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(Heads), ctypes.POINTER(Params), I32, I64, I32]
@@ -78,6 +114,17 @@ def lib() -> ctypes.CDLL:
     L.nsa_compress.restype = ctypes.c_int
     L.nsa_compress.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params),
                                P, P, P, SZ, P]
+    L.nsa_compress_append_plan.restype = ctypes.c_int
+    L.nsa_compress_append_plan.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(Params), P, P, P, P]
+    L.nsa_compress_append.restype = ctypes.c_int
+    L.nsa_compress_append.argtypes = [P, P, P, P, P, P, P, P, I32, I32, I32, ctypes.POINTER(Heads),
+                                      ctypes.POINTER(Params), P, P, P, P, SZ, P]
+    L.nsa_compress_paged.restype = ctypes.c_int
+    L.nsa_compress_paged.argtypes = [P, P, I32, I32, P, I32, P, P, P, P, P, P, I32, P, P, I32, I32, P, I32,
+                                     ctypes.POINTER(Heads), ctypes.POINTER(Params), P, P, SZ, P]
+    L.nsa_decode_paged.restype = ctypes.c_int
+    L.nsa_decode_paged.argtypes = [P, P, P, I32, I32, P, I32, P, P, I32, I32, P, I32, P, I32, I32, P,
+                                   ctypes.POINTER(Heads), ctypes.POINTER(Params), P, P, P, P, SZ, P]
     L.nsa_compress_noalloc.restype = ctypes.c_int
     L.nsa_compress_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
                                        ctypes.POINTER(Params), P, P, P]
@@ -97,7 +144,10 @@ def lib() -> ctypes.CDLL:
     L.nsa_status_string.argtypes = [ctypes.c_int]
     L.nsa_last_error_detail.restype = ctypes.c_char_p
     L.nsa_last_error_detail.argtypes = []
-    _lib = L
+    if hasattr(L, "nsa_test_set_fault"):
+        L.nsa_test_set_fault.restype = ctypes.c_int
+        L.nsa_test_set_fault.argtypes = [I32]
+    _loaded[path] = L
     return L
 
 
@@ -204,6 +254,43 @@ def nsa_decode(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens, max_le
     _check(s, "nsa_decode")
 
 
+def nsa_compress_paged(k_pool, v_pool, block_table, w_ck, pe_k, w_cv, pe_v, lens_prev, lens, heads: Heads,
+                       params: Params, k_cmp_pool, v_cmp_pool, cmp_block_table, ws, stream=None) -> int:
+    """Paged caches: pools [n_pages, page_size, H_kv, d] and [n_cmp_pages,
+    cmp_page_size, H_kv, d]; block tables device int32 [B, max_pages]; lens_prev
+    (None: one token less; zeros: build from scratch) and lens host int32 [B].
+    Returns the number of summaries written."""
+    n = ctypes.c_int32(0)
+    B = int(lens.numel())
+    _check(lib().nsa_compress_paged(_ptr(k_pool, torch.bfloat16), _ptr(v_pool, torch.bfloat16), int(k_pool.shape[0]),
+                                    int(k_pool.shape[1]), _ptr(block_table, torch.int32), int(block_table.shape[1]),
+                                    _ptr(w_ck, torch.float32), _ptr(pe_k, torch.float32), _ptr(w_cv, torch.float32),
+                                    _ptr(pe_v, torch.float32), _ptr(lens_prev, torch.int32, "cpu"),
+                                    _ptr(lens, torch.int32, "cpu"), B, _ptr(k_cmp_pool, torch.bfloat16),
+                                    _ptr(v_cmp_pool, torch.bfloat16), int(k_cmp_pool.shape[0]),
+                                    int(k_cmp_pool.shape[1]), _ptr(cmp_block_table, torch.int32),
+                                    int(cmp_block_table.shape[1]), ctypes.byref(heads), ctypes.byref(params),
+                                    ctypes.byref(n), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "nsa_compress_paged")
+    return int(n.value)
+
+
+def nsa_decode_paged(q, k_pool, v_pool, block_table, k_cmp_pool, v_cmp_pool, cmp_block_table, cache_lens,
+                     max_len: int, gates, heads: Heads, params: Params, out, sel_out=None, imp_out=None, ws=None,
+                     stream=None):
+    """Paged decode (layouts as nsa_compress_paged); cache_lens device int32 [B]."""
+    B = int(q.shape[0])
+    _check(lib().nsa_decode_paged(_ptr(q, torch.bfloat16), _ptr(k_pool, torch.bfloat16), _ptr(v_pool, torch.bfloat16),
+                                  int(k_pool.shape[0]), int(k_pool.shape[1]), _ptr(block_table, torch.int32),
+                                  int(block_table.shape[1]), _ptr(k_cmp_pool, torch.bfloat16),
+                                  _ptr(v_cmp_pool, torch.bfloat16), int(k_cmp_pool.shape[0]), int(k_cmp_pool.shape[1]),
+                                  _ptr(cmp_block_table, torch.int32), int(cmp_block_table.shape[1]),
+                                  _ptr(cache_lens, torch.int32), B, int(max_len), _ptr(gates, torch.float32),
+                                  ctypes.byref(heads), ctypes.byref(params), _ptr(out, torch.bfloat16),
+                                  _ptr(sel_out, torch.int32), _ptr(imp_out, torch.float32), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "nsa_decode_paged")
+
+
 def nsa_profile_enable(enable: bool):
     _check(lib().nsa_profile_enable(1 if enable else 0), "nsa_profile_enable")
 
@@ -273,52 +360,63 @@ def compress_cache(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, heads: Heads,
     return kc, vc
 
 
+def nsa_compress_append_plan(lens_prev, lens, Lmax: int, Lmax_cmp: int, params: Params):
+    """Host-only plan of the blocks completed by growth (C ABI of the same name).
+    lens_prev/lens: host int32 [B] (lens_prev may be None: one new token).
+    Returns (tok_offset int64 [B], seq_len int32 [B], cmp_offset int64 [B], n_blocks)."""
+    B = int(lens.numel())
+    tok = torch.empty(B, dtype=torch.int64)
+    sl = torch.empty(B, dtype=torch.int32)
+    co = torch.empty(B, dtype=torch.int64)
+    n = ctypes.c_int32(0)
+    _check(lib().nsa_compress_append_plan(_ptr(lens_prev, torch.int32, "cpu"), _ptr(lens, torch.int32, "cpu"), B,
+                                          int(Lmax), int(Lmax_cmp), ctypes.byref(params), _ptr(tok, None, "cpu"),
+                                          _ptr(sl, None, "cpu"), _ptr(co, None, "cpu"), ctypes.byref(n)),
+           "nsa_compress_append_plan")
+    return tok, sl, co, int(n.value)
+
+
+def nsa_compress_append(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens_prev, lens, heads: Heads, params: Params,
+                        k_cmp_cache, v_cmp_cache, ws, stream=None) -> int:
+    """Incremental decode: write the summaries of every block completed while the
+    batched caches grew from lens_prev (None: one token less) to lens, in place.
+    lens_prev/lens: host int32 [B]. Returns the number of summaries written."""
+    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
+    n = ctypes.c_int32(0)
+    _check(lib().nsa_compress_append(_ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                                     _ptr(w_ck, torch.float32), _ptr(pe_k, torch.float32), _ptr(w_cv, torch.float32),
+                                     _ptr(pe_v, torch.float32), _ptr(lens_prev, torch.int32, "cpu"),
+                                     _ptr(lens, torch.int32, "cpu"), B, Lmax, int(k_cmp_cache.shape[1]),
+                                     ctypes.byref(heads), ctypes.byref(params), _ptr(k_cmp_cache, torch.bfloat16),
+                                     _ptr(v_cmp_cache, torch.bfloat16), ctypes.byref(n), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "nsa_compress_append")
+    return int(n.value)
+
+
+def _host_i32(x):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.to("cpu", torch.int32).contiguous()
+    return torch.tensor([int(v) for v in x], dtype=torch.int32)
+
+
 def append_plan(lens, Lmax: int, Lmax_cmp: int, l: int = 32, s: int = 16, lens_prev=None):
-    """Offsets for incremental decode: when a sequence grows from P to L tokens
-    (P = L - 1 unless lens_prev is given), the compressed blocks i with
-    n_cmp(P) <= i < n_cmp(L) are new; their tokens form one segment that starts at
-    row b*Lmax + n_cmp(P)*s of the batched cache and holds (count - 1)*s + l tokens,
-    and their summaries go to rows b*Lmax_cmp + n_cmp(P) onwards. Returns
-    (tok_offset, seq_len, cmp_offset) for nsa_compress, with seq_len 0 for sequences
-    that completed no block."""
-    lens = [int(x) for x in lens]
-    prev = [L - 1 for L in lens] if lens_prev is None else [int(x) for x in lens_prev]
-    tok, sl, co = [], [], []
-    for b, (P, L) in enumerate(zip(prev, lens)):
-        i0, i1 = n_cmp(max(P, 0), l, s), n_cmp(L, l, s)
-        if i1 > i0:
-            tok.append(b * Lmax + i0 * s)
-            sl.append((i1 - 1 - i0) * s + l)
-            co.append(b * Lmax_cmp + i0)
-        else:
-            tok.append(b * Lmax)
-            sl.append(0)
-            co.append(b * Lmax_cmp)
-    return tok, sl, co
+    """Lists (tok_offset, seq_len, cmp_offset) of nsa_compress_append_plan."""
+    tok, sl, co, _ = nsa_compress_append_plan(_host_i32(lens_prev), _host_i32(lens), Lmax, Lmax_cmp,
+                                              make_params(l_cmp=l, stride=s))
+    return tok.tolist(), sl.tolist(), co.tolist()
 
 
 def compress_append(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, lens, k_cmp, v_cmp, heads: Heads, params: Params,
                     ws=None, lens_prev=None) -> int:
-    """Incremental decode: after the batched caches [B, Lmax, H_kv, d] grew from
-    `lens_prev` (default: one token less) to `lens` tokens, write the summaries of
-    every block completed in between into the compressed caches [B, Lmax_cmp, H_kv,
-    d], in place, with one nsa_compress call. Returns the number of blocks written
-    (0: nothing to do, no launch)."""
-    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
-    Lc = int(k_cmp.shape[1])
-    lens_l = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
-    prev_l = None if lens_prev is None else [int(x) for x in (lens_prev.tolist() if hasattr(lens_prev, "tolist")
-                                                                else lens_prev)]
-    tok, sl, co = append_plan(lens_l, Lmax, Lc, params.l_cmp, params.stride, lens_prev=prev_l)
-    n = sum(n_cmp(x, params.l_cmp, params.stride) for x in sl)
-    if n == 0:
-        return 0
+    """nsa_compress_append with the workspace allocated when not given. Returns
+    the number of blocks written (0: nothing to do, no launch)."""
     if ws is None:
-        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, B, 0, 0), k_cache.device)
-    nsa_compress(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, torch.tensor(tok, dtype=torch.int64),
-                 torch.tensor(sl, dtype=torch.int32), torch.tensor(co, dtype=torch.int64), heads, params, k_cmp,
-                 v_cmp, ws)
-    return n
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, int(k_cache.shape[0]), 0, 0),
+                             k_cache.device)
+    return nsa_compress_append(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, _host_i32(lens_prev), _host_i32(lens),
+                               heads, params, k_cmp, v_cmp, ws)
 
 
 def prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, ws=None, want_sel=False,

@@ -31,6 +31,34 @@ struct WsHeader {
 #define NSA_WAIT_LIMIT_NS 500000000ull   // 0.5 s of wall time per wait
 #endif
 
+// Index checks of the bounds-checking build (-DNSA_DEBUG_BOUNDS): a failed check
+// records DEV_ERR_BOUNDS and the site in the status word and the guarded access
+// is skipped; nsa_check_device_status() then reports it. In the library build
+// the condition is not evaluated and the access always happens.
+#ifdef NSA_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool cond, uint32_t* status, uint32_t site) {
+  if (!cond && status) {
+    atomicOr(status, DEV_ERR_BOUNDS);
+    atomicExch(status + 1, site);
+  }
+  return cond;
+}
+#define NSA_BOUNDS(cond, status, site) ::nsa::bounds_ok((cond), (status), (site))
+#else
+#define NSA_BOUNDS(cond, status, site) true
+#endif
+
+// Fault injection of the checking build (-DNSA_FAULT_INJECT): the host sets a
+// site; the producer named by it withholds one tile, so the waits on that tile
+// run out (bounded, NSA_WAIT_LIMIT_NS) and the kernel records DEV_ERR_TIMEOUT and
+// returns. Nothing is injected in the library build.
+enum : int { FAULT_NONE = 0, FAULT_DECODE_FINE_TILE = 1, FAULT_PREFILL_K_TILE = 2 };
+#ifdef NSA_FAULT_INJECT
+#define NSA_INJECT(args, site) ((args).fault_site == (site))
+#else
+#define NSA_INJECT(args, site) false
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

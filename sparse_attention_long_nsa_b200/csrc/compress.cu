@@ -133,9 +133,19 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
     {  // A: one 128-byte row per thread
       const int row = tid;
       const int ci = i0 + row;
-      const bool ok = ci < ncmp;
-      const __nv_bfloat16* src =
-          x + (size_t)(tok0 + (int64_t)(ok ? ci : 0) * a.s + r) * row_stride + (size_t)g * D_IN + e0;
+      bool ok = ci < ncmp;
+      int64_t xr = tok0 + (int64_t)(ok ? ci : 0) * a.s + r;   // token row (paged: index in the sequence)
+      if (a.x_pt.table) {
+        const int pg = a.x_pt.table[(int64_t)b * a.x_pt.max_pages + (int)(xr / a.x_pt.page_size)];
+        if (pg < 0 || pg >= a.x_pt.n_pages) {   // invalid page: zeros, and the error is recorded
+          if (ok) atomicOr(a.status, DEV_ERR_BOUNDS);
+          ok = false;
+          xr = 0;
+        } else {
+          xr = (int64_t)pg * a.x_pt.page_size + xr % a.x_pt.page_size;
+        }
+      }
+      const __nv_bfloat16* src = x + (size_t)xr * row_stride + (size_t)g * D_IN + e0;
 #pragma unroll
       for (int c = 0; c < 8; ++c) cp_async16_zfill(A + sw128(row, c), src + c * 8, ok);
     }
@@ -194,13 +204,21 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
     const int row = warp * 32 + lane;
     const int ci = i0 + row;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-    const size_t orow = ((size_t)(a.seqs.cmp_off[b] + ci) * a.H_kv + g) * D_OUT;
+    int64_t oe = a.seqs.cmp_off[b] + ci;   // output row (paged: entry index in the sequence)
+    bool oval = true;
+    if (a.out_pt.table && ci < ncmp) {
+      const int pg = a.out_pt.table[(int64_t)b * a.out_pt.max_pages + (int)(oe / a.out_pt.page_size)];
+      oval = pg >= 0 && pg < a.out_pt.n_pages;
+      if (!oval) atomicOr(a.status, DEV_ERR_BOUNDS);
+      oe = oval ? (int64_t)pg * a.out_pt.page_size + oe % a.out_pt.page_size : 0;
+    }
+    const size_t orow = ((size_t)oe * a.H_kv + g) * D_OUT;
 #pragma unroll 1
     for (int c0 = 0; c0 < D_OUT; c0 += 16) {
       float v[16];
       tmem_ld16(tmem_d + ((uint32_t)(warp * 32) << 16) + c0, v);
       tmem_ld_wait();
-      if (ci < ncmp) {
+      if (ci < ncmp && oval) {
         if (a.ksplit == 1) {
           uint32_t pk[8];
 #pragma unroll

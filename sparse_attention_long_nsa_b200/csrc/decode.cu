@@ -60,6 +60,14 @@ struct DecSmem {
 
 __device__ __forceinline__ int n_cmp_dev(int L, int l, int s) { return L >= l ? (L - l) / s + 1 : 0; }
 
+// tensor-map row of raw token `tok` / compressed entry `e` of sequence b
+__device__ __forceinline__ int kv_row(const DecodeArgs& a, int b, int tok) {
+  return a.kv_pt.table ? (int)paged_row(a.kv_pt, b, tok, a.status) : b * a.Lmax + tok;
+}
+__device__ __forceinline__ int cmp_row(const DecodeArgs& a, int b, int e) {
+  return a.cmp_pt.table ? (int)paged_row(a.cmp_pt, b, e, a.status) : b * a.Lmax_cmp + e;
+}
+
 struct PartLayout {
   // offsets in floats; every row of DV floats starts 16-byte aligned
   size_t cp_o, cp_ml, tp, fp_o, fp_ml, cnt, total;
@@ -236,7 +244,10 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
         mbar_arrive_expect_tx(&q_full[qi], (uint32_t)(DK / 64) * G * 128);
         for (int kb = 0; kb < DK / 64; ++kb)
           tma_load_3d(qbuf + qi * S::QBUF + kb * 2048, &mp.q, &q_full[qi], kb * 64, g * G, b);
-        const int row0 = b * a.Lmax_cmp + chunk * kCmpChunk;
+        if (!NSA_BOUNDS(chunk * kCmpChunk + ntl * kTileKeys <= a.Lmax_cmp + kTileKeys - 1, a.status, 513)) {
+          *abort_flag = 1;   // stop the consumers; the copies issued so far are drained below
+          break;
+        }
         for (int i = 0; i < ntl; ++i, ++u) {
           const int st = u % kD1Stages;
           if (u >= kD1Stages && !mbar_wait(&empty[st], ((u / kD1Stages) - 1) & 1, abort_flag, a.status, 401)) {
@@ -245,13 +256,14 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
           }
           TRC(0, u, 2);
           uint8_t* Ks = ring + st * S::STAGE;
+          // a 32-entry tile never straddles a page (page sizes are multiples of 32)
+          const int row = cmp_row(a, b, chunk * kCmpChunk + i * kTileKeys);
           stage_tag[st] = u;
           mbar_arrive_expect_tx(&full[st], S::STAGE);
           for (int kb = 0; kb < DK / 64; ++kb)
-            tma_load_3d(Ks + kb * (kTileKeys * 128), &mp.kc, &full[st], kb * 64, g, row0 + i * kTileKeys);
+            tma_load_3d(Ks + kb * (kTileKeys * 128), &mp.kc, &full[st], kb * 64, g, row);
           for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_3d(Ks + DK * kTileKeys * 2 + vb * (kTileKeys * 128), &mp.vc, &full[st], vb * 64, g,
-                        row0 + i * kTileKeys);
+            tma_load_3d(Ks + DK * kTileKeys * 2 + vb * (kTileKeys * 128), &mp.vc, &full[st], vb * 64, g, row);
         }
         ++it;
       }
@@ -421,7 +433,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
 #endif
   // K/V of one 32-key half of block blk into L2 (the stream reads them from there)
   auto prefetch_half = [&](int blk, int half) {
-    const int row = b * a.Lmax + blk * a.ls + half * kTileKeys;
+    const int row = kv_row(a, b, blk * a.ls + half * kTileKeys);   // pages hold whole blocks
     for (int kb = 0; kb < DK / 64; ++kb) tma_prefetch_3d(&mp.k, kb * 64, g, row);
     for (int vb = 0; vb < DV / 64; ++vb) tma_prefetch_3d(&mp.v, vb * 64, g, row);
   };
@@ -573,6 +585,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
         warp == 0)
       warp_topn_any(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, lane);
     __syncthreads();
+#ifdef NSA_DEBUG_BOUNDS
+    if (warp == 0 && lane < a.top_n) {   // ascending, in 0..jt, -1 only as padding
+      const int32_t* sl = a.sel + bg * a.top_n;
+      const int v = sl[lane];
+      const bool fine = v == -1 ? (lane + 1 >= a.top_n || sl[lane + 1] == -1)
+                                : (v >= 0 && v <= jt && (lane == 0 || sl[lane - 1] < v));
+      NSA_BOUNDS(fine, a.status, 512);
+    }
+    __syncthreads();
+#endif
   }
   TRD(5);
   if (warp == kDecConsumers && lane == 0) {   // selected blocks below the window, ahead of the stream
@@ -657,8 +679,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       for (int u = 0; u < nh; ++u) {
         const int st = u % kDecStages;
         if (u >= kDecStages && !mbar_wait(&empty[st], ((u / kDecStages) - 1) & 1, abort_flag, a.status, 411)) break;
+        if (u == 0 && NSA_INJECT(a, FAULT_DECODE_FINE_TILE)) {   // checking build: withhold the first tile
+          issued = 1;
+          continue;
+        }
         uint8_t* Ks = ring + st * S::STAGE;
-        const int row = b * a.Lmax + uni[u >> 1] * a.ls + (u & 1) * kTileKeys;
+        if (!NSA_BOUNDS(uni[u >> 1] >= 0 && uni[u >> 1] <= jt, a.status, 511)) {
+          *abort_flag = 1;   // stop the consumers; the copies issued so far are drained below
+          break;
+        }
+        const int row = kv_row(a, b, uni[u >> 1] * a.ls + (u & 1) * kTileKeys);
         mbar_arrive_expect_tx(&full[st], S::STAGE);
         for (int kb = 0; kb < DK / 64; ++kb)
           tma_load_3d(Ks + kb * (kTileKeys * 128), &mp.k, &full[st], kb * 64, g, row);

@@ -16,6 +16,7 @@ enum ProfSlot {
 };
 void prof_begin(int slot, cudaStream_t st);
 void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()
+int test_fault_site();                    // checking build: site set by nsa_test_set_fault (else 0)
 void prof_end(int slot, cudaStream_t st, int launches);
 
 // Per-launch sequence table, passed by value as a kernel parameter.
@@ -29,6 +30,24 @@ struct SeqTable {
 
 __host__ __device__ inline int n_cmp_of(int L, int l, int s) { return L >= l ? (L - l) / s + 1 : 0; }
 
+// Paged caches: token (or compressed entry) e of sequence b lives in physical page
+// table[b * max_pages + e / page_size] at row e % page_size of the pool
+// [n_pages * page_size, H_kv, d]. A null table means the contiguous batched
+// layout. Page ids outside [0, n_pages) are recorded as DEV_ERR_BOUNDS in the
+// status word and replaced by page 0 (the result is then not valid).
+struct PageTable {
+  const int32_t* table;   // device int32 [B, max_pages] or null
+  int page_size, max_pages, n_pages;
+};
+__device__ __forceinline__ int64_t paged_row(const PageTable& pt, int b, int e, uint32_t* status) {
+  int p = pt.table[(int64_t)b * pt.max_pages + e / pt.page_size];
+  if (p < 0 || p >= pt.n_pages) {
+    atomicOr(status, 2u);   // DEV_ERR_BOUNDS
+    p = 0;
+  }
+  return (int64_t)p * pt.page_size + e % pt.page_size;
+}
+
 // ----- compression (block summaries) -----
 struct CompressArgs {
   const void* x;          // bf16 [*, H_kv, d_in]
@@ -41,6 +60,9 @@ struct CompressArgs {
   float* part;            // fp32 [ksplit][rows_total][H_kv][d_out] partial sums (ksplit > 1)
   int64_t rows_total;     // output rows (packed: sum of n_cmp)
   uint32_t* status;
+  // paged caches (x_pt.table non-null): seqs.tok_off / cmp_off are then token and
+  // entry indices within sequence b, mapped through the tables
+  PageTable x_pt, out_pt;
   SeqTable seqs;
 };
 cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
@@ -69,6 +91,7 @@ struct PrefillArgs {
   int want_imp, want_sel; // caller asked for the importance / selection rows
   float scale_log2;       // softmax scale * log2(e)
   uint32_t* status;
+  int fault_site;         // checking build only: injected failure (FAULT_*), 0 = none
   SeqTable seqs;          // tile_prefix counts query tiles of 128/G tokens
 };
 struct PrefillMaps {
@@ -100,6 +123,9 @@ struct DecodeArgs {
   int n_sw_chunks;               // D3 splits per (b, g), 4 blocks of l_sel keys each
   float scale_log2;
   uint32_t* status;
+  int fault_site;         // checking build only: injected failure (FAULT_*), 0 = none
+  PageTable kv_pt;        // paged raw cache (table null: [B, Lmax] rows)
+  PageTable cmp_pt;       // paged compressed cache (table null: [B, Lmax_cmp] rows)
 };
 struct DecodeMaps {
   CUtensorMap k, v, kc, vc;

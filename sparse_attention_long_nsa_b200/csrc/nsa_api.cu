@@ -1,6 +1,7 @@
 // C-ABI host layer of libnsa.so: argument validation, workspace carving,
 // tensor-map encoding and the launch sequence of each entry point.
 // See include/nsa.h for the contract of every function.
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -194,6 +195,13 @@ const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_at
 namespace nsa {
 void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
 
+#ifdef NSA_FAULT_INJECT
+static int g_test_fault = 0;
+int test_fault_site() { return g_test_fault; }
+#else
+int test_fault_site() { return 0; }
+#endif
+
 void prof_begin(int slot, cudaStream_t st) {
   Profiler& p = prof();
   std::lock_guard<std::mutex> g(p.mu);
@@ -214,6 +222,14 @@ void prof_end(int slot, cudaStream_t st, int launches) {
 }  // namespace nsa
 
 extern "C" {
+
+#ifdef NSA_FAULT_INJECT
+nsa_status_t nsa_test_set_fault(int32_t site) {
+  if (site < FAULT_NONE || site > FAULT_PREFILL_K_TILE) return NSA_ERR_INVALID_ARG;
+  nsa::g_test_fault = site;
+  return NSA_OK;
+}
+#endif
 
 nsa_status_t nsa_profile_enable(int32_t enable) {
   Profiler& p = prof();
@@ -313,11 +329,16 @@ nsa_status_t nsa_check_device_status(void* workspace, void* stream) {
   return NSA_OK;
 }
 
-nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const float* pe_k, const float* w_cv,
-                          const float* pe_v, const int64_t* tok_offset, const int32_t* seq_len,
-                          const int64_t* cmp_offset, int32_t batch, const nsa_heads_t* heads,
-                          const nsa_params_t* params, void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes,
-                          void* stream) {
+}  // extern "C"
+
+namespace {
+// nsa_compress with optional page tables for the input tokens and the output
+// summaries (both null: the plain layouts of nsa_compress)
+nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, const float* pe_k, const float* w_cv,
+                             const float* pe_v, const int64_t* tok_offset, const int32_t* seq_len,
+                             const int64_t* cmp_offset, int32_t batch, const nsa_heads_t* heads,
+                             const nsa_params_t* params, void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes,
+                             void* stream, const PageTable& x_pt, const PageTable& out_pt) {
   nsa_status_t s = check_heads(heads);
   if (s != NSA_OK) return s;
   if ((s = check_params(params, false)) != NSA_OK) return s;
@@ -346,6 +367,7 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
     if (rows_total >= 0) rows_total = (cmp_offset[b] == rows_total) ? rows_total + nc : -1;
   }
   t.tile_prefix[batch] = tiles;
+  if (out_pt.table) rows_total = -1;   // paged output rows are not packed: no split of K
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -363,6 +385,8 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
   CompressArgs a{};
   a.H_kv = heads->H_kv; a.l = params->l_cmp; a.s = params->stride;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.x_pt = x_pt;
+  a.out_pt = out_pt;
   a.seqs = t;
   a.part = (float*)(ws + w.ksum);
   a.rows_total = rows_total > 0 ? rows_total : 0;
@@ -396,6 +420,107 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
   prof_end(P_COMPRESS_GEMM, st, launches);
   if (e != cudaSuccess) return cuda_fail(e, "compress gemm");
   return NSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const float* pe_k, const float* w_cv,
+                          const float* pe_v, const int64_t* tok_offset, const int32_t* seq_len,
+                          const int64_t* cmp_offset, int32_t batch, const nsa_heads_t* heads,
+                          const nsa_params_t* params, void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  const PageTable none{};
+  return compress_common(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, batch, heads, params, k_cmp,
+                         v_cmp, workspace, ws_bytes, stream, none, none);
+}
+
+nsa_status_t nsa_compress_paged(const void* k_pool, const void* v_pool, int32_t n_pages, int32_t page_size,
+                                const int32_t* block_table, int32_t max_pages, const float* w_ck, const float* pe_k,
+                                const float* w_cv, const float* pe_v, const int32_t* lens_prev, const int32_t* lens,
+                                int32_t batch, void* k_cmp_pool, void* v_cmp_pool, int32_t n_cmp_pages,
+                                int32_t cmp_page_size, const int32_t* cmp_block_table, int32_t max_cmp_pages,
+                                const nsa_heads_t* heads, const nsa_params_t* params, int32_t* n_blocks,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, false)) != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!block_table || !cmp_block_table || n_pages <= 0 || n_cmp_pages <= 0 || max_pages <= 0 ||
+      max_cmp_pages <= 0)
+    return NSA_ERR_INVALID_ARG;
+  if (page_size <= 0 || page_size % 64 != 0 || cmp_page_size <= 0 || cmp_page_size % 32 != 0)
+    return NSA_ERR_INVALID_ARG;
+  const int64_t cap = (int64_t)max_pages * page_size, ccap = (int64_t)max_cmp_pages * cmp_page_size;
+  if (cap > INT32_MAX || ccap < n_cmp_of((int)cap, params->l_cmp, params->stride)) return NSA_ERR_INVALID_ARG;
+  // plan the new blocks as nsa_compress_append_plan does, but with offsets inside
+  // each sequence (token index i0 * stride, entry index i0): the tables map them
+  int64_t tok[NSA_MAX_BATCH], coff[NSA_MAX_BATCH];
+  int32_t len[NSA_MAX_BATCH], n = 0;
+  s = nsa_compress_append_plan(lens_prev, lens, batch, (int32_t)cap, (int32_t)ccap, params, tok, len, coff, &n);
+  if (s != NSA_OK) return s;
+  for (int b = 0; b < batch; ++b) {
+    tok[b] -= (int64_t)b * cap;
+    coff[b] -= (int64_t)b * ccap;
+  }
+  if (n_blocks) *n_blocks = n;
+  if (n == 0) return NSA_OK;
+  const PageTable x_pt{block_table, page_size, max_pages, n_pages};
+  const PageTable out_pt{cmp_block_table, cmp_page_size, max_cmp_pages, n_cmp_pages};
+  return compress_common(k_pool, v_pool, w_ck, pe_k, w_cv, pe_v, tok, len, coff, batch, heads, params, k_cmp_pool,
+                         v_cmp_pool, workspace, ws_bytes, stream, x_pt, out_pt);
+}
+
+nsa_status_t nsa_compress_append_plan(const int32_t* lens_prev, const int32_t* lens, int32_t batch, int32_t Lmax,
+                                      int32_t Lmax_cmp, const nsa_params_t* params, int64_t* tok_offset,
+                                      int32_t* seq_len, int64_t* cmp_offset, int32_t* n_blocks) {
+  // host-only planning works for any block / stride pair (l a multiple of s);
+  // nsa_compress_append then checks what the kernels support
+  if (!params || params->l_cmp <= 0 || params->stride <= 0 || params->l_cmp % params->stride != 0)
+    return NSA_ERR_INVALID_ARG;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!lens || !tok_offset || !seq_len || !cmp_offset || Lmax <= 0 || Lmax_cmp < 0) return NSA_ERR_INVALID_ARG;
+  if (Lmax_cmp < n_cmp_of(Lmax, params->l_cmp, params->stride)) return NSA_ERR_INVALID_ARG;
+  int32_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = lens[b];
+    const int P = lens_prev ? lens_prev[b] : L - 1;
+    if (L < 0 || L > Lmax || P < -1 || P > L) return NSA_ERR_INVALID_ARG;
+    // blocks i with n_cmp(P) <= i < n_cmp(L) were completed by the growth; their
+    // tokens [i0*s, (i1-1)*s + l) form one segment of the batched cache
+    const int i0 = n_cmp_of(P > 0 ? P : 0, params->l_cmp, params->stride);
+    const int i1 = n_cmp_of(L, params->l_cmp, params->stride);
+    if (i1 > i0) {
+      tok_offset[b] = (int64_t)b * Lmax + (int64_t)i0 * params->stride;
+      seq_len[b] = (i1 - 1 - i0) * params->stride + params->l_cmp;
+      cmp_offset[b] = (int64_t)b * Lmax_cmp + i0;
+      total += i1 - i0;
+    } else {
+      tok_offset[b] = (int64_t)b * Lmax;
+      seq_len[b] = 0;
+      cmp_offset[b] = (int64_t)b * Lmax_cmp;
+    }
+  }
+  if (n_blocks) *n_blocks = total;
+  return NSA_OK;
+}
+
+nsa_status_t nsa_compress_append(const void* k_cache, const void* v_cache, const float* w_ck, const float* pe_k,
+                                 const float* w_cv, const float* pe_v, const int32_t* lens_prev, const int32_t* lens,
+                                 int32_t batch, int32_t Lmax, int32_t Lmax_cmp, const nsa_heads_t* heads,
+                                 const nsa_params_t* params, void* k_cmp_cache, void* v_cmp_cache,
+                                 int32_t* n_blocks, void* workspace, size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  int64_t tok[NSA_MAX_BATCH], coff[NSA_MAX_BATCH];
+  int32_t len[NSA_MAX_BATCH], n = 0;
+  s = nsa_compress_append_plan(lens_prev, lens, batch, Lmax, Lmax_cmp, params, tok, len, coff, &n);
+  if (s != NSA_OK) return s;
+  if (n_blocks) *n_blocks = n;
+  if (n == 0) return NSA_OK;   // no block completed: nothing is launched
+  return nsa_compress(k_cache, v_cache, w_ck, pe_k, w_cv, pe_v, tok, len, coff, batch, heads, params, k_cmp_cache,
+                      v_cmp_cache, workspace, ws_bytes, stream);
 }
 
 nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void* k_cmp, const void* v_cmp,
@@ -440,6 +565,7 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   a.nb_stride = w.nb;
   a.scale_log2 = softmax_scale(params, heads->d_k) * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.fault_site = test_fault_site();
   if (!prefill_fused_stages(a)) {
     snprintf(g_detail, sizeof(g_detail), "sequence too long for the fused prefill kernel (%d blocks)", w.nb);
     return NSA_ERR_UNSUPPORTED;
@@ -483,11 +609,17 @@ nsa_status_t nsa_prefill(const void* q, const void* k, const void* v, const void
   return NSA_OK;
 }
 
-nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* k_cmp_cache,
-                        const void* v_cmp_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
-                        int32_t Lmax_cmp, int32_t max_len, const float* gates, const nsa_heads_t* heads,
-                        const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out, void* workspace,
-                        size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// nsa_decode with optional page tables; `rows` / `crows` are the rows of the raw
+// and compressed tensors the maps cover (batch * Lmax or the pool's rows)
+nsa_status_t decode_common(const void* q, const void* k_cache, const void* v_cache, const void* k_cmp_cache,
+                           const void* v_cmp_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
+                           int32_t Lmax_cmp, int32_t max_len, const float* gates, const nsa_heads_t* heads,
+                           const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out, void* workspace,
+                           size_t ws_bytes, void* stream, const PageTable& kv_pt, const PageTable& cmp_pt,
+                           int64_t rows, int64_t crows) {
   nsa_status_t s = check_heads(heads);
   if (s != NSA_OK) return s;
   if ((s = check_params(params, true)) != NSA_OK) return s;
@@ -516,9 +648,11 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.part = (float*)(ws + w.part);
   a.ocmp = (float*)(ws + w.ocmp);
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.fault_site = test_fault_site();
+  a.kv_pt = kv_pt;
+  a.cmp_pt = cmp_pt;
   DecodeMaps m;
   memset(&m, 0, sizeof(m));
-  const int64_t rows = (int64_t)batch * Lmax, crows = (int64_t)batch * Lmax_cmp;
   // decode streams 32-key tiles
   if (!make_map_3d(&m.k, k_cache, heads->d_k, heads->H_kv, rows, 1, 32) ||
       !make_map_3d(&m.v, v_cache, heads->d_v, heads->H_kv, rows, 1, 32) ||
@@ -531,6 +665,41 @@ nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaError_t e = launch_decode(a, m, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode");
   return NSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nsa_status_t nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* k_cmp_cache,
+                        const void* v_cmp_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
+                        int32_t Lmax_cmp, int32_t max_len, const float* gates, const nsa_heads_t* heads,
+                        const nsa_params_t* params, void* out, int32_t* sel_out, float* imp_out, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  const PageTable none{};
+  return decode_common(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens, batch, Lmax, Lmax_cmp, max_len,
+                       gates, heads, params, out, sel_out, imp_out, workspace, ws_bytes, stream, none, none,
+                       (int64_t)batch * Lmax, (int64_t)batch * Lmax_cmp);
+}
+
+nsa_status_t nsa_decode_paged(const void* q, const void* k_pool, const void* v_pool, int32_t n_pages,
+                              int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                              const void* k_cmp_pool, const void* v_cmp_pool, int32_t n_cmp_pages,
+                              int32_t cmp_page_size, const int32_t* cmp_block_table, int32_t max_cmp_pages,
+                              const int32_t* cache_lens, int32_t batch, int32_t max_len, const float* gates,
+                              const nsa_heads_t* heads, const nsa_params_t* params, void* out, int32_t* sel_out,
+                              float* imp_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!block_table || !cmp_block_table || n_pages <= 0 || n_cmp_pages <= 0 || max_pages <= 0 || max_cmp_pages <= 0)
+    return NSA_ERR_INVALID_ARG;
+  if (page_size <= 0 || page_size % 64 != 0 || cmp_page_size <= 0 || cmp_page_size % 32 != 0)
+    return NSA_ERR_INVALID_ARG;
+  const int64_t cap = (int64_t)max_pages * page_size, ccap = (int64_t)max_cmp_pages * cmp_page_size;
+  const int64_t rows = (int64_t)n_pages * page_size, crows = (int64_t)n_cmp_pages * cmp_page_size;
+  if (cap > INT32_MAX || ccap > INT32_MAX || rows > INT32_MAX || crows > INT32_MAX) return NSA_ERR_UNSUPPORTED;
+  const PageTable kv_pt{block_table, page_size, max_pages, n_pages};
+  const PageTable cmp_pt{cmp_block_table, cmp_page_size, max_cmp_pages, n_cmp_pages};
+  return decode_common(q, k_pool, v_pool, k_cmp_pool, v_cmp_pool, cache_lens, batch, (int32_t)cap, (int32_t)ccap,
+                       max_len, gates, heads, params, out, sel_out, imp_out, workspace, ws_bytes, stream, kv_pt,
+                       cmp_pt, rows, crows);
 }
 
 }  // extern "C"

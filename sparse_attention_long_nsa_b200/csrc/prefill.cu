@@ -310,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         const int st = j % nks;
         if (j >= nks && !mbar_wait(&bars->k_empty[st], ((j / nks) - 1) & 1, abort_flag, a.status, 401))
           return false;
+        if (j == 0 && NSA_INJECT(a, FAULT_PREFILL_K_TILE)) {   // checking build: withhold the first tile
+          issued = 1;
+          return true;
+        }
         TR(j, 0);
         uint8_t* Ks = kring + (size_t)st * 8192;   // chunk kb of slot st at kb * nks * 8 KB + st * 8 KB
         mbar_arrive_expect_tx(&bars->k_full[st], K_BYTES);
@@ -325,7 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       for (int i = 0; i < nkw && ok; ++i) ok = load(j++, &mp.k, (int)(tok0 + key0w + i * kKeys));
       if (ok) ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 402);
       const int nu = ok ? bars->nu : 0;
-      for (int u = 0; u < nu && ok; ++u) ok = load(j++, &mp.k, (int)(tok0 + (int64_t)uni[u] * a.ls));
+      for (int u = 0; u < nu && ok; ++u) {
+        if (!NSA_BOUNDS(uni[u] >= 0 && uni[u] <= jt_max, a.status, 501)) {
+          *abort_flag = 1;   // stop the other roles; the copies issued so far are drained below
+          ok = false;
+          break;
+        }
+        ok = load(j++, &mp.k, (int)(tok0 + (int64_t)uni[u] * a.ls));
+      }
       if (!ok) {   // let the copies still in flight land before the CTA exits
         mbar_wait_drain(&bars->q_full, 0);
         for (int v = issued - nks < 0 ? 0 : issued - nks; v < issued; ++v)
@@ -355,7 +366,14 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       for (int i = 0; i < nkw && ok; ++i) ok = load(vi++, &mp.v, (int)(tok0 + key0w + i * kKeys));
       if (ok) ok = mbar_wait(&bars->sel_ready, 0, abort_flag, a.status, 404);
       const int nu = ok ? bars->nu : 0;
-      for (int u = 0; u < nu && ok; ++u) ok = load(vi++, &mp.v, (int)(tok0 + (int64_t)uni[u] * a.ls));
+      for (int u = 0; u < nu && ok; ++u) {
+        if (!NSA_BOUNDS(uni[u] >= 0 && uni[u] <= jt_max, a.status, 502)) {
+          *abort_flag = 1;   // stop the other roles; the copies issued so far are drained below
+          ok = false;
+          break;
+        }
+        ok = load(vi++, &mp.v, (int)(tok0 + (int64_t)uni[u] * a.ls));
+      }
       if (!ok)
         for (int v = issued - nvs < 0 ? 0 : issued - nvs; v < issued; ++v)
           mbar_wait_drain(&bars->v_full[v % nvs], (v / nvs) & 1);
@@ -690,7 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       __syncwarp();
       if (lane < a.top_n) {
         const int jb = srow[lane];
-        if (jb >= 0) atomicOr(&bm[jb * MW + (tk >> 5)], 1u << (tk & 31));
+        if (jb >= 0 && NSA_BOUNDS(jb <= jq && (lane == 0 || srow[lane - 1] < jb), a.status, 503))
+          atomicOr(&bm[jb * MW + (tk >> 5)], 1u << (tk & 31));
         if (a.imp_smem && a.want_sel) gsel[lane] = jb;
       }
       if (a.imp_smem && a.want_imp) {

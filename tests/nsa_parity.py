@@ -13,6 +13,17 @@ Acceptance (NSA forward, fp64 oracle vs bf16/fp32 GPU path):
                  output rows are then compared against the oracle rerun with it.
 Stage-wise: the oracle's steps 2-7 consume the GPU's bf16 compressed K/V, so a
 selection is never flipped by the compression rounding alone.
+End to end (e2e_rows): the oracle also runs on its own fp64 compression of the
+fp32 weights. The GPU rounds the compressed keys to bf16 (relative 2^-9), which
+moves a logit by about 2^-9 and a block score by about 1e-3 relative, so there
+a selection may differ only where the oracle's own scores of the swapped blocks
+are within E2E_TIE (1e-2) of each other, the GPU's set must follow from its own
+scores, and the output rows are compared with the oracle rerun on that set.
+The outputs then also carry the compressed branch's inherited error: the bf16
+compressed keys and values differ from the fp64 ones by a relative RMS of about
+0.8u*sqrt(2) = 4.4e-3 (u = 2^-8: bf16 block tokens and weights in the l*d-term
+sums, and the rounding of the summaries), so the end-to-end bound is max-abs
+2e-2 and relative RMS E2E_RRMS = 1e-2 (the stage-wise 5e-3 plus that term).
 """
 from __future__ import annotations
 
@@ -27,6 +38,8 @@ TOL_MAX = 2e-2
 TOL_RRMS = 5e-3
 TOL_IMP = 1e-4
 NEAR_TIE = 1e-5
+E2E_TIE = 1e-2
+E2E_RRMS = 1e-2
 
 
 def heads_of(cfg):
@@ -121,7 +134,34 @@ def check_selection_and_outputs(keyed_rows, gpu_sel, gpu_imp, gpu_out, orc, reru
     return assert_close(gpu_out, want, "output")
 
 
-def run_prefill_case(cfg, seqlens, n_random_rows=64, seed=None, param_over=None, gates=None, rng_seed=0):
+def check_end_to_end(keyed_rows, gpu_sel, gpu_imp, gpu_out, orc, rerun, op, H_kv, stats):
+    """GPU rows against the oracle run on its own fp64 compression (see header)."""
+    override = {}
+    for ri, (key, t) in enumerate(keyed_rows):
+        jt = t // op["l_sel"]
+        for g in range(H_kv):
+            gs = [int(x) for x in gpu_sel[ri, g] if x >= 0]
+            osel = orc["sel"][(key, g)]
+            if gs == osel:
+                continue
+            oimp = orc["imp"][(key, g)]
+            gimp = gpu_imp[ri, g, :jt + 1]
+            lost, extra = set(osel) - set(gs), set(gs) - set(osel)
+            a = min(float(oimp[j]) for j in lost)
+            b = max(float(oimp[j]) for j in extra)
+            assert a - b <= E2E_TIE * max(abs(a), abs(b), 1e-30), \
+                f"end to end: selection differs beyond the compression rounding at t={t} g={g}: gpu {gs} oracle {osel}"
+            resel = O.select(gimp.astype(np.float64), t, op["l_sel"], op["top_n"], op["force_first"],
+                             op["force_local"])
+            assert resel == gs, f"GPU selection not reproducible from its scores at t={t} g={g}"
+            override[(key, g)] = gs
+            stats["e2e_swaps"] = stats.get("e2e_swaps", 0) + 1
+    want = orc["out"] if not override else rerun(override)
+    return assert_close(gpu_out, want, "output (end to end)", tol_rrms=E2E_RRMS)
+
+
+def run_prefill_case(cfg, seqlens, n_random_rows=64, seed=None, param_over=None, gates=None, rng_seed=0,
+                     e2e_rows=0, k_cmp_fn=None):
     """Full GPU prefill (compress + prefill) on packed sequences; oracle on
     sampled rows of every sequence. Returns stats."""
     param_over = param_over or {}
@@ -133,6 +173,9 @@ def run_prefill_case(cfg, seqlens, n_random_rows=64, seed=None, param_over=None,
     op = oracle_params(cfg, **param_over)
     k_cmp, v_cmp = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], seqlens,
                                 heads, par)
+    stage_only = k_cmp_fn is not None
+    if stage_only:   # the case replaces the compressed keys (constructed inputs)
+        k_cmp = k_cmp_fn(k_cmp)
     cu = inp["cu_seqlens"]
     ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_PREFILL, heads, par, len(seqlens),
                                                     int(cu[-1]), max(seqlens)), "cuda")
@@ -152,7 +195,8 @@ def run_prefill_case(cfg, seqlens, n_random_rows=64, seed=None, param_over=None,
         kcg = f64(k_cmp[coff:coff + nc])
         vcg = f64(v_cmp[coff:coff + nc])
         coff += nc
-        if nc:
+        kco = vco = None
+        if nc and not stage_only:
             kco = O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"])
             vco = O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"])
             assert_close(kcg, kco, "k_cmp", relative_to_rms=True)
@@ -173,12 +217,28 @@ def run_prefill_case(cfg, seqlens, n_random_rows=64, seed=None, param_over=None,
                                            stats)
         stats.setdefault("max_abs", []).append(m)
         stats.setdefault("rrms", []).append(r)
+        stats.setdefault("gpu", []).append(dict(rows=rows, sel=gsel, imp=gimp))
+        if e2e_rows and nc and not stage_only:
+            pick = sorted(rng.choice(len(rows), size=min(e2e_rows, len(rows)), replace=False).tolist())
+            erows = [rows[i] for i in pick]
+            orc_e = O.prefill(qb, kb, vb, kco, vco, gb, op, rows=erows)
+
+            def rerun_e(override, qb=qb, kb=kb, vb=vb, kco=kco, vco=vco, gb=gb, erows=erows):
+                return O.prefill(qb, kb, vb, kco, vco, gb, op, rows=erows, sel_override=override)["out"]
+            m, r = check_end_to_end([(t, t) for t in erows], gsel[pick], gimp[pick], gout[pick], orc_e, rerun_e, op,
+                                    cfg.H_kv, stats)
+            stats.setdefault("e2e_max_abs", []).append(m)
+            stats.setdefault("e2e_rrms", []).append(r)
     return stats
 
 
-def run_decode_case(cfg, lens=None, batch_rows=None, seed=None, Lmax=None, param_over=None):
+def run_decode_case(cfg, lens=None, batch_rows=None, seed=None, Lmax=None, param_over=None, cmp_rows=None,
+                    kc_fn=None):
     """lens=None draws the configuration's own lengths; batch_rows may be a
-    function of the drawn lengths."""
+    function of the drawn lengths. cmp_rows (default: every checked sequence)
+    limits the sequences whose compressed caches are recomputed by the oracle
+    (a function of the lengths, like batch_rows); kc_fn replaces the compressed
+    key cache (constructed inputs)."""
     param_over = param_over or {}
     inp = W.make_decode_inputs(cfg, device="cuda", lens=lens, seed=seed, Lmax=Lmax)
     heads = heads_of(cfg)
@@ -187,6 +247,9 @@ def run_decode_case(cfg, lens=None, batch_rows=None, seed=None, Lmax=None, param
     lens_t = inp["cache_lens"]
     kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"],
                                 lens_t, heads, par)
+    if kc_fn is not None:
+        kc = kc_fn(kc)
+        cmp_rows = []
     max_len = int(inp["k_cache"].shape[1])
     ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_DECODE, heads, par, len(lens_t), 0, max_len), "cuda")
     out, sel, imp = nsa.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens_t.to("cuda"), max_len,
@@ -197,22 +260,37 @@ def run_decode_case(cfg, lens=None, batch_rows=None, seed=None, Lmax=None, param
     if callable(batch_rows):
         batch_rows = batch_rows([int(x) for x in lens_t])
     batch_rows = list(range(B)) if batch_rows is None else batch_rows
-    stats = {}
+    if callable(cmp_rows):
+        cmp_rows = cmp_rows([int(x) for x in lens_t])
+    cmp_rows = set(batch_rows if cmp_rows is None else cmp_rows)
     w_ck, pe_k, w_cv, pe_v = (f64(inp[x]) for x in ("w_ck", "pe_k", "w_cv", "pe_v"))
     gsel_all = sel.cpu().numpy()
     gimp_all = imp.cpu().numpy().astype(np.float64)
+    stats = {"gpu": dict(lens=[int(x) for x in lens_t], sel=gsel_all, imp=gimp_all)}
     gout_all = f64(out)
     for b in batch_rows:
         L = int(lens_t[b])
         nc = nsa.n_cmp(L, op["l_cmp"], op["stride"])
-        kb = f64(inp["k_cache"][b, :L])
-        vb = f64(inp["v_cache"][b, :L])
-        kcg = f64(kc[b, :nc])
-        vcg = f64(vc[b, :nc])
-        if nc:
-            assert_close(kcg, O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"]), "k_cmp cache", relative_to_rms=True)
-            assert_close(vcg, O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]), "v_cmp cache", relative_to_rms=True)
         t = L - 1
+        if nc and b in cmp_rows:
+            kb = f64(inp["k_cache"][b, :L])
+            vb = f64(inp["v_cache"][b, :L])
+            kco = O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"])
+            vco = O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"])
+            assert_close(f64(kc[b, :nc]), kco, "k_cmp cache", relative_to_rms=True)
+            assert_close(f64(vc[b, :nc]), vco, "v_cmp cache", relative_to_rms=True)
+            # end to end: the oracle on its own fp64 compressed caches
+            one = dict(q=inp["q"][b:b + 1], k=inp["k_cache"][b:b + 1], v=inp["v_cache"][b:b + 1],
+                       g=inp["gates"][b:b + 1])
+            orc_e = O.decode(one["q"], one["k"], one["v"], kco[None], vco[None], [L], one["g"], op)
+
+            def rerun_e(override, one=one, kco=kco, vco=vco, L=L, b=b):
+                ov = {(0, g): v for (bb, g), v in override.items()}
+                return O.decode(one["q"], one["k"], one["v"], kco[None], vco[None], [L], one["g"], op,
+                                sel_override=ov)["out"]
+            m, r = check_end_to_end([(0, t)], gsel_all[b:b + 1], gimp_all[b:b + 1], gout_all[b:b + 1], orc_e,
+                                    rerun_e, op, cfg.H_kv, stats)
+            stats.setdefault("e2e_max_abs", []).append(m)
         orc = O.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens_t, inp["gates"], op, batch_rows=[b])
 
         def rerun(override, b=b):

@@ -11,8 +11,8 @@ import sparse_attention_long_nsa_b200 as nsa
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _header_functions():
-    src = open(os.path.join(ROOT, "include", "nsa.h")).read()
+def _header_functions(name="nsa.h"):
+    src = open(os.path.join(ROOT, "include", name)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(nsa_[a-z_]+)\s*\(", src)))
 
@@ -31,6 +31,24 @@ def test_exports_every_declared_symbol(L):
     assert set(declared) == set(nsa.EXPORTED)
     for name in declared:
         assert hasattr(L, name), name
+
+
+def test_checking_build_exports(L):
+    """libnsa_check.so exports what nsa.h and nsa_check.h declare; the library
+    build does not export the test-only fault setter."""
+    if not os.path.exists(nsa.CHECK_LIB_PATH):
+        from sparse_attention_long_nsa_b200 import build
+        build.build_check()
+    C = ctypes.CDLL(nsa.CHECK_LIB_PATH)
+    declared = set(_header_functions("nsa.h")) | set(_header_functions("nsa_check.h"))
+    assert declared == set(nsa.CHECK_EXPORTED)
+    for name in declared:
+        assert hasattr(C, name), name
+    assert not hasattr(L, "nsa_test_set_fault")
+    C.nsa_test_set_fault.restype = ctypes.c_int
+    C.nsa_test_set_fault.argtypes = [ctypes.c_int32]
+    assert C.nsa_test_set_fault(99) == nsa.NSA_ERR_INVALID_ARG
+    assert C.nsa_test_set_fault(0) == nsa.NSA_OK
 
 
 def test_status_strings(L):
@@ -149,3 +167,35 @@ def test_append_plan_multi_token_growth():
             if new:
                 assert co[b] == b * Lc + new[0] and (tok[b] - b * Lmax) % s == 0
                 assert (tok[b] - b * Lmax) + sl[b] <= L   # the segment ends inside the grown cache
+
+
+def test_paged_entry_points_validate_on_host(L):
+    """Page sizes that would let a selection block (64 tokens) or a tile of 32
+    summaries straddle pages, missing tables and inconsistent lengths are
+    rejected on the host, before any launch (fake device pointers are never
+    dereferenced)."""
+    h, p = nsa.Heads(64, 4, 192, 128), nsa.make_params()
+    fake = ctypes.c_void_p(1 << 20)
+    lens = (ctypes.c_int32 * 2)(100, 200)
+    for page, cpage, table in ((48, 32, fake), (64, 16, fake), (64, 32, None), (0, 32, fake)):
+        st = L.nsa_decode_paged(fake, fake, fake, 10, page, table, 8, fake, fake, 10, cpage, fake, 8, fake, 2, 200,
+                                fake, ctypes.byref(h), ctypes.byref(p), fake, None, None, fake, 1 << 30, None)
+        assert st == nsa.NSA_ERR_INVALID_ARG, (page, cpage)
+        n = ctypes.c_int32(-1)
+        st = L.nsa_compress_paged(fake, fake, 10, page, table, 8, fake, fake, fake, fake, None, lens, 2, fake, fake,
+                                  10, cpage, fake, 8, ctypes.byref(h), ctypes.byref(p), ctypes.byref(n), fake,
+                                  1 << 30, None)
+        assert st == nsa.NSA_ERR_INVALID_ARG, (page, cpage)
+    # lengths beyond the tables' capacity (8 pages of 64 tokens)
+    big = (ctypes.c_int32 * 2)(100, 600)
+    st = L.nsa_compress_paged(fake, fake, 10, 64, fake, 8, fake, fake, fake, fake, None, big, 2, fake, fake, 10, 32,
+                              fake, 8, ctypes.byref(h), ctypes.byref(p), None, fake, 1 << 30, None)
+    assert st == nsa.NSA_ERR_INVALID_ARG
+    # append on a batched cache: lens above Lmax, lens_prev above lens
+    st = L.nsa_compress_append(fake, fake, fake, fake, fake, fake, None, big, 2, 512, 31, ctypes.byref(h),
+                               ctypes.byref(p), fake, fake, None, fake, 1 << 30, None)
+    assert st == nsa.NSA_ERR_INVALID_ARG
+    prev = (ctypes.c_int32 * 2)(101, 200)
+    st = L.nsa_compress_append(fake, fake, fake, fake, fake, fake, prev, lens, 2, 512, 31, ctypes.byref(h),
+                               ctypes.byref(p), fake, fake, None, fake, 1 << 30, None)
+    assert st == nsa.NSA_ERR_INVALID_ARG

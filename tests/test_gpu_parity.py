@@ -32,12 +32,65 @@ def test_prefill_gqa16_ragged(seqlens):
 
 
 def test_prefill_8k_sampled():
-    """The benched 8K prefill, in the same launch configuration, on sampled rows."""
-    NP.run_prefill_case(CFG["prefill_8k"], [8192], n_random_rows=160)
+    """The benched 8K prefill, in the same launch configuration, on sampled rows;
+    64 of them also end to end against the oracle's own fp64 compression."""
+    st = NP.run_prefill_case(CFG["prefill_8k"], [8192], n_random_rows=1024, e2e_rows=64)
+    assert st["e2e_max_abs"]
 
 
 def test_prefill_64k_sampled():
-    NP.run_prefill_case(CFG["prefill_64k"], [65536], n_random_rows=48)
+    """The 64K prefill in the benched launch configuration: 1024 random rows plus
+    the edges, 64 of them also end to end."""
+    st = NP.run_prefill_case(CFG["prefill_64k"], [65536], n_random_rows=1024, e2e_rows=64)
+    assert st["e2e_max_abs"]
+
+
+def _ties_checked(stats, op, H_kv):
+    """Every checked row whose free candidates hold exact ties at the selection
+    boundary picks the lowest indices among them (the GPU's set must equal the
+    oracle's selection rule applied to the GPU's own scores, compared exactly).
+    Returns how many (row, group) pairs had such a tie."""
+    n_tied = 0
+    for rec in stats["gpu"] if isinstance(stats["gpu"], list) else [stats["gpu"]]:
+        rows = rec["rows"] if "rows" in rec else [L - 1 for L in rec["lens"]]
+        for ri, t in enumerate(rows):
+            jt = t // op["l_sel"]
+            if jt + 1 <= op["top_n"]:
+                continue
+            for g in range(H_kv):
+                imp = rec["imp"][ri, g, :jt + 1].astype(np.float64)
+                gs = [int(x) for x in rec["sel"][ri, g] if x >= 0]
+                want = O.select(imp, t, op["l_sel"], op["top_n"], op["force_first"], op["force_local"])
+                assert gs == want, f"t={t} g={g}: gpu {gs}, lowest-index rule on the gpu's scores {want}"
+                forced = O.forced_blocks(t, op["l_sel"], op["force_first"], op["force_local"])
+                free = sorted((float(imp[j]) for j in range(jt + 1) if j not in forced), reverse=True)
+                need = op["top_n"] - len(forced)
+                if need < len(free) and free[need - 1] == free[need]:
+                    n_tied += 1
+    return n_tied
+
+
+def _zero_keys(kc):
+    return torch.zeros_like(kc)
+
+
+def test_prefill_beyond_64k_radix_topn_and_ties():
+    """66,000 tokens: 1032 candidate blocks, beyond the register top-n (the radix
+    select path); 256 random rows plus the edges. Then the same sequence with all
+    compressed keys zero: every compressed probability of a row is equal, so the
+    interior blocks tie exactly and the lowest indices must win."""
+    cfg = W.small_config(name="prefill_66k", T=66000, H_q=64, H_kv=4, d_k=192, d_v=128, seed=1005)
+    NP.run_prefill_case(cfg, [66000], n_random_rows=256)
+    st = NP.run_prefill_case(cfg, [66000], n_random_rows=64, k_cmp_fn=_zero_keys)
+    assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
+
+
+def test_prefill_exact_ties_register_topn():
+    """All compressed keys zero (exact ties between interior blocks) on the
+    register top-n path of the prefill (GQA 16 and GQA 4)."""
+    for cfg, T in ((CFG["prefill_8k"], 4000), (CFG["prefill_tiny_1k"], 1024)):
+        st = NP.run_prefill_case(cfg, [T], n_random_rows=256, k_cmp_fn=_zero_keys)
+        assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
 
 
 def _dense_ref(inp, G, scale):
@@ -131,18 +184,42 @@ def test_decode_matches_prefill_last_row():
     NP.assert_close(NP.f64(out_d[0]), NP.f64(out_p[T - 1]), "decode vs prefill")
 
 
-def test_decode_64k_sampled():
+def test_decode_64k_all_sequences():
+    """The benched 64K decode batch: every one of the 32 sequences (selection and
+    output); the compressed caches of four of them recomputed by the oracle, and
+    those four also end to end."""
     cfg = CFG["decode_64k"]
-    NP.run_decode_case(cfg, [cfg.T] * cfg.B, batch_rows=[0, 13, 31])
+    NP.run_decode_case(cfg, [cfg.T] * cfg.B, cmp_rows=[0, 7, 13, 31])
 
 
-def test_decode_varlen_sampled():
+def test_decode_varlen_all_sequences():
+    """The varlen decode batch (64 cache lengths drawn in [8192, 131072]): every
+    sequence; the shortest, median and longest compressed caches recomputed by
+    the oracle (and checked end to end)."""
     cfg = CFG["decode_varlen"]
 
     def pick(lens):
         order = np.argsort(lens)
         return [int(order[0]), int(order[len(lens) // 2]), int(order[-1])]
-    NP.run_decode_case(cfg, None, batch_rows=pick)
+    NP.run_decode_case(cfg, None, cmp_rows=pick)
+
+
+def test_decode_longest_caches_fallback_topn_and_ties():
+    """The longest supported cache (262,144 tokens: 4096 candidate blocks, beyond
+    the CTA-wide top-n, so the warp radix select runs) next to a 170,001-token and
+    a short cache; then the same caches with zero compressed keys (exact ties)."""
+    cfg = CFG["decode_64k"]
+    lens = [262144, 170001, 5000]
+    NP.run_decode_case(cfg, lens, seed=41, cmp_rows=[2])
+    st = NP.run_decode_case(cfg, lens, seed=41, kc_fn=_zero_keys)
+    assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
+
+
+def test_decode_exact_ties_cta_topn():
+    """Zero compressed keys on the CTA-wide top-n path (up to 2560 candidates)."""
+    cfg = CFG["decode_64k"]
+    st = NP.run_decode_case(cfg, [20000, 65536, 3001, 160000], seed=43, kc_fn=_zero_keys)
+    assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
 
 
 def test_decode_incremental_compressed_cache():
@@ -177,6 +254,43 @@ def test_decode_incremental_compressed_cache():
         NP.assert_close(NP.f64(vc[b, :nc]), O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]), "appended v_cmp",
                         relative_to_rms=True)
         # same kernel arithmetic per block: at most a bf16 rounding step apart from one call
+        d = (kc[b, :nc].float() - kc1[b, :nc].float()).abs()
+        assert float(d.max()) <= 2.0 ** -7 * float(kc1[b, :nc].float().abs().max())
+
+
+def test_decode_incremental_growth_by_chunks():
+    """Sequences that grow by several tokens at a time (7, 16, 33 and 500 per round,
+    one size per sequence) through nsa_compress_append with the previous lengths:
+    each call writes one segment of many blocks per sequence into the compressed
+    caches in place; the grown caches match the fp64 oracle and one call over the
+    whole cache."""
+    cfg = CFG["decode_64k"]
+    lens0, grow, rounds = [20, 100, 1001, 4090], [7, 16, 33, 500], 5
+    lens_end = [L + g * rounds for L, g in zip(lens0, grow)]
+    inp = W.make_decode_inputs(cfg, device="cuda", lens=lens_end, seed=37)
+    heads, par, op = NP.heads_of(cfg), NP.params_of(cfg), NP.oracle_params(cfg)
+    kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"],
+                                lens0, heads, par)
+    ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, len(lens0), 0, 0), "cuda")
+    written = 0
+    for r in range(1, rounds + 1):
+        prev = [L + g * (r - 1) for L, g in zip(lens0, grow)]
+        cur = [L + g * r for L, g in zip(lens0, grow)]
+        written += nsa.compress_append(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                       inp["pe_v"], cur, kc, vc, heads, par, ws=ws, lens_prev=prev)
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws)
+    assert written == sum(nsa.n_cmp(b) - nsa.n_cmp(a) for a, b in zip(lens0, lens_end))
+    kc1, vc1 = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                  inp["pe_v"], lens_end, heads, par)
+    w_ck, pe_k, w_cv, pe_v = (NP.f64(inp[x]) for x in ("w_ck", "pe_k", "w_cv", "pe_v"))
+    for b, L in enumerate(lens_end):
+        nc = nsa.n_cmp(L)
+        kb, vb = NP.f64(inp["k_cache"][b, :L]), NP.f64(inp["v_cache"][b, :L])
+        NP.assert_close(NP.f64(kc[b, :nc]), O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"]), "grown k_cmp",
+                        relative_to_rms=True)
+        NP.assert_close(NP.f64(vc[b, :nc]), O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]), "grown v_cmp",
+                        relative_to_rms=True)
         d = (kc[b, :nc].float() - kc1[b, :nc].float()).abs()
         assert float(d.max()) <= 2.0 ** -7 * float(kc1[b, :nc].float().abs().max())
 

@@ -5,14 +5,16 @@ fixed device array inside libnsa.so instead of a caller workspace.
 
 Called through the C ABI twice in a row (the array keeps the previous call's
 contents, so the second call checks that nothing stale leaks through) and
-compared with nsa_compress, which takes an explicit workspace, within the
-tolerance the parity tests use for compressed K/V. Kept in a file of its own
+compared with nsa_compress, which takes an explicit workspace, and with the
+fp64 oracle's compression, within the tolerance the parity tests use for
+compressed K/V. Kept in a file of its own
 that is collected last."""
 import pytest
 import torch
 
 import nsa_workloads as W
 import sparse_attention_long_nsa_b200 as nsa
+from oracle import nsa_oracle as O
 from tests import nsa_parity as NP
 
 pytestmark = pytest.mark.gpu
@@ -58,6 +60,18 @@ def test_noalloc_matches_workspace_entry_point(cfg_name, seqlens):
         torch.cuda.synchronize()
         NP.assert_close(NP.f64(k_out), NP.f64(ref_k), f"k_cmp (no-alloc call {call})", relative_to_rms=True)
         NP.assert_close(NP.f64(v_out), NP.f64(ref_v), f"v_cmp (no-alloc call {call})", relative_to_rms=True)
+    # and against the fp64 oracle's own compression of every sequence
+    op = NP.oracle_params(cfg)
+    w_ck, pe_k, w_cv, pe_v = (NP.f64(inp[x]) for x in ("w_ck", "pe_k", "w_cv", "pe_v"))
+    for b, L in enumerate(seqlens):
+        t0, c0, nc = int(tok[b]), int(cmp_off[b]), nsa.n_cmp(L, par.l_cmp, par.stride)
+        if nc == 0:
+            continue
+        kb, vb = NP.f64(inp["k"][t0:t0 + L]), NP.f64(inp["v"][t0:t0 + L])
+        NP.assert_close(NP.f64(k_out[c0:c0 + nc]), O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"]),
+                        "k_cmp (no-alloc) vs oracle", relative_to_rms=True)
+        NP.assert_close(NP.f64(v_out[c0:c0 + nc]), O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]),
+                        "v_cmp (no-alloc) vs oracle", relative_to_rms=True)
 
 
 def test_noalloc_rejects_invalid_arguments():
