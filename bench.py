@@ -441,6 +441,63 @@ def bench_decode(cfg, args, rank, ws, dev, pk):
     return res
 
 
+def backward_work(cfg):
+    """Useful FLOPs of the backward: per attended (query head, key) pair dV += P^T dO,
+    dP = dO V^T (2 d_v each), dQ += dZ K, dK += dZ^T Q (2 d_k each); the
+    compression's backward dx and dW (2 l d^2 each per compressed token and KV
+    head). The recomputed forward (S, O) is not counted."""
+    pc, ps, pw = prefill_pairs(cfg.T, cfg)
+    nc = (cfg.T - cfg.l_cmp) // cfg.stride + 1
+    attn = (pc + ps + pw) * cfg.H_q * 4 * (cfg.d_k + cfg.d_v)
+    comp = 2 * 2 * cfg.l_cmp * (cfg.d_k ** 2 + cfg.d_v ** 2) * nc * cfg.H_kv
+    return attn + comp
+
+
+def bench_backward(cfg, args, rank, ws, dev, pk):
+    """One step = nsa_prefill_backward of one sequence (the forward's compressed
+    keys and selection computed once before)."""
+    import sparse_attention_long_nsa_b200 as nsa
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
+                          cfg.force_local)
+    T = cfg.T
+    inp = W.make_prefill_inputs(cfg, device=dev, seed=cfg.seed + 97 * rank)
+    cu = inp["cu_seqlens"]
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], [T], heads, par)
+    out, sel = nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], cu, heads, par, want_sel=True)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed + 5)
+    dout = torch.randn(out.shape, generator=gen, device=dev).to(torch.bfloat16)
+    ws_b = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_BACKWARD, heads, par, 1, T, T), dev)
+    g = {n: torch.empty(tuple(x.shape), dtype=torch.float32, device=dev) for n, x in
+         (("dq", inp["q"]), ("dk", inp["k"]), ("dv", inp["v"]), ("dgates", inp["gates"]), ("dw_ck", inp["w_ck"]),
+          ("dpe_k", inp["pe_k"]), ("dw_cv", inp["w_cv"]), ("dpe_v", inp["pe_v"]))}
+    flush = _make_flush(dev)
+
+    def step():
+        nsa.nsa_prefill_backward(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], dout, sel, inp["w_ck"],
+                                 inp["pe_k"], inp["w_cv"], inp["pe_v"], cu, heads, par, g["dq"], g["dk"], g["dv"],
+                                 g["dgates"], g["dw_ck"], g["dpe_k"], g["dw_cv"], g["dpe_v"], ws_b)
+
+    step()
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws_b)
+    steps = max(3, min(args.steps, 10))
+    ms = timed_steps(step, steps, args.warmup, flush, ws)
+    kern, launches = _profiled(step, steps, args.warmup, flush, ws)
+    nsa.nsa_check_device_status(ws_b)
+    work = backward_work(cfg)
+    dominant = max(kern, key=lambda k: kern[k][0])
+    return {
+        "tokens_per_s": T * ws / (ms * 1e-3), "ms_per_step": ms, "useful_flop_per_step": work,
+        "tflops_useful": work / (ms * 1e-3) / 1e12 * ws,
+        "tc_frac_useful": work / (ms * 1e-3) / 1e12 / pk["tc"],
+        "tensor_path": "mma.sync (warp-level bf16 MMA, fp32 accumulation)",
+        "dominant_kernel": dominant,
+        "kernels_ms_per_step": {k: v[0] for k, v in kern.items()},
+        "launches_per_step": launches,
+    }
+
+
 def run_nsa(args, rank, ws):
     dev = torch.device("cuda", torch.cuda.current_device())
     pk = peaks()
@@ -458,6 +515,8 @@ def run_nsa(args, rank, ws):
     dec = bench_decode(DECODE, args, rank, ws, dev, pk)
     torch.cuda.empty_cache()
     dvar = bench_decode(DECODE_VARLEN, args, rank, ws, dev, pk)
+    torch.cuda.empty_cache()
+    bwd = bench_backward(PREFILL_8K, args, rank, ws, dev, pk)
     if rank != 0:
         return None
     cfg = PREFILL
@@ -496,9 +555,11 @@ def run_nsa(args, rank, ws):
                                      "d_k=192 d_v=128"),
         "decode_varlen": dict(dvar, workload="decode_varlen: B=64 x 1 query, cache lengths drawn uniformly in "
                                              "[8192, 131072] (seeded), H_q=64 H_kv=4, d_k=192 d_v=128"),
+        "prefill_backward_8k": dict(bwd, workload="backward of the 8K prefill (selection held fixed): dq, dk, "
+                                                   "dv, dgates, dW and dpe of the compression"),
         "cpu_baseline": cpu,
     }
-    for d in (res["prefill_8k"], res["decode"], res["decode_varlen"]):
+    for d in (res["prefill_8k"], res["decode"], res["decode_varlen"], res["prefill_backward_8k"]):
         d.pop("launches_per_step", None)
     return res
 

@@ -75,7 +75,7 @@ typedef struct {
   int32_t H_q, H_kv, d_k, d_v;
 } nsa_heads_t;
 
-enum { NSA_OP_COMPRESS = 0, NSA_OP_PREFILL = 1, NSA_OP_DECODE = 2 };
+enum { NSA_OP_COMPRESS = 0, NSA_OP_PREFILL = 1, NSA_OP_DECODE = 2, NSA_OP_BACKWARD = 3 };
 
 /* Bytes of workspace `op` needs. `batch` = number of sequences;
  * `total_tokens` = sum of sequence lengths (prefill; for NSA_OP_COMPRESS it sizes
@@ -261,6 +261,31 @@ nsa_status_t nsa_compress_paged(const void* k_pool, const void* v_pool, int32_t 
                                 const nsa_heads_t* heads, const nsa_params_t* params, int32_t* n_blocks,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of the causal NSA prefill ("Native Sparse Attention" lesson, section
+ * on native trainability: the top-n step is not differentiable and only decides
+ * which blocks are loaded; gradients flow through the compressed branch and the
+ * selected and window contributions). Gradients of L with dL/dout = dout with the
+ * selection held at `sel` (the forward's sel_out):
+ *   q, k, v, k_cmp, v_cmp, gates, cu_seqlens (HOST), batch, heads, params:
+ *            as given to nsa_compress / nsa_prefill (k_cmp/v_cmp its outputs)
+ *   dout     bf16 [N, H_q, d_v]
+ *   sel      int32 [N, H_kv, top_n], ascending, -1 padded (nsa_prefill sel_out)
+ *   w_ck, pe_k, w_cv, pe_v: the compression weights given to nsa_compress
+ *   dq       fp32 out [N, H_q, d_k];   dk fp32 out [N, H_kv, d_k]; dv [N, H_kv, d_v]
+ *   dgates   fp32 out [N, H_q, 3] (cmp, slc, win)
+ *   dw_ck, dw_cv  fp32 out [l_cmp*d, d];  dpe_k, dpe_v fp32 out [l_cmp, d]
+ * dk/dv include the compressed branch's share through the compression. The
+ * compressed-key gradients and dW are accumulated with atomic additions, so the
+ * low-order bits of dk, dv and dW may differ between calls. Workspace:
+ * nsa_workspace_size(NSA_OP_BACKWARD, heads, params, batch, N, max_len). */
+nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, const void* k_cmp,
+                                  const void* v_cmp, const float* gates, const void* dout, const int32_t* sel,
+                                  const float* w_ck, const float* pe_k, const float* w_cv, const float* pe_v,
+                                  const int32_t* cu_seqlens, int32_t batch, const nsa_heads_t* heads,
+                                  const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates,
+                                  float* dw_ck, float* dpe_k, float* dw_cv, float* dpe_v, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
 /* Opt-in per-kernel timing (no compute change). While enabled, every entry point
  * records a CUDA event pair on its stream around each of its kernel launches.
  * nsa_profile_read() waits for the recorded events, writes for each of the
@@ -268,7 +293,7 @@ nsa_status_t nsa_compress_paged(const void* k_pool, const void* v_pool, int32_t 
  * the previous read, and resets them. Slot names: nsa_profile_slot_name(). The
  * events are created on first use and reused; this is the only state the
  * library keeps between calls. Returns NSA_ERR_CUDA if an event query fails. */
-#define NSA_PROFILE_SLOTS 5
+#define NSA_PROFILE_SLOTS 9
 nsa_status_t nsa_profile_enable(int32_t enable);
 nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots);
 const char* nsa_profile_slot_name(int32_t slot);

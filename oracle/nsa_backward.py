@@ -78,12 +78,15 @@ def compress_backward(x, W, pe, dc, l: int, s: int):
     return dx, dW, dpe
 
 
-def backward(q, k, v, w_ck, pe_k, w_cv, pe_v, gates, dout, p, sel=None):
+def backward(q, k, v, w_ck, pe_k, w_cv, pe_v, gates, dout, p, sel=None, kc=None, vc=None):
     """Gradients of one causal NSA prefill sequence (Reading B1).
 
     q [T, H_q, d_k], k [T, H_kv, d_k], v [T, H_kv, d_v], compression weights as in
     nsa_oracle.prefill_full, gates [T, H_q, 3], dout [T, H_q, d_v]; `sel` maps
-    (t, kv head) -> block list (default: the forward's own selection).
+    (t, kv head) -> block list (default: the forward's own selection). `kc`, `vc`
+    (optional) are the compressed keys/values the attention steps use (stage-wise
+    checks feed the GPU's rounded ones, as the forward oracle takes them); the
+    compression's own backward always follows its definition from x, W and pe.
     Returns a dict with out, sel and the gradients dq, dk, dv, dw_ck, dpe_k,
     dw_cv, dpe_v, dgates.
     """
@@ -94,8 +97,8 @@ def backward(q, k, v, w_ck, pe_k, w_cv, pe_v, gates, dout, p, sel=None):
     T, H_q, d_k = q.shape
     H_kv, d_v = k.shape[1], v.shape[2]
     G = H_q // H_kv
-    kc = O.compress(k, w_ck, pe_k, l, s)
-    vc = O.compress(v, w_cv, pe_v, l, s)
+    kc = O.compress(k, w_ck, pe_k, l, s) if kc is None else f(kc)
+    vc = O.compress(v, w_cv, pe_v, l, s) if vc is None else f(vc)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)

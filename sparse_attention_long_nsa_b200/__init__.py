@@ -25,16 +25,16 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 CHECK_LIB_PATH = os.path.join(_PKG, "libnsa_check.so")
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_DEVICE_CHECK = range(6)
-NSA_OP_COMPRESS, NSA_OP_PREFILL, NSA_OP_DECODE = 0, 1, 2
+NSA_OP_COMPRESS, NSA_OP_PREFILL, NSA_OP_DECODE, NSA_OP_BACKWARD = 0, 1, 2, 3
 NSA_MAX_BATCH = 128
 NSA_NOALLOC_SCRATCH_BYTES = 4194304
 
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
             "nsa_compress_append_plan", "nsa_compress_append", "nsa_compress_paged", "nsa_compress_noalloc",
-            "nsa_decode_paged", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
+            "nsa_decode_paged", "nsa_prefill_backward", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
-NSA_PROFILE_SLOTS = 5
+NSA_PROFILE_SLOTS = 9
 # the checking build exports one more symbol (include/nsa_check.h)
 CHECK_EXPORTED = EXPORTED + ("nsa_test_set_fault",)
 FAULT_NONE, FAULT_DECODE_FINE_TILE, FAULT_PREFILL_K_TILE = 0, 1, 2
@@ -125,6 +125,9 @@ def _load(path: str) -> ctypes.CDLL:
     L.nsa_decode_paged.restype = ctypes.c_int
     L.nsa_decode_paged.argtypes = [P, P, P, I32, I32, P, I32, P, P, I32, I32, P, I32, P, I32, I32, P,
                                    ctypes.POINTER(Heads), ctypes.POINTER(Params), P, P, P, P, SZ, P]
+    L.nsa_prefill_backward.restype = ctypes.c_int
+    L.nsa_prefill_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
+                                       ctypes.POINTER(Params), P, P, P, P, P, P, P, P, P, SZ, P]
     L.nsa_compress_noalloc.restype = ctypes.c_int
     L.nsa_compress_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
                                        ctypes.POINTER(Params), P, P, P]
@@ -289,6 +292,23 @@ def nsa_decode_paged(q, k_pool, v_pool, block_table, k_cmp_pool, v_cmp_pool, cmp
                                   ctypes.byref(heads), ctypes.byref(params), _ptr(out, torch.bfloat16),
                                   _ptr(sel_out, torch.int32), _ptr(imp_out, torch.float32), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "nsa_decode_paged")
+
+
+def nsa_prefill_backward(q, k, v, k_cmp, v_cmp, gates, dout, sel, w_ck, pe_k, w_cv, pe_v, cu_seqlens, heads: Heads,
+                         params: Params, dq, dk, dv, dgates, dw_ck, dpe_k, dw_cv, dpe_v, ws, stream=None):
+    """Gradients of the prefill with the selection held at `sel` (nsa_prefill's
+    sel_out). dout bf16 [N, H_q, d_v]; every gradient fp32; cu_seqlens host int32."""
+    B = int(cu_seqlens.numel()) - 1
+    f32 = torch.float32
+    _check(lib().nsa_prefill_backward(_ptr(q, torch.bfloat16), _ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16),
+                                      _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16), _ptr(gates, f32),
+                                      _ptr(dout, torch.bfloat16), _ptr(sel, torch.int32), _ptr(w_ck, f32),
+                                      _ptr(pe_k, f32), _ptr(w_cv, f32), _ptr(pe_v, f32),
+                                      _ptr(cu_seqlens, torch.int32, "cpu"), B, ctypes.byref(heads),
+                                      ctypes.byref(params), _ptr(dq, f32), _ptr(dk, f32), _ptr(dv, f32),
+                                      _ptr(dgates, f32), _ptr(dw_ck, f32), _ptr(dpe_k, f32), _ptr(dw_cv, f32),
+                                      _ptr(dpe_v, f32), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "nsa_prefill_backward")
 
 
 def nsa_profile_enable(enable: bool):
@@ -460,6 +480,25 @@ def decode(q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, cache_lens_dev, max_le
     if want_imp:
         res.append(imp)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def prefill_backward(q, k, v, k_cmp, v_cmp, gates, dout, sel, w_ck, pe_k, w_cv, pe_v, cu_seqlens, heads: Heads,
+                     params: Params, ws=None) -> dict:
+    """Allocates the gradients (fp32) and the workspace, calls nsa_prefill_backward."""
+    cu = cu_seqlens.to("cpu", torch.int32).contiguous()
+    B = cu.numel() - 1
+    N = int(cu[-1])
+    max_len = int((cu[1:] - cu[:-1]).max()) if B > 0 else 0
+    dev = q.device
+    g = dict(dq=torch.empty_like(q, dtype=torch.float32), dk=torch.empty_like(k, dtype=torch.float32),
+             dv=torch.empty_like(v, dtype=torch.float32), dgates=torch.empty_like(gates),
+             dw_ck=torch.empty_like(w_ck), dpe_k=torch.empty_like(pe_k), dw_cv=torch.empty_like(w_cv),
+             dpe_v=torch.empty_like(pe_v))
+    if ws is None:
+        ws = alloc_workspace(nsa_workspace_size(NSA_OP_BACKWARD, heads, params, B, N, max_len), dev)
+    nsa_prefill_backward(q, k, v, k_cmp, v_cmp, gates, dout, sel, w_ck, pe_k, w_cv, pe_v, cu, heads, params,
+                         g["dq"], g["dk"], g["dv"], g["dgates"], g["dw_ck"], g["dpe_k"], g["dw_cv"], g["dpe_v"], ws)
+    return g
 
 
 def default_scale(d_k: int) -> float:

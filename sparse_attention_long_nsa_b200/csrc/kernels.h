@@ -12,7 +12,8 @@ constexpr int kMaxBatch = 128;
 // Opt-in per-kernel timing: CUDA events recorded on the launching stream around
 // each launch (see nsa_profile_enable / nsa_profile_read in include/nsa.h).
 enum ProfSlot {
-  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_FINE, P_COUNT
+  P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_FINE, P_BWD_INDEX, P_BWD_QUERY,
+  P_BWD_KEYS, P_BWD_COMPRESS, P_COUNT
 };
 void prof_begin(int slot, cudaStream_t st);
 void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()
@@ -131,6 +132,47 @@ struct DecodeMaps {
   CUtensorMap k, v, kc, vc;
   CUtensorMap q;   // q [B, H_q, d_k] with a box of one sequence's G heads
 };
+// ----- backward (prefill) -----
+struct BackwardArgs {
+  const void* q;          // bf16 [N, H_q, d_k]
+  const void* dout;       // bf16 [N, H_q, d_v]
+  const float* gates;     // fp32 [N, H_q, 3]
+  const int32_t* sel;     // int32 [N, H_kv, top_n] (the forward's selection)
+  float* dq;              // fp32 [N, H_q, d_k]
+  float* dk;              // fp32 [N, H_kv, d_k] (raw branches; the compression's share is added after)
+  float* dv;              // fp32 [N, H_kv, d_v]
+  float* dkc;             // fp32 [Nc, H_kv, d_k] (zeroed; compressed-key pass adds into it)
+  float* dvc;             // fp32 [Nc, H_kv, d_v]
+  float* dgates;          // fp32 [N, H_q, 3]
+  float* lse;             // fp32 [N, H_q, 3] per-branch log-sum-exp (log2 units), gate order
+  float* dd;              // fp32 [N, H_q, 3] per-branch <dout, O_b>, gate order
+  const int32_t* inv_off; // [n_lists + 1]: list (blk_prefix[b] + j) * H_kv + g
+  const int32_t* inv_tok; // tokens (index within the sequence) of every list
+  int H_q, H_kv, G, d_k, d_v;
+  int l, s, ls, top_n, window;
+  int nb_stride;          // selection blocks of the longest sequence
+  int tok_chunk;          // compressed-key pass: query tokens per CTA (grid.z splits)
+  float scale, scale_log2;
+  uint32_t* status;
+  SeqTable seqs;                        // tile_prefix: query tiles of 8 tokens
+  int32_t blk_prefix[kMaxBatch + 1];    // 64-key raw blocks per sequence (prefix)
+  int32_t cblk_prefix[kMaxBatch + 1];   // 64-entry compressed tiles per sequence (prefix)
+};
+struct BackwardMaps {
+  CUtensorMap k32, v32, kc32, vc32;     // 32-row boxes (query-side key tiles)
+  CUtensorMap k64, v64, kc64, vc64;     // 64-row boxes (key-side resident tiles)
+  CUtensorMap qg, dog;                  // one token's G heads of q / dout
+};
+size_t backward_query_smem(int d_k, int d_v, int nb);
+cudaError_t launch_backward_attn(const BackwardArgs& a, const BackwardMaps& m, int q_tiles, int raw_blocks,
+                                 int cmp_tiles, int cmp_z, cudaStream_t st);
+cudaError_t launch_inverted_index(const BackwardArgs& a, int64_t n_ent, int n_lists, int32_t* cnt, int32_t* off,
+                                  int32_t* cur, int32_t* slot, int32_t* tok, cudaStream_t st);
+cudaError_t launch_compress_backward(const float* dc, const void* x, const float* W, const float* pe, int d_in,
+                                     int d_out, int H_kv, int l, int s, const SeqTable& seqs,
+                                     const int32_t* ncmp_prefix, int64_t n_cmp_total, float* dx, float* dW,
+                                     float* dpe, float* colsum, cudaStream_t st);
+
 size_t decode_partials_floats(const DecodeArgs& a);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
 

@@ -103,6 +103,34 @@ PrefillWs prefill_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t N, int
   return w;
 }
 
+// backward workspace: per-branch lse and <dout, O_b>, fp32 gradients of the
+// compressed keys/values, the inverted selection index, column sums
+struct BackwardWs {
+  size_t lse, dd, dkc, dvc, cnt, off, cur, slot, tok, colsum, total;
+  int64_t n_lists, n_ent, ncmp;
+};
+BackwardWs backward_ws(const nsa_heads_t* h, const nsa_params_t* p, int batch, int64_t N, int64_t ncmp,
+                       int64_t nblk) {
+  BackwardWs w{};
+  w.n_lists = nblk * h->H_kv;
+  w.n_ent = N * h->H_kv * p->top_n;
+  w.ncmp = ncmp;
+  size_t off = 256;
+  w.lse = off; off = align256(off + (size_t)N * h->H_q * 3 * 4);
+  w.dd = off; off = align256(off + (size_t)N * h->H_q * 3 * 4);
+  w.dkc = off; off = align256(off + (size_t)ncmp * h->H_kv * h->d_k * 4);
+  w.dvc = off; off = align256(off + (size_t)ncmp * h->H_kv * h->d_v * 4);
+  w.cnt = off; off = align256(off + (size_t)w.n_lists * 4);
+  w.off = off; off = align256(off + (size_t)(w.n_lists + 1) * 4);
+  w.cur = off; off = align256(off + (size_t)w.n_lists * 4);
+  w.slot = off; off = align256(off + (size_t)w.n_ent * 4);
+  w.tok = off; off = align256(off + (size_t)w.n_ent * 4);
+  w.colsum = off; off = align256(off + 256 * 4);
+  w.total = off;
+  (void)batch;
+  return w;
+}
+
 void fill_decode_args(DecodeArgs& a, const nsa_heads_t* h, const nsa_params_t* p, int B, int Lmax,
                       int Lmax_cmp, int max_len) {
   a.B = B; a.Lmax = Lmax; a.Lmax_cmp = Lmax_cmp; a.max_len = max_len;
@@ -188,7 +216,8 @@ Profiler& prof() {
   return p;
 }
 
-const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_fine"};
+const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_fine",
+                                   "bwd_index", "bwd_query", "bwd_keys", "bwd_compress"};
 
 }  // namespace
 
@@ -294,6 +323,14 @@ size_t nsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_params_t* 
     case NSA_OP_PREFILL:
       if (check_params(params, true) != NSA_OK || total_tokens < 0 || max_len < 0) return 0;
       return prefill_ws(heads, params, total_tokens, max_len).total;
+    case NSA_OP_BACKWARD: {
+      if (check_params(params, true) != NSA_OK || total_tokens < 0) return 0;
+      // bounds of the packed compressed rows and selection blocks of any split
+      // of total_tokens into `batch` sequences
+      const int64_t ncmp = total_tokens / params->stride + batch;
+      const int64_t nblk = total_tokens / params->l_sel + batch;
+      return backward_ws(heads, params, batch, total_tokens, ncmp, nblk).total;
+    }
     case NSA_OP_DECODE: {
       if (check_params(params, true) != NSA_OK || max_len <= 0 || max_union_blocks(params) > 64) return 0;
       DecodeArgs a{};
@@ -700,6 +737,136 @@ nsa_status_t nsa_decode_paged(const void* q, const void* k_pool, const void* v_p
   return decode_common(q, k_pool, v_pool, k_cmp_pool, v_cmp_pool, cache_lens, batch, (int32_t)cap, (int32_t)ccap,
                        max_len, gates, heads, params, out, sel_out, imp_out, workspace, ws_bytes, stream, kv_pt,
                        cmp_pt, rows, crows);
+}
+
+nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, const void* k_cmp,
+                                  const void* v_cmp, const float* gates, const void* dout, const int32_t* sel,
+                                  const float* w_ck, const float* pe_k, const float* w_cv, const float* pe_v,
+                                  const int32_t* cu_seqlens, int32_t batch, const nsa_heads_t* heads,
+                                  const nsa_params_t* params, float* dq, float* dk, float* dv, float* dgates,
+                                  float* dw_ck, float* dpe_k, float* dw_cv, float* dpe_v, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, true)) != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !gates || !dout || !sel || !w_ck || !pe_k || !w_cv || !pe_v || !cu_seqlens || !dq ||
+      !dk || !dv || !dgates || !dw_ck || !dpe_k || !dw_cv || !dpe_v || !workspace)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(workspace) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return NSA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return NSA_ERR_INVALID_ARG;
+  int max_len = 0;
+  int64_t ncmp = 0, nblk = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (L < 0) return NSA_ERR_INVALID_ARG;
+    if (L > max_len) max_len = L;
+    ncmp += n_cmp_of(L, params->l_cmp, params->stride);
+    nblk += n_blk_of(L, params->l_sel);
+  }
+  const int64_t N = cu_seqlens[batch];
+  if (ncmp > 0 && (!k_cmp || !v_cmp || !aligned16(k_cmp) || !aligned16(v_cmp))) return NSA_ERR_INVALID_ARG;
+  const BackwardWs w = backward_ws(heads, params, batch, N, ncmp, nblk);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+  const int nb = n_blk_of(max_len, params->l_sel);
+  if (backward_query_smem(heads->d_k, heads->d_v, nb) > 232448) {
+    snprintf(g_detail, sizeof(g_detail), "sequence too long for the backward query kernel (%d blocks)", nb);
+    return NSA_ERR_UNSUPPORTED;
+  }
+  if (N == 0) return NSA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BackwardArgs a{};
+  a.q = q; a.dout = dout; a.gates = gates; a.sel = sel;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dgates = dgates;
+  a.dkc = (float*)(ws + w.dkc); a.dvc = (float*)(ws + w.dvc);
+  a.lse = (float*)(ws + w.lse); a.dd = (float*)(ws + w.dd);
+  a.inv_off = (const int32_t*)(ws + w.off); a.inv_tok = (const int32_t*)(ws + w.tok);
+  a.H_q = heads->H_q; a.H_kv = heads->H_kv; a.G = heads->H_q / heads->H_kv; a.d_k = heads->d_k; a.d_v = heads->d_v;
+  a.l = params->l_cmp; a.s = params->stride; a.ls = params->l_sel; a.top_n = params->top_n;
+  a.window = params->window;
+  a.nb_stride = nb;
+  a.tok_chunk = 2048;
+  a.scale = softmax_scale(params, heads->d_k);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  SeqTable t{};
+  t.n = batch;
+  int q_tiles = 0, raw = 0, ctile = 0;
+  int64_t coff = 0;
+  int32_t ncmp_prefix[NSA_MAX_BATCH + 1];
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+    const int nc = n_cmp_of(L, params->l_cmp, params->stride);
+    t.tile_prefix[b] = q_tiles;
+    t.tok_off[b] = cu_seqlens[b];
+    t.cmp_off[b] = coff;
+    t.len[b] = L;
+    a.blk_prefix[b] = raw;
+    a.cblk_prefix[b] = ctile;
+    ncmp_prefix[b] = (int32_t)coff;
+    q_tiles += (L + 7) / 8;
+    raw += n_blk_of(L, params->l_sel);
+    ctile += (nc + 63) / 64;
+    coff += nc;
+  }
+  t.tile_prefix[batch] = q_tiles;
+  a.blk_prefix[batch] = raw;
+  a.cblk_prefix[batch] = ctile;
+  ncmp_prefix[batch] = (int32_t)coff;
+  a.seqs = t;
+  const int cmp_z = (max_len + a.tok_chunk - 1) / a.tok_chunk;
+
+  BackwardMaps m;
+  memset(&m, 0, sizeof(m));
+  const void* kcb = ncmp > 0 ? k_cmp : k;
+  const void* vcb = ncmp > 0 ? v_cmp : v;
+  const int64_t crows = ncmp > 0 ? ncmp : N;
+  const int G = a.G;
+  if (!make_map_3d(&m.k32, k, heads->d_k, heads->H_kv, N, 1, 32) ||
+      !make_map_3d(&m.v32, v, heads->d_v, heads->H_kv, N, 1, 32) ||
+      !make_map_3d(&m.kc32, kcb, heads->d_k, heads->H_kv, crows, 1, 32) ||
+      !make_map_3d(&m.vc32, vcb, heads->d_v, heads->H_kv, crows, 1, 32) ||
+      !make_map_3d(&m.k64, k, heads->d_k, heads->H_kv, N, 1, 64) ||
+      !make_map_3d(&m.v64, v, heads->d_v, heads->H_kv, N, 1, 64) ||
+      !make_map_3d(&m.kc64, kcb, heads->d_k, heads->H_kv, crows, 1, 64) ||
+      !make_map_3d(&m.vc64, vcb, heads->d_v, heads->H_kv, crows, 1, 64) ||
+      !make_map_3d(&m.qg, q, heads->d_k, heads->H_q, N, G, 1) ||
+      !make_map_3d(&m.dog, dout, heads->d_v, heads->H_q, N, G, 1)) {
+    snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
+    return NSA_ERR_CUDA;
+  }
+  cudaError_t e = cudaSuccess;
+  if (ncmp > 0) {
+    e = cudaMemsetAsync(ws + w.dkc, 0, (size_t)ncmp * heads->H_kv * heads->d_k * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + w.dvc, 0, (size_t)ncmp * heads->H_kv * heads->d_v * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward memset");
+  }
+  prof_begin(P_BWD_INDEX, st);
+  e = launch_inverted_index(a, w.n_ent, (int)w.n_lists, (int32_t*)(ws + w.cnt), (int32_t*)(ws + w.off),
+                            (int32_t*)(ws + w.cur), (int32_t*)(ws + w.slot), (int32_t*)(ws + w.tok), st);
+  prof_end(P_BWD_INDEX, st, 3);
+  if (e != cudaSuccess) return cuda_fail(e, "backward index");
+  prof_begin(P_BWD_QUERY, st);
+  e = launch_backward_attn(a, m, q_tiles, 0, 0, 0, st);
+  prof_end(P_BWD_QUERY, st, 1);
+  if (e != cudaSuccess) return cuda_fail(e, "backward query pass");
+  prof_begin(P_BWD_KEYS, st);
+  e = launch_backward_attn(a, m, 0, raw, ctile, cmp_z, st);
+  prof_end(P_BWD_KEYS, st, ctile > 0 ? 2 : 1);
+  if (e != cudaSuccess) return cuda_fail(e, "backward key passes");
+  prof_begin(P_BWD_COMPRESS, st);
+  float* colsum = (float*)(ws + w.colsum);
+  e = launch_compress_backward(a.dkc, k, w_ck, pe_k, heads->d_k, heads->d_k, heads->H_kv, params->l_cmp,
+                               params->stride, t, ncmp_prefix, ncmp, dk, dw_ck, dpe_k, colsum, st);
+  if (e == cudaSuccess)
+    e = launch_compress_backward(a.dvc, v, w_cv, pe_v, heads->d_v, heads->d_v, heads->H_kv, params->l_cmp,
+                                 params->stride, t, ncmp_prefix, ncmp, dv, dw_cv, dpe_v, colsum, st);
+  prof_end(P_BWD_COMPRESS, st, 10);
+  if (e != cudaSuccess) return cuda_fail(e, "backward compression");
+  return NSA_OK;
 }
 
 }  // extern "C"
