@@ -16,6 +16,11 @@ Draw order (fixed so that any consumer reproduces the same tensors):
            pe_v the same way with d_v; gates = sigmoid(N(0,1)) of shape [T, H_q, 3].
   decode:  cache lengths first (varlen only: uniform integers in [lo, hi]); then q,
            the K cache, the V cache, W_ck, pe_k, W_cv, pe_v, gates, as above.
+  DSA:     (decode: cache lengths first, as above) q, k, v as above, then the
+           indexer's queries q_I [*, H_I, d_I] and keys k_I [*, d_I] ~ N(0,1)
+           rounded to FP8 E4M3, and its weights w_I [*, H_I] ~ N(0,1) fp32
+           ("Разреженное внимание — NSA и DSA", section "DSA: молниеносный
+           индексатор": a few small heads, FP8, weights that depend on the query).
 """
 from __future__ import annotations
 
@@ -147,3 +152,86 @@ def small_config(name="small", T=256, H_q=4, H_kv=1, d_k=64, d_v=64, **kw) -> NS
     base = dict(kind="prefill", B=1, T=T, H_q=H_q, H_kv=H_kv, d_k=d_k, d_v=d_v)
     base.update(kw)
     return NSAConfig(name=name, **base)
+
+
+@dataclasses.dataclass(frozen=True)
+class DSAConfig:
+    """A DSA workload (lightning indexer + token top-k + attention over the kept
+    tokens). H_I, d_I: indexer heads and head size; top_k: tokens kept per query."""
+    name: str
+    kind: str
+    B: int
+    T: int
+    H_q: int
+    H_kv: int
+    d_k: int
+    d_v: int
+    H_I: int = 8
+    d_I: int = 128
+    top_k: int = 2048
+    len_lo: Optional[int] = None
+    len_hi: Optional[int] = None
+    seed: int = 2000
+
+    @property
+    def G(self) -> int:
+        return self.H_q // self.H_kv
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d_k)
+
+
+DSA_CONFIGS = {
+    "dsa_prefill_tiny": DSAConfig("dsa_prefill_tiny", "prefill", 1, 1024, 4, 1, 64, 64, H_I=4, d_I=64, top_k=256,
+                                  seed=2000),
+    "dsa_prefill_8k": DSAConfig("dsa_prefill_8k", "prefill", 1, 8192, 64, 4, 192, 128, seed=2001),
+    "dsa_decode_64k": DSAConfig("dsa_decode_64k", "decode", 32, 65536, 64, 4, 192, 128, seed=2002),
+}
+
+
+def _fp8(x):
+    return x.to(torch.float8_e4m3fn)
+
+
+def make_dsa_prefill_inputs(cfg: DSAConfig, device="cpu", seqlens=None, seed=None):
+    """Packed DSA prefill inputs: q, k, v (bf16) as make_prefill_inputs, then qi
+    [N, H_I, d_I] and ki [N, d_I] (FP8 E4M3), wi [N, H_I] (fp32), cu_seqlens (host)."""
+    seqlens = list(seqlens) if seqlens is not None else [cfg.T] * cfg.B
+    N = int(sum(seqlens))
+    g = _gen(cfg.seed if seed is None else seed, device)
+    q = _normal((N, cfg.H_q, cfg.d_k), g, device).to(torch.bfloat16)
+    k = _normal((N, cfg.H_kv, cfg.d_k), g, device).to(torch.bfloat16)
+    v = _normal((N, cfg.H_kv, cfg.d_v), g, device).to(torch.bfloat16)
+    qi = _fp8(_normal((N, cfg.H_I, cfg.d_I), g, device))
+    ki = _fp8(_normal((N, cfg.d_I), g, device))
+    wi = _normal((N, cfg.H_I), g, device)
+    cu = [0]
+    for x in seqlens:
+        cu.append(cu[-1] + int(x))
+    return dict(q=q, k=k, v=v, qi=qi, ki=ki, wi=wi, cu_seqlens=torch.tensor(cu, dtype=torch.int32))
+
+
+def make_dsa_decode_inputs(cfg: DSAConfig, device="cpu", seed=None, lens=None, Lmax=None):
+    """DSA decode inputs: cache lengths (varlen draws first), q [B, H_q, d_k], the K/V
+    caches [B, Lmax, H_kv, d] (bf16), qi [B, H_I, d_I] and the indexer key cache
+    ki [B, Lmax, d_I] (FP8 E4M3), wi [B, H_I] (fp32)."""
+    g = _gen(cfg.seed if seed is None else seed, device)
+    if lens is None:
+        if cfg.len_lo is not None:
+            lens = torch.randint(cfg.len_lo, cfg.len_hi + 1, (cfg.B,), generator=g, device=device)
+            lens = lens.to("cpu").to(torch.int32)
+        else:
+            lens = torch.full((cfg.B,), cfg.T, dtype=torch.int32)
+    else:
+        lens = torch.as_tensor(lens, dtype=torch.int32)
+    B = int(lens.numel())
+    if Lmax is None:
+        Lmax = int(lens.max())
+    q = _normal((B, cfg.H_q, cfg.d_k), g, device).to(torch.bfloat16)
+    k_cache = _normal((B, Lmax, cfg.H_kv, cfg.d_k), g, device).to(torch.bfloat16)
+    v_cache = _normal((B, Lmax, cfg.H_kv, cfg.d_v), g, device).to(torch.bfloat16)
+    qi = _fp8(_normal((B, cfg.H_I, cfg.d_I), g, device))
+    ki_cache = _fp8(_normal((B, Lmax, cfg.d_I), g, device))
+    wi = _normal((B, cfg.H_I), g, device)
+    return dict(q=q, k_cache=k_cache, v_cache=v_cache, qi=qi, ki_cache=ki_cache, wi=wi, cache_lens=lens)

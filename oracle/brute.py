@@ -147,3 +147,33 @@ def nsa_prefill_brute(q, k, v, kc, vc, gates, p):
             sel_all[(t, g)] = sel_rows[t]
             imp_all[(t, g)] = imp[t, :t // ls + 1]
     return out, sel_all, imp_all
+
+
+# ---------------------------------------------------------------------------
+# DSA variant, dense formulation (tiny inputs only)
+# ---------------------------------------------------------------------------
+
+def dsa_brute(q, k, v, qi, wi, ki, top_k, scale):
+    """Second formulation of the DSA variant (dsa_oracle.py): the full score
+    matrix I = ReLU(einsum over indexer heads) weighted and summed, a causal mask,
+    a rank matrix from a lexicographic sort (score descending, index ascending),
+    the keep mask rank < top_k, then masked attention per head (-inf outside the
+    mask, max-subtracted softmax). Returns (out [T, H_q, d_v], keep [T, T] bool)."""
+    q, k, v, qi, wi, ki = (np.asarray(x, dtype=np.float64) for x in (q, k, v, qi, wi, ki))
+    T, H_q, _ = q.shape
+    H_kv = k.shape[1]
+    G = H_q // H_kv
+    dots = np.einsum("thd,sd->tsh", qi, ki)                 # [T, T, H_I]
+    I = np.einsum("tsh,th->ts", np.maximum(dots, 0.0), wi)  # [T, T]
+    causal = np.arange(T)[None, :] <= np.arange(T)[:, None]
+    keep = np.zeros((T, T), dtype=bool)
+    for t in range(T):
+        cand = np.nonzero(causal[t])[0]
+        order = np.lexsort((cand, -I[t, cand]))             # last key primary: score desc, then index
+        keep[t, cand[order[:top_k]]] = True
+    out = np.zeros((T, H_q, v.shape[2]))
+    for h in range(H_q):
+        g = h // G
+        o, _ = masked_attention(q[:, h], k[:, g], v[:, g], keep, scale)
+        out[:, h] = o
+    return out, keep
