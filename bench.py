@@ -498,6 +498,80 @@ def bench_backward(cfg, args, rank, ws, dev, pk):
     }
 
 
+def bench_dsa_decode(cfg, args, rank, ws, dev, pk):
+    """One step = nsa_dsa_decode of the batch. Bytes the method must read: every
+    cached indexer key (d_I FP8 bytes per token) and the K/V rows of the kept
+    tokens of every KV head."""
+    import sparse_attention_long_nsa_b200 as nsa
+    inp = W.make_dsa_decode_inputs(cfg, device=dev, seed=cfg.seed + 97 * rank)
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    dp = nsa.DsaParams(cfg.H_I, cfg.d_I, cfg.top_k, 0.0)
+    lens = [int(x) for x in inp["cache_lens"]]
+    B, Lmax = len(lens), int(inp["k_cache"].shape[1])
+    lens_d = inp["cache_lens"].to(dev)
+    out = torch.empty((B, cfg.H_q, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    ws_d = nsa.alloc_workspace(nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, heads, dp, B, 0, Lmax), dev)
+    flush = _make_flush(dev)
+
+    def step():
+        nsa.nsa_dsa_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["qi"], inp["wi"], inp["ki_cache"], lens_d,
+                           Lmax, dp, heads, out, None, None, ws_d)
+
+    step()
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws_d)
+    steps = max(args.steps, 20)
+    ms = timed_steps(step, steps, args.warmup, flush, ws)
+    kern, launches = _profiled(step, min(steps, 50), args.warmup, flush, ws)
+    idx_b = sum(L * cfg.d_I for L in lens)
+    kv_b = sum(min(L, cfg.top_k) * cfg.H_kv * (cfg.d_k + cfg.d_v) * 2 for L in lens)
+    gbs = (idx_b + kv_b) / (ms * 1e-3) / 1e9
+    return {
+        "tokens_per_s": B * ws / (ms * 1e-3), "ms_per_step": ms, "bytes_per_step": idx_b + kv_b,
+        "bytes_indexer_keys": idx_b, "bytes_kept_kv": kv_b, "hbm_gbs": gbs, "hbm_frac": gbs / pk["hbm"],
+        "hbm_peak_gbs": pk["hbm"], "kernels_ms_per_step": {k: v[0] for k, v in kern.items()},
+        "launches_per_step": launches,
+    }
+
+
+def bench_dsa_prefill(cfg, args, rank, ws, dev, pk):
+    """One step = nsa_dsa_prefill of one sequence. Useful FLOPs: the indexer on
+    every causal pair (2 H_I d_I, FP8) and attention over the kept tokens
+    (2 (d_k + d_v) per query head and kept token)."""
+    import sparse_attention_long_nsa_b200 as nsa
+    T = cfg.T
+    inp = W.make_dsa_prefill_inputs(cfg, device=dev, seed=cfg.seed + 97 * rank)
+    heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+    dp = nsa.DsaParams(cfg.H_I, cfg.d_I, cfg.top_k, 0.0)
+    cu = inp["cu_seqlens"]
+    out = torch.empty((T, cfg.H_q, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    ws_p = nsa.alloc_workspace(nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_PREFILL, heads, dp, 1, T, T), dev)
+    flush = _make_flush(dev)
+
+    def step():
+        nsa.nsa_dsa_prefill(inp["q"], inp["k"], inp["v"], inp["qi"], inp["wi"], inp["ki"], cu, dp, heads, out, None,
+                            None, ws_p)
+
+    step()
+    torch.cuda.synchronize()
+    nsa.nsa_check_device_status(ws_p)
+    steps = max(3, min(args.steps, 10))
+    ms = timed_steps(step, steps, args.warmup, flush, ws)
+    kern, launches = _profiled(step, steps, args.warmup, flush, ws)
+    pairs = T * (T + 1) // 2
+    kept = sum(min(t + 1, cfg.top_k) for t in range(T))
+    f_idx = pairs * 2 * cfg.H_I * cfg.d_I
+    f_att = kept * cfg.H_q * 2 * (cfg.d_k + cfg.d_v)
+    return {
+        "tokens_per_s": T * ws / (ms * 1e-3), "ms_per_step": ms, "useful_flop_per_step": f_idx + f_att,
+        "flop_indexer_fp8": f_idx, "flop_attention_bf16": f_att,
+        "tflops_useful": (f_idx + f_att) / (ms * 1e-3) / 1e12 * ws,
+        "tc_frac_useful_vs_bf16_peak": (f_idx + f_att) / (ms * 1e-3) / 1e12 / pk["tc"],
+        "tensor_path": "mma.sync (FP8 e4m3 indexer, bf16 attention)",
+        "kernels_ms_per_step": {k: v[0] for k, v in kern.items()}, "launches_per_step": launches,
+    }
+
+
 def run_nsa(args, rank, ws):
     dev = torch.device("cuda", torch.cuda.current_device())
     pk = peaks()
@@ -517,6 +591,10 @@ def run_nsa(args, rank, ws):
     dvar = bench_decode(DECODE_VARLEN, args, rank, ws, dev, pk)
     torch.cuda.empty_cache()
     bwd = bench_backward(PREFILL_8K, args, rank, ws, dev, pk)
+    torch.cuda.empty_cache()
+    dsa_d = bench_dsa_decode(W.DSA_CONFIGS["dsa_decode_64k"], args, rank, ws, dev, pk)
+    torch.cuda.empty_cache()
+    dsa_p = bench_dsa_prefill(W.DSA_CONFIGS["dsa_prefill_8k"], args, rank, ws, dev, pk)
     if rank != 0:
         return None
     cfg = PREFILL
@@ -557,9 +635,14 @@ def run_nsa(args, rank, ws):
                                              "[8192, 131072] (seeded), H_q=64 H_kv=4, d_k=192 d_v=128"),
         "prefill_backward_8k": dict(bwd, workload="backward of the 8K prefill (selection held fixed): dq, dk, "
                                                    "dv, dgates, dW and dpe of the compression"),
+        "dsa_decode_64k": dict(dsa_d, workload="DSA variant decode: B=32 x 1 query, cache 65536, H_q=64 H_kv=4, "
+                                               "d_k=192 d_v=128, indexer H_I=8 d_I=128 FP8, top-2048 tokens"),
+        "dsa_prefill_8k": dict(dsa_p, workload="DSA variant prefill: T=8192, heads as above, indexer H_I=8 d_I=128 "
+                                               "FP8, top-2048 tokens per query"),
         "cpu_baseline": cpu,
     }
-    for d in (res["prefill_8k"], res["decode"], res["decode_varlen"], res["prefill_backward_8k"]):
+    for d in (res["prefill_8k"], res["decode"], res["decode_varlen"], res["prefill_backward_8k"],
+              res["dsa_decode_64k"], res["dsa_prefill_8k"]):
         d.pop("launches_per_step", None)
     return res
 

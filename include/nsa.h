@@ -286,6 +286,54 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
                                   float* dw_ck, float* dpe_k, float* dw_cv, float* dpe_v, void* workspace,
                                   size_t ws_bytes, void* stream);
 
+/* DSA variant ("Разреженное внимание — NSA и DSA", section "DSA: молниеносный
+ * индексатор"): a lightning indexer scores every past token s <= t of query t,
+ *   I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s])   (H_I heads of size d_I, FP8)
+ * the top_k tokens by I are kept (ties to the lower index; every token when
+ * t + 1 <= top_k) and each query head attends to the raw keys/values of the kept
+ * tokens (GQA: head h uses KV head h / G; scale as in nsa_params_t; one
+ * selection serves all heads). Supported: H_I <= 16, d_I in {32, 64, 128},
+ * top_k <= 65536, the head dims of the NSA entry points. */
+typedef struct {
+  int32_t H_I, d_I, top_k;
+  float scale;   /* 0 => 1/sqrt(d_k) */
+} nsa_dsa_params_t;
+
+enum { NSA_OP_DSA_DECODE = 4, NSA_OP_DSA_PREFILL = 5 };
+
+/* Workspace bytes of nsa_dsa_decode (batch sequences, caches up to max_len) or
+ * nsa_dsa_prefill (total_tokens packed tokens, longest sequence max_len; the
+ * queries run in chunks whose score rows fill at most 2^26 floats). 0 for
+ * invalid arguments. */
+size_t nsa_dsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_dsa_params_t* dsa, int32_t batch,
+                              int64_t total_tokens, int32_t max_len);
+
+/* DSA decode: one query per sequence at position cache_lens[b] - 1.
+ *   q          bf16 [batch, H_q, d_k]
+ *   k_cache    bf16 [batch, Lmax, H_kv, d_k]; v_cache bf16 [batch, Lmax, H_kv, d_v]
+ *   qi         fp8 e4m3 [batch, H_I, d_I];  wi fp32 [batch, H_I]
+ *   ki_cache   fp8 e4m3 [batch, Lmax, d_I] (the indexer's key of every cached token)
+ *   cache_lens DEVICE int32 [batch], 1 <= len <= max_len <= Lmax (others are
+ *              recorded in the status word and skipped)
+ *   out        bf16 out [batch, H_q, d_v]
+ *   idx_out    int32 out or NULL: [batch, top_k] kept tokens, ascending, -1 padded
+ *   score_out  fp32 out or NULL: [batch, max_len] indexer scores (entries past the
+ *              query's own position are unspecified) */
+nsa_status_t nsa_dsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* qi, const float* wi,
+                            const void* ki_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
+                            int32_t max_len, const nsa_dsa_params_t* dsa, const nsa_heads_t* heads, void* out,
+                            int32_t* idx_out, float* score_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* DSA causal prefill over packed sequences (positions restart at 0 per sequence).
+ *   q bf16 [N, H_q, d_k]; k, v bf16 [N, H_kv, d_k / d_v]; qi fp8 [N, H_I, d_I];
+ *   wi fp32 [N, H_I]; ki fp8 [N, d_I]; cu_seqlens HOST int32 [batch + 1];
+ *   out bf16 out [N, H_q, d_v]; idx_out int32 out or NULL [N, top_k];
+ *   score_out fp32 out or NULL [N, max_len] (max_len = longest sequence). */
+nsa_status_t nsa_dsa_prefill(const void* q, const void* k, const void* v, const void* qi, const float* wi,
+                             const void* ki, const int32_t* cu_seqlens, int32_t batch, const nsa_dsa_params_t* dsa,
+                             const nsa_heads_t* heads, void* out, int32_t* idx_out, float* score_out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Opt-in per-kernel timing (no compute change). While enabled, every entry point
  * records a CUDA event pair on its stream around each of its kernel launches.
  * nsa_profile_read() waits for the recorded events, writes for each of the
@@ -293,7 +341,7 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
  * the previous read, and resets them. Slot names: nsa_profile_slot_name(). The
  * events are created on first use and reused; this is the only state the
  * library keeps between calls. Returns NSA_ERR_CUDA if an event query fails. */
-#define NSA_PROFILE_SLOTS 9
+#define NSA_PROFILE_SLOTS 12
 nsa_status_t nsa_profile_enable(int32_t enable);
 nsa_status_t nsa_profile_read(double* ms_out, int64_t* launches_out, int32_t n_slots);
 const char* nsa_profile_slot_name(int32_t slot);

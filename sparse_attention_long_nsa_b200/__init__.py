@@ -32,9 +32,11 @@ NSA_NOALLOC_SCRATCH_BYTES = 4194304
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
             "nsa_compress_append_plan", "nsa_compress_append", "nsa_compress_paged", "nsa_compress_noalloc",
-            "nsa_decode_paged", "nsa_prefill_backward", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
+            "nsa_decode_paged", "nsa_prefill_backward", "nsa_dsa_workspace_size", "nsa_dsa_decode",
+            "nsa_dsa_prefill", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
-NSA_PROFILE_SLOTS = 9
+NSA_PROFILE_SLOTS = 12
+NSA_OP_DSA_DECODE, NSA_OP_DSA_PREFILL = 4, 5
 # the checking build exports one more symbol (include/nsa_check.h)
 CHECK_EXPORTED = EXPORTED + ("nsa_test_set_fault",)
 FAULT_NONE, FAULT_DECODE_FINE_TILE, FAULT_PREFILL_K_TILE = 0, 1, 2
@@ -57,6 +59,12 @@ class Heads(ctypes.Structure):
     """nsa_heads_t"""
     _fields_ = [("H_q", ctypes.c_int32), ("H_kv", ctypes.c_int32), ("d_k", ctypes.c_int32),
                 ("d_v", ctypes.c_int32)]
+
+
+class DsaParams(ctypes.Structure):
+    """nsa_dsa_params_t"""
+    _fields_ = [("H_I", ctypes.c_int32), ("d_I", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
 
 
 def make_params(l_cmp=32, stride=16, l_sel=64, top_n=16, window=512, force_first=1, force_local=2,
@@ -128,6 +136,15 @@ def _load(path: str) -> ctypes.CDLL:
     L.nsa_prefill_backward.restype = ctypes.c_int
     L.nsa_prefill_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
                                        ctypes.POINTER(Params), P, P, P, P, P, P, P, P, P, SZ, P]
+    L.nsa_dsa_workspace_size.restype = SZ
+    L.nsa_dsa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(Heads), ctypes.POINTER(DsaParams), I32, I64,
+                                         I32]
+    L.nsa_dsa_decode.restype = ctypes.c_int
+    L.nsa_dsa_decode.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, ctypes.POINTER(DsaParams),
+                                 ctypes.POINTER(Heads), P, P, P, P, SZ, P]
+    L.nsa_dsa_prefill.restype = ctypes.c_int
+    L.nsa_dsa_prefill.argtypes = [P, P, P, P, P, P, P, I32, ctypes.POINTER(DsaParams), ctypes.POINTER(Heads), P, P,
+                                  P, P, SZ, P]
     L.nsa_compress_noalloc.restype = ctypes.c_int
     L.nsa_compress_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
                                        ctypes.POINTER(Params), P, P, P]
@@ -309,6 +326,36 @@ def nsa_prefill_backward(q, k, v, k_cmp, v_cmp, gates, dout, sel, w_ck, pe_k, w_
                                       _ptr(dgates, f32), _ptr(dw_ck, f32), _ptr(dpe_k, f32), _ptr(dw_cv, f32),
                                       _ptr(dpe_v, f32), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "nsa_prefill_backward")
+
+
+def nsa_dsa_workspace_size(op: int, heads: Heads, dp: DsaParams, batch: int, total_tokens: int, max_len: int) -> int:
+    return int(lib().nsa_dsa_workspace_size(op, ctypes.byref(heads), ctypes.byref(dp), batch, total_tokens, max_len))
+
+
+def nsa_dsa_decode(q, k_cache, v_cache, qi, wi, ki_cache, cache_lens, max_len: int, dp: DsaParams, heads: Heads, out,
+                   idx_out=None, score_out=None, ws=None, stream=None):
+    """DSA decode: q [B, H_q, d_k]; caches [B, Lmax, H_kv, d]; qi fp8 [B, H_I, d_I];
+    wi fp32 [B, H_I]; ki_cache fp8 [B, Lmax, d_I]; cache_lens device int32 [B]."""
+    B, Lmax = int(k_cache.shape[0]), int(k_cache.shape[1])
+    f8 = torch.float8_e4m3fn
+    _check(lib().nsa_dsa_decode(_ptr(q, torch.bfloat16), _ptr(k_cache, torch.bfloat16), _ptr(v_cache, torch.bfloat16),
+                                _ptr(qi, f8), _ptr(wi, torch.float32), _ptr(ki_cache, f8),
+                                _ptr(cache_lens, torch.int32), B, Lmax, int(max_len), ctypes.byref(dp),
+                                ctypes.byref(heads), _ptr(out, torch.bfloat16), _ptr(idx_out, torch.int32),
+                                _ptr(score_out, torch.float32), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)), "nsa_dsa_decode")
+
+
+def nsa_dsa_prefill(q, k, v, qi, wi, ki, cu_seqlens, dp: DsaParams, heads: Heads, out, idx_out=None, score_out=None,
+                    ws=None, stream=None):
+    """DSA prefill over packed sequences; cu_seqlens host int32 [B+1]."""
+    B = int(cu_seqlens.numel()) - 1
+    f8 = torch.float8_e4m3fn
+    _check(lib().nsa_dsa_prefill(_ptr(q, torch.bfloat16), _ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16),
+                                 _ptr(qi, f8), _ptr(wi, torch.float32), _ptr(ki, f8),
+                                 _ptr(cu_seqlens, torch.int32, "cpu"), B, ctypes.byref(dp), ctypes.byref(heads),
+                                 _ptr(out, torch.bfloat16), _ptr(idx_out, torch.int32), _ptr(score_out, torch.float32),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "nsa_dsa_prefill")
 
 
 def nsa_profile_enable(enable: bool):

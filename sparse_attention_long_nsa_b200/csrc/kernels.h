@@ -13,7 +13,7 @@ constexpr int kMaxBatch = 128;
 // each launch (see nsa_profile_enable / nsa_profile_read in include/nsa.h).
 enum ProfSlot {
   P_COMPRESS_PREP = 0, P_COMPRESS_GEMM, P_PREFILL_ATTN, P_DEC_CMP, P_DEC_FINE, P_BWD_INDEX, P_BWD_QUERY,
-  P_BWD_KEYS, P_BWD_COMPRESS, P_COUNT
+  P_BWD_KEYS, P_BWD_COMPRESS, P_DSA_INDEX, P_DSA_TOPK, P_DSA_ATTN, P_COUNT
 };
 void prof_begin(int slot, cudaStream_t st);
 void set_error_detail(const char* msg);   // text returned by nsa_last_error_detail()
@@ -172,6 +172,28 @@ cudaError_t launch_compress_backward(const float* dc, const void* x, const float
                                      int d_out, int H_kv, int l, int s, const SeqTable& seqs,
                                      const int32_t* ncmp_prefix, int64_t n_cmp_total, float* dx, float* dW,
                                      float* dpe, float* colsum, cudaStream_t st);
+
+// ----- DSA variant (lightning indexer + token top-k + attention) -----
+struct DsaArgs {
+  const void* q;          // bf16 [*, H_q, d_k]
+  const void* k;          // bf16 rows of the raw keys: token s of a query's sequence at row base + s
+  const void* v;
+  const void* qi;         // fp8 e4m3 [*, H_I, d_I] (row = the query row)
+  const void* ki;         // fp8 e4m3 [*, d_I] (row base + s)
+  const float* wi;        // fp32 [*, H_I]
+  void* out;              // bf16 [*, H_q, d_v]
+  float* scores;          // fp32 [slots, ld_scores] indexer scores of this chunk of queries
+  int32_t* idx;           // int32 [slots, top_k] kept tokens (ascending, -1 padded)
+  int64_t ld_scores;
+  int64_t q0;             // first query of this chunk
+  const int32_t* lens;    // decode: device int32 [B] (query b at len - 1, base b * Lmax); null for prefill
+  int Lmax, max_len;
+  SeqTable seqs;          // prefill: packed sequences (query n = token n)
+  int H_q, H_kv, G, H_I, top_k;
+  float scale_log2;
+  uint32_t* status;
+};
+cudaError_t launch_dsa(const DsaArgs& a, int n_slots, int max_keys, int d_k, int d_v, int d_i, cudaStream_t st);
 
 size_t decode_partials_floats(const DecodeArgs& a);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);

@@ -217,7 +217,8 @@ Profiler& prof() {
 }
 
 const char* kSlotNames[P_COUNT] = {"compress_prep", "compress_gemm", "prefill_attn", "dec_cmp", "dec_fine",
-                                   "bwd_index", "bwd_query", "bwd_keys", "bwd_compress"};
+                                   "bwd_index", "bwd_query", "bwd_keys", "bwd_compress", "dsa_index", "dsa_topk",
+                                   "dsa_attn"};
 
 }  // namespace
 
@@ -866,6 +867,127 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
                                  params->stride, t, ncmp_prefix, ncmp, dv, dw_cv, dpe_v, colsum, st);
   prof_end(P_BWD_COMPRESS, st, 10);
   if (e != cudaSuccess) return cuda_fail(e, "backward compression");
+  return NSA_OK;
+}
+
+// ---- DSA variant ----
+static nsa_status_t check_dsa(const nsa_heads_t* heads, const nsa_dsa_params_t* dp) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if (!dp || dp->H_I <= 0 || dp->d_I <= 0 || dp->top_k <= 0 || !(dp->scale >= 0.f)) return NSA_ERR_INVALID_ARG;
+  if (dp->H_I > 16 || (dp->d_I != 32 && dp->d_I != 64 && dp->d_I != 128) || dp->top_k > 65536)
+    return NSA_ERR_UNSUPPORTED;
+  return NSA_OK;
+}
+
+// queries per chunk of a prefill: the score rows of a chunk fill at most 2^26 floats
+static int64_t dsa_chunk(int64_t n_queries, int max_len) {
+  const int64_t c = (int64_t(1) << 26) / (max_len > 0 ? max_len : 1);
+  return n_queries < c ? n_queries : (c > 0 ? c : 1);
+}
+
+struct DsaWs {
+  size_t scores, idx, total;
+};
+static DsaWs dsa_ws(int64_t slots, int max_len, int top_k) {
+  DsaWs w{};
+  size_t off = 256;
+  w.scores = off; off = align256(off + (size_t)slots * max_len * 4);
+  w.idx = off; off = align256(off + (size_t)slots * top_k * 4);
+  w.total = off;
+  return w;
+}
+
+size_t nsa_dsa_workspace_size(int op, const nsa_heads_t* heads, const nsa_dsa_params_t* dp, int32_t batch,
+                              int64_t total_tokens, int32_t max_len) {
+  if (check_dsa(heads, dp) != NSA_OK || batch <= 0 || batch > NSA_MAX_BATCH || max_len <= 0) return 0;
+  if (op == NSA_OP_DSA_DECODE) return dsa_ws(batch, max_len, dp->top_k).total;
+  if (op == NSA_OP_DSA_PREFILL) {
+    if (total_tokens < 0) return 0;
+    return dsa_ws(dsa_chunk(total_tokens, max_len), max_len, dp->top_k).total;
+  }
+  return 0;
+}
+
+static void fill_dsa(DsaArgs& a, const void* q, const void* k, const void* v, const void* qi, const float* wi,
+                     const void* ki, void* out, const nsa_heads_t* heads, const nsa_dsa_params_t* dp, void* ws) {
+  a.q = q; a.k = k; a.v = v; a.qi = qi; a.wi = wi; a.ki = ki; a.out = out;
+  a.H_q = heads->H_q; a.H_kv = heads->H_kv; a.G = heads->H_q / heads->H_kv; a.H_I = dp->H_I; a.top_k = dp->top_k;
+  a.scale_log2 = (dp->scale > 0.f ? dp->scale : 1.0f / sqrtf((float)heads->d_k)) * 1.4426950408889634f;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+}
+
+nsa_status_t nsa_dsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* qi, const float* wi,
+                            const void* ki_cache, const int32_t* cache_lens, int32_t batch, int32_t Lmax,
+                            int32_t max_len, const nsa_dsa_params_t* dp, const nsa_heads_t* heads, void* out,
+                            int32_t* idx_out, float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_dsa(heads, dp);
+  if (s != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !qi || !wi || !ki_cache || !cache_lens || !out || !workspace)
+    return NSA_ERR_INVALID_ARG;
+  if (max_len <= 0 || Lmax < max_len) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(qi) || !aligned16(ki_cache) ||
+      !aligned16(out) || !aligned16(workspace))
+    return NSA_ERR_INVALID_ARG;
+  const DsaWs w = dsa_ws(batch, max_len, dp->top_k);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DsaArgs a{};
+  fill_dsa(a, q, k_cache, v_cache, qi, wi, ki_cache, out, heads, dp, ws);
+  a.scores = score_out ? score_out : (float*)(ws + w.scores);
+  a.idx = idx_out ? idx_out : (int32_t*)(ws + w.idx);
+  a.ld_scores = max_len;
+  a.q0 = 0;
+  a.lens = cache_lens;
+  a.Lmax = Lmax;
+  a.max_len = max_len;
+  cudaError_t e = launch_dsa(a, batch, max_len, heads->d_k, heads->d_v, dp->d_I, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "dsa decode");
+}
+
+nsa_status_t nsa_dsa_prefill(const void* q, const void* k, const void* v, const void* qi, const float* wi,
+                             const void* ki, const int32_t* cu_seqlens, int32_t batch, const nsa_dsa_params_t* dp,
+                             const nsa_heads_t* heads, void* out, int32_t* idx_out, float* score_out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  nsa_status_t s = check_dsa(heads, dp);
+  if (s != NSA_OK) return s;
+  if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !qi || !wi || !ki || !cu_seqlens || !out || !workspace) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qi) || !aligned16(ki) || !aligned16(out) ||
+      !aligned16(workspace))
+    return NSA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return NSA_ERR_INVALID_ARG;
+  SeqTable t{};
+  t.n = batch;
+  int max_len = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (L < 0) return NSA_ERR_INVALID_ARG;
+    if (L > max_len) max_len = L;
+    t.tok_off[b] = cu_seqlens[b];
+    t.len[b] = L;
+  }
+  const int64_t N = cu_seqlens[batch];
+  if (N == 0) return NSA_OK;
+  const int64_t chunk = dsa_chunk(N, max_len);
+  const DsaWs w = dsa_ws(chunk, max_len, dp->top_k);
+  if (ws_bytes < w.total) return NSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DsaArgs a{};
+  fill_dsa(a, q, k, v, qi, wi, ki, out, heads, dp, ws);
+  a.scores = (float*)(ws + w.scores);
+  a.ld_scores = max_len;
+  a.seqs = t;
+  a.max_len = max_len;
+  for (int64_t q0 = 0; q0 < N; q0 += chunk) {
+    const int n = (int)(N - q0 < chunk ? N - q0 : chunk);
+    a.q0 = q0;
+    a.idx = idx_out ? idx_out + q0 * dp->top_k : (int32_t*)(ws + w.idx);
+    a.scores = score_out ? score_out + q0 * max_len : (float*)(ws + w.scores);
+    cudaError_t e = launch_dsa(a, n, max_len, heads->d_k, heads->d_v, dp->d_I, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dsa prefill");
+  }
   return NSA_OK;
 }
 
