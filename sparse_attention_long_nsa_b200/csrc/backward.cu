@@ -23,8 +23,9 @@
 //   bwd_keys   CTA = 64 keys x one KV group (4 warps x 16 keys), keys resident,
 //              query tokens streamed through a TMA ring: raw keys take the window
 //              tokens and the tokens whose selection holds the block (an inverted
-//              index); compressed keys take every later token (split over
-//              grid.z, added atomically). Writes dk, dv (raw) / dk_cmp, dv_cmp.
+//              index); compressed keys take every later token. The token
+//              sequence of a block is split over grid.z; shares are added
+//              atomically into dk, dv (raw) / dk_cmp, dv_cmp.
 //   inv_*      the inverted selection index (counts, scan, fill).
 //   cmp_bwd_*  the compression backward: column sums -> dpe; dx per residue of
 //              the token index modulo the stride (no atomics) added into dk/dv;
@@ -400,12 +401,14 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_keys_kernel(const BackwardA
   const int nc = cmp_vis(L - 1, a.l, a.s);   // compressed keys of the sequence
   // tokens: raw keys: the window range, then the block's inverted selection list;
   // compressed keys: this CTA's chunk of the tokens that see key0
+  // the concatenated token sequence (window range, then the list) is split over
+  // grid.z in chunks of tok_chunk, so a block that every token selects (block 0,
+  // forced) spreads over many CTAs; the CTAs add their shares atomically
   int w_lo = 0, w_n = 0, s_n = 0;
   const int32_t* s_list = nullptr;
   if (CMP) {
-    const int first = key0 * a.s + a.l - 1;
-    w_lo = first + blockIdx.z * a.tok_chunk;
-    w_n = max(0, min(L, w_lo + a.tok_chunk) - w_lo);
+    w_lo = key0 * a.s + a.l - 1;
+    w_n = max(0, L - w_lo);
   } else {
     w_lo = key0;
     w_n = max(0, min(L - 1, key0 + 63 + a.window - 1) - key0 + 1);
@@ -414,8 +417,11 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_keys_kernel(const BackwardA
     s_n = a.inv_off[ent + 1] - o0;
     s_list = a.inv_tok + o0;
   }
-  const int n_tok = w_n + s_n;
-  auto tok_of = [&](int i) -> int { return i < w_n ? w_lo + i : s_list[i - w_n]; };
+  const int c0 = blockIdx.z * a.tok_chunk;
+  const int n_tok = max(0, min(w_n + s_n - c0, a.tok_chunk));
+  if (n_tok == 0) return;   // nothing for this CTA (before any set-up)
+  auto tok_of = [&](int i) -> int { return i + c0 < w_n ? w_lo + i + c0 : s_list[i + c0 - w_n]; };
+  auto is_win = [&](int i) -> bool { return i + c0 < w_n; };
 
   if (tid == 0) {
     for (int i = 0; i < kBkStages; ++i) {
@@ -481,30 +487,44 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_keys_kernel(const BackwardA
   for (int i = 0; i < DV / 8; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
   // fragment (nt, e) of a [16 keys x 16 rows] product: key row km, query row qr
   const int cq = (lane & 3) * 2;
+  // per query row of this lane (rows cq, cq+1, cq+8, cq+9): the token's lse,
+  // <dout, O_b> and gate, loaded one token ahead of their use
+  float nlse[4], ndd[4], ngt[4];
+  auto load_rows = [&](int i) {
+    const int t = tok_of(i);
+    const int br = CMP ? 0 : (is_win(i) ? 2 : 1);   // gate / lse slot: 0 cmp, 1 slc, 2 win
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int qr = cq + (x & 1) + 8 * (x >> 1);
+      if (qr < G) {
+        const size_t o = ((size_t)(tok0 + t) * a.H_q + g * G + qr) * 3 + br;
+        nlse[x] = a.lse[o];
+        ndd[x] = a.dd[o];
+        ngt[x] = a.gates[o];
+      } else {
+        nlse[x] = kNoKeys;
+        ndd[x] = 0.f;
+        ngt[x] = 0.f;
+      }
+    }
+  };
+  load_rows(0);
 #pragma unroll 1
   for (int i = 0; i < n_tok; ++i) {
     const int st = i % kBkStages;
+    float lse[4], dd[4], gt[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      lse[x] = nlse[x];
+      dd[x] = ndd[x];
+      gt[x] = ngt[x];
+    }
+    if (i + 1 < n_tok) load_rows(i + 1);
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (i / kBkStages) & 1, abort_flag, a.status, 624));
     if (ok) {
       const int t = tok_of(i);
-      const int br = CMP ? 0 : (i < w_n ? 2 : 1);   // gate / lse slot: 0 cmp, 1 slc, 2 win
+      const int br = CMP ? 0 : (is_win(i) ? 2 : 1);
       const uint32_t qst = smem_u32(ring + st * S::STAGE), dst = qst + S::QST;
-      // per query row of this lane: rows cq, cq+1, cq+8, cq+9
-      float lse[4], dd[4], gt[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int qr = cq + (x & 1) + 8 * (x >> 1);
-        if (qr < G) {
-          const size_t o = ((size_t)(tok0 + t) * a.H_q + g * G + qr) * 3 + br;
-          lse[x] = a.lse[o];
-          dd[x] = a.dd[o];
-          gt[x] = a.gates[o];
-        } else {
-          lse[x] = kNoKeys;
-          dd[x] = 0.f;
-          gt[x] = 0.f;
-        }
-      }
       float s[2][4], dp[2][4];
       warp_qk_sq<DK, 2>(kb_s, 8192, warp * 16, qst, s, lane);     // S^T = K Q^T
       warp_qk_sq<DV, 2>(vb_s, 8192, warp * 16, dst, dp, lane);    // dP^T = V dout^T
@@ -540,23 +560,13 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_keys_kernel(const BackwardA
     float* dvp = (CMP ? a.dvc : a.dv) + ((size_t)((CMP ? cmp0 : tok0) + key) * a.H_kv + g) * DV;
 #pragma unroll
     for (int i = 0; i < DK / 8; ++i) {
-      const float x0 = a.scale * dk[i][2 * hr], x1 = a.scale * dk[i][2 * hr + 1];
-      if (CMP) {
-        atomicAdd(dkp + i * 8 + cq, x0);
-        atomicAdd(dkp + i * 8 + cq + 1, x1);
-      } else {
-        *reinterpret_cast<float2*>(dkp + i * 8 + cq) = make_float2(x0, x1);
-      }
+      atomicAdd(dkp + i * 8 + cq, a.scale * dk[i][2 * hr]);
+      atomicAdd(dkp + i * 8 + cq + 1, a.scale * dk[i][2 * hr + 1]);
     }
 #pragma unroll
     for (int i = 0; i < DV / 8; ++i) {
-      const float x0 = dv[i][2 * hr], x1 = dv[i][2 * hr + 1];
-      if (CMP) {
-        atomicAdd(dvp + i * 8 + cq, x0);
-        atomicAdd(dvp + i * 8 + cq + 1, x1);
-      } else {
-        *reinterpret_cast<float2*>(dvp + i * 8 + cq) = make_float2(x0, x1);
-      }
+      atomicAdd(dvp + i * 8 + cq, dv[i][2 * hr]);
+      atomicAdd(dvp + i * 8 + cq + 1, dv[i][2 * hr + 1]);
     }
   }
 }
@@ -772,7 +782,7 @@ size_t backward_query_smem(int d_k, int d_v, int nb) {
 
 template <int DK, int DV>
 static cudaError_t launch_bwd_t(const BackwardArgs& a, const BackwardMaps& m, int q_tiles, int raw_blocks,
-                                int cmp_tiles, int cmp_z, cudaStream_t st) {
+                                int raw_z, int cmp_tiles, int cmp_z, cudaStream_t st) {
   cudaError_t e;
   const size_t sq = backward_query_smem(DK, DV, a.nb_stride);
   auto kq = bwd_query_kernel<DK, DV>;
@@ -784,20 +794,20 @@ static cudaError_t launch_bwd_t(const BackwardArgs& a, const BackwardMaps& m, in
   auto kc = bwd_keys_kernel<DK, DV, true>;
   if ((e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, SK::TOTAL)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, SK::TOTAL)) != cudaSuccess) return e;
-  if (raw_blocks > 0) kr<<<dim3(raw_blocks, a.H_kv, 1), kBkThreads, SK::TOTAL, st>>>(a, m);
+  if (raw_blocks > 0) kr<<<dim3(raw_blocks, a.H_kv, raw_z), kBkThreads, SK::TOTAL, st>>>(a, m);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (cmp_tiles > 0) kc<<<dim3(cmp_tiles, a.H_kv, cmp_z), kBkThreads, SK::TOTAL, st>>>(a, m);
   return cudaGetLastError();
 }
 
 cudaError_t launch_backward_attn(const BackwardArgs& a, const BackwardMaps& m, int q_tiles, int raw_blocks,
-                                 int cmp_tiles, int cmp_z, cudaStream_t st) {
-  if (a.d_k == 192 && a.d_v == 128) return launch_bwd_t<192, 128>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
-  if (a.d_k == 64 && a.d_v == 64) return launch_bwd_t<64, 64>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
-  if (a.d_k == 128 && a.d_v == 128) return launch_bwd_t<128, 128>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
-  if (a.d_k == 192 && a.d_v == 64) return launch_bwd_t<192, 64>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
-  if (a.d_k == 64 && a.d_v == 128) return launch_bwd_t<64, 128>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
-  if (a.d_k == 128 && a.d_v == 64) return launch_bwd_t<128, 64>(a, m, q_tiles, raw_blocks, cmp_tiles, cmp_z, st);
+                                 int raw_z, int cmp_tiles, int cmp_z, cudaStream_t st) {
+  if (a.d_k == 192 && a.d_v == 128) return launch_bwd_t<192, 128>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
+  if (a.d_k == 64 && a.d_v == 64) return launch_bwd_t<64, 64>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
+  if (a.d_k == 128 && a.d_v == 128) return launch_bwd_t<128, 128>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
+  if (a.d_k == 192 && a.d_v == 64) return launch_bwd_t<192, 64>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
+  if (a.d_k == 64 && a.d_v == 128) return launch_bwd_t<64, 128>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
+  if (a.d_k == 128 && a.d_v == 64) return launch_bwd_t<128, 64>(a, m, q_tiles, raw_blocks, raw_z, cmp_tiles, cmp_z, st);
   return cudaErrorInvalidValue;
 }
 

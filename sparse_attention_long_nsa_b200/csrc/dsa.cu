@@ -13,12 +13,14 @@
 // has one per sequence (t = len - 1), prefill one per token. Three kernels:
 //   dsa_index  CTA = one query x 4096 keys: the indexer on warp-level FP8 MMA
 //              (m16n8k32, e4m3 x e4m3 -> fp32): 16 rows = indexer heads, 8 keys
-//              per MMA column block; ReLU, weights and the head sum in registers
+//              per MMA column block; ReLU, weights and the head sum in registers;
+//              128-key tiles through a 3-stage cp.async ring
 //   dsa_topk   CTA = one query: radix select of the top_k-th score over the
-//              order-preserving bit pattern (12 + 12 + 8 bits, warp-aggregated
-//              shared-memory histograms), then one pass in token order that keeps
-//              every larger score and the first equal ones (ties to the lower
-//              index); the kept tokens come out ascending
+//              order-preserving bit pattern (four 8-bit digits, warp-private
+//              histograms with lanes of equal digits merged, float4 loads), then
+//              one pass in token order that keeps every larger score and the
+//              first equal ones (ties to the lower index); the kept tokens come
+//              out ascending
 //   dsa_attn   CTA = one query x one KV group: 8 warps take 256 kept tokens each,
 //              gather their K/V rows with 16-byte cp.async into swizzled tiles of
 //              16 keys and run an online softmax (16 rows = the group's heads);
@@ -32,7 +34,8 @@ namespace nsa {
 namespace {
 
 constexpr int kIdxChunk = 4096;     // keys per indexer CTA
-constexpr int kIdxTile = 64;        // keys per shared-memory tile
+constexpr int kIdxTile = 128;       // keys per shared-memory tile (32 per warp)
+constexpr int kIdxStages = 3;
 constexpr int kTopkThreads = 1024;
 constexpr int kAttnWarps = 8;
 constexpr int kAttnTile = 16;       // keys per gathered tile
@@ -84,7 +87,7 @@ __device__ __forceinline__ void mma_e4m3_16832(float* c, const uint32_t* av, uin
 template <int DI>
 __global__ void __launch_bounds__(128) dsa_index_kernel(const DsaArgs a) {
   constexpr int ROW = DI + 16;                 // padded smem row (bytes): conflict-free fragment loads
-  __shared__ __align__(16) uint8_t kt[2][kIdxTile * ROW];
+  extern __shared__ __align__(16) uint8_t kt[];   // [kIdxStages][kIdxTile * ROW]
   __shared__ float wsm[16];
   const int slot = blockIdx.y;
   int64_t qrow, base;
@@ -110,31 +113,32 @@ __global__ void __launch_bounds__(128) dsa_index_kernel(const DsaArgs a) {
       af[ks][3] = r0 + 8 < a.H_I ? *reinterpret_cast<const uint32_t*>(qi + (r0 + 8) * DI + ks * 32 + 16 + c4) : 0u;
     }
   }
-  auto load_tile = [&](int buf, int kb) {
-    constexpr int CH = DI / 16;   // 16-byte chunks per key
-    for (int i = tid; i < kIdxTile * CH; i += 128) {
-      const int r = i / CH, c = i % CH;
-      const int key = kb + r;
-      cp_async16_zfill(&kt[buf][r * ROW + c * 16], ki + (int64_t)min(key, k1 - 1) * DI + c * 16, key < k1);
+  const int n_tiles = (k1 - k0 + kIdxTile - 1) / kIdxTile;
+  auto load_tile = [&](int it) {   // one commit group per tile (empty past the end)
+    if (it < n_tiles) {
+      constexpr int CH = DI / 16;   // 16-byte chunks per key
+      uint8_t* dst = kt + (it % kIdxStages) * (kIdxTile * ROW);
+      const int kb = k0 + it * kIdxTile;
+      for (int i = tid; i < kIdxTile * CH; i += 128) {
+        const int r = i / CH, c = i % CH;
+        const int key = kb + r;
+        cp_async16_zfill(dst + r * ROW + c * 16, ki + (int64_t)min(key, k1 - 1) * DI + c * 16, key < k1);
+      }
     }
     cp_async_commit();
   };
-  const int n_tiles = (k1 - k0 + kIdxTile - 1) / kIdxTile;
-  load_tile(0, k0);
+  for (int it = 0; it < kIdxStages - 1; ++it) load_tile(it);
   __syncthreads();
   const float w0 = wsm[lane >> 2], w1 = wsm[(lane >> 2) + 8];
+  float* dst = a.scores + (int64_t)slot * a.ld_scores;
   for (int it = 0; it < n_tiles; ++it) {
-    if (it + 1 < n_tiles) {
-      load_tile((it + 1) & 1, k0 + (it + 1) * kIdxTile);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    load_tile(it + kIdxStages - 1);
+    cp_async_wait<kIdxStages - 1>();
     __syncthreads();
-    const uint8_t* tb = kt[it & 1];
+    const uint8_t* tb = kt + (it % kIdxStages) * (kIdxTile * ROW);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {   // this warp's 16 keys: two blocks of 8
-      const int kr = warp * 16 + nt * 8 + (lane >> 2);   // B column (key) of this lane
+    for (int nt = 0; nt < 4; ++nt) {   // this warp's 32 keys: four blocks of 8
+      const int kr = warp * 32 + nt * 8 + (lane >> 2);   // B column (key) of this lane
       float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ks = 0; ks < DI / 32; ++ks) {
@@ -151,23 +155,51 @@ __global__ void __launch_bounds__(128) dsa_index_kernel(const DsaArgs a) {
         s1 += __shfl_xor_sync(0xffffffffu, s1, off);
       }
       if (lane < 4) {
-        const int key = k0 + it * kIdxTile + warp * 16 + nt * 8 + lane * 2;
-        float* dst = a.scores + (int64_t)slot * a.ld_scores;
+        const int key = k0 + it * kIdxTile + warp * 32 + nt * 8 + lane * 2;
         if (key < k1) dst[key] = s0;
         if (key + 1 < k1) dst[key + 1] = s1;
       }
     }
-    __syncthreads();
+    __syncthreads();   // the stage is reloaded kIdxStages - 1 tiles later
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
 // top-k over one query's scores
 // ---------------------------------------------------------------------------
+// exclusive prefix of `v` over the CTA's threads in index order (32 warps);
+// `total` gets the CTA-wide sum. Uses wsum[32]; synchronises the CTA twice.
+__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* wsum, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += o;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = wsum[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    wsum[lane] = w;   // inclusive prefix over warps
+  }
+  __syncthreads();
+  total = wsum[31];
+  const uint32_t before = warp > 0 ? wsum[warp - 1] : 0u;
+  return before + x - v;
+}
+
 __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const DsaArgs a) {
-  __shared__ uint32_t hist[4096];
-  __shared__ uint32_t wsum[32];
-  __shared__ uint32_t sh[4];
+  __shared__ uint32_t whist[32][256];   // one histogram per warp: no contention between warps
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t wsum[2][32];       // one buffer per scan of a chunk (a warp may still read the other)
+  __shared__ uint32_t sel_bin[2];
   const int slot = blockIdx.x;
   int64_t qrow, base;
   int t;
@@ -180,69 +212,84 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const DsaArgs a)
     for (int i = tid; i < K; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
-  // radix select of the K-th largest key: bits [31:20], [19:8], [7:0]
+  // radix select of the K-th largest order key, 8 bits per pass from the top
   uint32_t prefix = 0u, pmask = 0u;
-  int need = K;   // how many of the elements matching the prefix are still to be taken from the top
-  const int shifts[3] = {20, 8, 0};
-  const int widths[3] = {12, 12, 8};
-  for (int p = 0; p < 3; ++p) {
-    const int sh_ = shifts[p], nb = 1 << widths[p];
-    for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0u;
-    __syncthreads();
-    for (int i0 = 0; i0 < n; i0 += kTopkThreads) {   // warp-uniform trip count (the ballots need every lane)
-      const int i = i0 + tid;
-      const uint32_t u = i < n ? ord_key(sc[i]) : 0u;
-      const bool m = i < n && (u & pmask) == prefix;
-      const uint32_t bin = (u >> sh_) & (uint32_t)(nb - 1);
+  uint32_t need = (uint32_t)K;   // elements still to take among those matching the prefix
+  const bool vec = (reinterpret_cast<uintptr_t>(sc) & 15u) == 0;
+  for (int sh_ = 24; sh_ >= 0; sh_ -= 8) {
+    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+    __syncwarp();
+    auto add = [&](float f, bool valid) {
+      const uint32_t u = ord_key(f);
+      const bool m = valid && (u & pmask) == prefix;
+      const uint32_t bin = (u >> sh_) & 255u;
       const uint32_t act = __ballot_sync(0xffffffffu, m);
       if (m) {   // lanes with the same bin add once
         const uint32_t peers = __match_any_sync(act, bin);
-        if ((uint32_t)lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+        if ((uint32_t)lane == (uint32_t)(__ffs(peers) - 1)) whist[warp][bin] += __popc(peers);
       }
-    }
-    __syncthreads();
-    // counts above each thread's bin range (bins taken from the top): each thread
-    // owns nb / 1024 consecutive bins (at least one)
-    const int per = nb >= kTopkThreads ? nb / kTopkThreads : 1;
-    const int lo = tid * per;
-    uint32_t mine = 0u;
-    if (lo < nb)
-      for (int i = 0; i < per; ++i) mine += hist[lo + i];
-    // suffix sum over threads (higher bins first): inclusive scan in reverse thread order
-    uint32_t v = mine;
-    // warp-level inclusive suffix scan (lane and the lanes above it)
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_down_sync(0xffffffffu, v, off);
-      if (lane + off < 32) v += o;
-    }
-    if (lane == 0) wsum[warp] = v;   // warp total (lane 0 holds the sum over the whole warp)
-    __syncthreads();
-    uint32_t above_warps = 0u;
-    for (int w2 = warp + 1; w2 < 32; ++w2) above_warps += wsum[w2];
-    const uint32_t incl = v + above_warps;      // elements in bins >= lo
-    const uint32_t excl = incl - mine;          // elements in bins above this thread's range
-    if (lo < nb && excl < (uint32_t)need && incl >= (uint32_t)need) {
-      uint32_t acc = excl;
-      for (int i = per - 1; i >= 0; --i) {
-        const uint32_t h = hist[lo + i];
-        if (acc + h >= (uint32_t)need) {
-          sh[0] = (uint32_t)(lo + i);
-          sh[1] = acc;   // elements strictly above the chosen bin
-          break;
+      __syncwarp();
+    };
+    if (vec) {
+      for (int i0 = 0; i0 < n; i0 += 4 * kTopkThreads) {   // warp-uniform trip count
+        const int i = i0 + 4 * tid;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i + 3 < n) f = *reinterpret_cast<const float4*>(sc + i);
+        else {
+          if (i < n) f.x = sc[i];
+          if (i + 1 < n) f.y = sc[i + 1];
+          if (i + 2 < n) f.z = sc[i + 2];
         }
-        acc += h;
+        add(f.x, i < n);
+        add(f.y, i + 1 < n);
+        add(f.z, i + 2 < n);
+        add(f.w, i + 3 < n);
+      }
+    } else {
+      for (int i0 = 0; i0 < n; i0 += kTopkThreads) add(i0 + tid < n ? sc[i0 + tid] : 0.f, i0 + tid < n);
+    }
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t c = 0u;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) c += whist[w][tid];
+      hist[tid] = c;
+    }
+    __syncthreads();
+    if (warp == 0) {   // the bin holding the need-th largest, counting from bin 255 down
+      uint32_t loc[8], sum = 0u;   // lane owns bins 255 - 8 lane - 7 .. 255 - 8 lane
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        loc[j] = hist[255 - 8 * lane - j];
+        sum += loc[j];
+      }
+      uint32_t x = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += o;
+      }
+      uint32_t acc = x - sum;   // elements in bins above this lane's range
+      if (acc < need && x >= need) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (acc + loc[j] >= need) {
+            sel_bin[0] = 255u - 8u * lane - (uint32_t)j;
+            sel_bin[1] = acc;
+            break;
+          }
+          acc += loc[j];
+        }
       }
     }
     __syncthreads();
-    const uint32_t bsel = sh[0];
-    need -= (int)sh[1];
-    prefix |= bsel << sh_;
-    pmask |= (uint32_t)(nb - 1) << sh_;
+    prefix |= sel_bin[0] << sh_;
+    pmask |= 255u << sh_;
+    need -= sel_bin[1];
     __syncthreads();
   }
-  // prefix is the K-th largest key; keep every larger key and the first `need`
-  // equal ones in token order
+  // prefix is the K-th largest key: keep the larger keys and the first `need` equal
+  // ones in token order; positions from CTA-wide scans of each 1024-element chunk
   const uint32_t thr = prefix;
   uint32_t taken = 0u, eq_seen = 0u;
   for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
@@ -250,29 +297,15 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const DsaArgs a)
     const uint32_t u = i < n ? ord_key(sc[i]) : 0u;
     const bool gt = i < n && u > thr;
     const bool eq = i < n && u == thr;
-    // block-wide exclusive ranks of eq and of the kept flags (index order)
-    const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) wsum[warp] = __popc(eqb);
-    __syncthreads();
-    uint32_t eq_before = eq_seen;
-    for (int w2 = 0; w2 < warp; ++w2) eq_before += wsum[w2];
-    eq_before += __popc(eqb & ((1u << lane) - 1u));
-    uint32_t eq_total = 0u;
-    for (int w2 = 0; w2 < 32; ++w2) eq_total += wsum[w2];
-    __syncthreads();
-    const bool keep = gt || (eq && eq_before < (uint32_t)need);
-    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) wsum[warp] = __popc(kb);
-    __syncthreads();
-    uint32_t pos = taken;
-    for (int w2 = 0; w2 < warp; ++w2) pos += wsum[w2];
-    pos += __popc(kb & ((1u << lane) - 1u));
-    uint32_t kt = 0u;
-    for (int w2 = 0; w2 < 32; ++w2) kt += wsum[w2];
+    uint32_t eq_total;
+    const uint32_t eq_before = eq_seen + cta_excl_scan(eq ? 1u : 0u, wsum[0], eq_total);
+    const bool keep = gt || (eq && eq_before < need);
+    uint32_t k_total;
+    const uint32_t pos = taken + cta_excl_scan(keep ? 1u : 0u, wsum[1], k_total);
     if (keep && NSA_BOUNDS(pos < (uint32_t)K, a.status, 701)) out[pos] = i;
-    taken += kt;
+    taken += k_total;
     eq_seen += eq_total;
-    __syncthreads();
+    if (taken >= (uint32_t)K) break;   // CTA-uniform: every thread holds the same totals
   }
 }
 
@@ -419,13 +452,19 @@ static cudaError_t launch_attn_t(const DsaArgs& a, int n_slots, cudaStream_t st)
 cudaError_t launch_dsa(const DsaArgs& a, int n_slots, int max_keys, int d_k, int d_v, int d_i, cudaStream_t st) {
   if (n_slots <= 0) return cudaSuccess;
   const dim3 gi((max_keys + kIdxChunk - 1) / kIdxChunk, n_slots);
+  const size_t ism = (size_t)kIdxStages * kIdxTile * (d_i + 16);
+  cudaError_t e = cudaSuccess;
+  if (d_i == 64) e = cudaFuncSetAttribute(dsa_index_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
+  else if (d_i == 128) e = cudaFuncSetAttribute(dsa_index_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
+  else if (d_i == 32) e = cudaFuncSetAttribute(dsa_index_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
+  if (e != cudaSuccess) return e;
   prof_begin(P_DSA_INDEX, st);
-  if (d_i == 64) dsa_index_kernel<64><<<gi, 128, 0, st>>>(a);
-  else if (d_i == 128) dsa_index_kernel<128><<<gi, 128, 0, st>>>(a);
-  else if (d_i == 32) dsa_index_kernel<32><<<gi, 128, 0, st>>>(a);
+  if (d_i == 64) dsa_index_kernel<64><<<gi, 128, ism, st>>>(a);
+  else if (d_i == 128) dsa_index_kernel<128><<<gi, 128, ism, st>>>(a);
+  else if (d_i == 32) dsa_index_kernel<32><<<gi, 128, ism, st>>>(a);
   else return cudaErrorInvalidValue;
   prof_end(P_DSA_INDEX, st, 1);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prof_begin(P_DSA_TOPK, st);
   dsa_topk_kernel<<<n_slots, kTopkThreads, 0, st>>>(a);

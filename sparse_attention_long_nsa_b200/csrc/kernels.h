@@ -139,7 +139,7 @@ struct BackwardArgs {
   const float* gates;     // fp32 [N, H_q, 3]
   const int32_t* sel;     // int32 [N, H_kv, top_n] (the forward's selection)
   float* dq;              // fp32 [N, H_q, d_k]
-  float* dk;              // fp32 [N, H_kv, d_k] (raw branches; the compression's share is added after)
+  float* dk;              // fp32 [N, H_kv, d_k] (zeroed; raw branches add into it, then the compression's share)
   float* dv;              // fp32 [N, H_kv, d_v]
   float* dkc;             // fp32 [Nc, H_kv, d_k] (zeroed; compressed-key pass adds into it)
   float* dvc;             // fp32 [Nc, H_kv, d_v]
@@ -151,7 +151,7 @@ struct BackwardArgs {
   int H_q, H_kv, G, d_k, d_v;
   int l, s, ls, top_n, window;
   int nb_stride;          // selection blocks of the longest sequence
-  int tok_chunk;          // compressed-key pass: query tokens per CTA (grid.z splits)
+  int tok_chunk;          // key passes: query tokens per CTA (grid.z splits)
   float scale, scale_log2;
   uint32_t* status;
   SeqTable seqs;                        // tile_prefix: query tiles of 8 tokens
@@ -165,7 +165,7 @@ struct BackwardMaps {
 };
 size_t backward_query_smem(int d_k, int d_v, int nb);
 cudaError_t launch_backward_attn(const BackwardArgs& a, const BackwardMaps& m, int q_tiles, int raw_blocks,
-                                 int cmp_tiles, int cmp_z, cudaStream_t st);
+                                 int raw_z, int cmp_tiles, int cmp_z, cudaStream_t st);
 cudaError_t launch_inverted_index(const BackwardArgs& a, int64_t n_ent, int n_lists, int32_t* cnt, int32_t* off,
                                   int32_t* cur, int32_t* slot, int32_t* tok, cudaStream_t st);
 cudaError_t launch_compress_backward(const float* dc, const void* x, const float* W, const float* pe, int d_in,

@@ -789,7 +789,7 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
   a.l = params->l_cmp; a.s = params->stride; a.ls = params->l_sel; a.top_n = params->top_n;
   a.window = params->window;
   a.nb_stride = nb;
-  a.tok_chunk = 2048;
+  a.tok_chunk = 256;
   a.scale = softmax_scale(params, heads->d_k);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws);
@@ -818,7 +818,10 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
   a.cblk_prefix[batch] = ctile;
   ncmp_prefix[batch] = (int32_t)coff;
   a.seqs = t;
+  // grid.z of the key passes: the longest token sequence of a block (raw: the
+  // window range plus every token of the sequence, as block 0 is chosen by all)
   const int cmp_z = (max_len + a.tok_chunk - 1) / a.tok_chunk;
+  const int raw_z = (max_len + 64 + params->window + a.tok_chunk - 1) / a.tok_chunk;
 
   BackwardMaps m;
   memset(&m, 0, sizeof(m));
@@ -839,7 +842,9 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed");
     return NSA_ERR_CUDA;
   }
-  cudaError_t e = cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(dk, 0, (size_t)N * heads->H_kv * heads->d_k * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, (size_t)N * heads->H_kv * heads->d_v * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward memset");
   if (ncmp > 0) {
     e = cudaMemsetAsync(ws + w.dkc, 0, (size_t)ncmp * heads->H_kv * heads->d_k * 4, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ws + w.dvc, 0, (size_t)ncmp * heads->H_kv * heads->d_v * 4, st);
@@ -851,11 +856,11 @@ nsa_status_t nsa_prefill_backward(const void* q, const void* k, const void* v, c
   prof_end(P_BWD_INDEX, st, 3);
   if (e != cudaSuccess) return cuda_fail(e, "backward index");
   prof_begin(P_BWD_QUERY, st);
-  e = launch_backward_attn(a, m, q_tiles, 0, 0, 0, st);
+  e = launch_backward_attn(a, m, q_tiles, 0, 0, 0, 0, st);
   prof_end(P_BWD_QUERY, st, 1);
   if (e != cudaSuccess) return cuda_fail(e, "backward query pass");
   prof_begin(P_BWD_KEYS, st);
-  e = launch_backward_attn(a, m, 0, raw, ctile, cmp_z, st);
+  e = launch_backward_attn(a, m, 0, raw, raw_z, ctile, cmp_z, st);
   prof_end(P_BWD_KEYS, st, ctile > 0 ? 2 : 1);
   if (e != cudaSuccess) return cuda_fail(e, "backward key passes");
   prof_begin(P_BWD_COMPRESS, st);
