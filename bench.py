@@ -51,6 +51,11 @@ L2_FLUSH_BYTES = 256 << 20
 # processed when the traffic grows in proportion: the 64K decode capture ran 8 of
 # the 32 sequences (the compressed stream is per sequence).
 NCU_TRAFFIC = {
+    # 64K prefill: captured on the same kernel with one KV group (H_q=16, H_kv=1,
+    # bench.py --case prefill64k_g1); the CTAs of different KV groups touch disjoint
+    # rows of q, k, v, out and the importance rows, so a launch's traffic is 4x
+    ("prefill_attn", "prefill_64k"): dict(bytes=(468.813568e6 + 393.771520e6) * 4, src="prefill.cu",
+                                          sha1="56daa6c2426ce88eb7504c70e3129703afa180fa"),
     ("prefill_attn", "prefill_8k"): dict(bytes=232.535808e6 + 102.639360e6, src="prefill.cu",
                                          sha1="fe74b5e0732b48a3b4ff97b468fa0b9e4100689f"),
     ("dec_cmp", "decode_64k"): dict(bytes=(84.101376e6 + 2.978816e6) * 32 / 8, src="decode.cu",
