@@ -13,13 +13,15 @@
 //       blocks it touches. A dedicated warp merges the consumer warps' states
 //       while they go on with the next item.
 //   D2  (prologue of the D3 CTA of each (sequence, KV head), after waiting for
-//       D1 through programmatic dependent launch): merge the chunks, normalise,
-//       finish g_cmp * o_cmp, reduce the block sums over the group's heads into
-//       the importance, run the top-n selection over the CTA's warps.
+//       D1 through programmatic dependent launch): merge the chunks' softmax
+//       states, reduce the block sums over the group's heads into the
+//       importance, run the top-n selection over the CTA's warps.
 //   D3  dec_fine streams the union of the selected blocks and the window blocks
 //       once (the window is prefetched into L2 while D2 runs); four warps run
 //       the selected branch and four the window branch, each with its own
-//       softmax; it writes out = g_cmp o_cmp + g_slc o_slc + g_win o_win.
+//       softmax; the combine forms g_cmp o_cmp from the chunk outputs (L2) with
+//       the merge factors of D2 and writes out = g_cmp o_cmp + g_slc o_slc +
+//       g_win o_win.
 #include "common.cuh"
 #include "kernels.h"
 #include "topn.cuh"
@@ -36,7 +38,7 @@ constexpr int kNT = kTileKeys / 8;     // 8-key MMA n-tiles per tile
 constexpr int kDecStages = 8;
 constexpr int kDecBranchWarps = 4;                      // consumer warps per branch (selected, window)
 constexpr int kDecConsumers = 2 * kDecBranchWarps;
-constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+constexpr int kDecThreads = (kDecConsumers + 1) * 32;   // consumers, producer
 // compressed-key pass: consumer warps + producer warp
 constexpr int kD1Stages = 8;
 constexpr int kD1Consumers = 4;
@@ -462,42 +464,40 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
   __syncthreads();
   pdl_wait();   // the compressed pass (the previous kernel) has finished: its partials are visible
   // ---- D2 (in this CTA, before the ring is used): merge the compressed chunks of
-  // (b, g), finish g_cmp * o_cmp, form the importance, select the top-n blocks
+  // (b, g) (the factors are kept for the combine step), form the importance,
+  // select the top-n blocks
   {
     const PartLayout pl = part_layout(a);
     const int nc = n_cmp_dev(L, a.l, a.s);
     const int nch = (nc + kCmpChunk - 1) / kCmpChunk;   // <= 32 (checked on the host)
     const int ntl = (nc + kTileKeys - 1) / kTileKeys;
     float* Mh = reinterpret_cast<float*>(ring);   // [16] max per head
-    float* Li = Mh + 16;                          // [16] 1 / denominator
-    float* Fc = Mh + 32;                          // [nch][16] chunk factors
-    float* Ft = Fc + a.n_cmp_chunks * 16;         // [ntl][16] tile factors (incl. 1/L)
+    // 1 / denominator and the chunk factors outlive the prologue (the o_cmp warp
+    // reads them while the ring streams): they sit behind Q (<= 6 KB) in its area
+    float* Li = reinterpret_cast<float*>(qs + 8192);   // [16]
+    float* Fc = Li + 16;                               // [nch][16] chunk factors (<= 2 KB)
+    float* Ft = Mh + 16;                               // [ntl][16] tile factors (incl. 1/L)
     float* imp_s = Ft + pl.n_tiles * 16;          // [nb_stride]
-    const float* cpo = a.part + pl.cp_o + bg * a.n_cmp_chunks * G * DV;
     const float* cpm = a.part + pl.cp_ml + bg * a.n_cmp_chunks * G * 2;
     const float* tp = a.part + pl.tp + bg * pl.n_tiles * kTP * G;
-    // the tile partials and chunk outputs come into shared memory with two bulk
-    // copies when they fit next to the scratch (otherwise they are read in place)
-    uint32_t* ck = reinterpret_cast<uint32_t*>(imp_s + ((a.nb_stride + 3) & ~3));   // top-n scratch [5][32]
-    int* ci = reinterpret_cast<int*>(ck + 5 * 32);
-    float* tp_s = reinterpret_cast<float*>(ci + 5 * 32);
+    // the tile partials come into shared memory with bulk copies when they fit
+    // next to the scratch (otherwise they are read in place)
+    constexpr int kTopnWarps = 8;   // slices of the CTA-wide top-n
+    uint32_t* ck = reinterpret_cast<uint32_t*>(imp_s + ((a.nb_stride + 3) & ~3));   // top-n scratch [8][32]
+    int* ci = reinterpret_cast<int*>(ck + kTopnWarps * 32);
+    float* tp_s = reinterpret_cast<float*>(ci + kTopnWarps * 32);
     const uint32_t tp_bytes = (uint32_t)(((size_t)ntl * kTP * G * 4 + 15) & ~size_t(15));
-    float* cpo_s = tp_s + tp_bytes / 4;
-    const uint32_t cpo_bytes = (uint32_t)((size_t)nch * G * DV * 4);
-    const bool bulk = (size_t)((uint8_t*)cpo_s - ring) + cpo_bytes <= (size_t)S::BODY && nc > 0;
+    const bool bulk = (size_t)((uint8_t*)tp_s - ring) + tp_bytes <= (size_t)S::BODY && nc > 0;
     if (bulk) {
-      if (warp == 0) {   // 16 KB pieces from several lanes keep more copies in flight
-        if (lane == 0) mbar_arrive_expect_tx(d2bar, tp_bytes + cpo_bytes);
+      if (warp == 0) {   // 8 KB pieces from several lanes keep more copies in flight
+        if (lane == 0) mbar_arrive_expect_tx(d2bar, tp_bytes);
         __syncwarp();
-        constexpr uint32_t kPiece = 16384;
-        const uint32_t ntp = (tp_bytes + kPiece - 1) / kPiece, ncp = (cpo_bytes + kPiece - 1) / kPiece;
-        for (uint32_t i = lane; i < ntp + ncp; i += 32) {
-          const bool is_tp = i < ntp;
-          const uint32_t off = (is_tp ? i : i - ntp) * kPiece;
-          const uint32_t tot = is_tp ? tp_bytes : cpo_bytes;
-          const uint32_t n = min(kPiece, tot - off);
-          if (is_tp) bulk_load(reinterpret_cast<uint8_t*>(tp_s) + off, reinterpret_cast<const uint8_t*>(tp) + off, n, d2bar);
-          else bulk_load(reinterpret_cast<uint8_t*>(cpo_s) + off, reinterpret_cast<const uint8_t*>(cpo) + off, n, d2bar);
+        constexpr uint32_t kPiece = 8192;
+        const uint32_t ntp = (tp_bytes + kPiece - 1) / kPiece;
+        for (uint32_t i = lane; i < ntp; i += 32) {
+          const uint32_t off = i * kPiece;
+          const uint32_t n = min(kPiece, tp_bytes - off);
+          bulk_load(reinterpret_cast<uint8_t*>(tp_s) + off, reinterpret_cast<const uint8_t*>(tp) + off, n, d2bar);
         }
       }
       const bool got = mbar_wait(d2bar, 0, abort_flag, a.status, 410);
@@ -506,7 +506,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
         return;
       }
       tp = tp_s;
-      cpo = cpo_s;
     }
     TRD(1);
     // one warp per head, the chunks in its lanes
@@ -535,21 +534,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       const int tj = idx / G, h = idx % G;
       Ft[tj * 16 + h] = exp2f(tp[(size_t)tj * kTP * G + h] - Mh[h]) * Li[h];
     }
-    // g_cmp * o_cmp, 4 values per thread
-    for (int idx = tid; idx < G * (DV / 4); idx += kDecThreads) {
-      const int h = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int c = 0; c < nch; ++c) {
-        const float fc = Fc[c * 16 + h];
-        const float4 v = *reinterpret_cast<const float4*>(cpo + ((size_t)c * G + h) * DV + c4);
-        acc.x += fc * v.x; acc.y += fc * v.y; acc.z += fc * v.z; acc.w += fc * v.w;
-      }
-      const int hq = g * G + h;
-      const float sc = a.gates[((size_t)b * a.H_q + hq) * 3 + 0] * Li[h];
-      *reinterpret_cast<float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4) =
-          make_float4(sc * acc.x, sc * acc.y, sc * acc.z, sc * acc.w);
-    }
+    // (g_cmp * o_cmp is formed in the combine step, from the chunk outputs in L2)
     __syncthreads();
     TRD(3);
     // importance of blocks 0..jt: tile tj holds blocks kBlkPerTile*tj .. + kBlkPerTile
@@ -579,7 +564,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
     }
     __syncthreads();
     TRD(4);
-    constexpr int kTopnWarps = 5;   // the top-n scratch holds five warps' candidates
     if (!cta_topn(imp_s, jt, a.top_n, a.force_first, a.force_local, a.sel + bg * a.top_n, ck, ci, kTopnWarps,
                   warp, lane) &&
         warp == 0)
@@ -737,16 +721,48 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_fine_kernel(const DecodeAr
       if (lane == 0) mbar_arrive(&empty[st]);
     }
     rs.finish();
+    // g_cmp * o_cmp of this thread's (row, 4 columns) items of the combine, from the
+    // chunk outputs (L2) and the merge factors kept behind Q: formed before the
+    // barrier, so their loads overlap the warps that are still streaming
+    constexpr int kItems = 2;   // G * DV / 4 <= 512 items over 256 threads
+    float4 ocm[kItems];
+    {
+      const PartLayout pl = part_layout(a);
+      const int nch = (n_cmp_dev(L, a.l, a.s) + kCmpChunk - 1) / kCmpChunk;
+      const float* cpo = a.part + pl.cp_o + bg * a.n_cmp_chunks * G * DV;
+      const float* Li = reinterpret_cast<const float*>(qs + 8192);
+      const float* Fc = Li + 16;
+#pragma unroll
+      for (int it = 0; it < kItems; ++it) {
+        const int idx = tid + it * kDecConsumers * 32;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < G * (DV / 4)) {
+          const int row = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
+#pragma unroll 8
+          for (int c = 0; c < nch; ++c) {   // independent L2 loads, issued together
+            const float fc = Fc[c * 16 + row];
+            const float4 v = *reinterpret_cast<const float4*>(cpo + ((size_t)c * G + row) * DV + c4);
+            acc.x += fc * v.x; acc.y += fc * v.y; acc.z += fc * v.z; acc.w += fc * v.w;
+          }
+          const float scg = a.gates[((size_t)b * a.H_q + g * G + row) * 3 + 0] * Li[row];
+          acc = make_float4(scg * acc.x, scg * acc.y, scg * acc.z, scg * acc.w);
+        }
+        ocm[it] = acc;
+      }
+    }
     named_bar_sync(1, kDecConsumers * 32);   // every block consumed: the ring is free
     TRD(7);
     float* stg = reinterpret_cast<float*>(ring);
     rs.stage(stg + warp * 16 * (DV + 2), lane);   // [branch][warp of branch][16][DV + 2]
     named_bar_sync(1, kDecConsumers * 32);
     // merge the four warps of each branch and combine: thread per (row, 4 columns)
-    for (int idx = tid; idx < G * (DV / 4); idx += kDecConsumers * 32) {
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int idx = tid + it * kDecConsumers * 32;
+      if (idx >= G * (DV / 4)) break;
       const int row = idx / (DV / 4), c4 = (idx % (DV / 4)) * 4;
       const int hq = g * G + row;
-      float4 res = *reinterpret_cast<const float4*>(a.ocmp + ((size_t)b * a.H_q + hq) * DV + c4);
+      float4 res = ocm[it];
 #pragma unroll
       for (int br = 0; br < 2; ++br) {
         const float* base = stg + (size_t)br * kDecBranchWarps * 16 * (DV + 2);
