@@ -458,9 +458,10 @@ def backward_work(cfg):
     return attn + comp
 
 
-def bench_backward(cfg, args, rank, ws, dev, pk):
-    """One step = nsa_prefill_backward of one sequence (the forward's compressed
-    keys and selection computed once before)."""
+def _backward_setup(cfg, dev, rank):
+    """Inputs, the forward's compressed keys and selection, gradient buffers and
+    a workspace for one nsa_prefill_backward of one sequence; returns the step
+    closure and the workspace."""
     import sparse_attention_long_nsa_b200 as nsa
     heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
     par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
@@ -476,13 +477,22 @@ def bench_backward(cfg, args, rank, ws, dev, pk):
     g = {n: torch.empty(tuple(x.shape), dtype=torch.float32, device=dev) for n, x in
          (("dq", inp["q"]), ("dk", inp["k"]), ("dv", inp["v"]), ("dgates", inp["gates"]), ("dw_ck", inp["w_ck"]),
           ("dpe_k", inp["pe_k"]), ("dw_cv", inp["w_cv"]), ("dpe_v", inp["pe_v"]))}
-    flush = _make_flush(dev)
 
     def step():
         nsa.nsa_prefill_backward(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], dout, sel, inp["w_ck"],
                                  inp["pe_k"], inp["w_cv"], inp["pe_v"], cu, heads, par, g["dq"], g["dk"], g["dv"],
                                  g["dgates"], g["dw_ck"], g["dpe_k"], g["dw_cv"], g["dpe_v"], ws_b)
 
+    return step, ws_b
+
+
+def bench_backward(cfg, args, rank, ws, dev, pk):
+    """One step = nsa_prefill_backward of one sequence (the forward's compressed
+    keys and selection computed once before)."""
+    import sparse_attention_long_nsa_b200 as nsa
+    T = cfg.T
+    step, ws_b = _backward_setup(cfg, dev, rank)
+    flush = _make_flush(dev)
     step()
     torch.cuda.synchronize()
     nsa.nsa_check_device_status(ws_b)
@@ -786,7 +796,9 @@ def _decode_case(cfg, dev, lens=None):
 #                  DRAM-traffic capture that stays a few GB on the device
 #   decode         8 sequences of the 64K decode workload
 #   decode_varlen  the varlen decode batch
-CASES = ("prefill", "prefill64k_g1", "decode", "decode_varlen")
+#   backward       the backward of a 2048-token sequence with the 8K heads
+#   dsa_decode     8 sequences of the 64K DSA decode workload
+CASES = ("prefill", "prefill64k_g1", "decode", "decode_varlen", "backward", "dsa_decode")
 
 
 def run_case(case):
@@ -798,8 +810,24 @@ def run_case(case):
         _prefill_case(dataclasses.replace(PREFILL, name="prefill_64k_g1", H_q=16, H_kv=1), dev)
     elif case == "decode":
         _decode_case(DECODE, dev, lens=[DECODE.T] * 8)
-    else:
+    elif case == "decode_varlen":
         _decode_case(DECODE_VARLEN, dev)
+    elif case == "backward":
+        step, _ = _backward_setup(dataclasses.replace(PREFILL_8K, T=2048), dev, 0)
+        for _ in range(2):
+            step()
+    else:
+        import sparse_attention_long_nsa_b200 as nsa
+        cfg = W.DSA_CONFIGS["dsa_decode_64k"]
+        inp = W.make_dsa_decode_inputs(cfg, device=dev, lens=[cfg.T] * 8)
+        heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
+        dp = nsa.DsaParams(cfg.H_I, cfg.d_I, cfg.top_k, 0.0)
+        out = torch.empty((8, cfg.H_q, cfg.d_v), dtype=torch.bfloat16, device=dev)
+        ws = nsa.alloc_workspace(nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, heads, dp, 8, 0, cfg.T), dev)
+        lens = inp["cache_lens"].to(dev)
+        for _ in range(2):
+            nsa.nsa_dsa_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["qi"], inp["wi"], inp["ki_cache"], lens,
+                               cfg.T, dp, heads, out, None, None, ws)
     torch.cuda.synchronize()
 
 

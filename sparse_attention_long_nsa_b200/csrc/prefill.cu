@@ -27,10 +27,11 @@
 // Every tile is 64 keys. Q sits in shared memory (A operand of S = Q.K^T); S has
 // four buffers in tensor memory and the softmax writes its bf16 P over the S
 // columns it has read (A operand of O += P.V). K and V stream through TMA rings.
-// Roles (384 threads): warps 0-7 softmax: warp w owns the 32 rows of tensor-
-// memory lane quarter w % 4 and key columns 32 (w / 4) .. + 31 of every tile; the
-// two warps of a quarter trade their partial row maxima once per tile, so both
-// hold the same reference max. Warp 8 loads Q and the K tiles, warp 11 the V
+// Roles (384 threads): warps 0-7 softmax: warp w owns 16 rows, tensor-memory
+// lanes 32 (w % 4) + 16 (w / 4) .. + 15, and all 64 keys of every tile; its two
+// half-warps hold keys 0-31 and 32-63 of the same rows and trade row maxima and
+// sums by shuffles. With G = 16 a warp's rows are one token, so a selected block
+// that token did not pick costs the warp nothing. Warp 8 loads Q and the K tiles, warp 11 the V
 // tiles (separate rings: a K tile is released as soon as its S is computed);
 // warp 9 issues the S = Q.K^T products (tiles in pairs, up to four tiles ahead
 // of the softmax); warp 10 the O += P.V products. Every wait is time-bounded; on
@@ -61,8 +62,6 @@ struct FBars {
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];   // K ring: released once S = Q.K^T is computed
   uint64_t v_full[kMaxStages], v_empty[kMaxStages];   // V ring: released once O += P.V is computed
   uint64_t q_full, s_full[kSBuf], s_free[kSBuf], p_full[kSBuf], pv_done[kSBuf], ob_free, sel_ready, drain, smx;
-  uint64_t xbar[4];      // end-of-phase exchange between the two warps of a row quarter
-  uint64_t pbar[4];      // per-tile max exchange between the two warps of a row quarter
   uint32_t tmem_base;
   int abort;
   int nu;
@@ -108,17 +107,19 @@ __device__ __forceinline__ float tree_sum(const float* v) {
   return a[0];
 }
 
-// one warp scales `ncols` tensor-memory columns of its 32 rows, starting at `col`
-__device__ __noinline__ void tmem_scale_cols(uint32_t col, int ncols, float alpha) {
-  for (int c = 0; c < ncols; c += 16) {
+// one warp scales 2 * HALF tensor-memory columns of its 16 rows starting at
+// `col`: each half-warp scales HALF columns (the upper one from col + HALF)
+template <int HALF>
+__device__ __noinline__ void tmem_scale_cols(uint32_t col, float alpha) {
+  for (int c = 0; c < HALF; c += 16) {
     float ov[16];
-    tmem_ld16(col + c, ov);
+    tmem_ld16_h<HALF>(col + c, ov);
     tmem_ld_wait();
     uint32_t w[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(ov[i] * alpha);
-    tmem_st8(col + c, w);
-    tmem_st8(col + c + 8, w + 8);
+    tmem_st8_h<HALF>(col + c, w);
+    tmem_st8_h<HALF>(col + c + 8, w + 8);
   }
   tmem_st_wait();
 }
@@ -189,11 +190,11 @@ __device__ __forceinline__ float importance32(const float* h, float cin, int lan
 }  // namespace
 
 // Optional in-kernel timeline (compiled only with -DNSA_PREFILL_TRACE): lane 0
-// of every warp of a few CTAs (KV head 0, query tiles 255, 511, 767, 1023)
+// of every warp of four CTAs (KV head 0, the last query tile of each quarter of the grid)
 // records clock64() at fixed points of each tile's life; nsa_prefill_trace_read
 // copies the records out. Off in the library build.
 #ifdef NSA_PREFILL_TRACE
-constexpr int kTrTiles = 192;
+constexpr int kTrTiles = 320;
 __device__ unsigned long long g_trace[4][12][kTrTiles][4];
 __device__ unsigned long long g_trace_phase[4][12][8];
 #define TR(j, k)                                                                            \
@@ -211,12 +212,11 @@ __device__ unsigned long long g_trace_phase[4][12][8];
 #endif
 
 
-// dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | exchange [2][2][128] f32 |
-// per-tile maxima [2][2][128] f32 | block masks [nb][MW] | union [nb] | importance carries [nb/8 + 2][128/G] f32 |
+// dynamic shared memory: Q [d_k/64][128 rows][128 B] | K ring | V ring | bars | block masks [nb][MW] | union [nb] | importance carries [nb/8 + 2][128/G] f32 |
 // (when it fits) importance [128/G][nb] f32 | selections [128/G][32] i32
 __host__ __device__ inline size_t fused_fixed_bytes(int nb, int G) {
   const int tok = 128 / G, mw = (tok + 31) / 32;
-  return sizeof(FBars) + 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4 + (size_t)nb * mw * 4 + (size_t)nb * 4 +
+  return sizeof(FBars) + (size_t)nb * mw * 4 + (size_t)nb * 4 +
          (size_t)(nb / 8 + 2) * tok * 4 + 64;
 }
 
@@ -232,11 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   uint8_t* kring = smem + 128 * DK * 2;
   uint8_t* vring = kring + (size_t)nks * K_BYTES;
   FBars* bars = reinterpret_cast<FBars*>(vring + (size_t)nvs * V_BYTES);
-  float* xch = reinterpret_cast<float*>(bars + 1);                 // [slot][warpgroup][row]
-  float* pxch = xch + 512;                                         // [slot][warpgroup][row] per-tile maxima
   const int G = a.G;
   const int TOK = 128 / G, MW = (TOK + 31) / 32;
-  uint32_t* bm = reinterpret_cast<uint32_t*>(pxch + 512);          // [nb][MW] token bits per block
+  uint32_t* bm = reinterpret_cast<uint32_t*>(bars + 1);            // [nb][MW] token bits per block
   int* uni = reinterpret_cast<int*>(bm + (size_t)a.nb_stride * MW);  // union of selected blocks
   float* cbuf = reinterpret_cast<float*>(uni + a.nb_stride);      // [32-key half][token] carried mass
   float* imp_s = cbuf + (size_t)(a.nb_stride / 8 + 2) * TOK;      // [token][nb] when a.imp_smem
@@ -257,7 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
   const int nkw = (t_last - key0w) / kKeys + 1;                              // window tiles
   const int first_w = 2 * nkc, first_s = first_w + nkw;
 #ifdef NSA_PREFILL_TRACE
-  const int tr_cta = (g == 0 && (tile & 255) == 255) ? (tile >> 8) & 3 : -1;
+  const int tr_q = (int)gridDim.x / 4;
+  const int tr_cta = (g == 0 && tr_q > 0 && (tile + 1) % tr_q == 0) ? (tile + 1) / tr_q - 1 : -1;
 #endif
   TRP(0);
 
@@ -282,10 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     mbar_init(&bars->sel_ready, 1);
     mbar_init(&bars->drain, 2);   // one commit per MMA issuer
     mbar_init(&bars->smx, kSmThreads);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&bars->xbar[i], 64);
-      mbar_init(&bars->pbar[i], 64);
-    }
     bars->abort = 0;
     bars->nu = 0;
     fence_mbar_init();
@@ -499,22 +494,23 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // Warp w owns the 32 rows of tensor-memory lane quarter q4 = w % 4 and key
-    // columns 32*wg .. 32*wg + 31 (wg = w / 4) of every tile. The two warps of a
-    // quarter split each tile: they trade their partial row maxima once per tile
-    // (which also orders both warps' S reads before either writes P over the
-    // buffer), so both hold the same reference max, and each keeps the softmax
-    // denominator of its own columns until the end of the phase.
-    const int wg = warp >> 2;
-    const int q4 = warp & 3;          // row quarter = TMEM lane quarter
-    const int r = q4 * 32 + lane;     // row = TMEM lane
+    // Warp w owns the 16 rows 32 * (w % 4) + 16 * (w / 4) .. + 15 (tensor-memory
+    // lanes; a warp reaches only its own lane quarter w % 4). Lane i holds row
+    // i % 16 and key columns 32 * kh .. + 31 of every tile (kh = i / 16): the two
+    // half-warps split each tile's keys and trade row maxima and sums by
+    // shuffles; each keeps the softmax denominator of its own columns until the
+    // end of the phase. A half-warp's P store covers S columns the other half has
+    // read, and both reads finish (tcgen05.wait::ld) before either store.
+    const int kh = lane >> 4;         // key half
+    const int q4 = warp & 3;          // TMEM lane quarter
+    const int r = q4 * 32 + (warp >> 2) * 16 + (lane & 15);   // row = TMEM lane
     const int tt = r / G, hh = r % G;
     const int t = t0 + tt;
     const bool valid = t < L;
     const int64_t n = tok0 + t;
     const int hq = g * G + hh;
-    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t colh = 32u * (uint32_t)wg;   // this warp's key columns inside a tile
+    const uint32_t lane_base = (uint32_t)(r - (lane & 15)) << 16;
+    const uint32_t colh = 32u * (uint32_t)kh;   // this thread's key columns inside a tile
     const float sc = a.scale_log2;    // raw score -> log2 units
     float gc = 0.f, gsl = 0.f, gw = 0.f;
     if (valid) {
@@ -531,28 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     auto uwait = [&](uint64_t* bar, int parity, uint32_t site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)parity, abort_flag, a.status, site));
     };
-    int xcnt = 0;
-    // value of the partner warp for this row (both warps of the quarter call it in step)
-    auto exchange = [&](float mine) -> float {
-      const int slot = xcnt & 1;
-      xch[(slot * 2 + wg) * 128 + r] = mine;
-      mbar_arrive(&bars->xbar[q4]);
-      const bool w = uwait(&bars->xbar[q4], xcnt & 1, 421);
-      ++xcnt;
-      if (!w) ok = false;
-      return xch[(slot * 2 + (1 - wg)) * 128 + r];
-    };
-    // per-tile max with the partner warp (called by both warps for every online
-    // and C2 tile, whether or not they read S, so the phases stay in step)
-    int pxs = 0;
-    auto pair_max = [&](float mine) -> float {
-      const int slot = pxs & 1;
-      pxch[(slot * 2 + wg) * 128 + r] = mine;
-      mbar_arrive(&bars->pbar[q4]);
-      if (!uwait(&bars->pbar[q4], pxs & 1, 428)) ok = false;
-      ++pxs;
-      return fmaxf(mine, pxch[(slot * 2 + (1 - wg)) * 128 + r]);
-    };
+    // the other key half's value for this row
+    auto exchange = [&](float mine) -> float { return __shfl_xor_sync(0xffffffffu, mine, 16); };
+    auto pair_max = [&](float mine) -> float { return fmaxf(mine, exchange(mine)); };
     // A thread holds the 32 scores of its row and columns for the current tile.
     float sv[32];
     int cur_j = 0;
@@ -568,28 +545,28 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     };
     // raw scores of this warp's 32 keys of the current tile (two loads, one wait)
     auto ld32 = [&]() {
-      const uint32_t src = tmem + lane_base + col_s(cur_b) + colh;
-      tmem_ld16(src, sv);
-      tmem_ld16(src + 16, sv + 16);
+      const uint32_t src = tmem + lane_base + col_s(cur_b);
+      tmem_ld16_h<32>(src, sv);
+      tmem_ld16_h<32>(src + 16, sv + 16);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 32; ++c) asm volatile("" : "+f"(sv[c]));   // no use before the wait
     };
     // bf16 P (sv * scale) of keys colh .. colh + 31 into columns colh/2 .. colh/2 + 15
-    // (P of key pair (2c, 2c+1) sits in column c; both warps' S reads are done)
+    // (P of key pair (2c, 2c+1) sits in column c; the warp's S reads are done)
     auto st32 = [&](float scale) {
 #pragma unroll
       for (int c = 0; c < 16; c += 8) {
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(sv[2 * (c + i)] * scale, sv[2 * (c + i) + 1] * scale);
-        tmem_st8(tmem + lane_base + col_s(cur_b) + colh / 2 + c, pk);
+        tmem_st8_h<16>(tmem + lane_base + col_s(cur_b) + c, pk);
       }
     };
     auto st32_zero = [&]() {
       const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int c = 0; c < 16; c += 8) tmem_st8(tmem + lane_base + col_s(cur_b) + colh / 2 + c, z);
+      for (int c = 0; c < 16; c += 8) tmem_st8_h<16>(tmem + lane_base + col_s(cur_b) + c, z);
     };
     // all S reads of the tile are done (and its P written)
     auto tile_done = [&](bool with_p) {
@@ -633,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     if (nkc > 0) {   // merge the two warps' (max, sum) in a fixed order
       const float m_o = exchange(m);
       const float l_o = exchange(lp);
-      const float m0 = wg == 0 ? m : m_o, m1 = wg == 0 ? m_o : m;
-      const float l0 = wg == 0 ? lp : l_o, l1 = wg == 0 ? l_o : lp;
+      const float m0 = kh == 0 ? m : m_o, m1 = kh == 0 ? m_o : m;
+      const float l0 = kh == 0 ? lp : l_o, l1 = kh == 0 ? l_o : lp;
       const float mm = fmaxf(m0, m1);
       const float lc = l0 * ex2((m0 - mm) * sc) + l1 * ex2((m1 - mm) * sc);
       linv = lc > 0.f ? 1.f / lc : 0.f;
@@ -653,7 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const int c0 = i * kKeys + (int)colh;
       const bool part = !__all_sync(0xffffffffu, c0 + 32 <= nvis);
       if (ok) ld32();
-      pair_max(0.f);   // both warps' S reads precede the P stores
       if (part) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
@@ -663,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       if (ok) st32(gc);
       TR(j, 1);
       const bool wr = valid && ok;
-      const int B0 = 16 * i + 8 * wg;
+      const int B0 = 16 * i + 8 * kh;
       float carry;
       switch (G) {
         case 16: carry = importance32<16>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
@@ -672,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         case 2: carry = importance32<2>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
         default: carry = importance32<1>(sv, 0.f, lane, wr, imp_row, B0, jt); break;
       }
-      if (wr && hh == 0) cbuf[(2 * i + wg) * TOK + tt] = carry;
+      if (wr && hh == 0) cbuf[(2 * i + kh) * TOK + tt] = carry;
       if (ok) tile_done(true);
     }
 
@@ -764,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       m_ref = ref;
       if (__any_sync(0xffffffffu, had && alpha != 1.f)) {
         if (!wait_pv(j - 1)) return false;
-        tmem_scale_cols(tmem + lane_base + kColOB + wg * (DV / 2), DV / 2, had ? alpha : 1.f);
+        tmem_scale_cols<DV / 2>(tmem + lane_base + kColOB, had ? alpha : 1.f);
       }
       lp *= alpha;
       if (skip) {
@@ -782,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
     // denominator of the phase, both warps' columns summed in a fixed order
     auto phase_sum = [&]() -> float {
       const float other = exchange(lp);
-      return wg == 0 ? lp + other : other + lp;
+      return kh == 0 ? lp + other : other + lp;
     };
 
     // ---------------- W: window keys into O_B, then O_A += g_win / l * O_B
@@ -809,16 +785,16 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const float sw = lw > 0.f ? gw / lw : 0.f;
 #pragma unroll 1
       for (int c = 0; c < DV / 2; c += 16) {
-        const uint32_t cb = lane_base + wg * (DV / 2) + c;
+        const uint32_t cb = lane_base + c;
         float ob[16], oa[16];
-        tmem_ld16(tmem + kColOB + cb, ob);
-        if (nkc > 0) tmem_ld16(tmem + kColOA + cb, oa);
+        tmem_ld16_h<DV / 2>(tmem + kColOB + cb, ob);
+        if (nkc > 0) tmem_ld16_h<DV / 2>(tmem + kColOA + cb, oa);
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = __float_as_uint((nkc > 0 ? oa[e] : 0.f) + sw * ob[e]);
-        tmem_st8(tmem + kColOA + cb, w);
-        tmem_st8(tmem + kColOA + cb + 8, w + 8);
+        tmem_st8_h<DV / 2>(tmem + kColOA + cb, w);
+        tmem_st8_h<DV / 2>(tmem + kColOA + cb + 8, w + 8);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -850,13 +826,13 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       const float ls_ = nu > 0 ? phase_sum() : 0.f;
       if (ok && nu > 0) ok = wait_pv(first_s + nu - 1);
       const float ss = ls_ > 0.f ? gsl / ls_ : 0.f;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + hq) * DV + wg * (DV / 2);
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + ((size_t)n * a.H_q + hq) * DV + kh * (DV / 2);
 #pragma unroll 1
       for (int c = 0; c < DV / 2; c += 16) {
-        const uint32_t cb = lane_base + wg * (DV / 2) + c;
+        const uint32_t cb = lane_base + c;
         float ob[16], oa[16];
-        tmem_ld16(tmem + kColOB + cb, ob);
-        tmem_ld16(tmem + kColOA + cb, oa);
+        tmem_ld16_h<DV / 2>(tmem + kColOB + cb, ob);
+        tmem_ld16_h<DV / 2>(tmem + kColOA + cb, oa);
         tmem_ld_wait();
         if (valid && ok) {
           uint4 pk0, pk1;
@@ -935,7 +911,7 @@ extern "C" int nsa_prefill_trace_read(void* tiles, void* phases) {
   return 0;
 }
 extern "C" int nsa_prefill_trace_clear() {
-  static unsigned long long z[4 * 12 * 192 * 4];
+  static unsigned long long z[4 * 12 * nsa::kTrTiles * 4];
   if (cudaMemcpyToSymbol(nsa::g_trace, z, sizeof(nsa::g_trace)) != cudaSuccess) return 1;
   if (cudaMemcpyToSymbol(nsa::g_trace_phase, z, sizeof(nsa::g_trace_phase)) != cudaSuccess) return 1;
   return 0;

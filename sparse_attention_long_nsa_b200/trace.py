@@ -1,13 +1,14 @@
 """In-kernel timelines of the prefill and decode kernels.
 
-    python -m sparse_attention_long_nsa_b200.trace prefill   # 8K prefill
+    python -m sparse_attention_long_nsa_b200.trace prefill      # 8K prefill
+    python -m sparse_attention_long_nsa_b200.trace prefill64k   # 64K prefill, one KV group
     python -m sparse_attention_long_nsa_b200.trace decode    # 64K decode, B=32
 
 Builds a copy of libnsa.so with the compile-time trace points on
 (-DNSA_PREFILL_TRACE -DNSA_DECODE_TRACE) into _build/trace/, runs the workload a
 few times and prints a summary of the last launch:
 
-* prefill: for four CTAs (KV head 0, query tiles 255, 511, 767, 1023), the clock64
+* prefill: for four CTAs (KV head 0, the last query tile of each quarter), the clock64
   at the end of each phase (C1, C2, top-n, W, S) and, per 64-key tile, when its S
   was ready for the softmax, when the softmax finished it, and when the S and P.V
   products were issued; then the mean tile period and softmax latency of the
@@ -55,10 +56,13 @@ def build_trace_lib() -> str:
     return lib
 
 
-def _prefill(nsa, L):
+def _prefill(nsa, L, long=False):
+    import dataclasses
     import torch
     import nsa_workloads as W
     cfg = W.CONFIGS["prefill_8k"]
+    if long:
+        cfg = dataclasses.replace(W.CONFIGS["prefill_64k"], H_q=16, H_kv=1)
     inp = W.make_prefill_inputs(cfg, device="cuda")
     heads = nsa.Heads(cfg.H_q, cfg.H_kv, cfg.d_k, cfg.d_v)
     par = nsa.make_params(cfg.l_cmp, cfg.stride, cfg.l_sel, cfg.top_n, cfg.window, cfg.force_first,
@@ -68,7 +72,7 @@ def _prefill(nsa, L):
     for _ in range(4):
         nsa.prefill(inp["q"], inp["k"], inp["v"], kc, vc, inp["gates"], inp["cu_seqlens"], heads, par)
     torch.cuda.synchronize()
-    tiles = np.zeros((4, 12, 192, 4), np.uint64)
+    tiles = np.zeros((4, 12, 320, 4), np.uint64)
     ph = np.zeros((4, 12, 8), np.uint64)
     assert L.nsa_prefill_trace_read(tiles.ctypes.data_as(ctypes.c_void_p), ph.ctypes.data_as(ctypes.c_void_p)) == 0
     tiles, ph = tiles.astype(np.int64), ph.astype(np.int64)
@@ -77,16 +81,22 @@ def _prefill(nsa, L):
         if t0 == 0:
             continue
         P = [int(ph[c, 0, k] - t0) for k in range(1, 6)]
-        print(f"query tile {c * 256 + 255}: phase ends (cycles) C1 {P[0]}  C2 {P[1]}  top-n {P[2]}  W {P[3]}  "
-              f"S {P[4]}")
+        nt = cfg.T * cfg.H_q // cfg.H_kv // 128
+        print(f"query tile {(c + 1) * (nt // 4) - 1}: phase ends (cycles) C1 {P[0]}  C2 {P[1]}  top-n {P[2]}  "
+              f"W {P[3]}  S {P[4]}")
         rows = []
-        for j in range(192):
+        for j in range(320):
             sr = [tiles[c, w, j, 0] for w in range(8) if tiles[c, w, j, 0]]
             dn = [tiles[c, w, j, 3] for w in range(8) if tiles[c, w, j, 3]]
             if not sr:
                 break
             rows.append((j, min(sr) - t0, max(dn) - t0 if dn else -1, tiles[c, 9, j, 0] - t0 if tiles[c, 9, j, 0] else -1,
                          tiles[c, 10, j, 2] - t0 if tiles[c, 10, j, 2] else -1))
+        for name, lo, hi in (("C1", 0, P[0]), ("C2", P[0], P[1]), ("W", P[2], P[3])):
+            ph_t = [r for r in rows if lo <= r[1] < hi]
+            if len(ph_t) > 2:
+                print(f"  {name}: {len(ph_t)} tiles, period "
+                      f"{(ph_t[-1][1] - ph_t[0][1]) / (len(ph_t) - 1):.0f} cycles/tile")
         s_tiles = [r for r in rows if r[1] >= P[3]]
         if len(s_tiles) > 2:
             per = (s_tiles[-1][1] - s_tiles[0][1]) / (len(s_tiles) - 1)
@@ -146,7 +156,10 @@ def main():
     L.nsa_decode_trace_read.argtypes = [ctypes.c_void_p]
     L.nsa_decode_cspan_read.argtypes = [ctypes.c_void_p]
     L.nsa_decode_fspan_read.argtypes = [ctypes.c_void_p]
-    (_prefill if what == "prefill" else _decode)(nsa, L)
+    if what == "decode":
+        _decode(nsa, L)
+    else:
+        _prefill(nsa, L, long=what == "prefill64k")
 
 
 if __name__ == "__main__":
