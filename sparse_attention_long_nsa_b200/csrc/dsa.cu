@@ -16,11 +16,12 @@
 //              per MMA column block; ReLU, weights and the head sum in registers;
 //              128-key tiles through a 3-stage cp.async ring
 //   dsa_topk   CTA = one query: radix select of the top_k-th score over the
-//              order-preserving bit pattern (four 8-bit digits, warp-private
-//              histograms with lanes of equal digits merged, float4 loads), then
-//              one pass in token order that keeps every larger score and the
-//              first equal ones (ties to the lower index); the kept tokens come
-//              out ascending
+//              order-preserving bit pattern (digits of 12, 12 and 8 bits, shared-
+//              memory histograms; each warp reads a contiguous run of scores with
+//              coalesced float4 loads), then one pass in token order that keeps
+//              every larger score and the first equal ones (ties to the lower
+//              index); per-warp counts and lane scans place the kept tokens in
+//              ascending order
 //   dsa_attn   CTA = one query x one KV group: 8 warps take 256 kept tokens each,
 //              gather their K/V rows with 16-byte cp.async into swizzled tiles of
 //              16 keys and run an online softmax (16 rows = the group's heads);
@@ -37,6 +38,7 @@ constexpr int kIdxChunk = 4096;     // keys per indexer CTA
 constexpr int kIdxTile = 128;       // keys per shared-memory tile (32 per warp)
 constexpr int kIdxStages = 3;
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkBins = 4096;     // 12-bit digits in the first two radix passes
 constexpr int kAttnWarps = 8;
 constexpr int kAttnTile = 16;       // keys per gathered tile
 
@@ -195,11 +197,53 @@ __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* wsum, ui
   return before + x - v;
 }
 
+// The bin b of hist[0..nbins) with above(b) < need <= above(b) + hist[b], where
+// above(b) counts the elements in the bins above b; sel = {b, above(b)}. Thread
+// i owns bins nbins - 1 - (per i .. per i + per - 1), so the CTA scan runs from
+// the top bin down. Synchronises the CTA.
+__device__ __forceinline__ void topk_find_bin(const uint32_t* hist, int nbins, uint32_t need, uint32_t* wsum,
+                                              uint32_t* sel) {
+  const int tid = threadIdx.x;
+  const int per = nbins >= kTopkThreads ? nbins / kTopkThreads : 1;
+  const bool own = tid * per < nbins;
+  uint32_t sum = 0u;
+  if (own)
+    for (int j = 0; j < per; ++j) sum += hist[nbins - 1 - (tid * per + j)];
+  uint32_t total;
+  uint32_t above = cta_excl_scan(sum, wsum, total);
+  if (own && above < need && above + sum >= need) {
+    for (int j = 0; j < per; ++j) {
+      const int bin = nbins - 1 - (tid * per + j);
+      if (above + hist[bin] >= need) {
+        sel[0] = (uint32_t)bin;
+        sel[1] = above;
+        break;
+      }
+      above += hist[bin];
+    }
+  }
+  __syncthreads();
+}
+
+// exclusive prefix of v over the lanes of a warp; `total` gets the warp's sum
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t& total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += o;
+  }
+  total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
 __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const DsaArgs a) {
-  __shared__ uint32_t whist[32][256];   // one histogram per warp: no contention between warps
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t wsum[2][32];       // one buffer per scan of a chunk (a warp may still read the other)
-  __shared__ uint32_t sel_bin[2];
+  constexpr int kWarps = kTopkThreads / 32;
+  __shared__ uint32_t hist[kTopkBins];
+  __shared__ uint32_t wsum[32];
+  __shared__ uint32_t sel[2];
+  __shared__ uint32_t wcnt[2][kWarps];   // per warp: keys above the threshold, keys equal to it
   const int slot = blockIdx.x;
   int64_t qrow, base;
   int t;
@@ -212,100 +256,113 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const DsaArgs a)
     for (int i = tid; i < K; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
-  // radix select of the K-th largest order key, 8 bits per pass from the top
-  uint32_t prefix = 0u, pmask = 0u;
-  uint32_t need = (uint32_t)K;   // elements still to take among those matching the prefix
+  // warp w owns the scores [wb, we) (a multiple of 128 long); it reads them in
+  // chunks of 128, lane l taking 4 consecutive scores (float4 when aligned), so
+  // every load is coalesced and the chunks go in token order
+  const int span = ((n + kWarps - 1) / kWarps + 127) & ~127;
+  const int wb = min(n, warp * span), we = min(n, wb + span);
   const bool vec = (reinterpret_cast<uintptr_t>(sc) & 15u) == 0;
-  for (int sh_ = 24; sh_ >= 0; sh_ -= 8) {
-    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
-    __syncwarp();
-    auto add = [&](float f, bool valid) {
-      const uint32_t u = ord_key(f);
-      const bool m = valid && (u & pmask) == prefix;
-      const uint32_t bin = (u >> sh_) & 255u;
-      const uint32_t act = __ballot_sync(0xffffffffu, m);
-      if (m) {   // lanes with the same bin add once
-        const uint32_t peers = __match_any_sync(act, bin);
-        if ((uint32_t)lane == (uint32_t)(__ffs(peers) - 1)) whist[warp][bin] += __popc(peers);
-      }
-      __syncwarp();
-    };
-    if (vec) {
-      for (int i0 = 0; i0 < n; i0 += 4 * kTopkThreads) {   // warp-uniform trip count
-        const int i = i0 + 4 * tid;
-        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i + 3 < n) f = *reinterpret_cast<const float4*>(sc + i);
-        else {
-          if (i < n) f.x = sc[i];
-          if (i + 1 < n) f.y = sc[i + 1];
-          if (i + 2 < n) f.z = sc[i + 2];
-        }
-        add(f.x, i < n);
-        add(f.y, i + 1 < n);
-        add(f.z, i + 2 < n);
-        add(f.w, i + 3 < n);
-      }
+  auto load4 = [&](int i, uint32_t* u) {   // keys of i .. i + 3 (0 beyond we: never selected)
+    if (vec && i + 3 < we) {
+      const float4 v = *reinterpret_cast<const float4*>(sc + i);
+      u[0] = ord_key(v.x);
+      u[1] = ord_key(v.y);
+      u[2] = ord_key(v.z);
+      u[3] = ord_key(v.w);
     } else {
-      for (int i0 = 0; i0 < n; i0 += kTopkThreads) add(i0 + tid < n ? sc[i0 + tid] : 0.f, i0 + tid < n);
-    }
-    __syncthreads();
-    if (tid < 256) {
-      uint32_t c = 0u;
-#pragma unroll 8
-      for (int w = 0; w < 32; ++w) c += whist[w][tid];
-      hist[tid] = c;
-    }
-    __syncthreads();
-    if (warp == 0) {   // the bin holding the need-th largest, counting from bin 255 down
-      uint32_t loc[8], sum = 0u;   // lane owns bins 255 - 8 lane - 7 .. 255 - 8 lane
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        loc[j] = hist[255 - 8 * lane - j];
-        sum += loc[j];
-      }
-      uint32_t x = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += o;
-      }
-      uint32_t acc = x - sum;   // elements in bins above this lane's range
-      if (acc < need && x >= need) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + loc[j] >= need) {
-            sel_bin[0] = 255u - 8u * lane - (uint32_t)j;
-            sel_bin[1] = acc;
-            break;
-          }
-          acc += loc[j];
-        }
-      }
+      for (int e = 0; e < 4; ++e) u[e] = i + e < we ? ord_key(sc[i + e]) : 0u;
     }
+  };
+  auto visit = [&](auto&& f) {
+    for (int i = wb + 4 * lane; i < we; i += 128) {
+      uint32_t u[4];
+      load4(i, u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e < we) f(u[e]);
+    }
+  };
+  auto clear = [&](int nbins) {
+    for (int i = tid; i < nbins; i += kTopkThreads) hist[i] = 0u;
     __syncthreads();
-    prefix |= sel_bin[0] << sh_;
-    pmask |= 255u << sh_;
-    need -= sel_bin[1];
-    __syncthreads();
+  };
+  // radix select of the K-th largest order key: bits 31..20, 19..8, 7..0
+  clear(kTopkBins);
+  visit([&](uint32_t u) { atomicAdd(&hist[u >> 20], 1u); });
+  __syncthreads();
+  topk_find_bin(hist, kTopkBins, (uint32_t)K, wsum, sel);
+  const uint32_t b1 = sel[0];
+  uint32_t need = (uint32_t)K - sel[1];
+  __syncthreads();
+  clear(kTopkBins);
+  visit([&](uint32_t u) {
+    if ((u >> 20) == b1) atomicAdd(&hist[(u >> 8) & 4095u], 1u);
+  });
+  __syncthreads();
+  topk_find_bin(hist, kTopkBins, need, wsum, sel);
+  const uint32_t hi24 = (b1 << 12) | sel[0];
+  need -= sel[1];
+  __syncthreads();
+  clear(256);
+  visit([&](uint32_t u) {
+    if ((u >> 8) == hi24) atomicAdd(&hist[u & 255u], 1u);
+  });
+  __syncthreads();
+  topk_find_bin(hist, 256, need, wsum, sel);
+  const uint32_t thr = (hi24 << 8) | sel[0];
+  need -= sel[1];   // keys equal to thr still to take, in token order
+  // every key above thr and the first `need` equal ones, in token order: the
+  // warps' counts give each warp its starting rank and position, then each
+  // chunk's ranks come from lane scans
+  uint32_t gt = 0u, eq = 0u;
+  visit([&](uint32_t u) {
+    gt += u > thr ? 1u : 0u;
+    eq += u == thr ? 1u : 0u;
+  });
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, off);
+    eq += __shfl_xor_sync(0xffffffffu, eq, off);
   }
-  // prefix is the K-th largest key: keep the larger keys and the first `need` equal
-  // ones in token order; positions from CTA-wide scans of each 1024-element chunk
-  const uint32_t thr = prefix;
-  uint32_t taken = 0u, eq_seen = 0u;
-  for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
-    const int i = c0 + tid;
-    const uint32_t u = i < n ? ord_key(sc[i]) : 0u;
-    const bool gt = i < n && u > thr;
-    const bool eq = i < n && u == thr;
-    uint32_t eq_total;
-    const uint32_t eq_before = eq_seen + cta_excl_scan(eq ? 1u : 0u, wsum[0], eq_total);
-    const bool keep = gt || (eq && eq_before < need);
-    uint32_t k_total;
-    const uint32_t pos = taken + cta_excl_scan(keep ? 1u : 0u, wsum[1], k_total);
-    if (keep && NSA_BOUNDS(pos < (uint32_t)K, a.status, 701)) out[pos] = i;
-    taken += k_total;
-    eq_seen += eq_total;
-    if (taken >= (uint32_t)K) break;   // CTA-uniform: every thread holds the same totals
+  if (lane == 0) {
+    wcnt[0][warp] = gt;
+    wcnt[1][warp] = eq;
+  }
+  __syncthreads();
+  uint32_t gt_base = 0u, eq_rank = 0u;
+  for (int w = 0; w < warp; ++w) {
+    gt_base += wcnt[0][w];
+    eq_rank += wcnt[1][w];
+  }
+  uint32_t pos = gt_base + min(eq_rank, need);
+  for (int i = wb + 4 * lane; i - 4 * lane < we; i += 128) {   // warp-uniform trip count
+    uint32_t u[4];
+    load4(i, u);
+    uint32_t ne = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ne += (i + e < we && u[e] == thr) ? 1u : 0u;
+    uint32_t ne_tot;
+    uint32_t r = eq_rank + warp_excl_scan(ne, ne_tot);
+    bool keep[4];
+    uint32_t nk = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool in = i + e < we;
+      keep[e] = in && u[e] > thr;
+      if (in && u[e] == thr) keep[e] = r++ < need;
+      nk += keep[e] ? 1u : 0u;
+    }
+    uint32_t nk_tot;
+    uint32_t p = pos + warp_excl_scan(nk, nk_tot);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (keep[e]) {
+        if (NSA_BOUNDS(p < (uint32_t)K, a.status, 701)) out[p] = i + e;
+        ++p;
+      }
+    eq_rank += ne_tot;
+    pos += nk_tot;
   }
 }
 
