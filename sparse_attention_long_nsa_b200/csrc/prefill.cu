@@ -866,6 +866,18 @@ bool prefill_fused_stages(PrefillArgs& a) {
   int n = (int)(budget / (kb + vb));
   if (n > kMaxStages) n = kMaxStages;
   if (n < 2) return false;
+  // long sequences: keep the importance on chip by giving up V stages (down to
+  // two) before spilling it to the workspace
+  const size_t ib = imp_smem_bytes(a.nb_stride, a.G);
+  if (budget < (size_t)n * (kb + vb) + ib) {
+    for (int nv = n - 1; nv >= 2; --nv)
+      if (budget >= (size_t)n * kb + (size_t)nv * vb + ib) {
+        a.imp_smem = 1;
+        a.n_stages = n & ~1;
+        a.n_vstages = nv;
+        return true;
+      }
+  }
   budget -= (size_t)n * (kb + vb);
   // the tile's importance and selections stay on chip when the room is left over
   a.imp_smem = budget >= imp_smem_bytes(a.nb_stride, a.G) ? 1 : 0;

@@ -85,6 +85,14 @@ def test_prefill_beyond_64k_radix_topn_and_ties():
     assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
 
 
+def test_prefill_importance_through_workspace():
+    """80,000 tokens (1250 candidate blocks): the tile's importance rows no longer
+    fit in shared memory next to two V stages, so they go through the fp32
+    workspace; 128 random rows plus the edges."""
+    cfg = W.small_config(name="prefill_80k", T=80000, H_q=16, H_kv=1, d_k=192, d_v=128, seed=1006)
+    NP.run_prefill_case(cfg, [80000], n_random_rows=128)
+
+
 def test_prefill_exact_ties_register_topn():
     """All compressed keys zero (exact ties between interior blocks) on the
     register top-n path of the prefill (GQA 16 and GQA 4)."""
