@@ -170,13 +170,22 @@ nsa_status_t nsa_compress_append(const void* k_cache, const void* v_cache, const
  *    call's contents (each call clears the status word it needs zeroed). Calls
  *    whose work overlaps on the GPU (different streams, or different host
  *    threads) race on the array and must be serialised by the caller.
- *  - nsa_check_device_status() does not apply (the status word is internal). */
+ *  - Device errors: nsa_check_device_status() does not apply (the status word
+ *    is inside the array); nsa_noalloc_check_status() reads and clears it. */
 #define NSA_NOALLOC_SCRATCH_BYTES 4194304
 nsa_status_t nsa_compress_noalloc(const void* k, const void* v, const float* w_ck, const float* pe_k,
                                   const float* w_cv, const float* pe_v, const int64_t* tok_offset,
                                   const int32_t* seq_len, const int64_t* cmp_offset, int32_t batch,
                                   const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
                                   void* v_cmp, void* stream);
+
+/* The status word of nsa_compress_noalloc's built-in scratch on the current
+ * device: synchronises `stream`, reads the word and clears it. Returns NSA_OK,
+ * NSA_ERR_DEVICE_CHECK (a kernel of the last call on this device recorded a
+ * failed bounded wait or index check; its outputs are not valid) or
+ * NSA_ERR_CUDA. It synchronises, so it cannot run during stream capture; call
+ * it after the captured work has run. Allocates nothing. */
+nsa_status_t nsa_noalloc_check_status(void* stream);
 
 /* Causal NSA prefill over packed variable-length sequences (NSA-ru "NSA: три
  * ветви"; NSA-lesson "Concept"). Positions restart at 0 in every sequence.

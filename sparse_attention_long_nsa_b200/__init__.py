@@ -32,6 +32,7 @@ NSA_NOALLOC_SCRATCH_BYTES = 4194304
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
             "nsa_compress_append_plan", "nsa_compress_append", "nsa_compress_paged", "nsa_compress_noalloc",
+            "nsa_noalloc_check_status",
             "nsa_decode_paged", "nsa_prefill_backward", "nsa_dsa_workspace_size", "nsa_dsa_decode",
             "nsa_dsa_prefill", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
@@ -145,6 +146,8 @@ def _load(path: str) -> ctypes.CDLL:
     L.nsa_dsa_prefill.restype = ctypes.c_int
     L.nsa_dsa_prefill.argtypes = [P, P, P, P, P, P, P, I32, ctypes.POINTER(DsaParams), ctypes.POINTER(Heads), P, P,
                                   P, P, SZ, P]
+    L.nsa_noalloc_check_status.restype = ctypes.c_int
+    L.nsa_noalloc_check_status.argtypes = [P]
     L.nsa_compress_noalloc.restype = ctypes.c_int
     L.nsa_compress_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads),
                                        ctypes.POINTER(Params), P, P, P]
@@ -246,6 +249,12 @@ def nsa_compress_noalloc(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_
                                    ctypes.byref(params), _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16),
                                    _stream(stream))
     _check(s, "nsa_compress_noalloc")
+
+
+def nsa_noalloc_check_status(stream=None):
+    """Synchronise the stream, read and clear the status word of
+    nsa_compress_noalloc's built-in scratch on the current device."""
+    _check(lib().nsa_noalloc_check_status(_stream(stream)), "nsa_noalloc_check_status")
 
 
 def nsa_prefill(q, k, v, k_cmp, v_cmp, gates, cu_seqlens, heads: Heads, params: Params, out, sel_out=None,

@@ -84,3 +84,11 @@ extern "C" nsa_status_t nsa_compress_noalloc(const void* k, const void* v, const
   return nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, batch, heads, params, k_cmp,
                       v_cmp, scratch, (size_t)NSA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" nsa_status_t nsa_noalloc_check_status(void* stream) {
+  void* scratch = nullptr;
+  nsa_status_t s = scratch_address(&scratch);
+  if (s != NSA_OK) return s;
+  // the array's header is the status word of an ordinary workspace
+  return nsa_check_device_status(scratch, stream);
+}

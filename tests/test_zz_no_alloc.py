@@ -74,6 +74,55 @@ def test_noalloc_matches_workspace_entry_point(cfg_name, seqlens):
                         "v_cmp (no-alloc) vs oracle", relative_to_rms=True)
 
 
+def test_noalloc_under_graph_capture():
+    """After one eager call (which resolves the scratch address), the call is
+    captured into a CUDA graph and replayed on new inputs copied into the captured
+    tensors. Neither an eager call nor a replay allocates (torch's allocator and
+    the device's free memory are unchanged across them); the replay matches
+    nsa_compress on the new inputs, and the status word reads clean."""
+    cfg = W.CONFIGS["prefill_tiny_1k"]
+    seqlens = [1024, 31, 333]
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    tok, lens, cmp_off, total = _offsets(seqlens, par)
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=7)
+    k_out = torch.empty((total, cfg.H_kv, cfg.d_k), dtype=torch.bfloat16, device="cuda")
+    v_out = torch.empty((total, cfg.H_kv, cfg.d_v), dtype=torch.bfloat16, device="cuda")
+    args = (inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], tok, lens, cmp_off, heads, par,
+            k_out, v_out)
+    nsa.nsa_compress_noalloc(*args)
+    torch.cuda.synchronize()
+    nsa.nsa_noalloc_check_status()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    nsa.nsa_compress_noalloc(*args)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0 and torch.cuda.mem_get_info()[0] == free0
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=side):
+        nsa.nsa_compress_noalloc(*args, stream=side)
+    torch.cuda.synchronize()
+    new = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=8)
+    for name in ("k", "v", "w_ck", "pe_k", "w_cv", "pe_v"):
+        inp[name].copy_(new[name])
+    k_out.fill_(float("nan"))
+    v_out.fill_(float("nan"))
+    torch.cuda.synchronize()
+    alloc1, free1 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc1 and torch.cuda.mem_get_info()[0] == free1
+    nsa.nsa_noalloc_check_status()
+    ws = nsa.alloc_workspace(nsa.nsa_workspace_size(nsa.NSA_OP_COMPRESS, heads, par, len(seqlens), 0, 0), "cuda")
+    ref_k, ref_v = torch.empty_like(k_out), torch.empty_like(v_out)
+    nsa.nsa_compress(new["k"], new["v"], new["w_ck"], new["pe_k"], new["w_cv"], new["pe_v"], tok, lens, cmp_off,
+                     heads, par, ref_k, ref_v, ws)
+    torch.cuda.synchronize()
+    NP.assert_close(NP.f64(k_out), NP.f64(ref_k), "k_cmp (graph replay)", relative_to_rms=True)
+    NP.assert_close(NP.f64(v_out), NP.f64(ref_v), "v_cmp (graph replay)", relative_to_rms=True)
+    del graph
+
+
 def test_noalloc_rejects_invalid_arguments():
     cfg = W.CONFIGS["prefill_8k"]
     par = NP.params_of(cfg)
