@@ -118,6 +118,34 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
                           const nsa_heads_t* heads, const nsa_params_t* params, void* k_cmp,
                           void* v_cmp, void* workspace, size_t ws_bytes, void* stream);
 
+/* The compression's weights in the form the GEMM reads (NSA-ru "NSA: три
+ * ветви", compression branch): W^T of both maps rounded to bf16 and the fp32
+ * position terms sum(pe * W). nsa_compress forms them from the fp32 weights on
+ * every call; a caller whose weights stay fixed across calls (inference, or
+ * training between optimizer steps) forms them once with nsa_compress_prepare
+ * and passes them to nsa_compress_prepared, which then runs only the GEMM. The
+ * results are identical.
+ * nsa_compress_weights_size: bytes of the prepared form (0 for invalid
+ * arguments). */
+size_t nsa_compress_weights_size(const nsa_heads_t* heads, const nsa_params_t* params);
+
+/* Fill `prepared` (device, 256-byte aligned, prepared_bytes >=
+ * nsa_compress_weights_size) from w_ck, pe_k, w_cv, pe_v (the layouts of
+ * nsa_compress). The caller owns `prepared`; it holds no pointer to the inputs.
+ * NSA_ERR_INVALID_ARG for null or misaligned pointers, NSA_ERR_WORKSPACE when
+ * prepared_bytes is too small, NSA_ERR_UNSUPPORTED for head sizes the GEMM is
+ * not built for. */
+nsa_status_t nsa_compress_prepare(const float* w_ck, const float* pe_k, const float* w_cv, const float* pe_v,
+                                  const nsa_heads_t* heads, const nsa_params_t* params, void* prepared,
+                                  size_t prepared_bytes, void* stream);
+
+/* nsa_compress with weights from nsa_compress_prepare (same heads and params):
+ * the same outputs, arguments and errors, without the per-call conversion. */
+nsa_status_t nsa_compress_prepared(const void* k, const void* v, const void* prepared,
+                                   const int64_t* tok_offset, const int32_t* seq_len, const int64_t* cmp_offset,
+                                   int32_t batch, const nsa_heads_t* heads, const nsa_params_t* params,
+                                   void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes, void* stream);
+
 /* Incremental decode (NSA-ru "NSA: три ветви", compression branch: a summary
  * exists for every whole block of l_cmp tokens at stride `stride`; the cache
  * grows one token, or several, at a time). When sequence b of a batched cache

@@ -32,7 +32,7 @@ NSA_NOALLOC_SCRATCH_BYTES = 4194304
 # every symbol include/nsa.h declares
 EXPORTED = ("nsa_workspace_size", "nsa_workspace_init", "nsa_check_device_status", "nsa_compress",
             "nsa_compress_append_plan", "nsa_compress_append", "nsa_compress_paged", "nsa_compress_noalloc",
-            "nsa_noalloc_check_status",
+            "nsa_noalloc_check_status", "nsa_compress_weights_size", "nsa_compress_prepare", "nsa_compress_prepared",
             "nsa_decode_paged", "nsa_prefill_backward", "nsa_dsa_workspace_size", "nsa_dsa_decode",
             "nsa_dsa_prefill", "nsa_prefill", "nsa_decode", "nsa_profile_enable", "nsa_profile_read", "nsa_profile_slot_name",
             "nsa_status_string", "nsa_last_error_detail")
@@ -123,6 +123,13 @@ def _load(path: str) -> ctypes.CDLL:
     L.nsa_compress.restype = ctypes.c_int
     L.nsa_compress.argtypes = [P, P, P, P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params),
                                P, P, P, SZ, P]
+    L.nsa_compress_weights_size.restype = SZ
+    L.nsa_compress_weights_size.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Params)]
+    L.nsa_compress_prepare.restype = ctypes.c_int
+    L.nsa_compress_prepare.argtypes = [P, P, P, P, ctypes.POINTER(Heads), ctypes.POINTER(Params), P, SZ, P]
+    L.nsa_compress_prepared.restype = ctypes.c_int
+    L.nsa_compress_prepared.argtypes = [P, P, P, P, P, P, I32, ctypes.POINTER(Heads), ctypes.POINTER(Params),
+                                        P, P, P, SZ, P]
     L.nsa_compress_append_plan.restype = ctypes.c_int
     L.nsa_compress_append_plan.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(Params), P, P, P, P]
     L.nsa_compress_append.restype = ctypes.c_int
@@ -235,6 +242,29 @@ def nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, 
                            _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream))
     _check(s, "nsa_compress")
+
+
+def nsa_compress_weights_size(heads: Heads, params: Params) -> int:
+    return int(lib().nsa_compress_weights_size(ctypes.byref(heads), ctypes.byref(params)))
+
+
+def nsa_compress_prepare(w_ck, pe_k, w_cv, pe_v, heads: Heads, params: Params, prepared, stream=None):
+    s = lib().nsa_compress_prepare(_ptr(w_ck, torch.float32), _ptr(pe_k, torch.float32), _ptr(w_cv, torch.float32),
+                                   _ptr(pe_v, torch.float32), ctypes.byref(heads), ctypes.byref(params),
+                                   _ptr(prepared), prepared.numel() * prepared.element_size(), _stream(stream))
+    _check(s, "nsa_compress_prepare")
+
+
+def nsa_compress_prepared(k, v, prepared, tok_offset, seq_len, cmp_offset, heads: Heads, params: Params, k_cmp, v_cmp,
+                          ws, stream=None):
+    """nsa_compress with weights from nsa_compress_prepare."""
+    B = int(seq_len.numel())
+    s = lib().nsa_compress_prepared(_ptr(k, torch.bfloat16), _ptr(v, torch.bfloat16), _ptr(prepared),
+                                    _ptr(tok_offset, torch.int64, "cpu"), _ptr(seq_len, torch.int32, "cpu"),
+                                    _ptr(cmp_offset, torch.int64, "cpu"), B, ctypes.byref(heads),
+                                    ctypes.byref(params), _ptr(k_cmp, torch.bfloat16), _ptr(v_cmp, torch.bfloat16),
+                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(s, "nsa_compress_prepared")
 
 
 def nsa_compress_noalloc(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, heads: Heads,
@@ -398,8 +428,16 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return ws
 
 
-def compress(k, v, w_ck, pe_k, w_cv, pe_v, seqlens, heads: Heads, params: Params, ws=None, out=None):
-    """Packed prefill layout: sequences back to back in k/v. Returns (k_cmp, v_cmp)."""
+def compress_prepare(w_ck, pe_k, w_cv, pe_v, heads: Heads, params: Params) -> torch.Tensor:
+    """The compression weights in prepared form (a device byte tensor)."""
+    prepared = torch.empty(nsa_compress_weights_size(heads, params), dtype=torch.uint8, device=w_ck.device)
+    nsa_compress_prepare(w_ck, pe_k, w_cv, pe_v, heads, params, prepared)
+    return prepared
+
+
+def compress(k, v, w_ck, pe_k, w_cv, pe_v, seqlens, heads: Heads, params: Params, ws=None, out=None, prepared=None):
+    """Packed prefill layout: sequences back to back in k/v. Returns (k_cmp, v_cmp).
+    With `prepared` (from compress_prepare) the weight arguments are not read."""
     seqlens = [int(x) for x in seqlens]
     tok = torch.tensor([sum(seqlens[:b]) for b in range(len(seqlens))], dtype=torch.int64)
     ncs = [n_cmp(L, params.l_cmp, params.stride) for L in seqlens]
@@ -414,8 +452,12 @@ def compress(k, v, w_ck, pe_k, w_cv, pe_v, seqlens, heads: Heads, params: Params
     if ws is None:
         ws = alloc_workspace(nsa_workspace_size(NSA_OP_COMPRESS, heads, params, len(seqlens), sum(seqlens), 0),
                              dev)
-    nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok, torch.tensor(seqlens, dtype=torch.int32), cmp_off, heads,
-                 params, k_cmp, v_cmp, ws)
+    if prepared is not None:
+        nsa_compress_prepared(k, v, prepared, tok, torch.tensor(seqlens, dtype=torch.int32), cmp_off, heads, params,
+                              k_cmp, v_cmp, ws)
+    else:
+        nsa_compress(k, v, w_ck, pe_k, w_cv, pe_v, tok, torch.tensor(seqlens, dtype=torch.int32), cmp_off, heads,
+                     params, k_cmp, v_cmp, ws)
     return k_cmp[:total], v_cmp[:total]
 
 

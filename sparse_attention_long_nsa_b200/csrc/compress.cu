@@ -50,13 +50,24 @@ __global__ void compress_transpose_kernel(const float* __restrict__ w, const flo
   }
 }
 
+// 32 columns per CTA of 32 x 8 threads: thread (x, y) adds the tiles
+// y, y + 8, ... of column x, then the 8 partial sums are added in order y = 0..7
 __global__ void compress_bias_kernel(const float* __restrict__ partial, int KT, int N,
                                      float* __restrict__ bias) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  __shared__ float acc[8][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int n = blockIdx.x * 32 + tx;
   float s = 0.f;
-  for (int kt = 0; kt < KT; ++kt) s += partial[(size_t)kt * N + n];
-  bias[n] = s;
+  if (n < N)
+    for (int kt = ty; kt < KT; kt += 8) s += partial[(size_t)kt * N + n];
+  acc[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && n < N) {
+    float t = acc[0][tx];
+#pragma unroll
+    for (int y = 1; y < 8; ++y) t += acc[y][tx];
+    bias[n] = t;
+  }
 }
 
 cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
@@ -64,7 +75,7 @@ cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, 
   dim3 grid((N + 31) / 32, (K + 31) / 32);
   compress_transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(
       w, pe, K, N, static_cast<__nv_bfloat16*>(wt_bf16), partial);
-  compress_bias_kernel<<<(N + 127) / 128, 128, 0, st>>>(partial, (K + 31) / 32, N, bias);
+  compress_bias_kernel<<<(N + 31) / 32, dim3(32, 8), 0, st>>>(partial, (K + 31) / 32, N, bias);
   return cudaGetLastError();
 }
 
@@ -88,8 +99,9 @@ __device__ __forceinline__ int find_seq(const SeqTable& t, int tile) {
   return b;
 }
 
+// one map (m = 0 keys, 1 values) of KV head g
 template <int D_IN, int D_OUT>
-__global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArgs a) {
+__device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m, int g) {
   using S = CompressSmem<D_OUT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -100,14 +112,13 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x;
   const int b = find_seq(a.seqs, tile);
-  const int g = blockIdx.y;
   const int L = a.seqs.len[b];
   const int ncmp = n_cmp_of(L, a.l, a.s);
   const int i0 = (tile - a.seqs.tile_prefix[b]) * kTileM;
   const int64_t tok0 = a.seqs.tok_off[b];
   const int K = a.l * D_IN;
-  const int kb0 = blockIdx.z * a.kb_per_split;                 // this CTA's share of K
-  const int nkb = min(K / 64 - kb0, a.kb_per_split);
+  const int kb0 = blockIdx.z * a.kb_per_split[m];              // this CTA's share of K
+  const int nkb = min(K / 64 - kb0, a.kb_per_split[m]);
   constexpr uint32_t TM_COLS = D_OUT <= 64 ? 64 : (D_OUT <= 128 ? 128 : 256);
 
   if (tid == 0) {
@@ -121,8 +132,8 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
 
-  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
-  const __nv_bfloat16* wt = static_cast<const __nv_bfloat16*>(a.wt);
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x[m]);
+  const __nv_bfloat16* wt = static_cast<const __nv_bfloat16*>(a.wt[m]);
   const size_t row_stride = (size_t)a.H_kv * D_IN;   // elements between tokens
 
   auto load_stage = [&](int st, int kb) {
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
     // epilogue: warp w owns accumulator rows 32w .. 32w+31 (TMEM lanes)
     const int row = warp * 32 + lane;
     const int ci = i0 + row;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out[m]);
     int64_t oe = a.seqs.cmp_off[b] + ci;   // output row (paged: entry index in the sequence)
     bool oval = true;
     if (a.out_pt.table && ci < ncmp) {
@@ -219,16 +230,16 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
       tmem_ld16(tmem_d + ((uint32_t)(warp * 32) << 16) + c0, v);
       tmem_ld_wait();
       if (ci < ncmp && oval) {
-        if (a.ksplit == 1) {
+        if (a.ksplit[m] == 1) {
           uint32_t pk[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            pk[j] = pack_bf16x2(v[2 * j] + a.bias[c0 + 2 * j], v[2 * j + 1] + a.bias[c0 + 2 * j + 1]);
+            pk[j] = pack_bf16x2(v[2 * j] + a.bias[m][c0 + 2 * j], v[2 * j + 1] + a.bias[m][c0 + 2 * j + 1]);
           uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         } else {
-          float4* dst = reinterpret_cast<float4*>(a.part + (size_t)blockIdx.z * a.rows_total * a.H_kv * D_OUT + orow + c0);
+          float4* dst = reinterpret_cast<float4*>(a.part[m] + (size_t)blockIdx.z * a.rows_total * a.H_kv * D_OUT + orow + c0);
 #pragma unroll
           for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
@@ -240,49 +251,67 @@ __global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArg
   if (warp == 0) tmem_dealloc(tmem_d, TM_COLS);
 }
 
-template <int D_IN, int D_OUT>
+// keys and values of every KV head in one launch (grid.y = 2 H_kv); a CTA whose
+// split index is beyond its map's split count has nothing to do
+template <int DK, int DV>
+__global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArgs a) {
+  const int m = blockIdx.y >= a.H_kv ? 1 : 0;
+  if ((int)blockIdx.z >= a.ksplit[m]) return;
+  if (m == 0) compress_gemm_body<DK, DK>(a, 0, blockIdx.y);
+  else compress_gemm_body<DV, DV>(a, 1, blockIdx.y - a.H_kv);
+}
+
+template <int DK, int DV>
 static cudaError_t launch_gemm_t(const CompressArgs& a, int n_tiles, cudaStream_t st) {
-  using S = CompressSmem<D_OUT>;
-  auto kern = compress_gemm_kernel<D_IN, D_OUT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
+  constexpr int smem = CompressSmem<DK>::TOTAL > CompressSmem<DV>::TOTAL ? CompressSmem<DK>::TOTAL
+                                                                        : CompressSmem<DV>::TOTAL;
+  auto kern = compress_gemm_kernel<DK, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(n_tiles, a.H_kv, a.ksplit);
-  kern<<<grid, 128, S::TOTAL, st>>>(a);
+  dim3 grid(n_tiles, 2 * a.H_kv, a.ksplit[0] > a.ksplit[1] ? a.ksplit[0] : a.ksplit[1]);
+  kern<<<grid, 128, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-// out[r, :] = bf16(sum_z part[z, r, :] + bias) over the packed output rows, the
+// out[r, :] = bf16(sum_z part[z, r, :] + bias) over the packed output rows of
+// both maps (float4 indices [0, n4k) keys, then [n4k, n4k + n4v) values), the
 // partial sums added in a fixed order (deterministic)
-__global__ void compress_finalize_kernel(const float* __restrict__ part, int ksplit, int64_t n4, int d_out,
-                                         const float* __restrict__ bias, __nv_bfloat16* __restrict__ out) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
-  if (i >= n4) return;
-  float4 acc = reinterpret_cast<const float4*>(part)[i];
-  for (int z = 1; z < ksplit; ++z) {
-    const float4 v = reinterpret_cast<const float4*>(part)[(size_t)z * n4 + i];
+__global__ void compress_finalize_kernel(const CompressArgs a, int64_t n4k, int64_t n4v, int dk, int dv) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+  if (i >= n4k + n4v) return;
+  const int m = i < n4k ? 0 : 1;
+  if (m == 1) i -= n4k;
+  const int64_t n4 = m == 0 ? n4k : n4v;
+  const int d_out = m == 0 ? dk : dv;
+  const float4* part = reinterpret_cast<const float4*>(a.part[m]);
+  float4 acc = part[i];
+  for (int z = 1; z < a.ksplit[m]; ++z) {
+    const float4 v = part[(size_t)z * n4 + i];
     acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
   }
   const int c = (int)((i * 4) % d_out);
+  const float* bias = a.bias[m];
   uint2 pk;
   pk.x = pack_bf16x2(acc.x + bias[c], acc.y + bias[c + 1]);
   pk.y = pack_bf16x2(acc.z + bias[c + 2], acc.w + bias[c + 3]);
-  reinterpret_cast<uint2*>(out)[i] = pk;
+  reinterpret_cast<uint2*>(a.out[m])[i] = pk;
 }
 
-cudaError_t launch_compress_finalize(int d_out, const CompressArgs& a, cudaStream_t st) {
-  const int64_t n4 = a.rows_total * a.H_kv * d_out / 4;
-  if (n4 <= 0) return cudaSuccess;
-  compress_finalize_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(a.part, a.ksplit, n4, d_out, a.bias,
-                                                                          static_cast<__nv_bfloat16*>(a.out));
+cudaError_t launch_compress_finalize(int d_k, int d_v, const CompressArgs& a, cudaStream_t st) {
+  const int64_t n4k = a.ksplit[0] > 1 ? a.rows_total * a.H_kv * d_k / 4 : 0;
+  const int64_t n4v = a.ksplit[1] > 1 ? a.rows_total * a.H_kv * d_v / 4 : 0;
+  if (n4k + n4v <= 0) return cudaSuccess;
+  compress_finalize_kernel<<<(unsigned)((n4k + n4v + 255) / 256), 256, 0, st>>>(a, n4k, n4v, d_k, d_v);
   return cudaGetLastError();
 }
 
-cudaError_t launch_compress_gemm(int d_in, int d_out, const CompressArgs& a, int n_tiles,
-                                 cudaStream_t st) {
+cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, int n_tiles, cudaStream_t st) {
   if (n_tiles <= 0) return cudaSuccess;
-  if (d_in == 64 && d_out == 64) return launch_gemm_t<64, 64>(a, n_tiles, st);
-  if (d_in == 128 && d_out == 128) return launch_gemm_t<128, 128>(a, n_tiles, st);
-  if (d_in == 192 && d_out == 192) return launch_gemm_t<192, 192>(a, n_tiles, st);
+#define NSA_CMP_CASE(DK, DV) \
+  if (d_k == DK && d_v == DV) return launch_gemm_t<DK, DV>(a, n_tiles, st);
+  NSA_CMP_CASE(192, 128) NSA_CMP_CASE(64, 64) NSA_CMP_CASE(128, 128) NSA_CMP_CASE(192, 64)
+  NSA_CMP_CASE(64, 128) NSA_CMP_CASE(128, 64) NSA_CMP_CASE(192, 192) NSA_CMP_CASE(128, 192) NSA_CMP_CASE(64, 192)
+#undef NSA_CMP_CASE
   return cudaErrorInvalidValue;
 }
 

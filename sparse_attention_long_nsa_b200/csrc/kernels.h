@@ -50,15 +50,17 @@ __device__ __forceinline__ int64_t paged_row(const PageTable& pt, int b, int e, 
 }
 
 // ----- compression (block summaries) -----
+// Both maps in one launch: index 0 = keys (d = d_k), 1 = values (d = d_v);
+// grid.y = 2 H_kv (y < H_kv: keys of KV head y, else values of head y - H_kv).
 struct CompressArgs {
-  const void* x;          // bf16 [*, H_kv, d_in]
-  const void* wt;         // bf16 [d_out, l*d_in] (W transposed, rounded)
-  const float* bias;      // fp32 [d_out] = vec(pe) . W
-  void* out;              // bf16 [*, H_kv, d_out]
+  const void* x[2];       // bf16 [*, H_kv, d]
+  const void* wt[2];      // bf16 [d, l*d] (W transposed, rounded)
+  const float* bias[2];   // fp32 [d] = vec(pe) . W
+  void* out[2];           // bf16 [*, H_kv, d]
   int H_kv, l, s;
-  int ksplit;             // split of the K = l*d_in reduction over grid.z (1: no split)
-  int kb_per_split;       // 64-wide K blocks per split
-  float* part;            // fp32 [ksplit][rows_total][H_kv][d_out] partial sums (ksplit > 1)
+  int ksplit[2];          // split of the K = l*d reduction over grid.z (1: no split)
+  int kb_per_split[2];    // 64-wide K blocks per split
+  float* part[2];         // fp32 [ksplit][rows_total][H_kv][d] partial sums (ksplit > 1)
   int64_t rows_total;     // output rows (packed: sum of n_cmp)
   uint32_t* status;
   // paged caches (x_pt.table non-null): seqs.tok_off / cmp_off are then token and
@@ -68,9 +70,8 @@ struct CompressArgs {
 };
 cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
                                  float* partial, float* bias, cudaStream_t st);
-cudaError_t launch_compress_gemm(int d_in, int d_out, const CompressArgs& a, int n_tiles,
-                                 cudaStream_t st);
-cudaError_t launch_compress_finalize(int d_out, const CompressArgs& a, cudaStream_t st);
+cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, int n_tiles, cudaStream_t st);
+cudaError_t launch_compress_finalize(int d_k, int d_v, const CompressArgs& a, cudaStream_t st);
 
 // ----- prefill -----
 struct PrefillArgs {

@@ -66,7 +66,7 @@ float softmax_scale(const nsa_params_t* p, int d_k) {
 int n_blk_of(int L, int ls) { return (L + ls - 1) / ls; }
 
 // ---- workspace layouts ----
-constexpr int kMaxKSplit = 16;
+constexpr int kMaxKSplit = 4;   // more splits cost more in partial sums than they gain in CTAs
 struct CompressWs {
   size_t wt_k, wt_v, part_k, part_v, bias_k, bias_v, ksum, total;
 };
@@ -82,9 +82,8 @@ CompressWs compress_ws(const nsa_heads_t* h, const nsa_params_t* p, int64_t rows
   w.part_v = off; off = align256(off + ((Kv + 31) / 32) * h->d_v * 4);
   w.bias_k = off; off = align256(off + (size_t)h->d_k * 4);
   w.bias_v = off; off = align256(off + (size_t)h->d_v * 4);
-  w.ksum = off;
-  const size_t dmax = (size_t)(h->d_k > h->d_v ? h->d_k : h->d_v);
-  if (rows > 0) off = align256(off + (size_t)kMaxKSplit * (size_t)rows * h->H_kv * dmax * 4);
+  w.ksum = off;   // split-K partial sums of both maps: [ksplit][rows][H_kv][d_k], then the same with d_v
+  if (rows > 0) off = align256(off + (size_t)kMaxKSplit * (size_t)rows * h->H_kv * (h->d_k + h->d_v) * 4);
   w.total = off;
   return w;
 }
@@ -370,21 +369,36 @@ nsa_status_t nsa_check_device_status(void* workspace, void* stream) {
 }  // extern "C"
 
 namespace {
+// bf16 W^T and the position terms of both maps at base + (the offsets of w) - shift
+// (shift 0: a workspace; 256: a prepared blob, which has no workspace header)
+cudaError_t prepare_weights(const float* w_ck, const float* pe_k, const float* w_cv, const float* pe_v,
+                            const nsa_heads_t* heads, const nsa_params_t* params, uint8_t* base, size_t shift,
+                            const CompressWs& w, cudaStream_t st) {
+  const int Kk = params->l_cmp * heads->d_k, Kv = params->l_cmp * heads->d_v;
+  cudaError_t e = launch_compress_prep(w_ck, pe_k, Kk, heads->d_k, base + (w.wt_k - shift),
+                                       (float*)(base + (w.part_k - shift)), (float*)(base + (w.bias_k - shift)), st);
+  if (e == cudaSuccess)
+    e = launch_compress_prep(w_cv, pe_v, Kv, heads->d_v, base + (w.wt_v - shift),
+                             (float*)(base + (w.part_v - shift)), (float*)(base + (w.bias_v - shift)), st);
+  return e;
+}
+
 // nsa_compress with optional page tables for the input tokens and the output
-// summaries (both null: the plain layouts of nsa_compress)
+// summaries (both null: the plain layouts of nsa_compress) and optional prepared
+// weights (null: formed from the fp32 weights into the workspace)
 nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, const float* pe_k, const float* w_cv,
                              const float* pe_v, const int64_t* tok_offset, const int32_t* seq_len,
                              const int64_t* cmp_offset, int32_t batch, const nsa_heads_t* heads,
                              const nsa_params_t* params, void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes,
-                             void* stream, const PageTable& x_pt, const PageTable& out_pt) {
+                             void* stream, const PageTable& x_pt, const PageTable& out_pt,
+                             const uint8_t* prepared = nullptr) {
   nsa_status_t s = check_heads(heads);
   if (s != NSA_OK) return s;
   if ((s = check_params(params, false)) != NSA_OK) return s;
   if (heads->d_k != 64 && heads->d_k != 128 && heads->d_k != 192) return NSA_ERR_UNSUPPORTED;
   if (batch <= 0 || batch > NSA_MAX_BATCH) return batch <= 0 ? NSA_ERR_INVALID_ARG : NSA_ERR_UNSUPPORTED;
-  if (!k || !v || !w_ck || !pe_k || !w_cv || !pe_v || !tok_offset || !seq_len || !cmp_offset || !k_cmp ||
-      !v_cmp || !workspace)
-    return NSA_ERR_INVALID_ARG;
+  if (!k || !v || !tok_offset || !seq_len || !cmp_offset || !k_cmp || !v_cmp || !workspace) return NSA_ERR_INVALID_ARG;
+  if (!prepared && (!w_ck || !pe_k || !w_cv || !pe_v)) return NSA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(workspace))
     return NSA_ERR_INVALID_ARG;
   const CompressWs w = compress_ws(heads, params, 0);
@@ -409,15 +423,17 @@ nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, co
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int Kk = params->l_cmp * heads->d_k, Kv = params->l_cmp * heads->d_v;
-  prof_begin(P_COMPRESS_PREP, st);
-  cudaError_t e = launch_compress_prep(w_ck, pe_k, Kk, heads->d_k, ws + w.wt_k, (float*)(ws + w.part_k),
-                                       (float*)(ws + w.bias_k), st);
-  if (e == cudaSuccess)
-    e = launch_compress_prep(w_cv, pe_v, Kv, heads->d_v, ws + w.wt_v, (float*)(ws + w.part_v),
-                             (float*)(ws + w.bias_v), st);
-  prof_end(P_COMPRESS_PREP, st, 4);
-  if (e != cudaSuccess) return cuda_fail(e, "compress prep");
+  // the prepared weights: in the workspace (formed now) or the caller's blob,
+  // whose offsets are the workspace's less its 256-byte header
+  const uint8_t* wbase = prepared ? prepared : ws;
+  const size_t wshift = prepared ? 256 : 0;
+  cudaError_t e = cudaSuccess;
+  if (!prepared) {
+    prof_begin(P_COMPRESS_PREP, st);
+    e = prepare_weights(w_ck, pe_k, w_cv, pe_v, heads, params, ws, 0, w, st);
+    prof_end(P_COMPRESS_PREP, st, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "compress prep");
+  }
   if (tiles == 0) return NSA_OK;
 
   CompressArgs a{};
@@ -426,36 +442,35 @@ nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, co
   a.x_pt = x_pt;
   a.out_pt = out_pt;
   a.seqs = t;
-  a.part = (float*)(ws + w.ksum);
   a.rows_total = rows_total > 0 ? rows_total : 0;
+  a.x[0] = k; a.wt[0] = wbase + (w.wt_k - wshift); a.bias[0] = (const float*)(wbase + (w.bias_k - wshift));
+  a.x[1] = v; a.wt[1] = wbase + (w.wt_v - wshift); a.bias[1] = (const float*)(wbase + (w.bias_v - wshift));
+  a.out[0] = k_cmp;
+  a.out[1] = v_cmp;
   // split K when the row tiles alone leave SMs idle, the rows are packed and the
-  // workspace has room for the partial sums
+  // workspace has room for the partial sums of both maps
   int ks = 1;
   if (rows_total > 0) {
-    const int ctas = tiles * heads->H_kv;
+    const int ctas = tiles * heads->H_kv * 2;
     ks = (2 * 148 + ctas - 1) / ctas;
     if (ks > kMaxKSplit) ks = kMaxKSplit;
-    const size_t dmax = (size_t)(heads->d_k > heads->d_v ? heads->d_k : heads->d_v);
-    while (ks > 1 && w.ksum + (size_t)ks * rows_total * heads->H_kv * dmax * 4 > ws_bytes) ks >>= 1;
+    const size_t dsum = (size_t)(heads->d_k + heads->d_v);
+    while (ks > 1 && w.ksum + (size_t)ks * rows_total * heads->H_kv * dsum * 4 > ws_bytes) ks >>= 1;
   }
-  int launches = 0;
-  auto run = [&](const void* x, const void* wt, const float* bias, void* out, int d) -> cudaError_t {
-    a.x = x; a.wt = wt; a.bias = bias; a.out = out;
-    const int nkb = params->l_cmp * d / 64;
-    a.kb_per_split = (nkb + ks - 1) / ks;
-    a.ksplit = (nkb + a.kb_per_split - 1) / a.kb_per_split;
-    cudaError_t err = launch_compress_gemm(d, d, a, tiles, st);
-    ++launches;
-    if (err == cudaSuccess && a.ksplit > 1) {
-      err = launch_compress_finalize(d, a, st);
-      ++launches;
-    }
-    return err;
-  };
+  const int dm[2] = {heads->d_k, heads->d_v};
+  bool split = false;
+  for (int m = 0; m < 2; ++m) {
+    const int nkb = params->l_cmp * dm[m] / 64;
+    a.kb_per_split[m] = (nkb + ks - 1) / ks;
+    a.ksplit[m] = (nkb + a.kb_per_split[m] - 1) / a.kb_per_split[m];
+    split |= a.ksplit[m] > 1;
+  }
+  a.part[0] = (float*)(ws + w.ksum);
+  a.part[1] = a.part[0] + (size_t)a.ksplit[0] * a.rows_total * heads->H_kv * heads->d_k;
   prof_begin(P_COMPRESS_GEMM, st);
-  e = run(k, ws + w.wt_k, (const float*)(ws + w.bias_k), k_cmp, heads->d_k);
-  if (e == cudaSuccess) e = run(v, ws + w.wt_v, (const float*)(ws + w.bias_v), v_cmp, heads->d_v);
-  prof_end(P_COMPRESS_GEMM, st, launches);
+  e = launch_compress_gemm(heads->d_k, heads->d_v, a, tiles, st);
+  if (e == cudaSuccess && split) e = launch_compress_finalize(heads->d_k, heads->d_v, a, st);
+  prof_end(P_COMPRESS_GEMM, st, split ? 2 : 1);
   if (e != cudaSuccess) return cuda_fail(e, "compress gemm");
   return NSA_OK;
 }
@@ -471,6 +486,39 @@ nsa_status_t nsa_compress(const void* k, const void* v, const float* w_ck, const
   const PageTable none{};
   return compress_common(k, v, w_ck, pe_k, w_cv, pe_v, tok_offset, seq_len, cmp_offset, batch, heads, params, k_cmp,
                          v_cmp, workspace, ws_bytes, stream, none, none);
+}
+
+size_t nsa_compress_weights_size(const nsa_heads_t* heads, const nsa_params_t* params) {
+  if (check_heads(heads) != NSA_OK || check_params(params, false) != NSA_OK) return 0;
+  return compress_ws(heads, params, 0).ksum - 256;
+}
+
+nsa_status_t nsa_compress_prepare(const float* w_ck, const float* pe_k, const float* w_cv, const float* pe_v,
+                                  const nsa_heads_t* heads, const nsa_params_t* params, void* prepared,
+                                  size_t prepared_bytes, void* stream) {
+  nsa_status_t s = check_heads(heads);
+  if (s != NSA_OK) return s;
+  if ((s = check_params(params, false)) != NSA_OK) return s;
+  if (heads->d_k != 64 && heads->d_k != 128 && heads->d_k != 192) return NSA_ERR_UNSUPPORTED;
+  if (!w_ck || !pe_k || !w_cv || !pe_v || !prepared || (reinterpret_cast<uintptr_t>(prepared) & 255u) != 0)
+    return NSA_ERR_INVALID_ARG;
+  const CompressWs w = compress_ws(heads, params, 0);
+  if (prepared_bytes < w.ksum - 256) return NSA_ERR_WORKSPACE;
+  cudaError_t e = prepare_weights(w_ck, pe_k, w_cv, pe_v, heads, params, static_cast<uint8_t*>(prepared), 256, w,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "nsa_compress_prepare");
+  return NSA_OK;
+}
+
+nsa_status_t nsa_compress_prepared(const void* k, const void* v, const void* prepared,
+                                   const int64_t* tok_offset, const int32_t* seq_len, const int64_t* cmp_offset,
+                                   int32_t batch, const nsa_heads_t* heads, const nsa_params_t* params,
+                                   void* k_cmp, void* v_cmp, void* workspace, size_t ws_bytes, void* stream) {
+  if (!prepared || (reinterpret_cast<uintptr_t>(prepared) & 255u) != 0) return NSA_ERR_INVALID_ARG;
+  const PageTable none{};
+  return compress_common(k, v, nullptr, nullptr, nullptr, nullptr, tok_offset, seq_len, cmp_offset, batch, heads,
+                         params, k_cmp, v_cmp, workspace, ws_bytes, stream, none, none,
+                         static_cast<const uint8_t*>(prepared));
 }
 
 nsa_status_t nsa_compress_paged(const void* k_pool, const void* v_pool, int32_t n_pages, int32_t page_size,

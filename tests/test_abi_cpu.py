@@ -122,6 +122,30 @@ def test_decode_and_compress_validation(L):
                           None) == nsa.NSA_ERR_WORKSPACE
 
 
+def test_prepared_weights_validate_on_host(L):
+    """The prepared-weights entry points size their blob and reject bad arguments
+    before any launch (fake device pointers are never dereferenced)."""
+    h = nsa.Heads(64, 4, 192, 128)
+    p = nsa.make_params()
+    n = L.nsa_compress_weights_size(ctypes.byref(h), ctypes.byref(p))
+    # bf16 W^T of both maps and the fp32 position terms at least
+    assert n >= 2 * (32 * 192 * 192 + 32 * 128 * 128) + 4 * (192 + 128)
+    assert L.nsa_compress_weights_size(ctypes.byref(nsa.Heads(64, 5, 192, 128)), ctypes.byref(p)) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.nsa_compress_prepare(fake, fake, fake, fake, ctypes.byref(h), ctypes.byref(p), None, n,
+                                  None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_prepare(fake, fake, fake, fake, ctypes.byref(h), ctypes.byref(p),
+                                  ctypes.c_void_p((1 << 20) + 16), n, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_prepare(fake, fake, fake, fake, ctypes.byref(h), ctypes.byref(p), fake, n - 1,
+                                  None) == nsa.NSA_ERR_WORKSPACE
+    i64 = (ctypes.c_int64 * 1)(0)
+    i32 = (ctypes.c_int32 * 1)(100)
+    assert L.nsa_compress_prepared(fake, fake, None, i64, i32, i64, 1, ctypes.byref(h), ctypes.byref(p), fake, fake,
+                                   fake, 1 << 30, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_prepared(fake, fake, fake, i64, i32, i64, 1, ctypes.byref(h), ctypes.byref(p), fake, fake,
+                                   fake, 8, None) == nsa.NSA_ERR_WORKSPACE
+
+
 def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(nsa, "_lib", None)
     monkeypatch.setattr(nsa, "LIB_PATH", "/nonexistent/libnsa.so")

@@ -93,6 +93,24 @@ def test_prefill_importance_through_workspace():
     NP.run_prefill_case(cfg, [80000], n_random_rows=128)
 
 
+def test_compress_prepared_weights_match():
+    """nsa_compress_prepared with weights from nsa_compress_prepare writes the same
+    bits as nsa_compress (the same conversion, once instead of per call), over
+    several sequences, for two head shapes."""
+    for cfg_name, seqlens in (("prefill_8k", [1500, 64, 700, 31]), ("prefill_tiny_1k", [1024, 333])):
+        cfg = CFG[cfg_name]
+        heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+        inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=31)
+        args = (inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], seqlens, heads, par)
+        kc, vc = nsa.compress(*args)
+        prepared = nsa.compress_prepare(inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], heads, par)
+        for _ in range(2):   # the blob is read, not consumed
+            kp, vp = nsa.compress(*args, prepared=prepared)
+            torch.cuda.synchronize()
+            assert torch.equal(kp.view(torch.int16), kc.view(torch.int16))
+            assert torch.equal(vp.view(torch.int16), vc.view(torch.int16))
+
+
 def test_prefill_exact_ties_register_topn():
     """All compressed keys zero (exact ties between interior blocks) on the
     register top-n path of the prefill (GQA 16 and GQA 4)."""
