@@ -13,8 +13,8 @@
 // thread), read back with tcgen05.ld for the bias-add + bf16 epilogue. When the
 // rows give too few CTAs to fill the GPU, the K = l*d_in reduction is split over
 // grid.z into fp32 partial sums that a small kernel adds in a fixed order.
-// Operand rows are a strided gather (row i starts at token i*s), so they are
-// fetched with cp.async rather than a tensor map.
+// The A rows are a strided gather (row i starts at token i*s), fetched with
+// cp.async (one thread per row); the B tile (64 columns of W^T) is one TMA box.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -101,12 +101,13 @@ __device__ __forceinline__ int find_seq(const SeqTable& t, int tile) {
 
 // one map (m = 0 keys, 1 values) of KV head g
 template <int D_IN, int D_OUT>
-__device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m, int g) {
+__device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, const CompressMaps& mp, int m, int g) {
   using S = CompressSmem<D_OUT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + kCmpStages * S::STAGE);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + kCmpStages + 1);
+  uint64_t* b_full = mma_done + kCmpStages + 1;   // the B tile of a stage has landed (TMA)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_full + kCmpStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -123,6 +124,8 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
 
   if (tid == 0) {
     for (int i = 0; i <= kCmpStages; ++i) mbar_init(&mma_done[i], 1);
+    for (int i = 0; i < kCmpStages; ++i) mbar_init(&b_full[i], 1);
+    prefetch_tmap(&mp.w[m]);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -133,7 +136,6 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
   const uint32_t tmem_d = *tmem_slot;
 
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x[m]);
-  const __nv_bfloat16* wt = static_cast<const __nv_bfloat16*>(a.wt[m]);
   const size_t row_stride = (size_t)a.H_kv * D_IN;   // elements between tokens
 
   auto load_stage = [&](int st, int kb) {
@@ -160,15 +162,16 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
 #pragma unroll
       for (int c = 0; c < 8; ++c) cp_async16_zfill(A + sw128(row, c), src + c * 8, ok);
     }
-    // B: D_OUT rows of W^T, 8 chunks each
-    for (int idx = tid; idx < D_OUT * 8; idx += 128) {
-      const int n = idx >> 3, c = idx & 7;
-      cp_async16(Bm + sw128(n, c), wt + (size_t)n * K + f0 + c * 8);
+    // B: the 64 columns of all D_OUT rows of W^T, one TMA box (128-byte swizzle)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&b_full[st], (uint32_t)S::B_BYTES);
+      tma_load_3d(Bm, &mp.w[m], &b_full[st], f0, 0, 0);
     }
   };
 
   const uint32_t idesc = umma_idesc_bf16(kTileM, D_OUT, false, false);
   bool ok = true;
+  int loaded = 0;   // K blocks whose loads were issued
   for (int kb = 0; kb < nkb + kCmpStages - 1; ++kb) {
     if (kb < nkb) {
       const int st = kb % kCmpStages;
@@ -177,7 +180,10 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
           ok = false;
         }
       }
-      if (ok) load_stage(st, kb);
+      if (ok) {
+        load_stage(st, kb);
+        loaded = kb + 1;
+      }
     }
     cp_async_commit();
     const int c = kb - (kCmpStages - 1);
@@ -186,6 +192,11 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
       fence_proxy_async_smem();
       __syncthreads();
       if (*abort_flag) { ok = false; break; }
+      if (tid == 0) {
+        const int st = c % kCmpStages;
+        if (!mbar_wait(&b_full[st], (c / kCmpStages) & 1, abort_flag, a.status, 104)) ok = false;
+      }
+      if (__syncthreads_or(!ok)) { ok = false; break; }
       if (tid == 0) {
         tc_fence_after();
         const int st = c % kCmpStages;
@@ -203,8 +214,13 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
   }
   cp_async_wait<0>();
   // all MMAs done: commit a final barrier (also on the abort path, so that no
-  // product is still running when tensor memory is released)
-  if (tid == 0) umma_commit(&mma_done[kCmpStages]);
+  // product is still running when tensor memory is released); the B tiles still
+  // in flight land first
+  if (tid == 0) {
+    for (int v = loaded - kCmpStages < 0 ? 0 : loaded - kCmpStages; v < loaded; ++v)
+      mbar_wait_drain(&b_full[v % kCmpStages], (v / kCmpStages) & 1);
+    umma_commit(&mma_done[kCmpStages]);
+  }
   __syncthreads();
   if (ok && !*abort_flag) ok = mbar_wait(&mma_done[kCmpStages], 0, abort_flag, a.status, 102);
   else if (tid == 0) mbar_wait_drain(&mma_done[kCmpStages], 0);
@@ -254,22 +270,23 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, int m,
 // keys and values of every KV head in one launch (grid.y = 2 H_kv); a CTA whose
 // split index is beyond its map's split count has nothing to do
 template <int DK, int DV>
-__global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArgs a) {
+__global__ void __launch_bounds__(128, 1) compress_gemm_kernel(const CompressArgs a,
+                                                                const __grid_constant__ CompressMaps mp) {
   const int m = blockIdx.y >= a.H_kv ? 1 : 0;
   if ((int)blockIdx.z >= a.ksplit[m]) return;
-  if (m == 0) compress_gemm_body<DK, DK>(a, 0, blockIdx.y);
-  else compress_gemm_body<DV, DV>(a, 1, blockIdx.y - a.H_kv);
+  if (m == 0) compress_gemm_body<DK, DK>(a, mp, 0, blockIdx.y);
+  else compress_gemm_body<DV, DV>(a, mp, 1, blockIdx.y - a.H_kv);
 }
 
 template <int DK, int DV>
-static cudaError_t launch_gemm_t(const CompressArgs& a, int n_tiles, cudaStream_t st) {
+static cudaError_t launch_gemm_t(const CompressArgs& a, const CompressMaps& mp, int n_tiles, cudaStream_t st) {
   constexpr int smem = CompressSmem<DK>::TOTAL > CompressSmem<DV>::TOTAL ? CompressSmem<DK>::TOTAL
                                                                         : CompressSmem<DV>::TOTAL;
   auto kern = compress_gemm_kernel<DK, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles, 2 * a.H_kv, a.ksplit[0] > a.ksplit[1] ? a.ksplit[0] : a.ksplit[1]);
-  kern<<<grid, 128, smem, st>>>(a);
+  kern<<<grid, 128, smem, st>>>(a, mp);
   return cudaGetLastError();
 }
 
@@ -305,10 +322,11 @@ cudaError_t launch_compress_finalize(int d_k, int d_v, const CompressArgs& a, cu
   return cudaGetLastError();
 }
 
-cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, int n_tiles, cudaStream_t st) {
+cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, const CompressMaps& mp, int n_tiles,
+                                 cudaStream_t st) {
   if (n_tiles <= 0) return cudaSuccess;
 #define NSA_CMP_CASE(DK, DV) \
-  if (d_k == DK && d_v == DV) return launch_gemm_t<DK, DV>(a, n_tiles, st);
+  if (d_k == DK && d_v == DV) return launch_gemm_t<DK, DV>(a, mp, n_tiles, st);
   NSA_CMP_CASE(192, 128) NSA_CMP_CASE(64, 64) NSA_CMP_CASE(128, 128) NSA_CMP_CASE(192, 64)
   NSA_CMP_CASE(64, 128) NSA_CMP_CASE(128, 64) NSA_CMP_CASE(192, 192) NSA_CMP_CASE(128, 192) NSA_CMP_CASE(64, 192)
 #undef NSA_CMP_CASE

@@ -70,7 +70,11 @@ struct CompressArgs {
 };
 cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, void* wt_bf16,
                                  float* partial, float* bias, cudaStream_t st);
-cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, int n_tiles, cudaStream_t st);
+struct CompressMaps {
+  CUtensorMap w[2];   // W^T of both maps: boxes of 64 columns x all d rows (128-byte swizzle)
+};
+cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, const CompressMaps& mp, int n_tiles,
+                                 cudaStream_t st);
 cudaError_t launch_compress_finalize(int d_k, int d_v, const CompressArgs& a, cudaStream_t st);
 
 // ----- prefill -----

@@ -467,8 +467,16 @@ nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, co
   }
   a.part[0] = (float*)(ws + w.ksum);
   a.part[1] = a.part[0] + (size_t)a.ksplit[0] * a.rows_total * heads->H_kv * heads->d_k;
+  // W^T of both maps in boxes of 64 columns x d rows
+  CompressMaps mp;
+  memset(&mp, 0, sizeof(mp));
+  if (!make_map_3d(&mp.w[0], a.wt[0], params->l_cmp * heads->d_k, 1, heads->d_k, 1, heads->d_k) ||
+      !make_map_3d(&mp.w[1], a.wt[1], params->l_cmp * heads->d_v, 1, heads->d_v, 1, heads->d_v)) {
+    snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed (compression)");
+    return NSA_ERR_CUDA;
+  }
   prof_begin(P_COMPRESS_GEMM, st);
-  e = launch_compress_gemm(heads->d_k, heads->d_v, a, tiles, st);
+  e = launch_compress_gemm(heads->d_k, heads->d_v, a, mp, tiles, st);
   if (e == cudaSuccess && split) e = launch_compress_finalize(heads->d_k, heads->d_v, a, st);
   prof_end(P_COMPRESS_GEMM, st, split ? 2 : 1);
   if (e != cudaSuccess) return cuda_fail(e, "compress gemm");
