@@ -328,7 +328,7 @@ cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, const 
 #define NSA_CMP_CASE(DK, DV) \
   if (d_k == DK && d_v == DV) return launch_gemm_t<DK, DV>(a, mp, n_tiles, st);
   NSA_CMP_CASE(192, 128) NSA_CMP_CASE(64, 64) NSA_CMP_CASE(128, 128) NSA_CMP_CASE(192, 64)
-  NSA_CMP_CASE(64, 128) NSA_CMP_CASE(128, 64) NSA_CMP_CASE(192, 192) NSA_CMP_CASE(128, 192) NSA_CMP_CASE(64, 192)
+  NSA_CMP_CASE(64, 128) NSA_CMP_CASE(128, 64)
 #undef NSA_CMP_CASE
   return cudaErrorInvalidValue;
 }

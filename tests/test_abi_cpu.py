@@ -146,6 +146,18 @@ def test_prepared_weights_validate_on_host(L):
                                    fake, 8, None) == nsa.NSA_ERR_WORKSPACE
 
 
+def test_unsupported_head_sizes_rejected_on_host(L):
+    """A value head size of 192 (or any size outside the built ones) is rejected
+    before any launch."""
+    P = ctypes.c_void_p(16)
+    i64 = (ctypes.c_int64 * 1)(0)
+    i32 = (ctypes.c_int32 * 1)(100)
+    p = nsa.make_params()
+    for h in (nsa.Heads(8, 2, 64, 192), nsa.Heads(8, 2, 192, 192), nsa.Heads(8, 2, 96, 64)):
+        assert L.nsa_compress(P, P, P, P, P, P, i64, i32, i64, 1, ctypes.byref(h), ctypes.byref(p), P, P, P,
+                              1 << 30, None) == nsa.NSA_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(nsa, "_lib", None)
     monkeypatch.setattr(nsa, "LIB_PATH", "/nonexistent/libnsa.so")

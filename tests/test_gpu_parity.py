@@ -172,6 +172,34 @@ def test_prefill_deterministic():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("d_k,d_v", [(dk, dv) for dk in (64, 128, 192) for dv in (64, 128)])
+def test_compress_every_head_size_pair(d_k, d_v):
+    """Keys and values of every supported (d_k, d_v) pair share one GEMM launch
+    (one instantiation per pair; d_v = 192 is rejected on the host, checked in
+    the CPU tests): both maps against the fp64 oracle over two
+    sequences, one of them with a ragged tail; the K reduction is split (few row
+    tiles)."""
+    seqlens = [600, 77]
+    cfg = W.small_config(T=sum(seqlens), H_q=8, H_kv=2, d_k=d_k, d_v=d_v, seed=41)
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    inp = W.make_prefill_inputs(cfg, device="cuda", seqlens=seqlens, seed=41)
+    kc, vc = nsa.compress(inp["k"], inp["v"], inp["w_ck"], inp["pe_k"], inp["w_cv"], inp["pe_v"], seqlens, heads,
+                          par)
+    torch.cuda.synchronize()
+    op = NP.oracle_params(cfg)
+    w_ck, pe_k, w_cv, pe_v = (NP.f64(inp[x]) for x in ("w_ck", "pe_k", "w_cv", "pe_v"))
+    t0 = c0 = 0
+    for L in seqlens:
+        nc = nsa.n_cmp(L, par.l_cmp, par.stride)
+        kb, vb = NP.f64(inp["k"][t0:t0 + L]), NP.f64(inp["v"][t0:t0 + L])
+        NP.assert_close(NP.f64(kc[c0:c0 + nc]), O.compress(kb, w_ck, pe_k, op["l_cmp"], op["stride"]),
+                        f"k_cmp d_k={d_k}", relative_to_rms=True)
+        NP.assert_close(NP.f64(vc[c0:c0 + nc]), O.compress(vb, w_cv, pe_v, op["l_cmp"], op["stride"]),
+                        f"v_cmp d_v={d_v}", relative_to_rms=True)
+        t0 += L
+        c0 += nc
+
+
 def test_compress_mean_pool_on_gpu():
     """Averaging weights, no position embedding, stride = block: the compressed
     keys are the block means (up to bf16 rounding of the weights 1/32)."""
