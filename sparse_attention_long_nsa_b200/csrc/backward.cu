@@ -68,8 +68,6 @@ struct BqSmem {
   static constexpr int K_BYTES = kBqKeys * DK * 2;
   static constexpr int V_BYTES = kBqKeys * DV * 2;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int ROWS = kBqWarps * 3 * 16 * 2 * 4;   // per-warp lse / <dout,O> of each branch
-  static constexpr int FIXED = Q_BYTES + DO_BYTES + kBqStages * STAGE + ROWS + 256 * 8 + 512;
 };
 
 // dout . O over the lane's two rows (o normalised by 1/l), from the bf16 dout

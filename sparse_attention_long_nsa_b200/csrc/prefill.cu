@@ -16,10 +16,10 @@
 //   C1  compressed keys, pass 1: row max and softmax denominator
 //   C2  compressed keys, pass 2: normalised probabilities p; importance of every
 //       selection block (p spread by token overlap, summed over the group's
-//       heads); O_A = g_cmp * P.V_cmp
+//       heads); O_A = P.V_cmp
 //   --  top-n per token (forced first / local blocks, ties to the lower index),
 //       union of the tile's selections
-//   W   window keys, online softmax into O_B; O_A += g_win / l * O_B
+//   W   window keys, online softmax into O_B; O_A = g_cmp O_A + g_win / l * O_B
 //   S   union blocks, each row masked to its own token's selection (and to
 //       keys <= t inside the current block); online softmax into O_B;
 //       out = bf16(O_A + g_slc / l * O_B)
@@ -606,20 +606,21 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       lp = lp * ex2((m - mn) * sc) + tree_sum<32>(sv);
       m = mn;
     }
-    float linv = 0.f, mo_c = 0.f;
-    if (nkc > 0) {   // merge the two warps' (max, sum) in a fixed order
+    // p = 2^(s sc - m sc - log2 l): the denominator is folded into the exponent
+    // (-inf when no compressed key is visible: p = 0)
+    float mo_c = -INFINITY;
+    if (nkc > 0) {   // merge the two key halves' (max, sum) in a fixed order
       const float m_o = exchange(m);
       const float l_o = exchange(lp);
       const float m0 = kh == 0 ? m : m_o, m1 = kh == 0 ? m_o : m;
       const float l0 = kh == 0 ? lp : l_o, l1 = kh == 0 ? l_o : lp;
       const float mm = fmaxf(m0, m1);
       const float lc = l0 * ex2((m0 - mm) * sc) + l1 * ex2((m1 - mm) * sc);
-      linv = lc > 0.f ? 1.f / lc : 0.f;
-      mo_c = -mm * sc;
+      mo_c = lc > 0.f ? -mm * sc - log2f(lc) : -INFINITY;
     }
 
     TRP(1);
-    // ---------------- C2: probabilities, importance, O_A = g_cmp * P.V_cmp
+    // ---------------- C2: probabilities, importance, O_A = P.V_cmp (g_cmp applied in the W merge)
     // compressed key i' = 4u' + u spans tokens [16i', 16i' + 32): u in {0,1,2} puts
     // 2p on selection block u', u = 3 puts p on u' and u' + 1 (overlap / stride).
     // The 32 keys of a warp cover 8 selection blocks; the mass its last key
@@ -635,8 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         for (int c = 0; c < 32; ++c) sv[c] = (c0 + c < nvis) ? sv[c] : -INFINITY;
       }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo_c)) * linv;
-      if (ok) st32(gc);
+      for (int c = 0; c < 32; ++c) sv[c] = ex2(fmaf(sv[c], sc, mo_c));
+      if (ok) st32(1.f);
       TR(j, 1);
       const bool wr = valid && ok;
       const int B0 = 16 * i + 8 * kh;
@@ -761,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       return kh == 0 ? lp + other : other + lp;
     };
 
-    // ---------------- W: window keys into O_B, then O_A += g_win / l * O_B
+    // ---------------- W: window keys into O_B, then O_A = g_cmp O_A + g_win / l * O_B
     const int wlo = t - a.window + 1;
     lp = 0.f;
     for (int i = 0; i < nkw; ++i) {
@@ -792,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = __float_as_uint((nkc > 0 ? oa[e] : 0.f) + sw * ob[e]);
+        for (int e = 0; e < 16; ++e) w[e] = __float_as_uint((nkc > 0 ? gc * oa[e] : 0.f) + sw * ob[e]);
         tmem_st8_h<DV / 2>(tmem + kColOA + cb, w);
         tmem_st8_h<DV / 2>(tmem + kColOA + cb + 8, w + 8);
       }
