@@ -65,6 +65,7 @@ struct FBars {
   uint32_t tmem_base;
   int abort;
   int nu;
+  int ucnt[8];   // blocks per softmax warp's range of the union
 };
 
 __device__ __forceinline__ int seq_of_tile(const SeqTable& t, int tile) {
@@ -695,18 +696,31 @@ __global__ void __launch_bounds__(kThreads, 1) nsa_prefill_kernel(const PrefillA
       }
     }
     sm_sync();
-    if (warp == 0 && ok) {
-      int cnt = 0;
-      for (int j0 = 0; j0 <= jt_max; j0 += 32) {
-        const int jb = j0 + lane;
+    // the union of the tile's selections, ascending: each softmax warp takes a
+    // contiguous range of 32-block chunks, counts its blocks, and after a sync
+    // writes them at the offset of the warps before it
+    {
+      const int nch32 = (jt_max + 32) / 32, cpw = (nch32 + 7) / 8;
+      const int c_lo = min(nch32, warp * cpw), c_hi = min(nch32, c_lo + cpw);
+      auto chunk_bits = [&](int c) -> uint32_t {
+        const int jb = c * 32 + lane;
         bool any = false;
         if (jb <= jt_max)
           for (int w = 0; w < MW; ++w) any |= bm[jb * MW + w] != 0u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, any);
-        if (any) uni[cnt + __popc(bal & ((1u << lane) - 1u))] = jb;
-        cnt += __popc(bal);
+        return __ballot_sync(0xffffffffu, any);
+      };
+      int cnt = 0;
+      for (int c = c_lo; c < c_hi; ++c) cnt += __popc(chunk_bits(c));
+      if (lane == 0) bars->ucnt[warp] = cnt;
+      sm_sync();
+      int off = 0;
+      for (int w = 0; w < warp; ++w) off += bars->ucnt[w];
+      for (int c = c_lo; c < c_hi; ++c) {
+        const uint32_t bal = chunk_bits(c);
+        if ((bal >> lane) & 1u) uni[off + __popc(bal & ((1u << lane) - 1u))] = c * 32 + lane;
+        off += __popc(bal);
       }
-      if (lane == 0) bars->nu = cnt;
+      if (warp == 7 && lane == 0) bars->nu = off;   // the total: warp 7's range ends last
     }
     sm_sync();
     TRP(3);

@@ -86,6 +86,59 @@ __device__ __forceinline__ void warp_topn(const float* imp, int jt, int top_n, i
   for (int i = pos + lane; i < top_n; i += 32) out[i] = -1;
 }
 
+// Same selection with the scores in registers (PER per lane, block i*32 + lane in
+// key[i]) and the threshold found by a 32-step radix search over the order keys
+// instead of arg-max rounds: every step counts the keys at or above a candidate
+// threshold with one warp reduction, so the chain is 32 short steps whatever the
+// number of free slots. Then every key above the threshold and the first equal
+// ones in block order are taken (ties to the lower index), output ascending.
+template <int PER>
+__device__ __forceinline__ void warp_topn_radix(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
+                                                int lane) {
+  const int K = jt + 1;
+  if (K <= top_n) {
+    for (int i = lane; i < top_n; i += 32) out[i] = i < K ? i : -1;
+    return;
+  }
+  const int need = top_n - ff - fl;   // K > top_n >= ff + fl: forced sets are disjoint
+  uint32_t key[PER];
+  uint32_t forced = 0u;   // bit i: block i*32 + lane is forced
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = i * 32 + lane;
+    const bool cand = j < K && j >= ff && j <= jt - fl;
+    key[i] = cand ? order_key(imp[j]) : 0u;   // every real score maps above 0
+    if (j < K && (j < ff || j > jt - fl)) forced |= 1u << i;
+  }
+  uint32_t x = 0u;   // the need-th largest key
+  if (need > 0) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t y = x | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) c += key[i] >= y ? 1 : 0;
+      if ((int)__reduce_add_sync(0xffffffffu, (uint32_t)c) >= need) x = y;
+    }
+  }
+  int gt = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) gt += (need > 0 && key[i] > x) ? 1 : 0;
+  int ties_left = need - (int)__reduce_add_sync(0xffffffffu, (uint32_t)gt);
+  int pos = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const bool eq = need > 0 && key[i] == x && key[i] != 0u;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take_eq = eq && __popc(eqm & ((1u << lane) - 1u)) < ties_left;
+    ties_left -= min(__popc(eqm), max(ties_left, 0));
+    const bool chosen = ((forced >> i) & 1u) || (need > 0 && key[i] > x) || take_eq;
+    const uint32_t cm = __ballot_sync(0xffffffffu, chosen);
+    if (chosen) out[pos + __popc(cm & ((1u << lane) - 1u))] = i * 32 + lane;
+    pos += __popc(cm);
+  }
+  for (int i = pos + lane; i < top_n; i += 32) out[i] = -1;
+}
+
 // Same selection for any jt, reading the scores from memory on every pass
 // instead of holding them in registers (used beyond 1024 candidate blocks).
 __device__ __forceinline__ void warp_topn_mem(const float* imp, int jt, int top_n, int ff, int fl, int32_t* out,
@@ -140,8 +193,8 @@ __device__ __forceinline__ void warp_topn_any(const float* imp, int jt, int top_
   else if (per <= 2) warp_topn<2>(imp, jt, top_n, ff, fl, out, lane);
   else if (per <= 4) warp_topn<4>(imp, jt, top_n, ff, fl, out, lane);
   else if (per <= 8) warp_topn<8>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 16) warp_topn<16>(imp, jt, top_n, ff, fl, out, lane);
-  else if (per <= 32) warp_topn<32>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 16) warp_topn_radix<16>(imp, jt, top_n, ff, fl, out, lane);
+  else if (per <= 32) warp_topn_radix<32>(imp, jt, top_n, ff, fl, out, lane);
   else warp_topn_mem(imp, jt, top_n, ff, fl, out, lane);
 }
 

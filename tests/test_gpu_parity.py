@@ -119,6 +119,15 @@ def test_prefill_exact_ties_register_topn():
         assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
 
 
+def test_prefill_exact_ties_register_radix_topn():
+    """All compressed keys zero at 40,000 tokens (625 candidate blocks, the
+    register radix top-n): interior blocks tie exactly and the lowest indices
+    must win."""
+    cfg = W.small_config(name="prefill_40k", T=40000, H_q=64, H_kv=4, d_k=192, d_v=128, seed=1007)
+    st = NP.run_prefill_case(cfg, [40000], n_random_rows=64, k_cmp_fn=_zero_keys)
+    assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
+
+
 def _dense_ref(inp, G, scale):
     q = inp["q"].double().permute(1, 0, 2)[None]
     k = inp["k"].double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
