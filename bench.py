@@ -54,10 +54,10 @@ NCU_TRAFFIC = {
     # 64K prefill: captured on the same kernel with one KV group (H_q=16, H_kv=1,
     # bench.py --case prefill64k_g1); the CTAs of different KV groups touch disjoint
     # rows of q, k, v, out and the importance rows, so a launch's traffic is 4x
-    ("prefill_attn", "prefill_64k"): dict(bytes=(461.869824e6 + 258.854912e6) * 4, src="prefill.cu",
-                                          sha1="c9c8d330971ef494595604d121cfa62c60cfd170"),
-    ("prefill_attn", "prefill_8k"): dict(bytes=232.406272e6 + 104.760832e6, src="prefill.cu",
-                                         sha1="c9c8d330971ef494595604d121cfa62c60cfd170"),
+    ("prefill_attn", "prefill_64k"): dict(bytes=(461.753856e6 + 258.821632e6) * 4, src="prefill.cu",
+                                          sha1="07cb49eb164ddb0d6a742f1adc53272e9921193a"),
+    ("prefill_attn", "prefill_8k"): dict(bytes=232.378368e6 + 102.237440e6, src="prefill.cu",
+                                         sha1="07cb49eb164ddb0d6a742f1adc53272e9921193a"),
     ("dec_cmp", "decode_64k"): dict(bytes=(84.101120e6 + 2.445312e6) * 32 / 8, src="decode.cu",
                                     sha1="50df1c75c656cb16dff4c30e0bf690d06dd95c02"),
 }
