@@ -347,7 +347,7 @@ def bench_prefill(cfg, args, rank, ws, dev, pk, e2e=False, clocks=False):
             "frac": (achieved / pk["tc"]) if achieved else None,
             "peak_source": f"{pk['src']} bf16 dense (burst)",
             # the same against NVIDIA's dense bf16 figure (2.25 PFLOP/s), for context;
-            # `frac` (measured cuBLAS burst) is the figure targets are judged on
+            # `frac` (measured cuBLAS burst) is the figure the targets refer to
             "frac_vs_2250_nominal": (achieved / 2250.0) if achieved else None,
             "traffic": ncu_traffic(dominant, cfg.name),
             "ms_per_launch": dom_ms,

@@ -1,7 +1,8 @@
 """Plain float64 CPU oracle for the NSA (Native Sparse Attention) forward pass.
 
-TEST INFRASTRUCTURE ONLY. This module is the checker, not the product: only the
-tests, the package's smoke check and the bench's CPU-baseline leg may import it.
+TEST INFRASTRUCTURE ONLY. This module is the reference the kernels are checked
+against, not the product: only the tests, the package's smoke check and the
+bench's CPU-baseline leg may import it.
 It shares no code with the CUDA path (no kernels, headers, helpers or tables) and
 imports nothing from it.
 

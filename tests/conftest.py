@@ -14,7 +14,7 @@ def pytest_configure(config):
 
 def pytest_collection_modifyitems(config, items):
     # GPU tests are skipped (not failed) when no device is present, so the CPU
-    # suite stays green; on a GPU machine they run for real.
+    # suite stays green; on a machine with a GPU they run for real.
     try:
         import torch
         has_gpu = torch.cuda.is_available()
