@@ -13,8 +13,10 @@
 // thread), read back with tcgen05.ld for the bias-add + bf16 epilogue. When the
 // rows give too few CTAs to fill the GPU, the K = l*d_in reduction is split over
 // grid.z into fp32 partial sums that a small kernel adds in a fixed order.
-// The A rows are a strided gather (row i starts at token i*s), fetched with
-// cp.async (one thread per row); the B tile (64 columns of W^T) is one TMA box.
+// The A rows are a strided gather (row i starts at token i*s): one TMA box over a
+// (channel, token mod s, token div s) view of the packed tokens, or cp.async rows
+// (paged input, last partial group of s tokens); the B tile (64 columns of W^T)
+// is one TMA box.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -138,11 +140,27 @@ __device__ __forceinline__ void compress_gemm_body(const CompressArgs& a, const 
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x[m]);
   const size_t row_stride = (size_t)a.H_kv * D_IN;   // elements between tokens
 
+  // The A tile of a K block (token offset r) is rows i0 .. i0+127 of the view
+  // (channel, token mod s, token div s) of the packed tokens: one TMA box when
+  // every row this CTA writes lies in whole groups of s tokens inside the view
+  // (rows past its end read zeros and are never written out); otherwise (paged
+  // input, or a last partial group) one cp.async row per thread.
+  const int64_t last_tok = tok0 + (int64_t)(min(i0 + kTileM, ncmp) - 1) * a.s + a.l - 1;
+  const bool a_tma = a.x_chunks > 0 && !a.x_pt.table && last_tok < (int64_t)a.x_chunks * a.s;
   auto load_stage = [&](int st, int kb) {
     uint8_t* A = smem + st * S::STAGE;
     uint8_t* Bm = A + S::A_BYTES;
     const int f0 = (kb0 + kb) * 64;
     const int r = f0 / D_IN, e0 = f0 % D_IN;
+    if (a_tma) {
+      if (tid == 0) {
+        const int64_t t_row0 = tok0 + (int64_t)i0 * a.s + r;   // token of row i0
+        mbar_arrive_expect_tx(&b_full[st], (uint32_t)(S::A_BYTES + S::B_BYTES));
+        tma_load_3d(A, &mp.x[m], &b_full[st], g * D_IN + e0, (int)(t_row0 % a.s), (int)(t_row0 / a.s));
+        tma_load_3d(Bm, &mp.w[m], &b_full[st], f0, 0, 0);
+      }
+      return;
+    }
     {  // A: one 128-byte row per thread
       const int row = tid;
       const int ci = i0 + row;

@@ -62,6 +62,7 @@ struct CompressArgs {
   int kb_per_split[2];    // 64-wide K blocks per split
   float* part[2];         // fp32 [ksplit][rows_total][H_kv][d] partial sums (ksplit > 1)
   int64_t rows_total;     // output rows (packed: sum of n_cmp)
+  int x_chunks;           // whole groups of s tokens in the x view (0: no view, cp.async rows)
   uint32_t* status;
   // paged caches (x_pt.table non-null): seqs.tok_off / cmp_off are then token and
   // entry indices within sequence b, mapped through the tables
@@ -72,6 +73,7 @@ cudaError_t launch_compress_prep(const float* w, const float* pe, int K, int N, 
                                  float* partial, float* bias, cudaStream_t st);
 struct CompressMaps {
   CUtensorMap w[2];   // W^T of both maps: boxes of 64 columns x all d rows (128-byte swizzle)
+  CUtensorMap x[2];   // keys / values as (channel, token mod s, token div s): boxes of 64 channels x 128 rows
 };
 cudaError_t launch_compress_gemm(int d_k, int d_v, const CompressArgs& a, const CompressMaps& mp, int n_tiles,
                                  cudaStream_t st);

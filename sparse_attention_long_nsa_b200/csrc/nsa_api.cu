@@ -190,6 +190,23 @@ bool make_map_3d(CUtensorMap* m, const void* base, int dim, int heads, int64_t r
   return r == CUDA_SUCCESS;
 }
 
+// The packed tokens [rows, heads, dim] viewed as (channel, token mod s, token
+// div s) over the first `chunks` whole groups of s tokens: a box of 64 channels
+// x 1 x 128 groups holds 128 rows that start s tokens apart (128-byte swizzle).
+bool make_map_xview(CUtensorMap* m, const void* base, int dim, int heads, int s, int64_t chunks) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t c = (cuuint64_t)dim * heads;
+  cuuint64_t gdim[3] = {c, (cuuint64_t)s, (cuuint64_t)chunks};
+  cuuint64_t gstride[2] = {c * 2, c * 2 * (cuuint64_t)s};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---- opt-in profiler ----
 struct ProfRec {
   int slot, launches;
@@ -467,13 +484,25 @@ nsa_status_t compress_common(const void* k, const void* v, const float* w_ck, co
   }
   a.part[0] = (float*)(ws + w.ksum);
   a.part[1] = a.part[0] + (size_t)a.ksplit[0] * a.rows_total * heads->H_kv * heads->d_k;
-  // W^T of both maps in boxes of 64 columns x d rows
+  // W^T of both maps in boxes of 64 columns x d rows; k and v as views of whole
+  // groups of s tokens up to the end of the last sequence (contiguous input only)
   CompressMaps mp;
   memset(&mp, 0, sizeof(mp));
   if (!make_map_3d(&mp.w[0], a.wt[0], params->l_cmp * heads->d_k, 1, heads->d_k, 1, heads->d_k) ||
       !make_map_3d(&mp.w[1], a.wt[1], params->l_cmp * heads->d_v, 1, heads->d_v, 1, heads->d_v)) {
     snprintf(g_detail, sizeof(g_detail), "cuTensorMapEncodeTiled failed (compression)");
     return NSA_ERR_CUDA;
+  }
+  a.x_chunks = 0;
+  if (!x_pt.table) {
+    int64_t rows_x = 0;
+    for (int bb = 0; bb < batch; ++bb)
+      if (tok_offset[bb] + seq_len[bb] > rows_x) rows_x = tok_offset[bb] + seq_len[bb];
+    const int64_t chunks = rows_x / params->stride;
+    if (chunks > 0 && chunks < (int64_t)1 << 31 &&
+        make_map_xview(&mp.x[0], k, heads->d_k, heads->H_kv, params->stride, chunks) &&
+        make_map_xview(&mp.x[1], v, heads->d_v, heads->H_kv, params->stride, chunks))
+      a.x_chunks = (int)chunks;
   }
   prof_begin(P_COMPRESS_GEMM, st);
   e = launch_compress_gemm(heads->d_k, heads->d_v, a, mp, tiles, st);
