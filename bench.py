@@ -58,8 +58,8 @@ NCU_TRAFFIC = {
                                           sha1="07cb49eb164ddb0d6a742f1adc53272e9921193a"),
     ("prefill_attn", "prefill_8k"): dict(bytes=232.378368e6 + 102.237440e6, src="prefill.cu",
                                          sha1="07cb49eb164ddb0d6a742f1adc53272e9921193a"),
-    ("dec_cmp", "decode_64k"): dict(bytes=(84.101120e6 + 2.445312e6) * 32 / 8, src="decode.cu",
-                                    sha1="50df1c75c656cb16dff4c30e0bf690d06dd95c02"),
+    ("dec_cmp", "decode_64k"): dict(bytes=(84.105216e6 + 2.525952e6) * 32 / 8, src="decode.cu",
+                                    sha1="f05f46f2bc4b9132a6e51ff729d2b9e41367e4aa"),
 }
 
 

@@ -36,8 +36,11 @@
  *  - Supported: d_k in {64, 128, 192}, d_v in {64, 128}, G in {1, 2, 4, 8, 16},
  *    l_cmp = 32, stride = 16, l_sel = 64, 1 <= top_n <= 32, window >= 1,
  *    force_first + force_local <= top_n, batch <= NSA_MAX_BATCH.
- *  - Workspace: the first 256 bytes hold a device status word. Call
- *    nsa_workspace_init() once on a new workspace before its first use.
+ *  - Workspace: the first 256 bytes hold a device status word and the work
+ *    counters of the decode pass (back to 0 at the end of every decode call).
+ *    Call nsa_workspace_init() once on a new workspace before its first use.
+ *    A workspace serves one call at a time: calls that share one must be
+ *    ordered (same stream, or events between streams).
  */
 #ifndef NSA_H_
 #define NSA_H_

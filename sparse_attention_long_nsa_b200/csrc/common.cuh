@@ -24,7 +24,9 @@ enum : uint32_t {
 struct WsHeader {
   uint32_t status;
   uint32_t timeout_site;
-  uint32_t pad[62];
+  uint32_t sched_next;    // next work item of a dynamically scheduled kernel (0 between launches)
+  uint32_t sched_done;    // CTAs of that kernel that have finished (0 between launches)
+  uint32_t pad[60];
 };
 
 #ifndef NSA_WAIT_LIMIT_NS

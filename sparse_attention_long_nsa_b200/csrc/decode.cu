@@ -153,8 +153,8 @@ __device__ unsigned long long g_fspan[512][3];
 size_t decode_partials_floats(const DecodeArgs& a) { return part_layout(a).total; }
 
 // ---------------------------------------------------------------------------
-// D1: compressed keys, split into 512-key chunks. Persistent: one CTA per SM walks
-// the (sequence, KV head, chunk) items round-robin; the producer warp keeps the
+// D1: compressed keys, split into 512-key chunks. Persistent: one CTA per SM takes
+// (sequence, KV head, chunk) items from a shared counter; the producer warp keeps the
 // ring full across item boundaries (Q of the next item double-buffered), so the
 // HBM stream never drains between items.
 // ---------------------------------------------------------------------------
@@ -189,6 +189,13 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
   // barrier only once the stage holds its tile (consecutive tiles of one warp are
   // not consecutive uses of a stage, so a parity wait alone could alias)
   volatile int* stage_tag = abort_flag + 1;    // [kD1Stages]
+  volatile int* q_item = stage_tag + kD1Stages;  // [2] item of each Q slot (-1: no more items)
+  volatile int* stg_item = q_item + 2;           // item of the staged states (-1: no more)
+  // items are handed out by a counter in the workspace header, so CTAs whose
+  // stream runs faster take more of them; the last CTA to finish sets the
+  // counter back to 0 for the next launch
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.status);
+  int* item_ctr = reinterpret_cast<int*>(&hdr->sched_next);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G;
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     b = bg / a.H_kv;
     const int L = a.lens[b];
     if (L < 1 || L > a.max_len) {
-      if (chunk == 0 && g == 0 && tid == 0) atomicOr(a.status, DEV_ERR_BOUNDS);
+      if (chunk == 0 && g == 0) atomicOr(a.status, DEV_ERR_BOUNDS);   // called by the producer only
       return 0;
     }
     const int nc = n_cmp_dev(L, a.l, a.s);
@@ -237,12 +244,15 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     if (lane == 0) {
       int u = 0, it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      while (ok) {
+        const int item = atomicAdd(item_ctr, 1);
+        if (item >= n_items) break;
         int b, g, chunk;
         const int ntl = item_tiles(item, b, g, chunk);
         if (ntl == 0) continue;
         const int qi = it & 1;
         if (it >= 2 && !mbar_wait(&q_empty[qi], ((it >> 1) - 1) & 1, abort_flag, a.status, 403)) break;
+        q_item[qi] = item;   // published by the arrival on q_full
         mbar_arrive_expect_tx(&q_full[qi], (uint32_t)(DK / 64) * G * 128);
         for (int kb = 0; kb < DK / 64; ++kb)
           tma_load_3d(qbuf + qi * S::QBUF + kb * 2048, &mp.q, &q_full[qi], kb * 64, g * G, b);
@@ -269,6 +279,14 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
         }
         ++it;
       }
+      // no more items: an empty Q slot tells the consumers
+      if (ok && !*abort_flag) {
+        const int qi = it & 1;
+        if (it < 2 || mbar_wait(&q_empty[qi], ((it >> 1) - 1) & 1, abort_flag, a.status, 408)) {
+          q_item[qi] = -1;
+          mbar_arrive(&q_full[qi]);
+        }
+      }
       if (*abort_flag) {
         // let the copies still in flight land before the CTA exits
         for (int v = u - kD1Stages < 0 ? 0 : u - kD1Stages; v < u; ++v)
@@ -278,33 +296,40 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     }
   } else if (warp == kD1Consumers + 1) {
     // ------------------------------------------------------------ merger
-    int it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      int b, g, chunk;
-      const int ntl = item_tiles(item, b, g, chunk);
-      if (ntl == 0) continue;
+    for (int it = 0;; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(stg_full, it & 1, abort_flag, a.status, 407))) break;
+      const int item = *stg_item;
+      if (item < 0) break;
+      const int chunk = item % a.n_cmp_chunks;
+      const int g = (item / a.n_cmp_chunks) % a.H_kv, b = (item / a.n_cmp_chunks) / a.H_kv;
       const size_t ci = ((size_t)b * a.H_kv + g) * a.n_cmp_chunks + chunk;
       merge_warps_w32<DV, kD1Consumers>(stg, G, a.part + pl.cp_o + ci * G * DV, a.part + pl.cp_ml + ci * G * 2, lane);
       __syncwarp();
       mbar_arrive(stg_free);
-      ++it;
     }
   } else {
     // ------------------------------------------------------------ consumers
     float* ps = pscr + warp * 16 * kTileKeys;
     int u_base = 0, it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      int b, g, chunk;
-      const int ntl = item_tiles(item, b, g, chunk);
-      if (ntl == 0) continue;
+    while (ok) {
       const int qi = it & 1;
-      const int nc = n_cmp_dev(a.lens[b], a.l, a.s);
-      const int c0 = chunk * kCmpChunk;
-      // every warp reaches the three item-end barriers even when a wait gave up
       if (warp == 0) TRC(1, it, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qi], (it >> 1) & 1, abort_flag, a.status, 404));
+      if (!ok) break;
+      const int item = q_item[qi];
+      if (item < 0) {   // no more items: release the merger
+        if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(stg_free, (it - 1) & 1, abort_flag, a.status, 409))) break;
+        if (warp == 0 && lane == 0) *stg_item = -1;
+        mbar_arrive(stg_full);
+        break;
+      }
+      const int chunk = item % a.n_cmp_chunks;
+      const int g = (item / a.n_cmp_chunks) % a.H_kv, b = (item / a.n_cmp_chunks) / a.H_kv;
+      const int nc = n_cmp_dev(a.lens[b], a.l, a.s);
+      const int c0 = chunk * kCmpChunk;
+      const int ntl = min(kTilesPerChunk, (nc - c0 + kTileKeys - 1) / kTileKeys);
+      // every warp reaches the three item-end barriers even when a wait gave up
       if (warp == 0) TRC(1, it, 1);
       const uint32_t qbase = smem_u32(qbuf + qi * S::QBUF);
       RowState<DV> rs;
@@ -380,6 +405,7 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
       if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(stg_free, (it - 1) & 1, abort_flag, a.status, 406)))
         ok = false;
       if (ok) rs.stage(stg + warp * 16 * (DV + 2), lane);
+      if (warp == 0 && lane == 0) *stg_item = item;   // published by the arrival on stg_full
       mbar_arrive(stg_full);
       __syncwarp();
       if (lane == 0) mbar_arrive(&q_empty[qi]);
@@ -390,6 +416,15 @@ __global__ void __launch_bounds__(kD1Threads, 1) dec_cmp_kernel(const DecodeArgs
     }
   }
   __syncthreads();
+  if (tid == 0) {
+    // this CTA's producer has stopped taking items; the last CTA out resets the
+    // counters (kernels after this one in the stream see the reset)
+    __threadfence();
+    if (atomicAdd(&hdr->sched_done, 1u) == gridDim.x - 1) {
+      atomicExch(&hdr->sched_next, 0u);
+      atomicExch(&hdr->sched_done, 0u);
+    }
+  }
 #ifdef NSA_DECODE_TRACE
   if (threadIdx.x == 0 && blockIdx.x < 256) g_cspan[blockIdx.x][1] = globaltimer_ns();
 #endif

@@ -285,6 +285,33 @@ def test_decode_exact_ties_cta_topn():
     assert _ties_checked(st, cfg.params(), cfg.H_kv) > 0
 
 
+def test_decode_work_counter_returns_to_zero():
+    """The compressed decode pass takes its (sequence, KV head, chunk) items from
+    a counter in the workspace header. After every call the counter words are 0
+    again, so calls that reuse one workspace (with fewer items than SMs, and with
+    more) give the same bytes as a call on a fresh workspace."""
+    cfg = CFG["decode_64k"]
+    heads, par = NP.heads_of(cfg), NP.params_of(cfg)
+    for lens in ([1, 700, 20000], [65536] * 8 + [3001, 160000]):
+        inp = W.make_decode_inputs(cfg, device="cuda", lens=lens, seed=47)
+        lens_t = inp["cache_lens"].to("cuda")
+        kc, vc = nsa.compress_cache(inp["k_cache"], inp["v_cache"], inp["w_ck"], inp["pe_k"], inp["w_cv"],
+                                    inp["pe_v"], inp["cache_lens"], heads, par)
+        max_len = int(inp["k_cache"].shape[1])
+        nbytes = nsa.nsa_workspace_size(nsa.NSA_OP_DECODE, heads, par, len(lens), 0, max_len)
+        outs = []
+        for ws in [nsa.alloc_workspace(nbytes, "cuda")] * 3 + [nsa.alloc_workspace(nbytes, "cuda")]:
+            out, sel = nsa.decode(inp["q"], inp["k_cache"], inp["v_cache"], kc, vc, lens_t, max_len, inp["gates"],
+                                  heads, par, ws=ws, want_sel=True)
+            torch.cuda.synchronize()
+            nsa.nsa_check_device_status(ws)
+            hdr = ws[:16].cpu().numpy().view(np.uint32)
+            assert hdr[2] == 0 and hdr[3] == 0, hdr
+            outs.append((out.clone(), sel.clone()))
+        for out, sel in outs[1:]:
+            assert torch.equal(out, outs[0][0]) and torch.equal(sel, outs[0][1])
+
+
 def test_decode_incremental_compressed_cache():
     """A decode loop that appends one token per sequence and step and compresses each
     newly completed block (compress_append) builds the same compressed caches as the
