@@ -438,7 +438,8 @@ def bench_decode(cfg, args, rank, ws, dev, pk):
     }
     if len(set(lens_l)) > 1:
         # load balance of the ragged batch: bytes per sequence, and the compressed
-        # pass's 512-key work items per CTA of its persistent grid
+        # pass's 512-key work items over its persistent grid (each CTA takes the
+        # next item from a counter, so the count per CTA is not fixed)
         items = sum(cfg.H_kv * -(-nsa.n_cmp(L) // 512) for L in lens_l)
         n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
         grid = min(items, n_sm)
@@ -447,7 +448,7 @@ def bench_decode(cfg, args, rank, ws, dev, pk):
             "bytes_per_seq_min": min(per_seq), "bytes_per_seq_max": max(per_seq),
             "bytes_per_seq_mean": sum(per_seq) / len(per_seq),
             "dec_cmp_items": items, "dec_cmp_ctas": grid,
-            "dec_cmp_items_per_cta_max": -(-items // grid), "dec_cmp_items_per_cta_mean": items / grid,
+            "dec_cmp_assignment": "first come, from a counter", "dec_cmp_items_per_cta_mean": items / grid,
             "dec_fine_ctas": B * cfg.H_kv,
         }
     return res
