@@ -235,3 +235,99 @@ def test_paged_entry_points_validate_on_host(L):
     st = L.nsa_compress_append(fake, fake, fake, fake, fake, fake, prev, lens, 2, 512, 31, ctypes.byref(h),
                                ctypes.byref(p), fake, fake, None, fake, 1 << 30, None)
     assert st == nsa.NSA_ERR_INVALID_ARG
+
+
+def _call_backward(L, heads, params, cu, ptr=16, ws_bytes=1 << 62, batch=None):
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    P = ctypes.c_void_p(ptr)
+    return L.nsa_prefill_backward(*([P] * 12), cu_arr, len(cu) - 1 if batch is None else batch, ctypes.byref(heads),
+                                  ctypes.byref(params), *([P] * 8), P, ws_bytes, None)
+
+
+def test_backward_argument_validation_launches_nothing(L):
+    """Every call below is rejected on the host (or has no tokens), so nothing is
+    launched and the fake pointers are never dereferenced."""
+    h = nsa.Heads(64, 4, 192, 128)
+    p = nsa.make_params()
+    assert _call_backward(L, h, p, [0, 100], ptr=0) == nsa.NSA_ERR_INVALID_ARG           # null pointers
+    assert _call_backward(L, h, p, [0, 100], ptr=8) == nsa.NSA_ERR_INVALID_ARG           # misaligned
+    assert _call_backward(L, h, p, [3, 100]) == nsa.NSA_ERR_INVALID_ARG                  # cu_seqlens[0] != 0
+    assert _call_backward(L, h, p, [0, 100, 40]) == nsa.NSA_ERR_INVALID_ARG              # negative length
+    assert _call_backward(L, h, p, [0, 100], batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert _call_backward(L, h, p, [0, 100], batch=nsa.NSA_MAX_BATCH + 1) == nsa.NSA_ERR_UNSUPPORTED
+    assert _call_backward(L, h, p, [0, 100], ws_bytes=256) == nsa.NSA_ERR_WORKSPACE
+    assert _call_backward(L, nsa.Heads(64, 4, 96, 128), p, [0, 100]) == nsa.NSA_ERR_UNSUPPORTED
+    assert _call_backward(L, h, nsa.make_params(top_n=2), [0, 100]) == nsa.NSA_ERR_INVALID_ARG
+    # a sequence whose block list does not fit the query kernel's shared memory
+    assert _call_backward(L, h, p, [0, 1 << 26]) == nsa.NSA_ERR_UNSUPPORTED
+    assert b"too long" in L.nsa_last_error_detail()
+    # no tokens: valid, nothing to do
+    assert _call_backward(L, h, p, [0, 0, 0]) == nsa.NSA_OK
+    # the size query grows with the tokens and rejects what the entry point rejects
+    small = nsa.nsa_workspace_size(nsa.NSA_OP_BACKWARD, h, p, 2, 300, 200)
+    assert 0 < small < nsa.nsa_workspace_size(nsa.NSA_OP_BACKWARD, h, p, 2, 3000, 2000)
+    assert nsa.nsa_workspace_size(nsa.NSA_OP_BACKWARD, nsa.Heads(64, 4, 96, 128), p, 2, 300, 200) == 0
+
+
+def _dsa(H_I=8, d_I=128, top_k=2048, scale=0.0):
+    return nsa.DsaParams(H_I, d_I, top_k, scale)
+
+
+def test_dsa_workspace_size_host_only(L):
+    h = nsa.Heads(64, 4, 192, 128)
+    dp = _dsa()
+    # decode: header + scores [batch, max_len] + kept tokens [batch, top_k], each 256-byte aligned
+    def a256(x):
+        return (x + 255) // 256 * 256
+    assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, h, dp, 32, 0, 65536) == \
+        256 + a256(32 * 65536 * 4) + a256(32 * 2048 * 4)
+    # prefill: the score rows of one chunk of queries fill at most 2^26 floats
+    ws = nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_PREFILL, h, dp, 1, 8192, 8192)
+    assert ws == 256 + a256(8192 * 8192 * 4) + a256(8192 * 2048 * 4)
+    ws_long = nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_PREFILL, h, dp, 1, 65536, 65536)
+    chunk = (1 << 26) // 65536
+    assert ws_long == 256 + a256(chunk * 65536 * 4) + a256(chunk * 2048 * 4)
+    for bad in (_dsa(H_I=0), _dsa(d_I=48), _dsa(H_I=17), _dsa(top_k=0), _dsa(top_k=65537), _dsa(scale=-1.0),
+                _dsa(scale=float("nan"))):
+        assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, h, bad, 1, 0, 100) == 0
+    assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, h, dp, 0, 0, 100) == 0
+    assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_DECODE, h, dp, 1, 0, 0) == 0
+    assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DSA_PREFILL, h, dp, 1, -1, 100) == 0
+    assert nsa.nsa_dsa_workspace_size(nsa.NSA_OP_DECODE, h, dp, 1, 0, 100) == 0
+
+
+def test_dsa_argument_validation_launches_nothing(L):
+    """As for the backward: every call is rejected before a launch."""
+    h = nsa.Heads(64, 4, 192, 128)
+    dp = _dsa()
+
+    def dec(ptr=16, batch=2, Lmax=1000, max_len=1000, dp=dp, heads=h, ws_bytes=1 << 40):
+        P = ctypes.c_void_p(ptr)
+        return L.nsa_dsa_decode(P, P, P, P, P, P, P, batch, Lmax, max_len, ctypes.byref(dp), ctypes.byref(heads), P,
+                                None, None, P, ws_bytes, None)
+
+    assert dec(ptr=0) == nsa.NSA_ERR_INVALID_ARG
+    assert dec(ptr=8) == nsa.NSA_ERR_INVALID_ARG
+    assert dec(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert dec(batch=nsa.NSA_MAX_BATCH + 1) == nsa.NSA_ERR_UNSUPPORTED
+    assert dec(max_len=0) == nsa.NSA_ERR_INVALID_ARG
+    assert dec(Lmax=500) == nsa.NSA_ERR_INVALID_ARG                     # max_len above Lmax
+    assert dec(ws_bytes=1024) == nsa.NSA_ERR_WORKSPACE
+    assert dec(dp=_dsa(d_I=96)) == nsa.NSA_ERR_UNSUPPORTED
+    assert dec(dp=_dsa(top_k=-1)) == nsa.NSA_ERR_INVALID_ARG
+    assert dec(heads=nsa.Heads(64, 4, 192, 96)) == nsa.NSA_ERR_UNSUPPORTED
+
+    def pre(cu, ptr=16, ws_bytes=1 << 40, dp=dp, batch=None):
+        cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+        P = ctypes.c_void_p(ptr)
+        return L.nsa_dsa_prefill(P, P, P, P, P, P, cu_arr, len(cu) - 1 if batch is None else batch,
+                                 ctypes.byref(dp), ctypes.byref(h), P, None, None, P, ws_bytes, None)
+
+    assert pre([0, 100], ptr=0) == nsa.NSA_ERR_INVALID_ARG
+    assert pre([0, 100], ptr=8) == nsa.NSA_ERR_INVALID_ARG
+    assert pre([5, 100]) == nsa.NSA_ERR_INVALID_ARG
+    assert pre([0, 100, 99]) == nsa.NSA_ERR_INVALID_ARG
+    assert pre([0, 100], batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert pre([0, 100], ws_bytes=4096) == nsa.NSA_ERR_WORKSPACE
+    assert pre([0, 100], dp=_dsa(H_I=32)) == nsa.NSA_ERR_UNSUPPORTED
+    assert pre([0, 0, 0]) == nsa.NSA_OK                                  # no tokens: nothing to do
