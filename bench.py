@@ -205,7 +205,9 @@ def dist_setup(n_gpus):
         rank = int(os.environ["RANK"])
         if backend == "nccl":
             torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        # a short limit: ranks waiting on one that failed end with an error, not a hang
+        limit = float(os.environ.get("NSA_PG_TIMEOUT_S", "120"))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=limit))
         return rank, ws
     return 0, 1
 
